@@ -1,0 +1,174 @@
+"""fp64 CPU oracle for decode attention.  TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never links, loads or calls
+it, and it shares no code with the library: the two meet only through the seeded
+input generators in ``mla_kv_cache_b200/workloads.py``, which hold none of the
+method's arithmetic.
+
+The arithmetic lives in ``kvattn_oracle.c`` (plain fp64 loops, three passes).  This
+module builds it with gcc, converts bf16 inputs to fp64 (exact), and calls it one
+batch element at a time so that a 2 GiB bf16 cache never has to exist in fp64 all
+at once.
+"""
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvattn_oracle.c")
+_LOCK = threading.Lock()
+_LIBS = {}
+
+
+def _lib_path(mutant=0, out_dir=None):
+    name = "libkvattn_oracle.so" if mutant == 0 else f"libkvattn_oracle_mutant{mutant}.so"
+    return os.path.join(out_dir or _HERE, name)
+
+
+def build(mutant=0, out_dir=None, force=False):
+    """Compile the oracle with gcc (OpenMP); returns the shared-library path."""
+    path = _lib_path(mutant, out_dir)
+    if (not force and os.path.exists(path)
+            and os.path.getmtime(path) >= os.path.getmtime(_SRC)):
+        return path
+    cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c11",
+           f"-DKVO_MUTANT={int(mutant)}", _SRC, "-o", path + ".tmp", "-lm"]
+    subprocess.run(cmd, check=True, capture_output=True)
+    os.replace(path + ".tmp", path)
+    return path
+
+
+def load(mutant=0, out_dir=None):
+    """Load (building first if needed) the oracle library; cached per variant."""
+    key = (mutant, out_dir)
+    with _LOCK:
+        if key in _LIBS:
+            return _LIBS[key]
+        lib = ctypes.CDLL(build(mutant, out_dir))
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int32)
+        ci, cd = ctypes.c_int, ctypes.c_double
+        lib.kvo_gqa_decode.argtypes = [dp, dp, dp, ip, ci, ci, ci, ci, ci, cd, dp, dp]
+        lib.kvo_gqa_decode.restype = ci
+        lib.kvo_mla_decode.argtypes = [dp, dp, dp, dp, ip, ci, ci, ci, ci, ci, cd, dp, dp]
+        lib.kvo_mla_decode.restype = ci
+        lib.kvo_num_threads.restype = ci
+        lib.kvo_mutant.restype = ci
+        _LIBS[key] = lib
+        return lib
+
+
+def num_threads():
+    """Threads the oracle's parallel regions use (OpenMP)."""
+    return int(load().kvo_num_threads())
+
+
+def _f64(x):
+    """Exact conversion of a torch tensor (any float dtype) or array to contiguous fp64."""
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu")
+        import torch
+        return np.ascontiguousarray(x.to(torch.float64).numpy())
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _lens(seq_lens):
+    if hasattr(seq_lens, "detach"):
+        seq_lens = seq_lens.detach().to("cpu").numpy()
+    return np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+
+
+def gqa_decode_f64(q, k, v, seq_lens, scale, lib=None):
+    """GQA/MQA/MHA decode on fp64 arrays.
+
+    q [B, n_q, d], k and v [B, n_kv, T_max, d], seq_lens [B].
+    Returns (out [B, n_q, d], lse [B, n_q]) as fp64 numpy arrays.
+    """
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    lens = _lens(seq_lens)
+    B, n_q, d = q.shape
+    n_kv, T_max = k.shape[1], k.shape[2]
+    assert k.shape == (B, n_kv, T_max, d) and v.shape == k.shape and lens.shape == (B,)
+    out = np.zeros((B, n_q, d))
+    lse = np.zeros((B, n_q))
+    rc = lib.kvo_gqa_decode(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double),
+                            _ptr(v, ctypes.c_double), _ptr(lens, ctypes.c_int32),
+                            B, n_q, n_kv, d, T_max, float(scale),
+                            _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle kvo_gqa_decode failed ({rc})")
+    return out, lse
+
+
+def mla_decode_f64(q_lat, q_rope, lat, rope, seq_lens, scale, lib=None):
+    """Absorbed MLA decode on fp64 arrays.
+
+    q_lat [B, H, d_c], q_rope [B, H, d_r], lat [B, T_max, d_c], rope [B, T_max, d_r]
+    (d_r may be 0).  Returns (out [B, H, d_c], lse [B, H]).
+    """
+    lib = lib or load()
+    q_lat, q_rope, lat, rope = _f64(q_lat), _f64(q_rope), _f64(lat), _f64(rope)
+    lens = _lens(seq_lens)
+    B, H, d_c = q_lat.shape
+    d_r = q_rope.shape[2]
+    T_max = lat.shape[1]
+    assert lat.shape == (B, T_max, d_c) and rope.shape == (B, T_max, d_r)
+    if d_r == 0:  # keep valid (never dereferenced) pointers for empty arrays
+        q_rope = np.zeros((1,))
+        rope = np.zeros((1,))
+    out = np.zeros((B, H, d_c))
+    lse = np.zeros((B, H))
+    rc = lib.kvo_mla_decode(_ptr(q_lat, ctypes.c_double), _ptr(q_rope, ctypes.c_double),
+                            _ptr(lat, ctypes.c_double), _ptr(rope, ctypes.c_double),
+                            _ptr(lens, ctypes.c_int32), B, H, d_c, d_r, T_max,
+                            float(scale), _ptr(out, ctypes.c_double),
+                            _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle kvo_mla_decode failed ({rc})")
+    return out, lse
+
+
+def gqa_decode(q, k_cache, v_cache, seq_lens, scale, batch_ids=None, lib=None):
+    """Oracle on bf16 (torch) inputs, one batch element at a time.
+
+    Only the first seq_lens[b] cache rows of each sequence are converted and read.
+    batch_ids selects a subset of sequences (all by default); results are returned
+    in that order as (out [len(ids), n_q, d], lse [len(ids), n_q]) fp64 arrays.
+    """
+    lens = _lens(seq_lens)
+    T_max = k_cache.shape[2]
+    ids = range(q.shape[0]) if batch_ids is None else batch_ids
+    outs, lses = [], []
+    for b in ids:
+        T = int(min(max(int(lens[b]), 0), T_max))
+        o, l = gqa_decode_f64(q[b:b + 1], k_cache[b:b + 1, :, :T], v_cache[b:b + 1, :, :T],
+                              np.array([T], dtype=np.int32), scale, lib=lib)
+        outs.append(o[0])
+        lses.append(l[0])
+    return np.stack(outs), np.stack(lses)
+
+
+def mla_decode(q_latent, q_rope, latent_cache, rope_cache, seq_lens, scale, batch_ids=None,
+               lib=None):
+    """Absorbed-MLA oracle on bf16 (torch) inputs, one batch element at a time."""
+    lens = _lens(seq_lens)
+    T_max = latent_cache.shape[1]
+    ids = range(q_latent.shape[0]) if batch_ids is None else batch_ids
+    outs, lses = [], []
+    for b in ids:
+        T = int(min(max(int(lens[b]), 0), T_max))
+        o, l = mla_decode_f64(q_latent[b:b + 1], q_rope[b:b + 1], latent_cache[b:b + 1, :T],
+                              rope_cache[b:b + 1, :T], np.array([T], dtype=np.int32), scale,
+                              lib=lib)
+        outs.append(o[0])
+        lses.append(l[0])
+    return np.stack(outs), np.stack(lses)

@@ -1,0 +1,211 @@
+/*
+ * kvattn_oracle.c -- plain fp64 CPU oracle for single-token decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or call
+ * this file: only the test suite, the smoke check and the benchmark's CPU-baseline
+ * leg use it.  It shares no source, header, table or helper with the CUDA library.
+ *
+ * What it computes is the plain definition of softmax attention for one query
+ * token, written out with naive loops and three passes (max, sum, weighted sum):
+ *
+ *   GQA / MQA / MHA  ("Attention variants: MQA, GQA, and MLA", sections
+ *   "MQA: one KV head for everyone" and "GQA: interpolating with groups";
+ *   "Grouped-Query Attention: Fewer KV Heads, Same Quality", section
+ *   "Writing the formula explicitly" and "The Unified View"):
+ *       head_i = softmax(q_i . K_j^T / sqrt(d)) V_j,  j = the group of head i.
+ *   The pages number heads and groups from 1 and write j = ceil(i * n_kv / n_q);
+ *   with 0-based indices that is j = h / (n_q / n_kv) (consecutive groups, the
+ *   same order as repeat_interleave).  The caller passes the scale explicitly.
+ *
+ *   Absorbed MLA  ("Attention variants: MQA, GQA, and MLA", section "MLA: cache
+ *   a latent, not the keys and values"): W_UK is folded into the query, so head h
+ *   scores  q_lat[h] . c_t + q_rope[h] . r_t  against the cached latent c_t and
+ *   the decoupled RoPE key r_t, and its output is the softmax-weighted sum of the
+ *   latents c_t (W_UV is applied downstream).  Keys and values are the same
+ *   latent vector; the RoPE part enters the score only.
+ *
+ * Readings where the pages are silent (stated once more in the design doc):
+ *   - decode attends to every cached position t < seq_lens[b]; no mask;
+ *   - lse is the natural log of sum_t exp(s_t) with s_t already scaled;
+ *   - an empty sequence (seq_lens[b] == 0) gives out = 0 and lse = -inf;
+ *   - inputs arrive as fp64 arrays (the bf16 values are converted exactly by the
+ *     caller before the call).
+ *
+ * Build:  gcc -O2 -fopenmp -shared -fPIC kvattn_oracle.c -o libkvattn_oracle.so -lm
+ * The optional -DKVO_MUTANT=n plants one deliberate mistake (used only by the
+ * test that proves the pins catch such mistakes); the default build has none.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#ifndef KVO_MUTANT
+#define KVO_MUTANT 0
+#endif
+
+/* Returns the version of the oracle's interface. */
+int kvo_version(void) { return 1; }
+
+/* Returns the planted-mistake id this build carries (0 for the real oracle). */
+int kvo_mutant(void) { return KVO_MUTANT; }
+
+/* Index of the KV head that query head h reads: consecutive groups of n_q/n_kv. */
+static int kv_head_of(int h, int n_q, int n_kv) {
+#if KVO_MUTANT == 1
+    (void)n_q;
+    return h % n_kv;                  /* planted mistake: strided groups */
+#else
+    return h / (n_q / n_kv);
+#endif
+}
+
+/*
+ * GQA / MQA / MHA decode.
+ *   q    [B, n_q, d]
+ *   k, v [B, n_kv, T_max, d]
+ *   seq_lens [B]   (positions t < seq_lens[b] are attended; values are clamped to [0, T_max])
+ *   out  [B, n_q, d],  lse [B, n_q]
+ * Returns 0 on success, -1 on bad arguments, -2 if scratch memory is unavailable.
+ */
+int kvo_gqa_decode(const double *q, const double *k, const double *v,
+                   const int32_t *seq_lens, int B, int n_q, int n_kv, int d,
+                   int T_max, double scale, double *out, double *lse) {
+    if (B < 0 || n_q <= 0 || n_kv <= 0 || d <= 0 || T_max < 0 || n_q % n_kv != 0)
+        return -1;
+    int failed = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < n_q; ++h) {
+            int T = seq_lens[b];
+            if (T < 0) T = 0;
+            if (T > T_max) T = T_max;
+#if KVO_MUTANT == 6
+            if (T > 1) T -= 1;                /* planted mistake: last position dropped */
+#endif
+            const int j = kv_head_of(h, n_q, n_kv);
+            const double *qh = q + ((size_t)b * n_q + h) * d;
+            const double *kb = k + ((size_t)b * n_kv + j) * (size_t)T_max * d;
+#if KVO_MUTANT == 5
+            const double *vb = k + ((size_t)b * n_kv + j) * (size_t)T_max * d; /* planted mistake: values read from K */
+#else
+            const double *vb = v + ((size_t)b * n_kv + j) * (size_t)T_max * d;
+#endif
+            double *oh = out + ((size_t)b * n_q + h) * d;
+            for (int i = 0; i < d; ++i) oh[i] = 0.0;
+            if (T == 0) {
+                lse[(size_t)b * n_q + h] = -INFINITY;
+                continue;
+            }
+            double *s = (double *)malloc(sizeof(double) * (size_t)T);
+            if (!s) {
+#pragma omp atomic write
+                failed = 1;
+                continue;
+            }
+            /* scores */
+            for (int t = 0; t < T; ++t) {
+                double acc = 0.0;
+                for (int i = 0; i < d; ++i) acc += qh[i] * kb[(size_t)t * d + i];
+#if KVO_MUTANT == 2
+                s[t] = acc;                    /* planted mistake: scale dropped */
+#else
+                s[t] = scale * acc;
+#endif
+            }
+            /* pass 1: max */
+            double m = s[0];
+            for (int t = 1; t < T; ++t) if (s[t] > m) m = s[t];
+            /* pass 2: normaliser */
+            double l = 0.0;
+            for (int t = 0; t < T; ++t) l += exp(s[t] - m);
+            /* pass 3: weighted sum of values */
+            for (int t = 0; t < T; ++t) {
+                const double w = exp(s[t] - m) / l;
+                for (int i = 0; i < d; ++i) oh[i] += w * vb[(size_t)t * d + i];
+            }
+#if KVO_MUTANT == 3
+            lse[(size_t)b * n_q + h] = m + log2(l);   /* planted mistake: base-2 log */
+#else
+            lse[(size_t)b * n_q + h] = m + log(l);
+#endif
+            free(s);
+        }
+    }
+    return failed ? -2 : 0;
+}
+
+/*
+ * Absorbed MLA decode.
+ *   q_lat  [B, H, d_c]      query already multiplied by W_UK (latent space)
+ *   q_rope [B, H, d_r]      rotated decoupled-RoPE query part
+ *   lat    [B, T_max, d_c]  cached latents c_t (one per token, shared by all heads)
+ *   rope   [B, T_max, d_r]  cached rotated RoPE keys r_t
+ *   out    [B, H, d_c],  lse [B, H]
+ * d_r may be 0 (then q_rope / rope are not read).
+ */
+int kvo_mla_decode(const double *q_lat, const double *q_rope, const double *lat,
+                   const double *rope, const int32_t *seq_lens, int B, int H,
+                   int d_c, int d_r, int T_max, double scale, double *out,
+                   double *lse) {
+    if (B < 0 || H <= 0 || d_c <= 0 || d_r < 0 || T_max < 0) return -1;
+    int failed = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            int T = seq_lens[b];
+            if (T < 0) T = 0;
+            if (T > T_max) T = T_max;
+            const double *ql = q_lat + ((size_t)b * H + h) * d_c;
+            const double *qr = d_r ? q_rope + ((size_t)b * H + h) * d_r : 0;
+            const double *cb = lat + (size_t)b * T_max * d_c;
+            const double *rb = d_r ? rope + (size_t)b * T_max * d_r : 0;
+            double *oh = out + ((size_t)b * H + h) * d_c;
+            for (int i = 0; i < d_c; ++i) oh[i] = 0.0;
+            if (T == 0) {
+                lse[(size_t)b * H + h] = -INFINITY;
+                continue;
+            }
+            double *s = (double *)malloc(sizeof(double) * (size_t)T);
+            if (!s) {
+#pragma omp atomic write
+                failed = 1;
+                continue;
+            }
+            for (int t = 0; t < T; ++t) {
+                double acc = 0.0;
+                for (int i = 0; i < d_c; ++i) acc += ql[i] * cb[(size_t)t * d_c + i];
+#if KVO_MUTANT != 4
+                for (int i = 0; i < d_r; ++i) acc += qr[i] * rb[(size_t)t * d_r + i];
+#endif                                         /* mutant 4: RoPE term dropped */
+                s[t] = scale * acc;
+            }
+            double m = s[0];
+            for (int t = 1; t < T; ++t) if (s[t] > m) m = s[t];
+            double l = 0.0;
+            for (int t = 0; t < T; ++t) l += exp(s[t] - m);
+            for (int t = 0; t < T; ++t) {
+                const double w = exp(s[t] - m) / l;
+                for (int i = 0; i < d_c; ++i) oh[i] += w * cb[(size_t)t * d_c + i];
+            }
+            lse[(size_t)b * H + h] = m + log(l);
+            free(s);
+        }
+    }
+    return failed ? -2 : 0;
+}
+
+/* Number of OpenMP threads a parallel region of this library uses. */
+int kvo_num_threads(void) {
+    int n = 1;
+#pragma omp parallel
+    {
+#pragma omp single
+        {
+#ifdef _OPENMP
+            extern int omp_get_num_threads(void);
+            n = omp_get_num_threads();
+#endif
+        }
+    }
+    return n;
+}

@@ -1,0 +1,275 @@
+"""Checks that pin the oracle to facts other than itself.
+
+Each check takes the oracle library handle (so the same check can be run against a
+build with a planted mistake) and raises AssertionError on failure.  None of them
+retypes the oracle's formula: they use values the pages print, closed forms,
+invariants, library routines the pages name (PyTorch's scaled_dot_product_attention
+with enable_gqa, as in "Attention variants: MQA, GQA, and MLA", section "Against the
+real libraries") and brute force in pure Python on tiny inputs.
+"""
+import math
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+import oracle
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _gqa_case(seed, B=2, n_q=8, n_kv=2, d=16, T=13, lens=None):
+    r = _rng(seed)
+    q = r.standard_normal((B, n_q, d))
+    k = r.standard_normal((B, n_kv, T, d))
+    v = r.standard_normal((B, n_kv, T, d))
+    if lens is None:
+        lens = r.integers(1, T + 1, size=B)
+    return q, k, v, np.asarray(lens, dtype=np.int32)
+
+
+# --------------------------------------------------------------------------------------
+# Group indexing: GQA equals MHA run on repeat_interleave'd K/V ("Attention variants:
+# MQA, GQA, and MLA", "Implementation, twice"; "KV cache variants: MHA, GQA, MLA",
+# "MHA vs GQA when group_size = 1").  The oracle treats every head independently with
+# the same arithmetic, so the two must agree bit for bit.
+# --------------------------------------------------------------------------------------
+def pin_gqa_equals_mha_on_repeated_kv(lib):
+    for seed, (n_q, n_kv) in enumerate([(8, 2), (8, 4), (8, 1), (6, 3), (12, 4)]):
+        q, k, v, lens = _gqa_case(100 + seed, n_q=n_q, n_kv=n_kv)
+        g = n_q // n_kv
+        o1, l1 = oracle.gqa_decode_f64(q, k, v, lens, 0.3, lib=lib)
+        o2, l2 = oracle.gqa_decode_f64(q, np.repeat(k, g, axis=1), np.repeat(v, g, axis=1),
+                                       lens, 0.3, lib=lib)
+        assert np.array_equal(o1, o2) and np.array_equal(l1, l2), (n_q, n_kv)
+
+
+# --------------------------------------------------------------------------------------
+# Library cross-check: PyTorch SDPA with enable_gqa=True in fp64 on the CPU, atol 1e-12,
+# the check the pages run ("Against the real libraries").  Decode = one query token,
+# no causal mask; positions >= seq_len are masked out.  The log-sum-exp is read off the
+# same routine by appending one extra token whose score is exactly 0 and whose value is
+# a one-hot in an extra dimension: its output weight is 1 / (1 + exp(lse)).
+# --------------------------------------------------------------------------------------
+def _sdpa_reference(q, k, v, lens, scale):
+    B, n_q, d = q.shape
+    n_kv, T = k.shape[1], k.shape[2]
+    qt = torch.from_numpy(q).reshape(B, n_q, 1, d)
+    kt = torch.from_numpy(k)
+    vt = torch.from_numpy(v)
+    # extra token: zero key (score exactly 0), value one-hot in an extra dimension
+    k_ext = torch.cat([kt, torch.zeros(B, n_kv, 1, d, dtype=torch.float64)], dim=2)
+    v_pad = torch.cat([vt, torch.zeros(B, n_kv, T, 1, dtype=torch.float64)], dim=3)
+    extra = torch.zeros(B, n_kv, 1, d + 1, dtype=torch.float64)
+    extra[..., d] = 1.0
+    v_ext = torch.cat([v_pad, extra], dim=2)
+    pos = torch.arange(T + 1)
+    mask = (pos[None, :] < torch.from_numpy(lens.astype(np.int64))[:, None]) | (pos[None, :] == T)
+    mask = mask[:, None, None, :]
+    plain = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask[..., :T], scale=scale,
+                                           enable_gqa=True)
+    ext = F.scaled_dot_product_attention(qt, k_ext, v_ext, attn_mask=mask, scale=scale,
+                                         enable_gqa=True)
+    w0 = ext[..., 0, d]
+    lse = torch.log((1.0 - w0) / w0)
+    return plain[:, :, 0, :].numpy(), lse.numpy()
+
+
+def pin_sdpa_enable_gqa(lib):
+    for seed, (n_q, n_kv, d, T) in enumerate([(8, 2, 32, 64), (4, 4, 8, 5), (16, 1, 16, 40),
+                                              (6, 2, 64, 17)]):
+        q, k, v, lens = _gqa_case(200 + seed, B=3, n_q=n_q, n_kv=n_kv, d=d, T=T)
+        scale = 1.0 / math.sqrt(d)
+        o, l = oracle.gqa_decode_f64(q, k, v, lens, scale, lib=lib)
+        o_ref, l_ref = _sdpa_reference(q, k, v, lens, scale)
+        assert np.allclose(o, o_ref, rtol=0, atol=1e-12), np.abs(o - o_ref).max()
+        assert np.allclose(l, l_ref, rtol=0, atol=1e-10), np.abs(l - l_ref).max()
+
+
+# --------------------------------------------------------------------------------------
+# Closed forms of the softmax-weighted sum.
+# --------------------------------------------------------------------------------------
+def pin_closed_forms(lib):
+    r = _rng(300)
+    d = 8
+    # T = 1: the only weight is 1, so out = v_0 and lse = s_0 = scale * q . k_0
+    q = r.standard_normal((1, 2, d)); k = r.standard_normal((1, 1, 1, d))
+    v = r.standard_normal((1, 1, 1, d))
+    o, l = oracle.gqa_decode_f64(q, k, v, [1], 0.5, lib=lib)
+    assert np.allclose(o[0], v[0, 0, 0][None, :], atol=1e-15)
+    assert np.allclose(l[0], 0.5 * (q[0] @ k[0, 0, 0]), atol=1e-14)
+    # identical keys: uniform weights, out = mean of the values, lse = s + ln T
+    T = 7
+    k = np.repeat(r.standard_normal((1, 1, 1, d)), T, axis=2)
+    v = r.standard_normal((1, 1, T, d))
+    o, l = oracle.gqa_decode_f64(q, k, v, [T], 0.25, lib=lib)
+    assert np.allclose(o[0], v[0, 0].mean(axis=0)[None, :], atol=1e-14)
+    assert np.allclose(l[0], 0.25 * (q[0] @ k[0, 0, 0]) + math.log(T), atol=1e-13)
+    # T = 2: weight of token 0 is the logistic function of s_0 - s_1, lse = logaddexp
+    k = r.standard_normal((1, 1, 2, d)); v = r.standard_normal((1, 1, 2, d))
+    o, l = oracle.gqa_decode_f64(q, k, v, [2], 0.7, lib=lib)
+    for h in range(2):
+        s0, s1 = 0.7 * q[0, h] @ k[0, 0, 0], 0.7 * q[0, h] @ k[0, 0, 1]
+        w0 = 1.0 / (1.0 + math.exp(s1 - s0))
+        assert np.allclose(o[0, h], w0 * v[0, 0, 0] + (1 - w0) * v[0, 0, 1], atol=1e-14)
+        assert abs(l[0, h] - np.logaddexp(s0, s1)) < 1e-13
+
+
+def pin_empty_sequence(lib):
+    q, k, v, _ = _gqa_case(310, B=2, T=4)
+    o, l = oracle.gqa_decode_f64(q, k, v, [0, 3], 1.0, lib=lib)
+    assert np.all(o[0] == 0.0) and np.all(np.isneginf(l[0]))
+    assert np.all(np.isfinite(l[1]))
+
+
+# --------------------------------------------------------------------------------------
+# Brute force in pure Python on tiny inputs (B=1, n_q=2, n_kv=1, d=2, T<=3 and a few
+# more): a direct evaluation of softmax(q K^T * scale) V with math.exp, no arrays.
+# --------------------------------------------------------------------------------------
+def _brute(q, k, v, lens, scale):
+    B, n_q, d = len(q), len(q[0]), len(q[0][0])
+    n_kv = len(k[0])
+    out = [[[0.0] * d for _ in range(n_q)] for _ in range(B)]
+    lse = [[0.0] * n_q for _ in range(B)]
+    for b in range(B):
+        for h in range(n_q):
+            j = h * n_kv // n_q          # the pages' ceil(i * g / h) with 1-based i
+            ws = []
+            for t in range(lens[b]):
+                s = scale * sum(q[b][h][i] * k[b][j][t][i] for i in range(d))
+                ws.append(math.exp(s))
+            z = sum(ws)
+            lse[b][h] = math.log(z) if z > 0 else -math.inf
+            for t in range(lens[b]):
+                for i in range(d):
+                    out[b][h][i] += ws[t] / z * v[b][j][t][i]
+    return np.array(out), np.array(lse)
+
+
+def pin_brute_force_tiny(lib):
+    shapes = [(1, 2, 1, 2, 1), (1, 2, 1, 2, 2), (1, 2, 1, 2, 3), (2, 4, 2, 3, 3),
+              (1, 6, 3, 2, 3), (2, 3, 3, 1, 2)]
+    for i, (B, n_q, n_kv, d, T) in enumerate(shapes):
+        q, k, v, lens = _gqa_case(400 + i, B=B, n_q=n_q, n_kv=n_kv, d=d, T=T)
+        o, l = oracle.gqa_decode_f64(q, k, v, lens, 0.9, lib=lib)
+        ob, lb = _brute(q.tolist(), k.tolist(), v.tolist(), lens.tolist(), 0.9)
+        assert np.allclose(o, ob, atol=1e-13), (i, np.abs(o - ob).max())
+        assert np.allclose(l, lb, atol=1e-13), (i, np.abs(l - lb).max())
+
+
+# --------------------------------------------------------------------------------------
+# Invariants.
+# --------------------------------------------------------------------------------------
+def pin_split_merge(lib):
+    """Attention over [0,T) equals the log-sum-exp merge of attention over any partition
+    of [0,T) into parts (empty parts included, lse = -inf, weight 0).  This is the
+    identity the split-KV combine relies on."""
+    q, k, v, _ = _gqa_case(500, B=1, n_q=4, n_kv=2, d=8, T=23)
+    T = 23
+    whole_o, whole_l = oracle.gqa_decode_f64(q, k, v, [T], 0.4, lib=lib)
+    for cuts in ([0, 5, 5, 17, 23], [0, 1, 2, 3, 23], [0, 23], [0, 11, 23, 23]):
+        parts = []
+        for a, b in zip(cuts[:-1], cuts[1:]):
+            ko = np.ascontiguousarray(k[:, :, a:b]); vo = np.ascontiguousarray(v[:, :, a:b])
+            if b == a:
+                ko = np.zeros((1, 2, 1, 8)); vo = np.zeros((1, 2, 1, 8))
+            parts.append(oracle.gqa_decode_f64(q, ko, vo, [b - a], 0.4, lib=lib))
+        lses = np.stack([p[1] for p in parts])          # [P, 1, n_q]
+        m = lses.max(axis=0)
+        total = m + np.log(np.exp(lses - m).sum(axis=0))
+        merged = sum(np.exp(p[1] - total)[..., None] * p[0] for p in parts)
+        assert np.allclose(total, whole_l, atol=1e-13)
+        assert np.allclose(merged, whole_o, atol=1e-13)
+
+
+def pin_permutation_invariance(lib):
+    q, k, v, _ = _gqa_case(600, B=1, n_q=4, n_kv=2, d=8, T=19)
+    perm = _rng(601).permutation(19)
+    o1, l1 = oracle.gqa_decode_f64(q, k, v, [19], 0.6, lib=lib)
+    o2, l2 = oracle.gqa_decode_f64(q, k[:, :, perm], v[:, :, perm], [19], 0.6, lib=lib)
+    assert np.allclose(o1, o2, atol=1e-14) and np.allclose(l1, l2, atol=1e-13)
+
+
+def pin_scale_equivariance(lib):
+    """Multiplying q by a and the scale by 1/a leaves every score, hence the result, unchanged."""
+    q, k, v, lens = _gqa_case(700)
+    o1, l1 = oracle.gqa_decode_f64(q, k, v, lens, 0.5, lib=lib)
+    o2, l2 = oracle.gqa_decode_f64(4.0 * q, k, v, lens, 0.125, lib=lib)
+    assert np.allclose(o1, o2, atol=1e-14) and np.allclose(l1, l2, atol=1e-13)
+
+
+# --------------------------------------------------------------------------------------
+# MLA.
+# --------------------------------------------------------------------------------------
+def pin_mla_absorbed_equals_explicit(lib):
+    """Absorbed MLA equals MLA with explicit per-head up-projections ("Attention
+    variants: MQA, GQA, and MLA", section "MLA: cache a latent, not the keys and values",
+    the score identity q.(c W_UK) = (q W_UK^T).c and the output identity
+    sum_s w_s c_s W_UV = (sum_s w_s c_s) W_UV).  The explicit path below reconstructs
+    per-head keys and values from the latents and never forms q W_UK^T."""
+    r = _rng(800)
+    H, d_c, d_h, d_r, T = 4, 24, 8, 6, 11
+    W_uk = r.standard_normal((H, d_c, d_h)) / math.sqrt(d_c)
+    W_uv = r.standard_normal((H, d_c, d_h)) / math.sqrt(d_c)
+    q_head = r.standard_normal((H, d_h))
+    q_rope = r.standard_normal((H, d_r))
+    c = r.standard_normal((T, d_c))
+    rr = r.standard_normal((T, d_r))
+    scale = 1.0 / math.sqrt(d_h + d_r)
+    # explicit: per-head K and V from the latents, RoPE key appended to K
+    explicit = np.zeros((H, d_h))
+    for h in range(H):
+        k_h = np.concatenate([c @ W_uk[h], rr], axis=1)          # [T, d_h + d_r]
+        v_h = c @ W_uv[h]                                        # [T, d_h]
+        qh = np.concatenate([q_head[h], q_rope[h]])
+        ref = F.scaled_dot_product_attention(torch.from_numpy(qh)[None, None, None],
+                                             torch.from_numpy(k_h)[None, None],
+                                             torch.from_numpy(v_h)[None, None], scale=scale)
+        explicit[h] = ref[0, 0, 0].numpy()
+    # absorbed: q_lat = W_UK q, attend over latents, then apply W_UV
+    q_lat = np.einsum("hcd,hd->hc", W_uk, q_head)
+    o_lat, _ = oracle.mla_decode_f64(q_lat[None], q_rope[None], c[None], rr[None], [T], scale,
+                                     lib=lib)
+    absorbed = np.einsum("hc,hcd->hd", o_lat[0], W_uv)
+    assert np.allclose(absorbed, explicit, atol=1e-12), np.abs(absorbed - explicit).max()
+
+
+def pin_mla_matches_sdpa(lib):
+    """MLA is MQA whose key is [c || r] and whose value is c (the same latent): checked
+    against SDPA with one KV head (values narrower than keys), fp64, atol 1e-12."""
+    r = _rng(810)
+    B, H, d_c, d_r, T = 2, 6, 16, 4, 9
+    ql = r.standard_normal((B, H, d_c)); qr = r.standard_normal((B, H, d_r))
+    c = r.standard_normal((B, T, d_c)); rr = r.standard_normal((B, T, d_r))
+    lens = np.array([9, 4], dtype=np.int32)
+    scale = 0.2
+    o, _ = oracle.mla_decode_f64(ql, qr, c, rr, lens, scale, lib=lib)
+    for b in range(B):
+        L = int(lens[b])
+        qfull = torch.from_numpy(np.concatenate([ql[b], qr[b]], axis=1))[None, :, None, :]
+        kfull = torch.from_numpy(np.concatenate([c[b, :L], rr[b, :L]], axis=1))[None, None]
+        val = torch.from_numpy(c[b, :L])[None, None]
+        ref = F.scaled_dot_product_attention(qfull, kfull, val, scale=scale, enable_gqa=True)
+        assert np.allclose(o[b], ref[0, :, 0].numpy(), atol=1e-12)
+
+
+def pin_mla_without_rope_is_mqa(lib):
+    """With no RoPE part, absorbed MLA is MQA with K = V = latent (one shared KV head)."""
+    r = _rng(820)
+    B, H, d_c, T = 2, 4, 12, 10
+    ql = r.standard_normal((B, H, d_c)); c = r.standard_normal((B, T, d_c))
+    lens = np.array([10, 6], dtype=np.int32)
+    o1, l1 = oracle.mla_decode_f64(ql, np.zeros((B, H, 0)), c, np.zeros((B, T, 0)), lens, 0.3,
+                                   lib=lib)
+    o2, l2 = oracle.gqa_decode_f64(ql, c[:, None], c[:, None], lens, 0.3, lib=lib)
+    assert np.allclose(o1, o2, atol=1e-14) and np.allclose(l1, l2, atol=1e-13)
+
+
+ALL_PINS = [
+    pin_gqa_equals_mha_on_repeated_kv, pin_sdpa_enable_gqa, pin_closed_forms,
+    pin_empty_sequence, pin_brute_force_tiny, pin_split_merge, pin_permutation_invariance,
+    pin_scale_equivariance, pin_mla_absorbed_equals_explicit, pin_mla_matches_sdpa,
+    pin_mla_without_rope_is_mqa,
+]

@@ -1,0 +1,23 @@
+"""Plant one mistake at a time in the oracle (CPU builds with -DKVO_MUTANT=n) and show
+that the pins catch each one: a strided group index, a dropped scale, a base-2 lse, a
+dropped RoPE term, values read from the key cache, a dropped last position."""
+import pytest
+
+import oracle
+from tests import oracle_pins
+
+MUTANTS = {1: "strided group index", 2: "scale dropped", 3: "base-2 log-sum-exp",
+           4: "MLA RoPE score term dropped", 5: "values read from K", 6: "last position dropped"}
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS), ids=lambda m: MUTANTS[m])
+def test_pins_catch_planted_mistake(mutant, tmp_path):
+    lib = oracle.load(mutant=mutant, out_dir=str(tmp_path))
+    assert lib.kvo_mutant() == mutant
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(lib)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught mutant {mutant} ({MUTANTS[mutant]})"
