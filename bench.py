@@ -1,0 +1,464 @@
+"""Decode-attention benchmark: one JSON line on stdout (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvattn|reference]
+                    [--config NAME] [--no-extra-configs] [--cpu-sample-s S]
+
+A step is one library call covering every sequence of one layer's decode step for the
+workload (all of its query heads, out and lse complete, split-KV combine included).
+The headline workload is the Llama-2-7B-shaped MHA layer (batch 32, 32/32 heads,
+head_dim 128, context 4096); the other workloads are measured on the same line under
+"configs".  Inputs are seeded synthetic tensors resident in HBM before the timed
+region; L2 is flushed (a 256 MiB device write) before every timed step and the flush
+is outside the step's CUDA-event interval.  With N > 1 (torchrun, one rank per GPU)
+every rank runs its own independent batch (replicas: the units of this path are
+independent sequences, there is no collective on the data path); the time is the
+maximum over ranks and the value is the bytes of all ranks over that time.
+
+Metric: decode-attention time per step, bytes per second and fraction of the measured
+HBM peak.  Bytes per step are the algorithmic minimum: q + the touched K/V (or latent +
+RoPE) cache rows + fp32 out + fp32 lse.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+from mla_kv_cache_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+HEADLINE = "mha_b32_h32_d128_t4096"
+METRIC = "decode-attention µs/step, KV-cache GB/s and % of B200 HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ----------------------------------------------------------------------------- bytes / flops
+def step_bytes(cfg, lens):
+    """Algorithmic bytes of one step: q + touched cache rows + out (fp32) + lse (fp32)."""
+    lens = [min(max(int(x), 0), cfg.max_seq_len) for x in lens]
+    if isinstance(cfg, wl.MLAConfig):
+        q = cfg.batch * cfg.n_heads * (cfg.latent_dim + cfg.rope_dim) * 2
+        kv = sum(lens) * (cfg.latent_dim + cfg.rope_dim) * 2
+        out = cfg.batch * cfg.n_heads * cfg.latent_dim * 4
+        lse = cfg.batch * cfg.n_heads * 4
+    else:
+        q = cfg.batch * cfg.n_q_heads * cfg.head_dim * 2
+        kv = 2 * sum(lens) * cfg.n_kv_heads * cfg.head_dim * 2
+        out = cfg.batch * cfg.n_q_heads * cfg.head_dim * 4
+        lse = cfg.batch * cfg.n_q_heads * 4
+    return {"total": q + kv + out + lse, "kv": kv, "q": q, "out": out + lse}
+
+
+def step_flops(cfg, lens):
+    """Algorithmic flops: 2 per multiply-add of the score and the value products."""
+    T = sum(min(max(int(x), 0), cfg.max_seq_len) for x in lens)
+    if isinstance(cfg, wl.MLAConfig):
+        return T * cfg.n_heads * 2 * ((cfg.latent_dim + cfg.rope_dim) + cfg.latent_dim)
+    return T * cfg.n_q_heads * 4 * cfg.head_dim
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "source": "measured (MEASURED_PEAKS.json)"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "source": "fallback (profiling recipe)"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def physical_gpu_id():
+    """nvidia-smi id (index or UUID) of the current CUDA device."""
+    cur = torch.cuda.current_device()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if cur < len(ids):
+            return ids[cur]
+    return str(cur)
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def dist_max(x):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dev = torch.device("cuda") if torch.cuda.is_available() else torch.device("cpu")
+        t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return float(x)
+
+
+def dist_barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def device_inputs(cfg, seed):
+    x = wl.make_inputs(cfg, seed=seed)
+    return x, {k: v.cuda() for k, v in x.items()}
+
+
+def make_call(cfg, d, out, lse, stream):
+    from mla_kv_cache_b200 import binding as kb
+    if isinstance(cfg, wl.MLAConfig):
+        return lambda: kb.kvattn_mla_decode(d["q_latent"], d["q_rope"], d["latent_cache"],
+                                            d["rope_cache"], d["seq_lens"], cfg.scale, out=out,
+                                            lse=lse, stream=stream)
+    return lambda: kb.kvattn_gqa_decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], cfg.scale,
+                                        out=out, lse=lse, stream=stream)
+
+
+def out_shapes(cfg):
+    if isinstance(cfg, wl.MLAConfig):
+        return (cfg.batch, cfg.n_heads, cfg.latent_dim), (cfg.batch, cfg.n_heads)
+    return (cfg.batch, cfg.n_q_heads, cfg.head_dim), (cfg.batch, cfg.n_q_heads)
+
+
+def time_device(call, stream, steps, warmup, flush):
+    """Per-step CUDA-event time (ms) of `call`, L2 flushed before each step (outside the
+    event interval).  Returns the list of step times."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            flush.zero_()
+            call()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            call()
+            ends[i].record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+
+def time_e2e(cfg, d, stream, steps, warmup, flush):
+    """End to end through the public API: every step copies the step's host inputs (q and
+    seq_lens, pinned) to the device, calls the library and reads out and lse back into
+    pinned host memory.  The KV cache is the decode loop's resident state in HBM."""
+    from mla_kv_cache_b200 import binding as kb
+    if isinstance(cfg, wl.MLAConfig):
+        names = ["q_latent", "q_rope", "seq_lens"]
+    else:
+        names = ["q", "seq_lens"]
+    host = {n: d[n].cpu().pin_memory() for n in names}
+    o_shape, l_shape = out_shapes(cfg)
+    out_h = torch.empty(o_shape, dtype=torch.float32).pin_memory()
+    lse_h = torch.empty(l_shape, dtype=torch.float32).pin_memory()
+    dev = dict(d)
+    out = torch.empty(o_shape, dtype=torch.float32, device="cuda")
+    lse = torch.empty(l_shape, dtype=torch.float32, device="cuda")
+    call = make_call(cfg, dev, out, lse, stream)
+
+    def step():
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        call()
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    times = time_device(step, stream, steps, warmup, flush)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = out_h.numel() * 4 + lse_h.numel() * 4
+    return times, h2d, d2h
+
+
+def cpu_baseline(cfg, x, budget_s):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload's sequences."""
+    import oracle
+    lens = x["seq_lens"].tolist()
+    order = list(range(cfg.batch))
+    done, t_used = [], 0.0
+    t0 = time.perf_counter()
+    for b in order:
+        if isinstance(cfg, wl.MLAConfig):
+            oracle.mla_decode(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"],
+                              x["seq_lens"], cfg.scale, batch_ids=[b])
+        else:
+            oracle.gqa_decode(x["q"], x["k_cache"], x["v_cache"], x["seq_lens"], cfg.scale,
+                              batch_ids=[b])
+        done.append(b)
+        t_used = time.perf_counter() - t0
+        if t_used >= budget_s:
+            break
+    sample_lens = [lens[b] for b in done]
+    sub = (wl.MLAConfig if isinstance(cfg, wl.MLAConfig) else wl.GQAConfig)
+    nbytes = step_bytes(cfg, lens)["total"] * (sum(sample_lens) / max(sum(lens), 1))
+    return {"value": nbytes / t_used / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(done)} of {cfg.batch} sequences of {cfg.name} (all their heads), "
+                      f"{t_used:.1f} s of fp64 CPU work incl. exact bf16->fp64 conversion; "
+                      f"bytes scaled by the sample's share of tokens",
+            "us_per_step_extrapolated": t_used * 1e6 * sum(lens) / max(sum(sample_lens), 1)}
+
+
+def measure_config(cfg, steps, warmup, flush, stream, seed, pk, world):
+    x, d = device_inputs(cfg, seed)
+    o_shape, l_shape = out_shapes(cfg)
+    out = torch.empty(o_shape, dtype=torch.float32, device="cuda")
+    lse = torch.empty(l_shape, dtype=torch.float32, device="cuda")
+    call = make_call(cfg, d, out, lse, stream)
+    dist_barrier()
+    torch.cuda.synchronize()
+    times = time_device(call, stream, steps, warmup, flush)
+    torch.cuda.synchronize()
+    dist_barrier()
+    ms = dist_max(sum(times) / len(times))
+    lens = x["seq_lens"].tolist()
+    nb = step_bytes(cfg, lens)
+    fl = step_flops(cfg, lens)
+    gbs = nb["total"] / (ms * 1e-3) / 1e9
+    res = {"us_per_step": ms * 1e3, "us_min": min(times) * 1e3, "gb_per_s": gbs,
+           "kv_gb_per_s": nb["kv"] / (ms * 1e-3) / 1e9, "bytes_per_step": nb["total"],
+           "hbm_frac": gbs / pk["hbm_gbs"], "tflops": fl / (ms * 1e-3) / 1e12,
+           "flops_per_step": fl}
+    if isinstance(cfg, wl.MLAConfig):
+        t_hbm = nb["total"] / (pk["hbm_gbs"] * 1e9)
+        t_tc = fl / (pk["bf16_tflops"] * 1e12)
+        res["roofline_us"] = max(t_hbm, t_tc) * 1e6
+        res["roofline_frac"] = res["roofline_us"] / res["us_per_step"]
+    return x, d, res, times
+
+
+def gpu_arm(args):
+    rank, world, local = dist_setup(args.gpus)
+    from mla_kv_cache_b200 import binding as kb
+    kb.lib()
+    pk = peaks()
+    stream = torch.cuda.Stream()
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    flush = torch.empty(max(256 << 20, 2 * l2), dtype=torch.uint8, device="cuda")
+    seed = 0 + rank * 1000   # each replica its own batch
+
+    head_cfg = wl.CONFIGS[args.config]
+    extras = {}
+    if not args.no_extra_configs:
+        for name in wl.CONFIG_ORDER:
+            if name == args.config:
+                continue
+            try:
+                _, _, res, _ = measure_config(wl.CONFIGS[name], max(args.steps // 10, 20),
+                                              args.warmup, flush, stream, seed, pk, world)
+            except Exception as e:  # an unsupported workload is reported, not hidden
+                res = {"error": str(e).splitlines()[0][:200]}
+            extras[name] = res
+            torch.cuda.empty_cache()
+
+    x, d, res, _ = measure_config(head_cfg, 20, args.warmup, flush, stream, seed, pk, world)
+    o_shape, l_shape = out_shapes(head_cfg)
+    out = torch.empty(o_shape, dtype=torch.float32, device="cuda")
+    lse = torch.empty(l_shape, dtype=torch.float32, device="cuda")
+    call = make_call(head_cfg, d, out, lse, stream)
+    # the timed region proper: exactly K steps, barrier + synchronize on both sides
+    with ClockSampler(physical_gpu_id()) as clk:
+        dist_barrier()
+        torch.cuda.synchronize()
+        times = time_device(call, stream, args.steps, args.warmup, flush)
+        torch.cuda.synchronize()
+        dist_barrier()
+    clocks = clk.summary()
+    ms = dist_max(sum(times) / len(times))
+    lens = x["seq_lens"].tolist()
+    nb = step_bytes(head_cfg, lens)
+    value = nb["total"] * world / (ms * 1e-3) / 1e9
+    e2e_times, h2d, d2h = time_e2e(head_cfg, d, stream, max(args.steps // 10, 20), args.warmup, flush)
+    e2e_ms = dist_max(sum(e2e_times) / len(e2e_times))
+    achieved = nb["total"] / (ms * 1e-3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            traffic = json.load(open(tpath)).get(args.config)
+        except Exception:
+            traffic = None
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, shapes of the workload)",
+        "config": {"workload": args.config, "batch": head_cfg.batch,
+                   "n_q_heads": head_cfg.n_q_heads, "n_kv_heads": head_cfg.n_kv_heads,
+                   "head_dim": head_cfg.head_dim, "seq_len": head_cfg.max_seq_len,
+                   "bytes_per_step": nb["total"],
+                   "l2": "flushed before every timed step (256 MiB device write, outside the timed interval)",
+                   "parallelism": f"replicas x{world}: one independent batch per GPU, no collective"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
+                     "peak_source": pk["source"] + " burst copy bandwidth",
+                     "timed_unit": "one library call: decode kernel + PDL-chained combine kernel"},
+        "e2e": {"value": nb["total"] * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "per step: pinned host q/seq_lens -> device, library call, out/lse -> pinned host; KV cache resident in HBM"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "configs": dict(extras, **{args.config: res}),
+    }
+    if rank == 0 and world == 1 and args.cpu_sample_s > 0:
+        line["cpu_baseline"] = cpu_baseline(head_cfg, x, args.cpu_sample_s)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    _finish()
+
+
+def reference_arm(args):
+    """The oracle on the host cores: same workload, metric and unit; each step is a
+    bounded sample of the workload (a few sequences), scaled by its share of tokens."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    cfg = wl.CONFIGS[args.config]
+    x = wl.make_inputs(cfg, seed=0)
+    lens = x["seq_lens"].tolist()
+    nb = step_bytes(cfg, lens)
+    per_step_seqs = max(1, min(cfg.batch, args.ref_sequences))
+    times, shares = [], []
+    for s in range(args.warmup + args.steps):
+        ids = [(s * per_step_seqs + i) % cfg.batch for i in range(per_step_seqs)]
+        t0 = time.perf_counter()
+        if isinstance(cfg, wl.MLAConfig):
+            oracle.mla_decode(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"],
+                              x["seq_lens"], cfg.scale, batch_ids=ids)
+        else:
+            oracle.gqa_decode(x["q"], x["k_cache"], x["v_cache"], x["seq_lens"], cfg.scale,
+                              batch_ids=ids)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+            shares.append(sum(lens[i] for i in ids) / max(sum(lens), 1))
+    # seconds for a whole step, extrapolated from the sampled share of tokens
+    full_s = statistics.mean(t / sh for t, sh in zip(times, shares))
+    value = nb["total"] / full_s / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16, shapes of the workload)",
+        "config": {"workload": args.config, "bytes_per_step": nb["total"]},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{per_step_seqs} of {cfg.batch} sequences per step (all heads), "
+                                   f"time scaled by their share of tokens"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _finish():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvattn", choices=["kvattn", "reference"])
+    ap.add_argument("--config", default=HEADLINE, choices=wl.CONFIG_ORDER)
+    ap.add_argument("--no-extra-configs", action="store_true")
+    ap.add_argument("--cpu-sample-s", type=float, default=10.0)
+    ap.add_argument("--ref-sequences", type=int, default=2)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,152 @@
+/*
+ * kvattn.h -- C ABI of the kvattn decode-attention library (NVIDIA B200, sm_100a).
+ *
+ * One decode step of attention for a batch of sequences: every sequence contributes
+ * one query token, which attends to all of that sequence's cached keys and values.
+ * Two forms share the library:
+ *
+ *  - kvattn_gqa_decode: multi-head (MHA), grouped-query (GQA) and multi-query (MQA)
+ *    attention.  n_kv_heads KV heads are each shared by a group of
+ *    g = n_q_heads / n_kv_heads consecutive query heads; query head h reads KV head
+ *    h / g.  ("Attention variants: MQA, GQA, and MLA", sections "MQA: one KV head for
+ *    everyone" and "GQA: interpolating with groups"; "Grouped-Query Attention: Fewer
+ *    KV Heads, Same Quality", section "Writing the formula explicitly", where the
+ *    1-based group index ceil(i * n_kv / n_q) is this h / g with 0-based indices.)
+ *
+ *  - kvattn_mla_decode: absorbed multi-head latent attention.  The key up-projection
+ *    is already folded into the query, every head scores the one cached latent per
+ *    token plus a decoupled RoPE key, and the output stays in latent space (the
+ *    value up-projection is applied by the caller).  ("Attention variants: MQA, GQA,
+ *    and MLA", section "MLA: cache a latent, not the keys and values".)
+ *
+ * For each sequence b and query head h, with T = seq_lens[b] and scaled scores
+ * s_t (t < T), both entry points write
+ *      out[b, h, :] = sum_t softmax(s)_t * value_t       (fp32)
+ *      lse[b, h]    = log(sum_t exp(s_t))                 (fp32, natural log)
+ * An empty sequence (T == 0) gives out = 0 and lse = -inf.
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked "device" must point to memory of the device that is current on
+ *    the calling host thread; "host" pointers to host memory.  The library never
+ *    frees, retains or reallocates caller memory.
+ *  - bf16 data is passed as uint16_t bit patterns (IEEE bfloat16).
+ *  - All arrays are dense and row-major in the shape given (last index fastest).
+ *  - Every device pointer must be 16-byte aligned (else KVATTN_ERR_MISALIGNED).
+ *  - out and lse are fully overwritten and must not overlap any input.
+ *  - stream is a cudaStream_t (NULL = the legacy default stream).  The call only
+ *    enqueues work: KVATTN_OK means the kernels were launched; their completion is
+ *    observed through the stream.  Arguments are checked on the host before any work
+ *    is enqueued; an argument error launches nothing.
+ *  - Functions never throw or abort; they return a kvattn_status.
+ *  - Scratch memory: the library keeps one workspace per device, grown with
+ *    cudaMalloc when a call needs more than it holds and kept until
+ *    kvattn_release_workspace().  A call that grows it is not capturable in a CUDA
+ *    graph; issue one call of the largest shape before capturing.  Calls that share a
+ *    device must be ordered (same stream, or synchronised): they share the workspace.
+ *  - Thread safety: entry points may be called from several host threads; the
+ *    workspace is guarded by a mutex, but see the ordering rule above.
+ */
+#ifndef KVATTN_H
+#define KVATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVATTN_VERSION 10000 /* major * 10000 + minor * 100 + patch */
+
+typedef enum {
+    KVATTN_OK = 0,
+    KVATTN_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, n_q % n_kv != 0, non-finite scale, overlap */
+    KVATTN_ERR_UNSUPPORTED = 2, /* valid but not implemented: head_dim, latent/rope width, size limits */
+    KVATTN_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned */
+    KVATTN_ERR_CUDA = 4,        /* a CUDA runtime call failed (see kvattn_last_error_detail) */
+    KVATTN_ERR_NO_MEMORY = 5    /* the workspace could not be allocated */
+} kvattn_status;
+
+/*
+ * GQA / MQA / MHA decode.
+ *   q         device bf16 [batch, n_q_heads, head_dim]   one query token per sequence
+ *   k_cache   device bf16 [batch, n_kv_heads, max_seq_len, head_dim]
+ *   v_cache   device bf16 [batch, n_kv_heads, max_seq_len, head_dim]
+ *             (the pages' cache layout (batch, kv_heads, seq, head_dim), "The KV cache
+ *             bill, worked numerically"; positions >= seq_lens[b] are never read)
+ *   seq_lens  device int32 [batch]   tokens cached for each sequence, 0..max_seq_len;
+ *             values outside that range are clamped on the device (the result for such
+ *             a sequence is then unspecified, but no memory outside the caches is read)
+ *   max_seq_len  cache capacity per sequence (the T stride of the caches), >= 1
+ *   batch, n_q_heads, n_kv_heads   > 0, n_q_heads % n_kv_heads == 0, batch <= 4096
+ *   head_dim  64 or 128 (others: KVATTN_ERR_UNSUPPORTED)
+ *   scale     finite score scale (the pages use 1/sqrt(head_dim))
+ *   out       device fp32 [batch, n_q_heads, head_dim]
+ *   lse       device fp32 [batch, n_q_heads]  (required, natural log)
+ *   stream    cudaStream_t
+ * Limits: batch * n_kv_heads * max_seq_len < 2^31.
+ */
+int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                      const int32_t *seq_lens, int max_seq_len, int batch, int n_q_heads,
+                      int n_kv_heads, int head_dim, float scale, float *out, float *lse,
+                      void *stream);
+
+/*
+ * Absorbed MLA decode (DeepSeek shape: latent_dim 512, rope_dim 64).
+ *   q_latent      device bf16 [batch, n_heads, latent_dim]  queries already multiplied
+ *                 by the key up-projection (they score the latents directly)
+ *   q_rope        device bf16 [batch, n_heads, rope_dim]    rotated decoupled-RoPE queries
+ *   latent_cache  device bf16 [batch, max_seq_len, latent_dim]  one latent per token,
+ *                 shared by all heads; it is both key (with the RoPE part) and value
+ *   rope_cache    device bf16 [batch, max_seq_len, rope_dim]    rotated RoPE keys
+ *   seq_lens      device int32 [batch], as for kvattn_gqa_decode
+ *   max_seq_len   cache capacity per sequence, >= 1
+ *   batch         > 0, <= 4096;  n_heads 1..128
+ *   latent_dim    512;  rope_dim 64 (others: KVATTN_ERR_UNSUPPORTED)
+ *   scale         finite score scale (DeepSeek: 1/sqrt(128 + 64))
+ *   out           device fp32 [batch, n_heads, latent_dim]  (latent space)
+ *   lse           device fp32 [batch, n_heads]
+ * Score of head h at token t: scale * (q_latent[h] . latent_t + q_rope[h] . rope_t).
+ * Precondition: |q_latent| and |latent_cache| values stay within the fp16 range
+ * (65504); the value product runs in fp16 on the tensor cores.
+ */
+int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
+                      const uint16_t *latent_cache, const uint16_t *rope_cache,
+                      const int32_t *seq_lens, int max_seq_len, int batch, int n_heads,
+                      int latent_dim, int rope_dim, float scale, float *out, float *lse,
+                      void *stream);
+
+/* Human-readable name of a kvattn_status value (static string, never NULL). */
+const char *kvattn_status_string(int status);
+
+/* Detail of the last KVATTN_ERR_CUDA / KVATTN_ERR_NO_MEMORY on this host thread. */
+const char *kvattn_last_error_detail(void);
+
+/* KVATTN_VERSION of the loaded library. */
+int kvattn_version(void);
+
+/* Frees the workspace of every device (waits for that device to be idle first). */
+void kvattn_release_workspace(void);
+
+/*
+ * Device-side error flags of the current device.  Every wait inside the kernels is
+ * bounded; a wait that runs out sets a bit here and the kernel returns early (its
+ * output is then invalid).  Bit 0: pipeline data wait, bit 1: pipeline slot wait,
+ * bit 2: cluster peer wait, bit 3: tensor-core completion wait.  Reading synchronises
+ * the device.  Returns a kvattn_status; *flags receives the bits.
+ */
+int kvattn_read_device_flags(unsigned int *flags);
+int kvattn_clear_device_flags(void);
+
+/*
+ * Test and tuning knob (process-wide): when workers > 0 the next calls use exactly
+ * that many workers (CTAs or CTA pairs) and at least min_tiles tiles per worker,
+ * which forces the split/combine path on small inputs.  workers == 0 restores the
+ * built-in heuristic.
+ */
+void kvattn_debug_set_workers(int workers, int min_tiles);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVATTN_H */

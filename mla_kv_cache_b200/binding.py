@@ -1,0 +1,185 @@
+"""Thin ctypes binding of libkvattn.so with the C entry points' names.
+
+Argument marshalling only: tensors are checked for device, dtype, shape and layout,
+their data pointers and the current CUDA stream are passed to the C ABI
+(include/kvattn.h), and a non-zero status is raised as KvattnError.  Every step of the
+computation runs in the library's CUDA kernels; there is no fallback of any kind.  If
+libkvattn.so is missing the first call raises (build it with
+``python -m mla_kv_cache_b200.build``).
+"""
+import ctypes
+import os
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkvattn.so")
+
+KVATTN_OK = 0
+KVATTN_ERR_INVALID_ARG = 1
+KVATTN_ERR_UNSUPPORTED = 2
+KVATTN_ERR_MISALIGNED = 3
+KVATTN_ERR_CUDA = 4
+KVATTN_ERR_NO_MEMORY = 5
+
+# Every function the header declares, with its ctypes signature.
+_c_u16p = ctypes.c_void_p
+_SIGNATURES = {
+    "kvattn_gqa_decode": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p]),
+    "kvattn_mla_decode": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p,
+                                         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p]),
+    "kvattn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "kvattn_last_error_detail": (ctypes.c_char_p, []),
+    "kvattn_version": (ctypes.c_int, []),
+    "kvattn_release_workspace": (None, []),
+    "kvattn_read_device_flags": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint)]),
+    "kvattn_clear_device_flags": (ctypes.c_int, []),
+    "kvattn_debug_set_workers": (None, [ctypes.c_int, ctypes.c_int]),
+}
+
+_lib = None
+_lock = threading.Lock()
+
+
+class KvattnError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        detail = ""
+        if status in (KVATTN_ERR_CUDA, KVATTN_ERR_NO_MEMORY):
+            detail = ": " + lib().kvattn_last_error_detail().decode()
+        super().__init__(f"{where} -> {lib().kvattn_status_string(status).decode()}{detail}")
+
+
+def lib():
+    """The loaded libkvattn.so (loaded on first use; raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(f"{LIB_PATH} is missing: run python -m mla_kv_cache_b200.build")
+                h = ctypes.CDLL(LIB_PATH)
+                for name, (res, args) in _SIGNATURES.items():
+                    f = getattr(h, name)
+                    f.restype = res
+                    f.argtypes = args
+                _lib = h
+    return _lib
+
+
+def _stream_handle(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(t, name, dtype, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def kvattn_gqa_decode(q, k_cache, v_cache, seq_lens, scale, out=None, lse=None, stream=None):
+    """GQA / MQA / MHA decode step (see include/kvattn.h, kvattn_gqa_decode).
+
+    q [B, n_q, d] bf16, k_cache / v_cache [B, n_kv, max_seq_len, d] bf16, seq_lens [B]
+    int32 -- all on the current CUDA device.  Returns (out [B, n_q, d] fp32,
+    lse [B, n_q] fp32); out / lse may be passed in preallocated.
+    """
+    import torch
+    B, n_q, d = q.shape
+    n_kv, T = k_cache.shape[1], k_cache.shape[2]
+    _check(q, "q", torch.bfloat16)
+    _check(k_cache, "k_cache", torch.bfloat16, (B, n_kv, T, d))
+    _check(v_cache, "v_cache", torch.bfloat16, (B, n_kv, T, d))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, n_q, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, n_q), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, (B, n_q, d))
+    _check(lse, "lse", torch.float32, (B, n_q))
+    st = lib().kvattn_gqa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                 seq_lens.data_ptr(), T, B, n_q, n_kv, d, float(scale),
+                                 out.data_ptr(), lse.data_ptr(), _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_gqa_decode")
+    return out, lse
+
+
+def kvattn_mla_decode(q_latent, q_rope, latent_cache, rope_cache, seq_lens, scale, out=None,
+                      lse=None, stream=None):
+    """Absorbed-MLA decode step (see include/kvattn.h, kvattn_mla_decode).
+
+    q_latent [B, H, 512], q_rope [B, H, 64], latent_cache [B, T, 512],
+    rope_cache [B, T, 64] bf16, seq_lens [B] int32.  Returns (out [B, H, 512] fp32,
+    lse [B, H] fp32).
+    """
+    import torch
+    B, H, dc = q_latent.shape
+    dr = q_rope.shape[2]
+    T = latent_cache.shape[1]
+    _check(q_latent, "q_latent", torch.bfloat16)
+    _check(q_rope, "q_rope", torch.bfloat16, (B, H, dr))
+    _check(latent_cache, "latent_cache", torch.bfloat16, (B, T, dc))
+    _check(rope_cache, "rope_cache", torch.bfloat16, (B, T, dr))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, H, dc), dtype=torch.float32, device=q_latent.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q_latent.device)
+    _check(out, "out", torch.float32, (B, H, dc))
+    _check(lse, "lse", torch.float32, (B, H))
+    st = lib().kvattn_mla_decode(q_latent.data_ptr(), q_rope.data_ptr(), latent_cache.data_ptr(),
+                                 rope_cache.data_ptr(), seq_lens.data_ptr(), T, B, H, dc, dr,
+                                 float(scale), out.data_ptr(), lse.data_ptr(),
+                                 _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_mla_decode")
+    return out, lse
+
+
+def kvattn_status_string(status):
+    return lib().kvattn_status_string(int(status)).decode()
+
+
+def kvattn_last_error_detail():
+    return lib().kvattn_last_error_detail().decode()
+
+
+def kvattn_version():
+    return int(lib().kvattn_version())
+
+
+def kvattn_release_workspace():
+    lib().kvattn_release_workspace()
+
+
+def kvattn_read_device_flags():
+    v = ctypes.c_uint(0)
+    st = lib().kvattn_read_device_flags(ctypes.byref(v))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_read_device_flags")
+    return int(v.value)
+
+
+def kvattn_clear_device_flags():
+    st = lib().kvattn_clear_device_flags()
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_clear_device_flags")
+
+
+def kvattn_debug_set_workers(workers, min_tiles=0):
+    lib().kvattn_debug_set_workers(int(workers), int(min_tiles))

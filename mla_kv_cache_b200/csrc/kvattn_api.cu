@@ -1,0 +1,364 @@
+// kvattn_api.cu -- the C ABI of kvattn (include/kvattn.h): argument checks, the work
+// plan, the per-device workspace, TMA descriptors and kernel launches.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/kvattn.h"
+#include "combine.cuh"
+#include "common.cuh"
+#include "gqa_decode.cuh"
+#include "mla_decode.cuh"
+
+using namespace kvattn;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxBatch = 4096;
+
+thread_local char t_detail[256] = "";
+
+int fail_cuda(cudaError_t e, const char *where) {
+    snprintf(t_detail, sizeof(t_detail), "%s: %s", where, cudaGetErrorString(e));
+    return KVATTN_ERR_CUDA;
+}
+
+struct DeviceState {
+    bool init = false;
+    int sms = 0;
+    int max_smem_optin = 0;
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mutex;
+int g_force_workers = 0;
+int g_force_min_tiles = 0;
+
+int device_state(DeviceState **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) {
+        snprintf(t_detail, sizeof(t_detail), "device ordinal %d out of range", dev);
+        return KVATTN_ERR_UNSUPPORTED;
+    }
+    DeviceState &s = g_dev[dev];
+    if (!s.init) {
+        e = cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return fail_cuda(e, "cudaDeviceGetAttribute(SMs)");
+        e = cudaDeviceGetAttribute(&s.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return fail_cuda(e, "cudaDeviceGetAttribute(smem)");
+        s.init = true;
+    }
+    *out = &s;
+    return KVATTN_OK;
+}
+
+// Grows the calling device's workspace to at least `bytes` (caller holds g_mutex).
+int ensure_workspace(DeviceState *s, size_t bytes, void **ws) {
+    if (s->ws_bytes < bytes) {
+        if (s->ws) {
+            cudaError_t e = cudaDeviceSynchronize();
+            if (e != cudaSuccess) return fail_cuda(e, "cudaDeviceSynchronize (workspace grow)");
+            cudaFree(s->ws);
+            s->ws = nullptr;
+            s->ws_bytes = 0;
+        }
+        size_t want = bytes < (1u << 20) ? (1u << 20) : bytes;
+        cudaError_t e = cudaMalloc(&s->ws, want);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            snprintf(t_detail, sizeof(t_detail), "cudaMalloc(%zu): %s", want, cudaGetErrorString(e));
+            return KVATTN_ERR_NO_MEMORY;
+        }
+        s->ws_bytes = want;
+    }
+    *ws = s->ws;
+    return KVATTN_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 tensor [dim2][dim1][dim0] (dim0 fastest), box {box0, box1, 1}.
+int make_map_3d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                uint32_t box0, uint32_t box1, CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) {
+        snprintf(t_detail, sizeof(t_detail), "cuTensorMapEncodeTiled unavailable");
+        return KVATTN_ERR_CUDA;
+    }
+    cuuint64_t dims[3] = {dim0, dim1, dim2};
+    cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(t_detail, sizeof(t_detail), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return KVATTN_ERR_CUDA;
+    }
+    return KVATTN_OK;
+}
+
+int launch_combine(int D, const CombineParams &cp, int units, int rows, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(units, rows, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (D == 64) {
+        cfg.blockDim = dim3(32, 1, 1);
+        e = cudaLaunchKernelEx(&cfg, combine_kernel<64, 2>, cp);
+    } else if (D == 128) {
+        cfg.blockDim = dim3(32, 1, 1);
+        e = cudaLaunchKernelEx(&cfg, combine_kernel<128, 4>, cp);
+    } else {
+        cfg.blockDim = dim3(128, 1, 1);
+        e = cudaLaunchKernelEx(&cfg, combine_kernel<512, 4>, cp);
+    }
+    if (e != cudaSuccess) return fail_cuda(e, "combine launch");
+    return KVATTN_OK;
+}
+
+template <int D, int MT>
+int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &vmap,
+            DeviceState *dev, int units_per_seq, cudaStream_t stream) {
+    using C = GqaCfg<D, MT>;
+    GqaParams p = base;
+    const int smem = C::smem_bytes(p.B);
+    if (smem > dev->max_smem_optin) {
+        snprintf(t_detail, sizeof(t_detail), "needs %d B shared memory", smem);
+        return KVATTN_ERR_UNSUPPORTED;
+    }
+    // Workers: one persistent CTA per SM unless the work is smaller than that.
+    const long long max_tiles =
+        (long long)p.B * units_per_seq * ((p.T_max + C::TILE - 1) / C::TILE);
+    p.min_tiles = g_force_min_tiles > 0 ? g_force_min_tiles : 4;
+    long long workers = g_force_workers > 0 ? g_force_workers : dev->sms;
+    const long long by_size = (max_tiles + p.min_tiles - 1) / p.min_tiles;
+    if (g_force_workers <= 0 && workers > by_size) workers = by_size;
+    if (workers < 1) workers = 1;
+    p.workers = (int)workers;
+
+    void *ws = nullptr;
+    const size_t meta_bytes = ((16 + (size_t)(p.B + 1) * 4) + 255) & ~size_t(255);
+    const size_t lse_bytes = (((size_t)p.workers * 2 * C::HEADS * 4) + 255) & ~size_t(255);
+    const size_t o_bytes = (size_t)p.workers * 2 * C::HEADS * D * 4;
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        int st = ensure_workspace(dev, meta_bytes + lse_bytes + o_bytes, &ws);
+        if (st != KVATTN_OK) return st;
+    }
+    p.ws_meta = ws;
+    p.ws_lse = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes);
+    p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes + lse_bytes);
+
+    auto kern = gqa_decode_kernel<D, MT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaFuncSetAttribute(gqa)");
+    kern<<<p.workers, C::NTHREADS, smem, stream>>>(p, kmap, vmap);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_cuda(e, "gqa decode launch");
+
+    CombineParams cp;
+    cp.ws_meta = p.ws_meta;
+    cp.ws_lse = p.ws_lse;
+    cp.ws_o = p.ws_o;
+    cp.out = p.out;
+    cp.lse = p.lse;
+    cp.B = p.B;
+    cp.n_q = p.n_q;
+    cp.units_per_seq = units_per_seq;
+    cp.heads_per_unit = C::HEADS;
+    cp.n_hb = p.n_hb;
+    cp.n_kv = p.n_kv;
+    cp.g = p.g;
+    const int rows = p.g < C::HEADS ? p.g : C::HEADS;
+    return launch_combine(D, cp, p.B * units_per_seq, rows, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                      const int32_t *seq_lens, int max_seq_len, int batch, int n_q_heads,
+                      int n_kv_heads, int head_dim, float scale, float *out, float *lse,
+                      void *stream) {
+    if (!q || !k_cache || !v_cache || !seq_lens || !out || !lse) return KVATTN_ERR_INVALID_ARG;
+    if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || max_seq_len <= 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if (n_q_heads % n_kv_heads != 0) return KVATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return KVATTN_ERR_UNSUPPORTED;
+    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
+    if ((long long)batch * n_kv_heads * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seq_lens) ||
+        !aligned16(out) || !aligned16(lse))
+        return KVATTN_ERR_MISALIGNED;
+    const size_t q_bytes = (size_t)batch * n_q_heads * head_dim * 2;
+    const size_t kv_bytes = (size_t)batch * n_kv_heads * max_seq_len * head_dim * 2;
+    const size_t out_bytes = (size_t)batch * n_q_heads * head_dim * 4;
+    const size_t lse_bytes = (size_t)batch * n_q_heads * 4;
+    const void *ins[4] = {q, k_cache, v_cache, seq_lens};
+    const size_t in_sz[4] = {q_bytes, kv_bytes, kv_bytes, (size_t)batch * 4};
+    for (int i = 0; i < 4; ++i)
+        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
+            return KVATTN_ERR_INVALID_ARG;
+    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+
+    DeviceState *dev = nullptr;
+    int st = device_state(&dev);
+    if (st != KVATTN_OK) return st;
+
+    const int g = n_q_heads / n_kv_heads;
+    const int MT = g <= 16 ? 1 : 2;
+    const int heads = 16 * MT;
+    const int n_hb = (g + heads - 1) / heads;
+
+    CUtensorMap kmap, vmap;
+    st = make_map_3d(&kmap, k_cache, head_dim, max_seq_len, (uint64_t)batch * n_kv_heads, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != KVATTN_OK) return st;
+    st = make_map_3d(&vmap, v_cache, head_dim, max_seq_len, (uint64_t)batch * n_kv_heads, 64, 64,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != KVATTN_OK) return st;
+
+    GqaParams p = {};
+    p.q = reinterpret_cast<const __nv_bfloat16 *>(q);
+    p.seq_lens = seq_lens;
+    p.out = out;
+    p.lse = lse;
+    p.B = batch;
+    p.n_q = n_q_heads;
+    p.n_kv = n_kv_heads;
+    p.T_max = max_seq_len;
+    p.g = g;
+    p.n_hb = n_hb;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    const int U = n_kv_heads * n_hb;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (head_dim == 128)
+        return MT == 1 ? run_gqa<128, 1>(p, kmap, vmap, dev, U, s) : run_gqa<128, 2>(p, kmap, vmap, dev, U, s);
+    return MT == 1 ? run_gqa<64, 1>(p, kmap, vmap, dev, U, s) : run_gqa<64, 2>(p, kmap, vmap, dev, U, s);
+}
+
+int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
+                      const uint16_t *latent_cache, const uint16_t *rope_cache,
+                      const int32_t *seq_lens, int max_seq_len, int batch, int n_heads,
+                      int latent_dim, int rope_dim, float scale, float *out, float *lse,
+                      void *stream) {
+    if (!q_latent || !q_rope || !latent_cache || !rope_cache || !seq_lens || !out || !lse)
+        return KVATTN_ERR_INVALID_ARG;
+    if (batch <= 0 || n_heads <= 0 || max_seq_len <= 0 || latent_dim <= 0 || rope_dim < 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
+    if (latent_dim != 512 || rope_dim != 64 || n_heads > 128) return KVATTN_ERR_UNSUPPORTED;
+    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
+    if ((long long)batch * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q_latent) || !aligned16(q_rope) || !aligned16(latent_cache) ||
+        !aligned16(rope_cache) || !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
+        return KVATTN_ERR_MISALIGNED;
+    const size_t ql_bytes = (size_t)batch * n_heads * latent_dim * 2;
+    const size_t qr_bytes = (size_t)batch * n_heads * rope_dim * 2;
+    const size_t lat_bytes = (size_t)batch * max_seq_len * latent_dim * 2;
+    const size_t rope_bytes = (size_t)batch * max_seq_len * rope_dim * 2;
+    const size_t out_bytes = (size_t)batch * n_heads * latent_dim * 4;
+    const size_t lse_bytes = (size_t)batch * n_heads * 4;
+    const void *ins[5] = {q_latent, q_rope, latent_cache, rope_cache, seq_lens};
+    const size_t in_sz[5] = {ql_bytes, qr_bytes, lat_bytes, rope_bytes, (size_t)batch * 4};
+    for (int i = 0; i < 5; ++i)
+        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
+            return KVATTN_ERR_INVALID_ARG;
+    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+
+    DeviceState *dev = nullptr;
+    int st = device_state(&dev);
+    if (st != KVATTN_OK) return st;
+    (void)stream;
+    snprintf(t_detail, sizeof(t_detail), "MLA decode kernel not built");
+    return KVATTN_ERR_UNSUPPORTED;
+}
+
+const char *kvattn_status_string(int status) {
+    switch (status) {
+        case KVATTN_OK: return "KVATTN_OK";
+        case KVATTN_ERR_INVALID_ARG: return "KVATTN_ERR_INVALID_ARG";
+        case KVATTN_ERR_UNSUPPORTED: return "KVATTN_ERR_UNSUPPORTED";
+        case KVATTN_ERR_MISALIGNED: return "KVATTN_ERR_MISALIGNED";
+        case KVATTN_ERR_CUDA: return "KVATTN_ERR_CUDA";
+        case KVATTN_ERR_NO_MEMORY: return "KVATTN_ERR_NO_MEMORY";
+        default: return "KVATTN_UNKNOWN_STATUS";
+    }
+}
+
+const char *kvattn_last_error_detail(void) { return t_detail; }
+
+int kvattn_version(void) { return KVATTN_VERSION; }
+
+void kvattn_release_workspace(void) {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    int cur = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess) return;
+    for (int d = 0; d < kMaxDevices; ++d) {
+        if (g_dev[d].ws) {
+            cudaSetDevice(d);
+            cudaDeviceSynchronize();
+            cudaFree(g_dev[d].ws);
+            g_dev[d].ws = nullptr;
+            g_dev[d].ws_bytes = 0;
+        }
+    }
+    cudaSetDevice(cur);
+}
+
+int kvattn_read_device_flags(unsigned int *flags) {
+    if (!flags) return KVATTN_ERR_INVALID_ARG;
+    cudaError_t e = cudaMemcpyFromSymbol(flags, kvattn::g_device_flags, sizeof(unsigned int));
+    if (e != cudaSuccess) return fail_cuda(e, "cudaMemcpyFromSymbol(flags)");
+    return KVATTN_OK;
+}
+
+int kvattn_clear_device_flags(void) {
+    const unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyToSymbol(kvattn::g_device_flags, &zero, sizeof(unsigned int));
+    if (e != cudaSuccess) return fail_cuda(e, "cudaMemcpyToSymbol(flags)");
+    return KVATTN_OK;
+}
+
+void kvattn_debug_set_workers(int workers, int min_tiles) {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    g_force_workers = workers > 0 ? workers : 0;
+    g_force_min_tiles = workers > 0 && min_tiles > 0 ? min_tiles : 0;
+}
+
+}  // extern "C"

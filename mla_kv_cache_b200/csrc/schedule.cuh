@@ -1,0 +1,104 @@
+// schedule.cuh -- how the decode work is cut into pieces for the workers.
+//
+// The work is a stream of KV tiles.  A "unit" is everything one worker would need to
+// finish one output block: for GQA one (sequence, KV head, head block), for MLA one
+// sequence.  Unit u of sequence b holds ceil(len_b / TILE) tiles.  Units are laid end
+// to end (sequence-major), and worker c takes the contiguous tile range
+// [c*W, min((c+1)*W, total)), W = max(ceil(total / workers), min_tiles).  A unit that a
+// worker covers completely is finished by that worker (final out/lse); a unit cut by
+// a worker boundary leaves one partial result per worker that touched it, and the
+// combine kernel merges those by log-sum-exp.
+//
+// Because seq_lens lives on the device, every CTA computes the same decomposition from
+// it (a prefix sum over the batch in shared memory); CTA 0 also publishes it (W, total,
+// the prefix) in the workspace for the combine kernel.  Tiles never straddle two
+// units, and a unit's last tile is loaded shifted back so that it ends at len_b: no
+// load ever touches a cache position >= len_b (a negative start row is zero-filled by
+// the TMA unit).
+#pragma once
+#include <stdint.h>
+
+namespace kvattn {
+
+struct Piece {
+    int b;              // sequence
+    int i;              // unit index within the sequence (GQA: kv_head * n_hb + head block)
+    int n_tiles;        // tiles of this unit
+    int lt0, lt1;       // tiles [lt0, lt1) of the unit belong to this piece
+    long long ustart;   // global tile index of the unit's first tile
+    bool whole;         // the piece is the entire unit
+    int slot;           // workspace slot of a partial piece: 0 or 1
+};
+
+__device__ __forceinline__ int tiles_of(int len, int tile) { return (len + tile - 1) / tile; }
+
+__device__ __forceinline__ int clamp_len(int len, int T_max) {
+    return len < 0 ? 0 : (len > T_max ? T_max : len);
+}
+
+// Warp 0 of the block fills s_prefix[0..B] with the exclusive prefix of tiles per
+// sequence.  The caller synchronises the block afterwards.
+__device__ __forceinline__ void build_tile_prefix(const int32_t *seq_lens, int B, int T_max,
+                                                  int tile, int *s_prefix, int lane) {
+    int running = 0;
+    if (lane == 0) s_prefix[0] = 0;
+    for (int base = 0; base < B; base += 32) {
+        const int idx = base + lane;
+        int v = idx < B ? tiles_of(clamp_len(__ldg(seq_lens + idx), T_max), tile) : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, v, off);
+            if (lane >= off) v += n;
+        }
+        if (idx < B) s_prefix[idx + 1] = running + v;
+        running += __shfl_sync(0xffffffffu, v, 31);
+    }
+}
+
+// Largest b in [0, B) with prefix[b] * U <= p  (p < total): the sequence holding tile p.
+__device__ __forceinline__ int find_seq(const int *s_prefix, int B, int U, long long p) {
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((long long)s_prefix[mid] * U <= p) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ Piece piece_at(const int *s_prefix, int B, int U, long long p,
+                                          long long p_end, long long worker_start) {
+    Piece pc;
+    pc.b = find_seq(s_prefix, B, U, p);
+    pc.n_tiles = s_prefix[pc.b + 1] - s_prefix[pc.b];
+    const long long base = (long long)s_prefix[pc.b] * U;
+    pc.i = (int)((p - base) / pc.n_tiles);
+    pc.ustart = base + (long long)pc.i * pc.n_tiles;
+    pc.lt0 = (int)(p - pc.ustart);
+    const long long rem = p_end - pc.ustart;
+    pc.lt1 = rem < pc.n_tiles ? (int)rem : pc.n_tiles;
+    pc.whole = (pc.lt0 == 0 && pc.lt1 == pc.n_tiles);
+    pc.slot = (pc.ustart <= worker_start) ? 0 : 1;
+    return pc;
+}
+
+// Tiles per worker, identical on every CTA and in the combine kernel.
+__device__ __forceinline__ long long tiles_per_worker(long long total, int workers, int min_tiles) {
+    long long w = (total + workers - 1) / workers;
+    if (w < min_tiles) w = min_tiles;
+    if (w < 1) w = 1;
+    return w;
+}
+
+// Layout of the published decomposition at the start of the workspace.
+struct MetaView {
+    long long *w_total;  // [0] = W, [1] = total
+    int *prefix;         // [B + 1]
+};
+__device__ __forceinline__ MetaView meta_view(void *ws) {
+    MetaView m;
+    m.w_total = reinterpret_cast<long long *>(ws);
+    m.prefix = reinterpret_cast<int *>(reinterpret_cast<long long *>(ws) + 2);
+    return m;
+}
+
+}  // namespace kvattn

@@ -1,0 +1,142 @@
+"""The C ABI on the CPU: the library loads, exports every function include/kvattn.h
+declares, and rejects bad arguments on the host before any device work (no compute
+call is made here: there is no GPU in this test)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mla_kv_cache_b200 import binding as kb
+from mla_kv_cache_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build(quiet=True)
+    return kb.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "kvattn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvattn_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("kvattn_gqa_decode", "kvattn_mla_decode", "kvattn_status_string",
+                     "kvattn_version", "kvattn_release_workspace"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in kb._SIGNATURES, f"binding lacks {name}"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.kvattn_version() == 10000
+    for code, name in [(0, "KVATTN_OK"), (1, "KVATTN_ERR_INVALID_ARG"), (2, "KVATTN_ERR_UNSUPPORTED"),
+                       (3, "KVATTN_ERR_MISALIGNED"), (4, "KVATTN_ERR_CUDA"), (5, "KVATTN_ERR_NO_MEMORY")]:
+        assert lib.kvattn_status_string(code).decode() == name
+    assert lib.kvattn_status_string(99).decode() == "KVATTN_UNKNOWN_STATUS"
+
+
+# Fake, never-dereferenced, 16-byte aligned "device" addresses far apart from each other.
+A = 1 << 40
+
+
+def gqa_args(**kw):
+    args = dict(q=A, k=2 * A, v=3 * A, lens=4 * A, T=512, B=1, nq=8, nkv=2, d=64, scale=0.125,
+                out=5 * A, lse=6 * A, stream=None)
+    args.update(kw)
+    return args
+
+
+def call_gqa(lib, a):
+    return lib.kvattn_gqa_decode(a["q"], a["k"], a["v"], a["lens"], a["T"], a["B"], a["nq"], a["nkv"],
+                                 a["d"], a["scale"], a["out"], a["lse"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(q=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(k=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(v=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(lens=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(out=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(lse=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(B=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(B=-3), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(nq=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(nkv=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(nq=8, nkv=3), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(T=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(d=96), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(d=256), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(B=4097), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(B=4096, nkv=8, nq=8, T=1 << 16), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(q=A + 8), kb.KVATTN_ERR_MISALIGNED),
+    (dict(k=2 * A + 2), kb.KVATTN_ERR_MISALIGNED),
+    (dict(out=5 * A + 4), kb.KVATTN_ERR_MISALIGNED),
+    (dict(lse=6 * A + 12), kb.KVATTN_ERR_MISALIGNED),
+    (dict(out=2 * A + 64), kb.KVATTN_ERR_INVALID_ARG),      # output overlaps the K cache
+    (dict(lse=A), kb.KVATTN_ERR_INVALID_ARG),              # lse overlaps q
+])
+def test_gqa_rejects_bad_arguments(lib, kw, expected):
+    assert call_gqa(lib, gqa_args(**kw)) == expected
+
+
+def mla_args(**kw):
+    args = dict(ql=A, qr=2 * A, lat=3 * A, rope=4 * A, lens=5 * A, T=4096, B=2, H=128, dc=512, dr=64,
+                scale=0.0722, out=6 * A, lse=7 * A, stream=None)
+    args.update(kw)
+    return args
+
+
+def call_mla(lib, a):
+    return lib.kvattn_mla_decode(a["ql"], a["qr"], a["lat"], a["rope"], a["lens"], a["T"], a["B"],
+                                 a["H"], a["dc"], a["dr"], a["scale"], a["out"], a["lse"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(ql=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(rope=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(lse=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(B=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(H=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(T=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(H=129), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(dc=256), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(dr=32), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(B=5000), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(lat=3 * A + 8), kb.KVATTN_ERR_MISALIGNED),
+    (dict(out=3 * A), kb.KVATTN_ERR_INVALID_ARG),
+])
+def test_mla_rejects_bad_arguments(lib, kw, expected):
+    assert call_mla(lib, mla_args(**kw)) == expected
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 2, 16, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        kb.kvattn_gqa_decode(q, k, k, torch.zeros(1, dtype=torch.int32), 0.125)
+
+
+def test_product_path_does_not_reference_the_oracle():
+    """The library sources and the binding never name the oracle (no CPU fallback)."""
+    pkg = os.path.join(ROOT, "mla_kv_cache_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
+                assert "kvattn_oracle" not in text, f
