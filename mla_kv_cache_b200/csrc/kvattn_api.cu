@@ -33,6 +33,11 @@ struct DeviceState {
     int max_smem_optin = 0;
     void *ws = nullptr;
     size_t ws_bytes = 0;
+    struct Func {
+        const void *kern;
+        int smem;
+    } funcs[16] = {};
+    int n_funcs = 0;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -102,9 +107,51 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+// Recently encoded tensor maps of this host thread (a decode loop calls the library
+// with the same cache tensors every step; encoding costs microseconds of host time).
+struct MapKey {
+    const void *base;
+    uint64_t d0, d1, d2;
+    uint32_t b0, b1;
+    int swz;
+    bool operator==(const MapKey &o) const {
+        return base == o.base && d0 == o.d0 && d1 == o.d1 && d2 == o.d2 && b0 == o.b0 && b1 == o.b1 &&
+               swz == o.swz;
+    }
+};
+struct MapEntry {
+    MapKey key;
+    CUtensorMap map;
+    bool valid;
+};
+constexpr int kMapCache = 16;
+thread_local MapEntry t_maps[kMapCache];
+thread_local int t_map_next = 0;
+
+int encode_map_3d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                  uint32_t box0, uint32_t box1, CUtensorMapSwizzle swz);
+
 // 3-D bf16 tensor [dim2][dim1][dim0] (dim0 fastest), box {box0, box1, 1}.
 int make_map_3d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
                 uint32_t box0, uint32_t box1, CUtensorMapSwizzle swz) {
+    const MapKey key{base, dim0, dim1, dim2, box0, box1, (int)swz};
+    for (int i = 0; i < kMapCache; ++i)
+        if (t_maps[i].valid && t_maps[i].key == key) {
+            *map = t_maps[i].map;
+            return KVATTN_OK;
+        }
+    int st = encode_map_3d(map, base, dim0, dim1, dim2, box0, box1, swz);
+    if (st != KVATTN_OK) return st;
+    MapEntry &e = t_maps[t_map_next];
+    t_map_next = (t_map_next + 1) % kMapCache;
+    e.key = key;
+    e.map = *map;
+    e.valid = true;
+    return KVATTN_OK;
+}
+
+int encode_map_3d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1, uint64_t dim2,
+                  uint32_t box0, uint32_t box1, CUtensorMapSwizzle swz) {
     auto fn = encode_fn();
     if (!fn) {
         snprintf(t_detail, sizeof(t_detail), "cuTensorMapEncodeTiled unavailable");
@@ -122,6 +169,25 @@ int make_map_3d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1
         return KVATTN_ERR_CUDA;
     }
     return KVATTN_OK;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device (the largest request
+// seen so far is kept).
+cudaError_t set_smem_limit(const void *kern, DeviceState *dev, int smem) {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    for (int i = 0; i < dev->n_funcs; ++i) {
+        auto &f = dev->funcs[i];
+        if (f.kern == kern) {
+            if (f.smem >= smem) return cudaSuccess;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e == cudaSuccess) f.smem = smem;
+            return e;
+        }
+    }
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess && dev->n_funcs < (int)(sizeof(dev->funcs) / sizeof(dev->funcs[0])))
+        dev->funcs[dev->n_funcs++] = {kern, smem};
+    return e;
 }
 
 int launch_combine(int D, const CombineParams &cp, int units, int rows, cudaStream_t stream) {
@@ -183,7 +249,7 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
     p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes + lse_bytes);
 
     auto kern = gqa_decode_kernel<D, MT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), dev, smem);
     if (e != cudaSuccess) return fail_cuda(e, "cudaFuncSetAttribute(gqa)");
     kern<<<p.workers, C::NTHREADS, smem, stream>>>(p, kmap, vmap);
     e = cudaGetLastError();
