@@ -145,6 +145,29 @@ int kvattn_clear_device_flags(void);
  */
 void kvattn_debug_set_workers(int workers, int min_tiles);
 
+/*
+ * kvattn_gqa_decode without any allocation by the library.  The pages have no
+ * counterpart to this call; it exists for callers that must not have a library call
+ * cudaMalloc: serving engines that reserve nearly all device memory for their own
+ * KV-cache pool, code being recorded into a CUDA graph, and loops that cannot afford
+ * cudaMalloc's implicit synchronisation.
+ *   Arguments, layouts, results and errors are those of kvattn_gqa_decode.
+ *   Scratch: a fixed 6 MiB array inside the library, present on every GPU that loads
+ *   the library until the process exits.  A plan that needs more (only possible with
+ *   kvattn_debug_set_workers forcing many workers) returns KVATTN_ERR_UNSUPPORTED with
+ *   the sizes in kvattn_last_error_detail.  It calls no cudaMalloc, cudaFree or other
+ *   allocating routine.
+ *   The first call on a device looks up the array's device address (once per device,
+ *   with that device current); make that first call before any stream capture.
+ *   All calls share the one array and it keeps the last call's contents: calls that
+ *   overlap on the GPU (different streams without ordering, or several host threads)
+ *   race on it and give wrong results.  Order them on one stream.
+ */
+int kvattn_gqa_decode_noalloc(const uint16_t *q, const uint16_t *k_cache,
+                              const uint16_t *v_cache, const int32_t *seq_lens, int max_seq_len,
+                              int batch, int n_q_heads, int n_kv_heads, int head_dim, float scale,
+                              float *out, float *lse, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -32,6 +32,11 @@ _SIGNATURES = {
                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_float, ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_void_p]),
+    "kvattn_gqa_decode_noalloc": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p,
+                                                 ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                 ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                                 ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_void_p]),
     "kvattn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvattn_last_error_detail": (ctypes.c_char_p, []),
     "kvattn_version": (ctypes.c_int, []),
@@ -148,6 +153,35 @@ def kvattn_mla_decode(q_latent, q_rope, latent_cache, rope_cache, seq_lens, scal
                                  _stream_handle(stream))
     if st != KVATTN_OK:
         raise KvattnError(st, "kvattn_mla_decode")
+    return out, lse
+
+
+def kvattn_gqa_decode_noalloc(q, k_cache, v_cache, seq_lens, scale, out=None, lse=None,
+                              stream=None):
+    """kvattn_gqa_decode without any allocation by the library (include/kvattn.h).
+
+    For callers that cannot let the library allocate device memory; the scratch is a
+    fixed array inside the library that all calls share, so calls must be ordered on
+    one stream.  out / lse are allocated here by torch only when not passed in.
+    """
+    import torch
+    B, n_q, d = q.shape
+    n_kv, T = k_cache.shape[1], k_cache.shape[2]
+    _check(q, "q", torch.bfloat16)
+    _check(k_cache, "k_cache", torch.bfloat16, (B, n_kv, T, d))
+    _check(v_cache, "v_cache", torch.bfloat16, (B, n_kv, T, d))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, n_q, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, n_q), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, (B, n_q, d))
+    _check(lse, "lse", torch.float32, (B, n_q))
+    st = lib().kvattn_gqa_decode_noalloc(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                         seq_lens.data_ptr(), T, B, n_q, n_kv, d, float(scale),
+                                         out.data_ptr(), lse.data_ptr(), _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_gqa_decode_noalloc")
     return out, lse
 
 
