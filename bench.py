@@ -8,8 +8,9 @@ workload (all of its query heads, out and lse complete, split-KV combine include
 The headline workload is the Llama-2-7B-shaped MHA layer (batch 32, 32/32 heads,
 head_dim 128, context 4096); the other workloads are measured on the same line under
 "configs".  Inputs are seeded synthetic tensors resident in HBM before the timed
-region; L2 is flushed (a 256 MiB device write) before every timed step and the flush
-is outside the step's CUDA-event interval.  With N > 1 (torchrun, one rank per GPU)
+region; L2 is flushed before every timed step (a 256 MiB device write, then a read of
+the same buffer so no dirty line is left to write back) and the flush is outside the
+step's CUDA-event interval.  With N > 1 (torchrun, one rank per GPU)
 every rank runs its own independent batch (replicas: the units of this path are
 independent sequences, there is no collective on the data path); the time is the
 maximum over ranks and the value is the bytes of all ranks over that time.
@@ -224,19 +225,27 @@ def out_shapes(cfg):
     return (cfg.batch, cfg.n_q_heads, cfg.head_dim), (cfg.batch, cfg.n_q_heads)
 
 
+def flush_l2(buf):
+    """Evict the step's data from L2: write a buffer twice the L2 size, then read it
+    back, so that L2 holds clean lines (no dirty write-back of the flush itself lands
+    inside the next timed step)."""
+    buf.zero_()
+    buf.view(torch.int64).amax()
+
+
 def time_device(call, stream, steps, warmup, flush):
     """Per-step CUDA-event time (ms) of `call`, L2 flushed before each step (outside the
     event interval).  Returns the list of step times."""
     with torch.cuda.stream(stream):
         for _ in range(warmup):
-            flush.zero_()
+            flush_l2(flush)
             call()
     torch.cuda.synchronize()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     with torch.cuda.stream(stream):
         for i in range(steps):
-            flush.zero_()
+            flush_l2(flush)
             # Keep the GPU busy (outside the timed interval) while the host enqueues the
             # step, so host-side Python latency is not counted as device time.
             torch.cuda._sleep(HOST_HIDE_CYCLES)
@@ -389,7 +398,7 @@ def gpu_arm(args):
                    "n_q_heads": head_cfg.n_q_heads, "n_kv_heads": head_cfg.n_kv_heads,
                    "head_dim": head_cfg.head_dim, "seq_len": head_cfg.max_seq_len,
                    "bytes_per_step": nb["total"],
-                   "l2": "flushed before every timed step (256 MiB device write, outside the timed interval)",
+                   "l2": "flushed before every timed step (256 MiB device write + read-back, outside the timed interval)",
                    "parallelism": f"replicas x{world}: one independent batch per GPU, no collective"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / pk["hbm_gbs"], "traffic": traffic,

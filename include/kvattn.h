@@ -100,7 +100,7 @@ int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
  *   rope_cache    device bf16 [batch, max_seq_len, rope_dim]    rotated RoPE keys
  *   seq_lens      device int32 [batch], as for kvattn_gqa_decode
  *   max_seq_len   cache capacity per sequence, >= 1
- *   batch         > 0, <= 4096;  n_heads 1..128
+ *   batch         > 0, <= 1024;  n_heads 1..128
  *   latent_dim    512;  rope_dim 64 (others: KVATTN_ERR_UNSUPPORTED)
  *   scale         finite score scale (DeepSeek: 1/sqrt(128 + 64))
  *   out           device fp32 [batch, n_heads, latent_dim]  (latent space)

@@ -175,7 +175,7 @@ gqa_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap,
     uint32_t cbar_uses = 0;
     auto consumer_sync = [&]() -> bool {
         mbar_arrive(cbar);
-        return mbar_wait(cbar, (cbar_uses++) & 1u, FLAG_FULL_WAIT, abort_flag);
+        return __all_sync(0xffffffffu, mbar_wait(cbar, (cbar_uses++) & 1u, FLAG_FULL_WAIT, abort_flag)) != 0;
     };
 
     int k = 0;
@@ -216,7 +216,11 @@ gqa_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap,
         for (int lt = pc.lt0; lt < pc.lt1; ++lt, ++k) {
             const int stage = k % C::NST;
             const uint32_t ph = (uint32_t)(k / C::NST) & 1u;
-            if (!mbar_wait(&full[stage], ph, FLAG_FULL_WAIT, abort_flag)) { aborted = true; break; }
+            // warp-uniform: the warp goes on to ldmatrix / mma.sync (warp-collective)
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], ph, FLAG_FULL_WAIT, abort_flag))) {
+                aborted = true;
+                break;
+            }
             const int y = min(lt * C::TILE, len - C::TILE);
             const int tok_lo = lt * C::TILE - y;                       // valid tile rows
             const int tok_hi = min((lt + 1) * C::TILE, len) - y;

@@ -38,6 +38,7 @@ struct DeviceState {
         int smem;
     } funcs[16] = {};
     int n_funcs = 0;
+    int mla_clusters = 0;   // co-resident MLA CTA pairs (0: not queried yet)
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -349,7 +350,7 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
         return KVATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
     if (latent_dim != 512 || rope_dim != 64 || n_heads > 128) return KVATTN_ERR_UNSUPPORTED;
-    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
+    if (batch > mla::MAX_BATCH) return KVATTN_ERR_UNSUPPORTED;
     if ((long long)batch * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
     if (!aligned16(q_latent) || !aligned16(q_rope) || !aligned16(latent_cache) ||
         !aligned16(rope_cache) || !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
@@ -370,9 +371,96 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
     DeviceState *dev = nullptr;
     int st = device_state(&dev);
     if (st != KVATTN_OK) return st;
-    (void)stream;
-    snprintf(t_detail, sizeof(t_detail), "MLA decode kernel not built");
-    return KVATTN_ERR_UNSUPPORTED;
+
+    MlaMaps maps;
+    st = make_map_3d(&maps.lat, latent_cache, 512, max_seq_len, batch, 64, mla::TILE,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != KVATTN_OK) return st;
+    st = make_map_3d(&maps.rope, rope_cache, 64, max_seq_len, batch, 64, mla::TILE,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != KVATTN_OK) return st;
+    st = make_map_3d(&maps.qlat, q_latent, 512, n_heads, batch, 64, mla::HR, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != KVATTN_OK) return st;
+    st = make_map_3d(&maps.qrope, q_rope, 64, n_heads, batch, 64, mla::HR, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != KVATTN_OK) return st;
+
+    MlaParams p = {};
+    p.seq_lens = seq_lens;
+    p.out = out;
+    p.lse = lse;
+    p.B = batch;
+    p.H = n_heads;
+    p.T_max = max_seq_len;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    const int smem = mla::smem_bytes(batch);
+    if (smem > dev->max_smem_optin) {
+        snprintf(t_detail, sizeof(t_detail), "needs %d B shared memory", smem);
+        return KVATTN_ERR_UNSUPPORTED;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(mla_decode_kernel), dev, smem);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaFuncSetAttribute(mla)");
+    // Workers are CTA pairs; a persistent grid must not exceed the pairs that can be
+    // resident at once (a pair needs two SMs of one GPC).
+    if (dev->mla_clusters == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(2 * (dev->sms / 2), 1, 1);
+        cfg.blockDim = dim3(mla::NTHREADS, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void *>(mla_decode_kernel), &cfg);
+        if (e != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = dev->sms / 2;
+        }
+        dev->mla_clusters = n < dev->sms / 2 ? n : dev->sms / 2;
+    }
+    const long long max_tiles = (long long)batch * ((max_seq_len + mla::TILE - 1) / mla::TILE);
+    p.min_tiles = g_force_min_tiles > 0 ? g_force_min_tiles : 4;
+    long long workers = g_force_workers > 0 ? g_force_workers : dev->mla_clusters;
+    const long long by_size = (max_tiles + p.min_tiles - 1) / p.min_tiles;
+    if (g_force_workers <= 0 && workers > by_size) workers = by_size;
+    if (workers < 1) workers = 1;
+    p.workers = (int)workers;
+
+    void *ws = nullptr;
+    const size_t meta_bytes = ((16 + (size_t)(batch + 1) * 4) + 255) & ~size_t(255);
+    const size_t wlse_bytes = (((size_t)p.workers * 2 * mla::HR * 4) + 255) & ~size_t(255);
+    const size_t wo_bytes = (size_t)p.workers * 2 * mla::HR * 512 * 4;
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        st = ensure_workspace(dev, meta_bytes + wlse_bytes + wo_bytes, &ws);
+        if (st != KVATTN_OK) return st;
+    }
+    p.ws_meta = ws;
+    p.ws_lse = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes);
+    p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes + wlse_bytes);
+
+    mla_decode_kernel<<<2 * p.workers, mla::NTHREADS, smem, s>>>(p, maps);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_cuda(e, "mla decode launch");
+
+    CombineParams cp;
+    cp.ws_meta = p.ws_meta;
+    cp.ws_lse = p.ws_lse;
+    cp.ws_o = p.ws_o;
+    cp.out = out;
+    cp.lse = lse;
+    cp.B = batch;
+    cp.n_q = n_heads;
+    cp.units_per_seq = 1;
+    cp.heads_per_unit = mla::HR;
+    cp.n_hb = 1;
+    cp.n_kv = 1;
+    cp.g = n_heads;
+    return launch_combine(512, cp, batch, n_heads, s);
 }
 
 const char *kvattn_status_string(int status) {

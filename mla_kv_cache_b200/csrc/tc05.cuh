@@ -17,6 +17,10 @@
 
 namespace kvattn {
 
+// Warp-uniform outcome of a per-lane wait: warps that go on to issue warp-collective
+// instructions (tcgen05.ld/st, ldmatrix, mma.sync) must never split on an abort.
+__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok) != 0; }
+
 // ---------------------------------------------------------------- cluster
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;

@@ -116,6 +116,7 @@ def call_mla(lib, a):
     (dict(dc=256), kb.KVATTN_ERR_UNSUPPORTED),
     (dict(dr=32), kb.KVATTN_ERR_UNSUPPORTED),
     (dict(B=5000), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(B=1025), kb.KVATTN_ERR_UNSUPPORTED),
     (dict(lat=3 * A + 8), kb.KVATTN_ERR_MISALIGNED),
     (dict(out=3 * A), kb.KVATTN_ERR_INVALID_ARG),
 ])

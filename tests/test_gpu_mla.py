@@ -1,0 +1,81 @@
+"""GPU parity of kvattn_mla_decode (tcgen05 CTA-pair kernel) against the fp64 oracle.
+
+Cache positions >= seq_len are NaN-filled; the full-size DeepSeek-shaped workload is
+compared on every sequence in the bench's launch configuration.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mla_kv_cache_b200 import binding as kb
+from mla_kv_cache_b200 import workloads as wl
+from tests.parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+SCALE = 1.0 / math.sqrt(192.0)
+
+
+@pytest.fixture(autouse=True)
+def _reset_knob():
+    kb.kvattn_debug_set_workers(0, 0)
+    kb.kvattn_clear_device_flags()
+    yield
+    kb.kvattn_debug_set_workers(0, 0)
+    assert kb.kvattn_read_device_flags() == 0, "a bounded wait ran out on the device"
+
+
+def run_case(cfg, seed=0, poison=True, q_gain=1.0):
+    x = wl.make_mla_inputs(cfg, seed=seed, poison_tail=poison)
+    if q_gain != 1.0:  # a power of two keeps the bf16 values exact
+        x["q_latent"] = (x["q_latent"].float() * q_gain).to(torch.bfloat16)
+        x["q_rope"] = (x["q_rope"].float() * q_gain).to(torch.bfloat16)
+    d = {k: v.cuda() for k, v in x.items()}
+    out, lse = kb.kvattn_mla_decode(d["q_latent"], d["q_rope"], d["latent_cache"], d["rope_cache"],
+                                    d["seq_lens"], cfg.scale)
+    torch.cuda.synchronize()
+    ro, rl = oracle.mla_decode(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"],
+                               x["seq_lens"], cfg.scale)
+    assert_close(out.cpu().numpy(), ro, f"{cfg.name} out")
+    assert_close(lse.cpu().numpy(), rl, f"{cfg.name} lse")
+    return out, lse
+
+
+def mla(name, B, H, T, lens=None):
+    return wl.MLAConfig(name, B, H, 512, 64, T, SCALE, seq_lens=tuple(lens) if lens else None)
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 63, 64, 65, 128, 200, 1000])
+def test_lengths(T):
+    run_case(mla(f"T{T}", 2, 128, T, lens=[T, max(T // 3, 1)]))
+
+
+@pytest.mark.parametrize("H", [1, 16, 64, 100, 128])
+def test_head_counts(H):
+    run_case(mla(f"H{H}", 3, H, 300, lens=[300, 129, 5]))
+
+
+def test_ragged_with_empty_sequences():
+    run_case(mla("ragged", 6, 128, 700, lens=[0, 1, 64, 65, 700, 0]))
+
+
+def test_sharp_softmax_rescales():
+    """Queries scaled by 4: the running max keeps growing by more than 2^8 between tiles,
+    which exercises the rescale of the TMEM accumulator."""
+    run_case(mla("sharp", 2, 128, 1500, lens=[1500, 400]), q_gain=4.0)
+
+
+@pytest.mark.parametrize("workers,min_tiles", [(1, 1), (2, 1), (3, 1), (7, 1), (40, 1)])
+def test_forced_splits(workers, min_tiles):
+    kb.kvattn_debug_set_workers(workers, min_tiles)
+    run_case(mla("split", 4, 128, 2000, lens=[2000, 1, 0, 777]))
+
+
+def test_workload_full_size():
+    run_case(wl.CONFIGS["mla_b32_h128_c512_r64_t4096"])
