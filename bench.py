@@ -67,6 +67,14 @@ def step_flops(cfg, lens):
     return T * cfg.n_q_heads * 4 * cfg.head_dim
 
 
+def workload_fields(cfg):
+    if isinstance(cfg, wl.MLAConfig):
+        return {"batch": cfg.batch, "n_heads": cfg.n_heads, "latent_dim": cfg.latent_dim,
+                "rope_dim": cfg.rope_dim, "seq_len": cfg.max_seq_len}
+    return {"batch": cfg.batch, "n_q_heads": cfg.n_q_heads, "n_kv_heads": cfg.n_kv_heads,
+            "head_dim": cfg.head_dim, "seq_len": cfg.max_seq_len}
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -394,9 +402,7 @@ def gpu_arm(args):
         "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16, shapes of the workload)",
-        "config": {"workload": args.config, "batch": head_cfg.batch,
-                   "n_q_heads": head_cfg.n_q_heads, "n_kv_heads": head_cfg.n_kv_heads,
-                   "head_dim": head_cfg.head_dim, "seq_len": head_cfg.max_seq_len,
+        "config": {"workload": args.config, **workload_fields(head_cfg),
                    "bytes_per_step": nb["total"],
                    "l2": "flushed before every timed step (256 MiB device write + read-back, outside the timed interval)",
                    "parallelism": f"replicas x{world}: one independent batch per GPU, no collective"},

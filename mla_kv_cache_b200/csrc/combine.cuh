@@ -10,7 +10,10 @@
 // may start early but wait (griddepcontrol.wait) until the decode grid has finished
 // and its writes are visible.  One CTA per (unit, head row); units covered entirely by
 // one worker were finished by that worker and are skipped; empty sequences get
-// out = 0, lse = -inf here.
+// out = 0, lse = -inf here.  The CTA's warps take the partials round robin, each keeps
+// a running (max, sum, weighted output) -- the same online rescaling as the decode
+// kernels -- with four partials' loads in flight, and the warps' states are merged at
+// the end through shared memory.
 #pragma once
 #include "common.cuh"
 #include "schedule.cuh"
@@ -31,9 +34,14 @@ struct CombineParams {
     int g;                 // query heads per KV head (GQA); n_heads for MLA
 };
 
-// VEC floats per thread, D / VEC threads per CTA.
-template <int D, int VEC>
-__global__ void __launch_bounds__(D / VEC) combine_kernel(const CombineParams p) {
+// D columns, D / 32 floats per lane; NW warps share the partials of one output row.
+template <int D, int NW>
+__global__ void __launch_bounds__(NW * 32) combine_kernel(const CombineParams p) {
+    constexpr int kCombineWarps = NW;
+    constexpr int VEC = D / 32;
+    __shared__ float s_m[kCombineWarps], s_s[kCombineWarps];
+    __shared__ float s_acc[kCombineWarps][D];
+
     pdl_wait_primary();
     const int u = blockIdx.x;                // unit = b * U + i
     const int r = blockIdx.y;                // row within the unit's head block
@@ -44,14 +52,14 @@ __global__ void __launch_bounds__(D / VEC) combine_kernel(const CombineParams p)
     const int hg = hb * p.heads_per_unit + r;
     if (hg >= p.g) return;
     const size_t gh = (size_t)b * p.n_q + (size_t)j * p.g + hg;
-    const int col = threadIdx.x * VEC;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int col = lane * VEC;
 
     const MetaView mv = meta_view(const_cast<void *>(p.ws_meta));
     const long long W = mv.w_total[0];
     const int n_tiles = mv.prefix[b + 1] - mv.prefix[b];
     if (n_tiles == 0) {
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) p.out[gh * D + col + v] = 0.f;
+        for (int c = threadIdx.x; c < D; c += blockDim.x) p.out[gh * D + c] = 0.f;
         if (threadIdx.x == 0) p.lse[gh] = -INFINITY;
         return;
     }
@@ -60,33 +68,70 @@ __global__ void __launch_bounds__(D / VEC) combine_kernel(const CombineParams p)
     const long long c_last = (ustart + n_tiles - 1) / W;
     if (c_first == c_last) return;            // finished by its only worker
 
-    float M = -INFINITY;
-    for (long long c = c_first; c <= c_last; ++c) {
-        const int slot = (ustart <= c * W) ? 0 : 1;
-        M = fmaxf(M, p.ws_lse[((size_t)c * 2 + slot) * p.heads_per_unit + r]);
-    }
+    float m = -INFINITY, S = 0.f;
     float acc[VEC];
 #pragma unroll
     for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
-    float S = 0.f;
-    for (long long c = c_first; c <= c_last; ++c) {
-        const int slot = (ustart <= c * W) ? 0 : 1;
-        const size_t part = ((size_t)c * 2 + slot) * p.heads_per_unit + r;
-        const float w = __expf(p.ws_lse[part] - M);
-        S += w;
-        const float *src = p.ws_o + part * D + col;
-        if (VEC == 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(src);
-            acc[0] += w * x.x; acc[1] += w * x.y; acc[2] += w * x.z; acc[3] += w * x.w;
-        } else {
+    constexpr int UNROLL = 4;
+    for (long long c0 = c_first + warp; c0 <= c_last; c0 += (long long)kCombineWarps * UNROLL) {
+        float ls[UNROLL];
+        float ov[UNROLL][VEC];
 #pragma unroll
-            for (int v = 0; v < VEC; ++v) acc[v] += w * src[v];
+        for (int q = 0; q < UNROLL; ++q) {
+            const long long c = c0 + (long long)q * kCombineWarps;
+            ls[q] = -INFINITY;
+            if (c <= c_last) {
+                const int slot = (ustart <= c * W) ? 0 : 1;
+                const size_t part = ((size_t)c * 2 + slot) * p.heads_per_unit + r;
+                ls[q] = p.ws_lse[part];
+                const float4 *src = reinterpret_cast<const float4 *>(p.ws_o + part * D + col);
+#pragma unroll
+                for (int v = 0; v < VEC / 4; ++v) {
+                    const float4 x = src[v];
+                    ov[q][4 * v] = x.x; ov[q][4 * v + 1] = x.y; ov[q][4 * v + 2] = x.z; ov[q][4 * v + 3] = x.w;
+                }
+                if (VEC % 4 != 0)
+                    for (int v = (VEC / 4) * 4; v < VEC; ++v) ov[q][v] = p.ws_o[part * D + col + v];
+            } else {
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) ov[q][v] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < UNROLL; ++q) {
+            if (ls[q] == -INFINITY) continue;
+            const float mn = fmaxf(m, ls[q]);
+            const float a = __expf(m - mn);       // 0 while m is still -inf
+            const float w = __expf(ls[q] - mn);
+            S = S * a + w;
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) acc[v] = acc[v] * a + w * ov[q][v];
+            m = mn;
         }
     }
-    const float inv = 1.f / S;
+    if (lane == 0) { s_m[warp] = m; s_s[warp] = S; }
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) p.out[gh * D + col + v] = acc[v] * inv;
-    if (threadIdx.x == 0) p.lse[gh] = M + __logf(S);
+    for (int v = 0; v < VEC; ++v) s_acc[warp][col + v] = acc[v];
+    __syncthreads();
+    if (warp != 0) return;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) M = fmaxf(M, s_m[w]);
+    float tot = 0.f;
+    float res[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) res[v] = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) {
+        const float f = (s_m[w] == -INFINITY) ? 0.f : __expf(s_m[w] - M);
+        tot += s_s[w] * f;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) res[v] += s_acc[w][col + v] * f;
+    }
+    const float inv = 1.f / tot;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) p.out[gh * D + col + v] = res[v] * inv;
+    if (lane == 0) p.lse[gh] = M + __logf(tot);
 }
 
 }  // namespace kvattn

@@ -6,11 +6,11 @@
 // ("Attention variants: MQA, GQA, and MLA", section "Against the real libraries": index
 // each query head into its group's KV tile instead of materialising the repeat).
 //
-// Warp roles (160 threads):
-//   warp 4, lane 0  producer: TMA tiled loads (128-byte swizzle, no multicast) of the K
+// Warp roles (160 threads; 288 when the group needs two m-tiles):
+//   last warp, lane 0  producer: TMA tiled loads (128-byte swizzle, no multicast) of the K
 //                   and V tiles into an NST-stage ring guarded by full/empty mbarriers;
 //                   the KV stream is tagged evict-first in L2.
-//   warps 0..3      consumers: the group's query heads are the M rows of warp-level
+//   other warps     consumers: the group's query heads are the M rows of warp-level
 //                   m16n8k16 bf16 MMAs (16 heads per m-tile, zero rows when g < 16).
 //                   Scores S = Q K^T and the update O += P V run on the tensor path;
 //                   the online softmax (running max m, running sum l, rescale of O by
@@ -45,8 +45,8 @@ struct GqaParams {
 template <int D, int MT>
 struct GqaCfg {
     static constexpr int TILE = 64;                       // tokens per pipeline stage
-    static constexpr int NST = (D == 128) ? 5 : 8;        // pipeline depth
-    static constexpr int NCW = 4;                         // consumer warps
+    static constexpr int NST = (D == 128) ? (MT == 1 ? 5 : 4) : 8;   // pipeline depth
+    static constexpr int NCW = 4 * MT;                    // consumer warps (16 tokens each)
     static constexpr int NTHREADS = (NCW + 1) * 32;
     static constexpr int NTS = NCW / MT;                  // token slots per tile
     static constexpr int TOK_PER_WARP = TILE / NTS;       // 16 or 32

@@ -191,7 +191,29 @@ cudaError_t set_smem_limit(const void *kern, DeviceState *dev, int smem) {
     return e;
 }
 
-int launch_combine(int D, const CombineParams &cp, int units, int rows, cudaStream_t stream) {
+template <int D>
+cudaError_t launch_combine_d(cudaLaunchConfig_t &cfg, const CombineParams &cp, int warps) {
+    cfg.blockDim = dim3(warps * 32, 1, 1);
+    switch (warps) {
+        case 1: return cudaLaunchKernelEx(&cfg, combine_kernel<D, 1>, cp);
+        case 2: return cudaLaunchKernelEx(&cfg, combine_kernel<D, 2>, cp);
+        case 4: return cudaLaunchKernelEx(&cfg, combine_kernel<D, 4>, cp);
+        default: return cudaLaunchKernelEx(&cfg, combine_kernel<D, 8>, cp);
+    }
+}
+
+// Warps per combine CTA from the partials one unit is expected to have (about four
+// partials per warp, so the loads of a warp overlap).
+int combine_warps(long long tiles_per_unit_max, long long total_tiles_max, int workers) {
+    const long long w = (total_tiles_max + workers - 1) / workers;
+    const long long parts = (tiles_per_unit_max + (w > 0 ? w : 1) - 1) / (w > 0 ? w : 1) + 1;
+    if (parts <= 4) return 1;
+    if (parts <= 8) return 2;
+    if (parts <= 16) return 4;
+    return 8;
+}
+
+int launch_combine(int D, const CombineParams &cp, int units, int rows, cudaStream_t stream, int warps) {
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -202,16 +224,12 @@ int launch_combine(int D, const CombineParams &cp, int units, int rows, cudaStre
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    if (D == 64) {
-        cfg.blockDim = dim3(32, 1, 1);
-        e = cudaLaunchKernelEx(&cfg, combine_kernel<64, 2>, cp);
-    } else if (D == 128) {
-        cfg.blockDim = dim3(32, 1, 1);
-        e = cudaLaunchKernelEx(&cfg, combine_kernel<128, 4>, cp);
-    } else {
-        cfg.blockDim = dim3(128, 1, 1);
-        e = cudaLaunchKernelEx(&cfg, combine_kernel<512, 4>, cp);
-    }
+    if (D == 64)
+        e = launch_combine_d<64>(cfg, cp, warps);
+    else if (D == 128)
+        e = launch_combine_d<128>(cfg, cp, warps);
+    else
+        e = launch_combine_d<512>(cfg, cp, warps);
     if (e != cudaSuccess) return fail_cuda(e, "combine launch");
     return KVATTN_OK;
 }
@@ -270,7 +288,8 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
     cp.n_kv = p.n_kv;
     cp.g = p.g;
     const int rows = p.g < C::HEADS ? p.g : C::HEADS;
-    return launch_combine(D, cp, p.B * units_per_seq, rows, stream);
+    return launch_combine(D, cp, p.B * units_per_seq, rows, stream,
+                          combine_warps((p.T_max + C::TILE - 1) / C::TILE, max_tiles, p.workers));
 }
 
 }  // namespace
@@ -385,6 +404,8 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
     if (st != KVATTN_OK) return st;
 
     MlaParams p = {};
+    p.q_latent = reinterpret_cast<const __nv_bfloat16 *>(q_latent);
+    p.q_rope = reinterpret_cast<const __nv_bfloat16 *>(q_rope);
     p.seq_lens = seq_lens;
     p.out = out;
     p.lse = lse;
@@ -460,7 +481,8 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
     cp.n_hb = 1;
     cp.n_kv = 1;
     cp.g = n_heads;
-    return launch_combine(512, cp, batch, n_heads, s);
+    return launch_combine(512, cp, batch, n_heads, s,
+                          combine_warps((max_seq_len + mla::TILE - 1) / mla::TILE, max_tiles, p.workers));
 }
 
 const char *kvattn_status_string(int status) {
@@ -610,7 +632,8 @@ int run_gqa_noalloc(const GqaParams &base, const CUtensorMap &kmap, const CUtens
     cp.n_kv = p.n_kv;
     cp.g = p.g;
     const int rows = p.g < C::HEADS ? p.g : C::HEADS;
-    return launch_combine(D, cp, p.B * units_per_seq, rows, stream);
+    return launch_combine(D, cp, p.B * units_per_seq, rows, stream,
+                          combine_warps((p.T_max + C::TILE - 1) / C::TILE, max_tiles, p.workers));
 }
 
 }  // namespace
