@@ -146,6 +146,17 @@ int kvattn_clear_device_flags(void);
 void kvattn_debug_set_workers(int workers, int min_tiles);
 
 /*
+ * Test and tuning knob (process-wide): which kernel kvattn_gqa_decode runs.
+ *   0  built-in choice (the tensor-memory kernel for head_dim 128 and groups of at
+ *      least 4 query heads, the warp-level kernel otherwise)
+ *   1  always the warp-level MMA kernel
+ *   2  always the tensor-memory (tcgen05) kernel; calls it cannot serve (head_dim 64,
+ *      or a batch too large for its shared memory) return KVATTN_ERR_UNSUPPORTED
+ * Other values mean 0.  kvattn_gqa_decode_noalloc always runs the warp-level kernel.
+ */
+void kvattn_debug_set_gqa_kernel(int which);
+
+/*
  * kvattn_gqa_decode without any allocation by the library.  The pages have no
  * counterpart to this call; it exists for callers that must not have a library call
  * cudaMalloc: serving engines that reserve nearly all device memory for their own

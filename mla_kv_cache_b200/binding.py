@@ -44,6 +44,7 @@ _SIGNATURES = {
     "kvattn_read_device_flags": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint)]),
     "kvattn_clear_device_flags": (ctypes.c_int, []),
     "kvattn_debug_set_workers": (None, [ctypes.c_int, ctypes.c_int]),
+    "kvattn_debug_set_gqa_kernel": (None, [ctypes.c_int]),
 }
 
 _lib = None
@@ -217,3 +218,8 @@ def kvattn_clear_device_flags():
 
 def kvattn_debug_set_workers(workers, min_tiles=0):
     lib().kvattn_debug_set_workers(int(workers), int(min_tiles))
+
+
+def kvattn_debug_set_gqa_kernel(which):
+    """0: built-in choice, 1: warp-level MMA kernel, 2: tcgen05 kernel."""
+    lib().kvattn_debug_set_gqa_kernel(int(which))

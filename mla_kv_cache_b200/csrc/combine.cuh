@@ -8,12 +8,14 @@
 //
 // Launched right after the decode kernel with programmatic dependent launch: the CTAs
 // may start early but wait (griddepcontrol.wait) until the decode grid has finished
-// and its writes are visible.  One CTA per (unit, head row); units covered entirely by
-// one worker were finished by that worker and are skipped; empty sequences get
-// out = 0, lse = -inf here.  The CTA's warps take the partials round robin, each keeps
-// a running (max, sum, weighted output) -- the same online rescaling as the decode
-// kernels -- with four partials' loads in flight, and the warps' states are merged at
-// the end through shared memory.
+// and its writes are visible.  Before that wait each CTA derives the work split from
+// seq_lens itself (the same integer arithmetic as the decode kernels, schedule.cuh), so
+// that after it the partials' loads go out at once.  One CTA per (unit, head row);
+// units covered entirely by one worker were finished by that worker and are skipped;
+// empty sequences get out = 0, lse = -inf here.  The CTA's warps take the partials
+// round robin, each keeps a running (max, sum, weighted output) -- the same online
+// rescaling as the decode kernels -- with up to eight partials' loads in flight, and the
+// warps' states are merged at the end through shared memory.
 #pragma once
 #include "common.cuh"
 #include "schedule.cuh"
@@ -21,7 +23,7 @@
 namespace kvattn {
 
 struct CombineParams {
-    const void *ws_meta;
+    const int32_t *seq_lens;
     const float *ws_lse;   // [workers, 2, heads_per_unit]
     const float *ws_o;     // [workers, 2, heads_per_unit, D]
     float *out;            // [B, n_q, D]
@@ -32,6 +34,10 @@ struct CombineParams {
     int n_hb;              // head blocks per group (GQA); 1 for MLA
     int n_kv;              // KV heads (GQA); 1 for MLA
     int g;                 // query heads per KV head (GQA); n_heads for MLA
+    int T_max;             // cache capacity per sequence
+    int tile;              // tokens per tile of the decode kernel
+    int workers;           // decode workers (CTAs or CTA pairs)
+    int min_tiles;         // the decode kernel's minimum tiles per worker
 };
 
 // D columns, D / 32 floats per lane; NW warps share the partials of one output row.
@@ -42,7 +48,6 @@ __global__ void __launch_bounds__(NW * 32) combine_kernel(const CombineParams p)
     __shared__ float s_m[kCombineWarps], s_s[kCombineWarps];
     __shared__ float s_acc[kCombineWarps][D];
 
-    pdl_wait_primary();
     const int u = blockIdx.x;                // unit = b * U + i
     const int r = blockIdx.y;                // row within the unit's head block
     const int b = u / p.units_per_seq;
@@ -55,24 +60,44 @@ __global__ void __launch_bounds__(NW * 32) combine_kernel(const CombineParams p)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int col = lane * VEC;
 
-    const MetaView mv = meta_view(const_cast<void *>(p.ws_meta));
-    const long long W = mv.w_total[0];
-    const int n_tiles = mv.prefix[b + 1] - mv.prefix[b];
+    // ---- the work split, from seq_lens (an input: readable before the decode grid ends)
+    int before = 0, all = 0;
+    for (int x = threadIdx.x; x < p.B; x += blockDim.x) {
+        const int t = tiles_of(clamp_len(__ldg(p.seq_lens + x), p.T_max), p.tile);
+        all += t;
+        if (x < b) before += t;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+        before += __shfl_xor_sync(0xffffffffu, before, off);
+        all += __shfl_xor_sync(0xffffffffu, all, off);
+    }
+    __shared__ int s_sum[2][kCombineWarps];
+    if (lane == 0) { s_sum[0][warp] = before; s_sum[1][warp] = all; }
+    __syncthreads();
+    before = 0;
+    all = 0;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) { before += s_sum[0][w]; all += s_sum[1][w]; }
+    const int n_tiles = tiles_of(clamp_len(__ldg(p.seq_lens + b), p.T_max), p.tile);
+    const long long W = tiles_per_worker((long long)all * p.units_per_seq, p.workers, p.min_tiles);
     if (n_tiles == 0) {
+        // nothing of this unit was touched by the decode kernel
         for (int c = threadIdx.x; c < D; c += blockDim.x) p.out[gh * D + c] = 0.f;
         if (threadIdx.x == 0) p.lse[gh] = -INFINITY;
         return;
     }
-    const long long ustart = (long long)mv.prefix[b] * p.units_per_seq + (long long)i * n_tiles;
+    const long long ustart = (long long)before * p.units_per_seq + (long long)i * n_tiles;
     const long long c_first = ustart / W;
     const long long c_last = (ustart + n_tiles - 1) / W;
     if (c_first == c_last) return;            // finished by its only worker
 
+    pdl_wait_primary();
     float m = -INFINITY, S = 0.f;
     float acc[VEC];
 #pragma unroll
     for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
-    constexpr int UNROLL = 4;
+    constexpr int UNROLL = D >= 512 ? 4 : 8;
     for (long long c0 = c_first + warp; c0 <= c_last; c0 += (long long)kCombineWarps * UNROLL) {
         float ls[UNROLL];
         float ov[UNROLL][VEC];

@@ -1,0 +1,579 @@
+// gqa_tc_decode.cuh -- decode attention for query-head groups that share a KV head
+// (GQA, MQA) on the sm_100a tensor cores (tcgen05, accumulators in tensor memory), with
+// the cached tokens on the MMA rows.
+//
+// What it computes is what gqa_decode.cuh computes ("Attention variants: MQA, GQA, and
+// MLA", sections "MQA: one KV head for everyone" and "GQA: interpolating with groups";
+// "Grouped-Query Attention: Fewer KV Heads, Same Quality", "The Unified View"):
+//     out[b, h] = softmax(scale * q[b, h] . K[b, j]^T) V[b, j],   j = h / g.
+//
+// Orientation.  A decode step has one query token per head, so the query side of a
+// group is g rows while the token side of a KV tile is long.  Both products are taken
+// transposed so that the 128 tokens of a tile fill the M = 128 rows of tcgen05.mma:
+//     S^T[t, h]  = K[t, :] . q[h, :]          A = K tile (K-major), B = query block (K-major)
+//     O^T[d, h] += sum_t V[t, d] P^T[t, h]    A = V tile read MN-major, B = P^T (MN-major)
+// S^T and O^T live in tensor memory: TMEM lane t holds token t's scores for every head
+// of the unit, lane d holds output dimension d of every head.  A unit is up to 64 query
+// heads of one group (the N of the value product); the score product uses
+// N = max(16, NR) where NR is the number of head columns the kernel processes.
+//
+// Per 128-token tile (one CTA per SM, persistent, stream-K over tiles, schedule.cuh):
+//   producer (warp 0)   TMA loads of the K and V tiles (two 128-byte-swizzled boxes of
+//                       [128 tokens x 64] each) into a 3-stage ring; the unit's query
+//                       block once per piece.  No multicast.
+//   MMA (warp 1)        the score product of the next tile (8 MMAs 128 x N x 16) into one
+//                       of two TMEM score buffers, then the value product of this tile
+//                       (16 MMAs 128 x 64 x 16) into O^T; completion by tcgen05.commit.
+//   softmax (warps 2-5) one thread per TMEM lane.  Per tile: scale and mask its token's
+//                       scores, reduce the per-head maxima over the 128 tokens (a
+//                       transposed shuffle reduction inside the warp, then the four warps
+//                       through shared memory), let the owner thread of each head update
+//                       its running max, and write P^T = 2^(s - m) into the K half of the
+//                       stage (the score product is done with it) as a bf16 high part and
+//                       a bf16 remainder; the value product multiplies V by both, so the
+//                       weights keep ~16 significant bits.  The running max moves lazily:
+//                       only when a head's tile maximum exceeds it by more than 2^8, and
+//                       then that head's column of O^T and its row sums are rescaled.
+// Each thread keeps its token slot's partial row sums per head; at the end of a piece
+// they are reduced the same way and every thread writes its output dimension of every
+// head (final output, or the worker's partial for the split combine).
+//
+// Every wait is bounded (common.cuh), including the softmax warps' own group barrier,
+// which is an mbarrier rather than a named barrier so that it can give up.
+#pragma once
+#include "common.cuh"
+#include "gqa_decode.cuh"
+#include "schedule.cuh"
+#include "tc05.cuh"
+
+namespace kvattn {
+namespace gqatc {
+
+constexpr int TILE = 128;                 // tokens per tile = MMA M
+constexpr int D = 128;                    // head dimension
+constexpr int HB = 64;                    // query heads per unit (value-product N)
+constexpr int NST = 3;                    // pipeline stages
+constexpr int CHUNK = TILE * 128;         // one [128 tokens x 64] bf16 box: 16 KB
+constexpr int KV_BYTES = 2 * CHUNK;       // a K or V tile: 32 KB
+constexpr int STAGE = 2 * KV_BYTES;       // K then V: 64 KB
+constexpr int QCHUNK = HB * 128;          // [64 heads x 64] bf16 box: 8 KB
+constexpr int QBUF = 2 * QCHUNK;          // the unit's query block: 16 KB
+constexpr int NTHREADS = 192;             // producer, MMA, 4 softmax warps
+constexpr int NSOFT = 128;
+constexpr uint32_t TM_S = 0;              // two 64-column score buffers
+constexpr uint32_t TM_O = 128;            // O^T: 64 columns
+constexpr uint32_t TM_COLS = 256;
+constexpr float RESCALE_LOG2 = 8.f;
+
+constexpr int OFF_ST = 0;
+constexpr int OFF_Q = OFF_ST + NST * STAGE;        // 196608
+constexpr int OFF_RED = OFF_Q + QBUF;              // [3][4][64] fp32: tile slots 0/1, piece end
+constexpr int OFF_MS = OFF_RED + 3 * 4 * HB * 4;   // [2][64] running max per head
+constexpr int OFF_AS = OFF_MS + 2 * HB * 4;        // [2][64] rescale factor per head
+constexpr int OFF_NF = OFF_AS + 2 * HB * 4;        // [2][64] bytes: head rescaled this tile
+constexpr int OFF_LINV = OFF_NF + 2 * HB;          // [64] 1 / row sum
+constexpr int OFF_BARS = OFF_LINV + HB * 4;
+constexpr int OFF_TMEMPTR = OFF_BARS + 256;
+constexpr int OFF_ABORT = OFF_TMEMPTR + 16;
+constexpr int OFF_PREFIX = OFF_ABORT + 16;
+constexpr int smem_bytes(int B) { return 1024 + OFF_PREFIX + (B + 1) * 4; }
+
+struct Bars {
+    uint64_t full[NST], empty[NST];
+    uint64_t qfull;       // the unit's query block landed
+    uint64_t qempty;      // every score MMA of the piece has read it
+    uint64_t sready[2];   // scores of a tile in TMEM buffer (tile & 1)
+    uint64_t sfree[2];    // the softmax threads have read that buffer
+    uint64_t pready[2];   // P^T written (and O^T rescaled): the value product may run
+    uint64_t odone[2];    // value product of a tile (parity tile & 1) finished
+    uint64_t ofree;       // the epilogue has read O^T
+    uint64_t grp;         // barrier of the 128 softmax threads
+};
+static_assert(sizeof(Bars) <= 256, "barrier block overflows its slot");
+
+template <int NR>
+struct Cfg {
+    static_assert(NR == 8 || NR == 16 || NR == 32 || NR == 64, "head columns per unit");
+    static constexpr int NQ = NR < 16 ? 16 : NR;           // score-product N (and columns read)
+    static constexpr int RW = NR >= 32 ? NR / 32 : 1;      // values a lane holds after the reduction
+    static constexpr int LPH = NR >= 32 ? 1 : 32 / NR;     // lanes holding the same head after it
+};
+
+struct Ctx {
+    uint8_t *smem;
+    Bars *bars;
+    volatile int *abort_flag;
+    const int *s_prefix;
+    uint32_t tmem;
+    int U;
+    long long p0, p1;
+};
+
+// One halving step of the transposed reduction: lanes whose bit `m` is set keep the
+// upper W values, the others the lower W, and each adds (or takes the max of) the half
+// its partner gave away.
+template <int W, bool MAX>
+__device__ __forceinline__ void xr_step(float *v, bool upper, int m) {
+#pragma unroll
+    for (int i = 0; i < W; ++i) {
+        const float send = upper ? v[i] : v[W + i];
+        const float keep = upper ? v[W + i] : v[i];
+        const float got = __shfl_xor_sync(0xffffffffu, send, m);
+        v[i] = MAX ? fmaxf(keep, got) : keep + got;
+    }
+}
+// Reduces NR per-lane values over the 32 lanes of the warp, per column.  Afterwards
+// lane l holds in v[i] the result for column RW * l + i (NR >= 32), or in v[0] the
+// result for column l / LPH (NR < 32).  NR - 1 shuffles for NR >= 32.
+template <int NR, bool MAX>
+__device__ __forceinline__ void warp_xreduce(float (&v)[NR], int lane) {
+    if constexpr (NR >= 2) xr_step<NR / 2, MAX>(v, (lane & 16) != 0, 16);
+    if constexpr (NR >= 4) xr_step<NR / 4, MAX>(v, (lane & 8) != 0, 8);
+    if constexpr (NR >= 8) xr_step<NR / 8, MAX>(v, (lane & 4) != 0, 4);
+    if constexpr (NR >= 16) xr_step<NR / 16, MAX>(v, (lane & 2) != 0, 2);
+    if constexpr (NR >= 32) xr_step<NR / 32, MAX>(v, (lane & 1) != 0, 1);
+    if constexpr (NR < 32) {
+#pragma unroll
+        for (int m = 16 / NR; m >= 1; m >>= 1) {
+            const float got = __shfl_xor_sync(0xffffffffu, v[0], m);
+            v[0] = MAX ? fmaxf(v[0], got) : v[0] + got;
+        }
+    }
+}
+// Stores the warp's reduced columns into row[0..NR).
+template <int NR>
+__device__ __forceinline__ void store_reduced(float *row, const float (&v)[NR], int lane) {
+    using C = Cfg<NR>;
+    if constexpr (NR >= 32) {
+#pragma unroll
+        for (int i = 0; i < C::RW; ++i) row[C::RW * lane + i] = v[i];
+    } else {
+        if ((lane & (C::LPH - 1)) == 0) row[lane / C::LPH] = v[0];
+    }
+}
+
+// NQ consecutive TMEM columns of this thread's lane.
+template <int NQ>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[NQ]) {
+    if constexpr (NQ == 16) {
+        tmem_ld16(taddr, v);
+    } else if constexpr (NQ == 32) {
+        tmem_ld32(taddr, v);
+    } else {
+        uint32_t a[32], b[32];
+        tmem_ld32(taddr, a);
+        tmem_ld32(taddr + 32, b);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) { v[i] = a[i]; v[32 + i] = b[i]; }
+    }
+}
+// ------------------------------------------------------------------ producer (warp 0, lane 0)
+__device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *kmap, const CUtensorMap *vmap,
+                                         const CUtensorMap *qmap, const Ctx &c) {
+    Bars *bars = c.bars;
+    const uint64_t pol = l2_policy_evict_first();
+    int k = 0, pi = 0;
+    bool ok = true;
+    for (long long pos = c.p0; pos < c.p1 && ok; ++pi) {
+        const Piece pc = piece_at(c.s_prefix, p.B, c.U, pos, c.p1, c.p0);
+        pos = pc.ustart + pc.lt1;
+        const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
+        const int j = pc.i / p.n_hb, hb = pc.i % p.n_hb;
+        const int z = pc.b * p.n_kv + j;
+        if (pi > 0 && !mbar_wait(&bars->qempty, (uint32_t)(pi - 1) & 1u, FLAG_EMPTY_WAIT, c.abort_flag)) {
+            ok = false;
+            break;
+        }
+        mbar_arrive_expect_tx(&bars->qfull, QBUF);
+        const int qrow = j * p.g + hb * HB;
+        tma_load_3d(c.smem + OFF_Q, qmap, &bars->qfull, 0, qrow, pc.b, pol);
+        tma_load_3d(c.smem + OFF_Q + QCHUNK, qmap, &bars->qfull, 64, qrow, pc.b, pol);
+        for (int lt = pc.lt0; lt < pc.lt1; ++lt, ++k) {
+            const int s = k % NST;
+            const uint32_t ph = (uint32_t)(k / NST) & 1u;
+            if (!mbar_wait(&bars->empty[s], ph ^ 1u, FLAG_EMPTY_WAIT, c.abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(&bars->full[s], STAGE);
+            const int y = min(lt * TILE, len - TILE);
+            uint8_t *st = c.smem + OFF_ST + s * STAGE;
+            tma_load_3d(st, kmap, &bars->full[s], 0, y, z, pol);
+            tma_load_3d(st + CHUNK, kmap, &bars->full[s], 64, y, z, pol);
+            tma_load_3d(st + KV_BYTES, vmap, &bars->full[s], 0, y, z, pol);
+            tma_load_3d(st + KV_BYTES + CHUNK, vmap, &bars->full[s], 64, y, z, pol);
+        }
+    }
+    if (!ok) {
+        // Let every copy already issued land before the CTA can exit.
+        for (int kk = (k > NST ? k - NST : 0); kk < k; ++kk)
+            mbar_wait_sleep(&bars->full[kk % NST], (uint32_t)(kk / NST) & 1u, FLAG_FULL_WAIT, nullptr);
+        if (pi > 0) mbar_wait_sleep(&bars->qfull, (uint32_t)(pi - 1) & 1u, FLAG_FULL_WAIT, nullptr);
+    }
+}
+
+// ------------------------------------------------------------------ MMA issuer (warp 1, lane 0)
+// Score product of tile kt into TMEM buffer (kt & 1).  The caller has seen the tile
+// land and the buffer freed.
+template <int NR>
+__device__ __forceinline__ void issue_scores(const Ctx &c, int kt) {
+    const int s = kt % NST, sb = kt & 1;
+    tc_fence_after();
+    constexpr uint32_t idesc = idesc_f16_major(128, Cfg<NR>::NQ, 1, 1, 0, 0);
+    const uint32_t st = smem_u32(c.smem + OFF_ST + s * STAGE);
+    const uint32_t qb = smem_u32(c.smem + OFF_Q);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t blk = kk >> 2, in = (kk & 3) * 32;
+        const uint64_t a = smem_desc_sw128(st + blk * CHUNK + in, 16, 1024);
+        const uint64_t b = smem_desc_sw128(qb + blk * QCHUNK + in, 16, 1024);
+        umma_ss(c.tmem + TM_S + 64 * sb, a, b, idesc, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&c.bars->sready[sb]);
+}
+
+// Value product of tile kt into O^T (first = the piece's first tile: overwrite).
+__device__ __forceinline__ void issue_values(const Ctx &c, int kt, bool first) {
+    const int s = kt % NST;
+    constexpr uint32_t idesc_pv = idesc_f16_major(128, HB, 1, 1, 1, 1);
+    tc_fence_after();
+    const uint32_t st = smem_u32(c.smem + OFF_ST + s * STAGE);
+#pragma unroll
+    for (int kk = 0; kk < TILE / 16; ++kk) {
+        // V^T: M = 128 dimensions in two 64-wide blocks 16 KB apart, K = 16 tokens
+        const uint64_t a = smem_desc_sw128(st + KV_BYTES + kk * 2048, CHUNK, 1024);
+        // P^T high part and remainder (in the K half of the stage): N = 64 heads
+        const uint64_t bh = smem_desc_sw128(st + kk * 2048, CHUNK, 1024);
+        const uint64_t bl = smem_desc_sw128(st + CHUNK + kk * 2048, CHUNK, 1024);
+        umma_ss(c.tmem + TM_O, a, bh, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+        umma_ss(c.tmem + TM_O, a, bl, idesc_pv, 1u);
+    }
+    umma_commit(&c.bars->empty[s]);
+    umma_commit(&c.bars->odone[kt & 1]);
+}
+
+// The issuer never blocks on one product while the other could go: it tests whether
+// the next score product (its tile landed, its TMEM buffer free) or the next value
+// product (P^T written; at a piece start, O^T read out) may run and issues whatever is
+// ready.  Score products run at most two tiles ahead of value products -- the order a
+// blocking loop would give -- which keeps every tested barrier within one phase of the
+// tested parity.  Idle time is bounded like every other wait.
+template <int NR>
+__device__ __forceinline__ void mma_issuer(const GqaParams &p, const Ctx &c) {
+    Bars *bars = c.bars;
+    int k = 0, pi = 0;
+    for (long long pos = c.p0; pos < c.p1; ++pi) {
+        const Piece pc = piece_at(c.s_prefix, p.B, c.U, pos, c.p1, c.p0);
+        pos = pc.ustart + pc.lt1;
+        const int nt = pc.lt1 - pc.lt0;
+        if (!mbar_wait(&bars->qfull, (uint32_t)pi & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
+        int nq = 0, nv = 0;
+        long long idle_since = clock64();
+        while (nv < nt) {
+            bool progressed = false;
+            if (nq < nt && nq < nv + 2) {
+                const int kt = k + nq;
+                if (mbar_test(&bars->full[kt % NST], (uint32_t)(kt / NST) & 1u) &&
+                    (kt < 2 || mbar_test(&bars->sfree[kt & 1], (uint32_t)((kt >> 1) - 1) & 1u))) {
+                    issue_scores<NR>(c, kt);
+                    ++nq;
+                    if (nq == nt) umma_commit(&bars->qempty);
+                    progressed = true;
+                }
+            }
+            if (nv < nq) {
+                const int kt = k + nv;
+                if (mbar_test(&bars->pready[kt & 1], (uint32_t)(kt >> 1) & 1u) &&
+                    (nv > 0 || pi == 0 || mbar_test(&bars->ofree, (uint32_t)(pi - 1) & 1u))) {
+                    issue_values(c, kt, nv == 0);
+                    ++nv;
+                    progressed = true;
+                }
+            }
+            if (progressed) {
+                idle_since = clock64();
+            } else {
+                if (*c.abort_flag) return;
+                if (clock64() - idle_since > kWaitLimitCycles) {
+                    atomicOr(&g_device_flags, FLAG_MMA_WAIT);
+                    *c.abort_flag = 1;
+                    return;
+                }
+            }
+        }
+        k += nt;
+    }
+}
+
+// ------------------------------------------------------------------ softmax (warps 2-5)
+template <int NR>
+__device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, int warp, int lane) {
+    using C = Cfg<NR>;
+    constexpr int NQ = C::NQ;
+    Bars *bars = c.bars;
+    const int q = warp & 3;               // TMEM lane quadrant
+    const int r = 32 * q + lane;          // token row of a tile / output dimension
+    const int st_id = (warp - 2) * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    float *red = reinterpret_cast<float *>(c.smem + OFF_RED);
+    float *ms = reinterpret_cast<float *>(c.smem + OFF_MS);
+    float *as = reinterpret_cast<float *>(c.smem + OFF_AS);
+    uint8_t *nf = c.smem + OFF_NF;
+    float *linv = reinterpret_cast<float *>(c.smem + OFF_LINV);
+    uint32_t grp_uses = 0;
+    auto grp_sync = [&]() -> bool {
+        mbar_arrive(&bars->grp);
+        const bool ok = mbar_wait(&bars->grp, grp_uses & 1u, FLAG_FULL_WAIT, c.abort_flag);
+        ++grp_uses;
+        return warp_all(ok);
+    };
+
+    int k = 0, pi = 0;
+    for (long long pos = c.p0; pos < c.p1; ++pi) {
+        const Piece pc = piece_at(c.s_prefix, p.B, c.U, pos, c.p1, c.p0);
+        pos = pc.ustart + pc.lt1;
+        const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
+        const int j = pc.i / p.n_hb, hb = pc.i % p.n_hb;
+        const int nt = pc.lt1 - pc.lt0;
+        float m_own = -INFINITY;              // running max of head st_id (owner threads)
+        float l_part[NR];
+#pragma unroll
+        for (int h = 0; h < NR; ++h) l_part[h] = 0.f;
+
+        for (int t = 0; t < nt; ++t) {
+            const int kt = k + t;
+            const int s = kt % NST, sb = kt & 1;
+            const int lt = pc.lt0 + t;
+            const int y = min(lt * TILE, len - TILE);
+            const int tok_lo = lt * TILE - y, tok_hi = min((lt + 1) * TILE, len) - y;
+            // ---- this token's scores
+            if (!warp_all(mbar_wait(&bars->sready[sb], (uint32_t)(kt >> 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
+                return;
+            tc_fence_after();
+            uint32_t sv[NQ];
+            tmem_ld_cols<NQ>(c.tmem + lane_base + TM_S + 64 * sb, sv);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&bars->sfree[sb]);
+            const bool valid = r >= tok_lo && r < tok_hi;
+            float sc[NR], v[NR];
+#pragma unroll
+            for (int h = 0; h < NR; ++h) {
+                sc[h] = valid ? __uint_as_float(sv[h]) * p.scale_log2 : -INFINITY;
+                v[h] = sc[h];
+            }
+            // ---- per-head maximum over the tile's 128 tokens
+            warp_xreduce<NR, true>(v, lane);
+            store_reduced<NR>(red + (sb * 4 + q) * HB, v, lane);
+            if (!grp_sync()) return;
+            if (st_id < NR) {
+                const float tm = fmaxf(fmaxf(red[(sb * 4 + 0) * HB + st_id], red[(sb * 4 + 1) * HB + st_id]),
+                                       fmaxf(red[(sb * 4 + 2) * HB + st_id], red[(sb * 4 + 3) * HB + st_id]));
+                float alpha = 1.f;
+                uint8_t need = 0;
+                if (t == 0) {
+                    m_own = tm;
+                } else if (tm > m_own + RESCALE_LOG2) {
+                    alpha = fast_exp2(m_own - tm);
+                    m_own = tm;
+                    need = 1;
+                }
+                ms[sb * HB + st_id] = m_own;
+                as[sb * HB + st_id] = alpha;
+                nf[sb * HB + st_id] = need;
+            }
+            if (!grp_sync()) return;
+            // ---- weights: P^T row r, high part and remainder, into the stage's K half
+            uint32_t anyw = 0;
+#pragma unroll
+            for (int h = 0; h < NR; h += 4) anyw |= *reinterpret_cast<const uint32_t *>(nf + sb * HB + h);
+            const bool rescale = anyw != 0;     // the same for every thread
+            const float *as_t = as + sb * HB;
+            if (rescale) {
+#pragma unroll
+                for (int h = 0; h < NR; h += 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(as_t + h);
+                    l_part[h] *= x.x; l_part[h + 1] *= x.y; l_part[h + 2] *= x.z; l_part[h + 3] *= x.w;
+                }
+            }
+            uint8_t *st = c.smem + OFF_ST + s * STAGE;
+            uint8_t *hrow = st + r * 128;
+            uint8_t *lrow = st + CHUNK + r * 128;
+#pragma unroll
+            for (int cc = 0; cc < NR / 8; ++cc) {
+                uint32_t hw[4], lw[4];
+                const float4 m0 = *reinterpret_cast<const float4 *>(ms + sb * HB + 8 * cc);
+                const float4 m1 = *reinterpret_cast<const float4 *>(ms + sb * HB + 8 * cc + 4);
+                const float mh[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int h = 8 * cc + 2 * e;
+                    const float a = fast_exp2(sc[h] - mh[2 * e]);
+                    const float b = fast_exp2(sc[h + 1] - mh[2 * e + 1]);
+                    l_part[h] += a;
+                    l_part[h + 1] += b;
+                    const float ah = bf16_round(a), bh = bf16_round(b);
+                    hw[e] = pack_bf16x2(ah, bh);
+                    lw[e] = pack_bf16x2(a - ah, b - bh);
+                }
+                const int slot = (cc ^ (r & 7)) << 4;
+                *reinterpret_cast<uint4 *>(hrow + slot) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(lrow + slot) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+            fence_proxy_async_smem();
+            // ---- rescale the affected heads' columns of O^T (after the previous value product)
+            if (rescale) {
+                if (!warp_all(mbar_wait(&bars->odone[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u, FLAG_MMA_WAIT,
+                                        c.abort_flag)))
+                    return;
+                tc_fence_after();
+#pragma unroll
+                for (int c0 = 0; c0 < NQ; c0 += 16) {
+                    uint32_t ov[16];
+                    tmem_ld16(c.tmem + lane_base + TM_O + c0, ov);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < 16; h += 4) {
+                        if (c0 + h < NR) {
+                            const float4 x = *reinterpret_cast<const float4 *>(as_t + c0 + h);
+                            ov[h] = __float_as_uint(__uint_as_float(ov[h]) * x.x);
+                            ov[h + 1] = __float_as_uint(__uint_as_float(ov[h + 1]) * x.y);
+                            ov[h + 2] = __float_as_uint(__uint_as_float(ov[h + 2]) * x.z);
+                            ov[h + 3] = __float_as_uint(__uint_as_float(ov[h + 3]) * x.w);
+                        }
+                    }
+                    tmem_st16(c.tmem + lane_base + TM_O + c0, ov);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(&bars->pready[sb]);
+        }
+        k += nt;
+
+        // ---- end of the piece: row sums, lse, output
+        float v[NR];
+#pragma unroll
+        for (int h = 0; h < NR; ++h) v[h] = l_part[h];
+        warp_xreduce<NR, false>(v, lane);
+        store_reduced<NR>(red + (2 * 4 + q) * HB, v, lane);
+        if (!grp_sync()) return;
+        const int h_real = min(HB, p.g - hb * HB);
+        const size_t head0 = (size_t)pc.b * p.n_q + (size_t)j * p.g + (size_t)hb * HB;
+        const size_t part = ((size_t)blockIdx.x * 2 + pc.slot) * HB;
+        if (st_id < NR) {
+            const float l = red[(8 + 0) * HB + st_id] + red[(8 + 1) * HB + st_id] + red[(8 + 2) * HB + st_id] +
+                            red[(8 + 3) * HB + st_id];
+            linv[st_id] = l > 0.f ? 1.f / l : 0.f;
+            const float lse_v = l > 0.f ? (m_own + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+            if (st_id < h_real) {
+                if (pc.whole)
+                    p.lse[head0 + st_id] = lse_v;
+                else
+                    p.ws_lse[part + st_id] = lse_v;
+            }
+        }
+        if (!grp_sync()) return;
+        const int klast = k - 1;
+        if (!warp_all(mbar_wait(&bars->odone[klast & 1], (uint32_t)(klast >> 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
+            return;
+        tc_fence_after();
+        float *dst = pc.whole ? p.out + head0 * D : p.ws_o + part * D;
+#pragma unroll
+        for (int c0 = 0; c0 < NQ; c0 += 16) {
+            uint32_t ov[16];
+            tmem_ld16(c.tmem + lane_base + TM_O + c0, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 16; ++h)
+                if (c0 + h < NR && c0 + h < h_real) dst[(size_t)(c0 + h) * D + r] = __uint_as_float(ov[h]) * linv[c0 + h];
+        }
+        tc_fence_before();
+        mbar_arrive(&bars->ofree);
+    }
+}
+
+}  // namespace gqatc
+
+template <int NR>
+__global__ void __launch_bounds__(gqatc::NTHREADS, 1)
+gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap,
+                     const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
+    using namespace gqatc;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars *bars = reinterpret_cast<Bars *>(smem + OFF_BARS);
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + OFF_TMEMPTR);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ABORT);
+    int *s_prefix = reinterpret_cast<int *>(smem + OFF_PREFIX);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int U = p.n_kv * p.n_hb;
+
+    if (tid == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        mbar_init(&bars->qfull, 1);
+        mbar_init(&bars->qempty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->sready[i], 1);
+            mbar_init(&bars->sfree[i], NSOFT);
+            mbar_init(&bars->pready[i], NSOFT);
+            mbar_init(&bars->odone[i], 1);
+        }
+        mbar_init(&bars->ofree, NSOFT);
+        mbar_init(&bars->grp, NSOFT);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_ptr), TM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == 2) build_tile_prefix(p.seq_lens, p.B, p.T_max, TILE, s_prefix, lane);
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+        prefetch_tensormap(&qmap);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    Ctx c;
+    c.smem = smem;
+    c.bars = bars;
+    c.abort_flag = abort_flag;
+    c.s_prefix = s_prefix;
+    c.tmem = *tmem_ptr;
+    c.U = U;
+    const long long total = (long long)s_prefix[p.B] * U;
+    const long long W = tiles_per_worker(total, p.workers, p.min_tiles);
+    if (blockIdx.x == 0) {
+        MetaView mv = meta_view(p.ws_meta);
+        if (tid == 0) { mv.w_total[0] = W; mv.w_total[1] = total; }
+        for (int i = tid; i <= p.B; i += NTHREADS) mv.prefix[i] = s_prefix[i];
+    }
+    // The combine kernel may be scheduled now; it waits for this grid to finish.
+    pdl_launch_dependents();
+    c.p0 = (long long)blockIdx.x * W;
+    c.p1 = (c.p0 + W < total) ? c.p0 + W : total;
+
+    if (c.p0 < total) {
+        if (warp == 0) {
+            if (lane == 0) producer(p, &kmap, &vmap, &qmap, c);
+        } else if (warp == 1) {
+            if (lane == 0) mma_issuer<NR>(p, c);
+        } else {
+            softmax_warps<NR>(p, c, warp, lane);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(c.tmem, TM_COLS);
+    }
+}
+
+}  // namespace kvattn

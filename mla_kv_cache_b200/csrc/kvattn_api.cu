@@ -11,6 +11,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "gqa_decode.cuh"
+#include "gqa_tc_decode.cuh"
 #include "mla_decode.cuh"
 
 using namespace kvattn;
@@ -44,6 +45,7 @@ DeviceState g_dev[kMaxDevices];
 std::mutex g_mutex;
 int g_force_workers = 0;
 int g_force_min_tiles = 0;
+int g_gqa_kernel = 0;   // 0: heuristic, 1: warp-level MMA kernel, 2: tcgen05 kernel
 
 int device_state(DeviceState **out) {
     int dev = 0;
@@ -275,7 +277,7 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
     if (e != cudaSuccess) return fail_cuda(e, "gqa decode launch");
 
     CombineParams cp;
-    cp.ws_meta = p.ws_meta;
+    cp.seq_lens = p.seq_lens;
     cp.ws_lse = p.ws_lse;
     cp.ws_o = p.ws_o;
     cp.out = p.out;
@@ -287,9 +289,85 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
     cp.n_hb = p.n_hb;
     cp.n_kv = p.n_kv;
     cp.g = p.g;
+    cp.T_max = p.T_max;
+    cp.tile = C::TILE;
+    cp.workers = p.workers;
+    cp.min_tiles = p.min_tiles;
     const int rows = p.g < C::HEADS ? p.g : C::HEADS;
     return launch_combine(D, cp, p.B * units_per_seq, rows, stream,
                           combine_warps((p.T_max + C::TILE - 1) / C::TILE, max_tiles, p.workers));
+}
+
+// The tcgen05 kernel (gqa_tc_decode.cuh): tokens on the MMA rows, up to 64 query heads
+// per unit, NR head columns processed.
+template <int NR>
+int run_gqa_tc(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &vmap,
+               const CUtensorMap &qmap, DeviceState *dev, int units_per_seq, cudaStream_t stream) {
+    GqaParams p = base;
+    const int smem = gqatc::smem_bytes(p.B);
+    if (smem > dev->max_smem_optin) {
+        snprintf(t_detail, sizeof(t_detail), "needs %d B shared memory", smem);
+        return KVATTN_ERR_UNSUPPORTED;
+    }
+    const long long max_tiles =
+        (long long)p.B * units_per_seq * ((p.T_max + gqatc::TILE - 1) / gqatc::TILE);
+    p.min_tiles = g_force_min_tiles > 0 ? g_force_min_tiles : 2;
+    long long workers = g_force_workers > 0 ? g_force_workers : dev->sms;
+    const long long by_size = (max_tiles + p.min_tiles - 1) / p.min_tiles;
+    if (g_force_workers <= 0 && workers > by_size) workers = by_size;
+    if (workers < 1) workers = 1;
+    p.workers = (int)workers;
+
+    void *ws = nullptr;
+    const size_t meta_bytes = ((16 + (size_t)(p.B + 1) * 4) + 255) & ~size_t(255);
+    const size_t lse_bytes = (((size_t)p.workers * 2 * gqatc::HB * 4) + 255) & ~size_t(255);
+    const size_t o_bytes = (size_t)p.workers * 2 * gqatc::HB * gqatc::D * 4;
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        int st = ensure_workspace(dev, meta_bytes + lse_bytes + o_bytes, &ws);
+        if (st != KVATTN_OK) return st;
+    }
+    p.ws_meta = ws;
+    p.ws_lse = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes);
+    p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes + lse_bytes);
+
+    auto kern = gqa_tc_decode_kernel<NR>;
+    cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), dev, smem);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaFuncSetAttribute(gqa tc)");
+    kern<<<p.workers, gqatc::NTHREADS, smem, stream>>>(p, kmap, vmap, qmap);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_cuda(e, "gqa tc decode launch");
+
+    CombineParams cp;
+    cp.seq_lens = p.seq_lens;
+    cp.ws_lse = p.ws_lse;
+    cp.ws_o = p.ws_o;
+    cp.out = p.out;
+    cp.lse = p.lse;
+    cp.B = p.B;
+    cp.n_q = p.n_q;
+    cp.units_per_seq = units_per_seq;
+    cp.heads_per_unit = gqatc::HB;
+    cp.n_hb = p.n_hb;
+    cp.n_kv = p.n_kv;
+    cp.g = p.g;
+    cp.T_max = p.T_max;
+    cp.tile = gqatc::TILE;
+    cp.workers = p.workers;
+    cp.min_tiles = p.min_tiles;
+    const int rows = p.g < gqatc::HB ? p.g : gqatc::HB;
+    return launch_combine(gqatc::D, cp, p.B * units_per_seq, rows, stream,
+                          combine_warps((p.T_max + gqatc::TILE - 1) / gqatc::TILE, max_tiles, p.workers));
+}
+
+// Which GQA kernel runs: the tcgen05 kernel for head_dim 128 once a group has a few
+// query heads (its tensor work per KV byte grows with the group, and the warp-level
+// MMA path runs out of tensor throughput first), the warp-level kernel otherwise.
+bool use_tc_kernel(int head_dim, int g, int batch, const DeviceState *dev) {
+    const bool possible = head_dim == 128 && gqatc::smem_bytes(batch) <= dev->max_smem_optin;
+    if (g_gqa_kernel == 1) return false;
+    if (g_gqa_kernel == 2) return possible;
+    return possible && g >= 4;
 }
 
 }  // namespace
@@ -327,17 +405,28 @@ int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
     if (st != KVATTN_OK) return st;
 
     const int g = n_q_heads / n_kv_heads;
+    if (g_gqa_kernel == 2 && !use_tc_kernel(head_dim, g, batch, dev)) {
+        snprintf(t_detail, sizeof(t_detail), "tcgen05 GQA kernel needs head_dim 128 and batch <= %d",
+                 (dev->max_smem_optin - gqatc::smem_bytes(0)) / 4);
+        return KVATTN_ERR_UNSUPPORTED;
+    }
+    const bool tc = use_tc_kernel(head_dim, g, batch, dev);
     const int MT = g <= 16 ? 1 : 2;
-    const int heads = 16 * MT;
+    const int heads = tc ? gqatc::HB : 16 * MT;
     const int n_hb = (g + heads - 1) / heads;
+    const uint32_t box_rows = tc ? gqatc::TILE : 64;
 
-    CUtensorMap kmap, vmap;
-    st = make_map_3d(&kmap, k_cache, head_dim, max_seq_len, (uint64_t)batch * n_kv_heads, 64, 64,
+    CUtensorMap kmap, vmap, qmap;
+    st = make_map_3d(&kmap, k_cache, head_dim, max_seq_len, (uint64_t)batch * n_kv_heads, 64, box_rows,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
-    st = make_map_3d(&vmap, v_cache, head_dim, max_seq_len, (uint64_t)batch * n_kv_heads, 64, 64,
+    st = make_map_3d(&vmap, v_cache, head_dim, max_seq_len, (uint64_t)batch * n_kv_heads, 64, box_rows,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
+    if (tc) {
+        st = make_map_3d(&qmap, q, head_dim, n_q_heads, batch, 64, gqatc::HB, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != KVATTN_OK) return st;
+    }
 
     GqaParams p = {};
     p.q = reinterpret_cast<const __nv_bfloat16 *>(q);
@@ -353,6 +442,12 @@ int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     const int U = n_kv_heads * n_hb;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tc) {
+        if (g > 32) return run_gqa_tc<64>(p, kmap, vmap, qmap, dev, U, s);
+        if (g > 16) return run_gqa_tc<32>(p, kmap, vmap, qmap, dev, U, s);
+        if (g > 8) return run_gqa_tc<16>(p, kmap, vmap, qmap, dev, U, s);
+        return run_gqa_tc<8>(p, kmap, vmap, qmap, dev, U, s);
+    }
     if (head_dim == 128)
         return MT == 1 ? run_gqa<128, 1>(p, kmap, vmap, dev, U, s) : run_gqa<128, 2>(p, kmap, vmap, dev, U, s);
     return MT == 1 ? run_gqa<64, 1>(p, kmap, vmap, dev, U, s) : run_gqa<64, 2>(p, kmap, vmap, dev, U, s);
@@ -469,7 +564,7 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
     if (e != cudaSuccess) return fail_cuda(e, "mla decode launch");
 
     CombineParams cp;
-    cp.ws_meta = p.ws_meta;
+    cp.seq_lens = p.seq_lens;
     cp.ws_lse = p.ws_lse;
     cp.ws_o = p.ws_o;
     cp.out = out;
@@ -481,6 +576,10 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
     cp.n_hb = 1;
     cp.n_kv = 1;
     cp.g = n_heads;
+    cp.T_max = p.T_max;
+    cp.tile = mla::TILE;
+    cp.workers = p.workers;
+    cp.min_tiles = p.min_tiles;
     return launch_combine(512, cp, batch, n_heads, s,
                           combine_warps((max_seq_len + mla::TILE - 1) / mla::TILE, max_tiles, p.workers));
 }
@@ -535,6 +634,11 @@ void kvattn_debug_set_workers(int workers, int min_tiles) {
     std::lock_guard<std::mutex> lk(g_mutex);
     g_force_workers = workers > 0 ? workers : 0;
     g_force_min_tiles = workers > 0 && min_tiles > 0 ? min_tiles : 0;
+}
+
+void kvattn_debug_set_gqa_kernel(int which) {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    g_gqa_kernel = (which == 1 || which == 2) ? which : 0;
 }
 
 }  // extern "C"
@@ -619,7 +723,7 @@ int run_gqa_noalloc(const GqaParams &base, const CUtensorMap &kmap, const CUtens
     if (e != cudaSuccess) return fail_cuda(e, "gqa decode launch");
 
     CombineParams cp;
-    cp.ws_meta = p.ws_meta;
+    cp.seq_lens = p.seq_lens;
     cp.ws_lse = p.ws_lse;
     cp.ws_o = p.ws_o;
     cp.out = p.out;
@@ -631,6 +735,10 @@ int run_gqa_noalloc(const GqaParams &base, const CUtensorMap &kmap, const CUtens
     cp.n_hb = p.n_hb;
     cp.n_kv = p.n_kv;
     cp.g = p.g;
+    cp.T_max = p.T_max;
+    cp.tile = C::TILE;
+    cp.workers = p.workers;
+    cp.min_tiles = p.min_tiles;
     const int rows = p.g < C::HEADS ? p.g : C::HEADS;
     return launch_combine(D, cp, p.B * units_per_seq, rows, stream,
                           combine_warps((p.T_max + C::TILE - 1) / C::TILE, max_tiles, p.workers));

@@ -23,20 +23,36 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA GPU", allow_module_level=True)
 
 
-@pytest.fixture(autouse=True)
-def _reset_knob():
+KERNELS = {"warp": 1, "tc": 2}   # warp-level MMA kernel, tcgen05 kernel
+_forced = {"kernel": 0}
+
+
+@pytest.fixture(autouse=True, params=list(KERNELS), ids=list(KERNELS))
+def kernel(request):
+    """Every test runs once per GQA kernel (the knob forces the choice)."""
     kb.kvattn_debug_set_workers(0, 0)
+    kb.kvattn_debug_set_gqa_kernel(KERNELS[request.param])
+    _forced["kernel"] = KERNELS[request.param]
     kb.kvattn_clear_device_flags()
-    yield
+    yield request.param
     kb.kvattn_debug_set_workers(0, 0)
+    kb.kvattn_debug_set_gqa_kernel(0)
+    _forced["kernel"] = 0
     assert kb.kvattn_read_device_flags() == 0, "a bounded wait ran out on the device"
 
 
-def run_case(cfg, seed=0, poison=True, batch_ids=None):
-    x = wl.make_gqa_inputs(cfg, seed=seed, poison_tail=poison)
+def decode(cfg, dev):
+    """kvattn_gqa_decode; skips the test when the forced kernel cannot serve the shape
+    (the tcgen05 kernel only takes head_dim 128)."""
+    if _forced["kernel"] == 2 and cfg.head_dim != 128:
+        pytest.skip("tcgen05 GQA kernel: head_dim 128 only")
+    return kb.kvattn_gqa_decode(dev["q"], dev["k_cache"], dev["v_cache"], dev["seq_lens"], cfg.scale)
+
+
+def run_case(cfg, seed=0, poison=True, batch_ids=None, inputs=None):
+    x = wl.make_gqa_inputs(cfg, seed=seed, poison_tail=poison) if inputs is None else inputs
     dev = {k: v.cuda() for k, v in x.items()}
-    out, lse = kb.kvattn_gqa_decode(dev["q"], dev["k_cache"], dev["v_cache"], dev["seq_lens"],
-                                    cfg.scale)
+    out, lse = decode(cfg, dev)
     torch.cuda.synchronize()
     ids = list(range(cfg.batch)) if batch_ids is None else list(batch_ids)
     ro, rl = oracle.gqa_decode(x["q"], x["k_cache"], x["v_cache"], x["seq_lens"], cfg.scale,
@@ -95,10 +111,11 @@ def test_repeat_invariance():
     cfg = small("rep", 2, 16, 2, 128, 500, lens=[500, 77])
     x = wl.make_gqa_inputs(cfg, seed=5)
     d = {k: v.cuda() for k, v in x.items()}
-    o1, l1 = kb.kvattn_gqa_decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], cfg.scale)
-    k2 = d["k_cache"].repeat_interleave(8, dim=1).contiguous()
-    v2 = d["v_cache"].repeat_interleave(8, dim=1).contiguous()
-    o2, l2 = kb.kvattn_gqa_decode(d["q"], k2, v2, d["seq_lens"], cfg.scale)
+    o1, l1 = decode(cfg, d)
+    d2 = dict(d)
+    d2["k_cache"] = d["k_cache"].repeat_interleave(8, dim=1).contiguous()
+    d2["v_cache"] = d["v_cache"].repeat_interleave(8, dim=1).contiguous()
+    o2, l2 = decode(cfg, d2)
     assert_close(o1.cpu().numpy(), o2.cpu().numpy().astype(np.float64), "repeat out")
     assert_close(l1.cpu().numpy(), l2.cpu().numpy().astype(np.float64), "repeat lse")
 
@@ -111,6 +128,8 @@ def test_nonzero_stream_and_reuse():
     with torch.cuda.stream(s):
         outs = [kb.kvattn_gqa_decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], cfg.scale,
                                      stream=s) for _ in range(3)]
+        if _forced["kernel"] == 2:
+            assert cfg.head_dim == 128
     s.synchronize()
     for o, l in outs[1:]:
         assert torch.equal(o, outs[0][0]) and torch.equal(l, outs[0][1])
@@ -120,3 +139,24 @@ def test_nonzero_stream_and_reuse():
 def test_workload_full_size(name):
     """The GQA/MHA/MQA workloads at full size, every sequence, bench launch configuration."""
     run_case(wl.CONFIGS[name], poison=True)
+
+
+@pytest.mark.parametrize("direction", [1.0, -1.0], ids=["rising", "falling"])
+def test_running_max_moves(direction):
+    """Scores that ramp steeply along the sequence (about 20 in log2 units per 128
+    tokens): with a rising ramp every tile raises every head's running max by far more
+    than the rescale threshold, so O and the row sums are rescaled on most tiles; with a
+    falling ramp the first tile holds the max and later weights underflow to zero."""
+    cfg = small("ramp", 2, 32, 2, 128, 1500, lens=[1500, 700])
+    g = torch.Generator().manual_seed(3)
+    B, n_q, n_kv, d, T = cfg.batch, cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.max_seq_len
+    q = (0.5 + 0.1 * torch.randn(B, n_q, d, generator=g)).to(torch.bfloat16)
+    t = torch.arange(T, dtype=torch.float32).view(1, 1, T, 1)
+    ramp = 0.019 * (t if direction > 0 else (T - 1 - t))
+    k = (ramp + 0.3 * torch.randn(B, n_kv, T, d, generator=g)).to(torch.bfloat16)
+    v = torch.randn(B, n_kv, T, d, generator=g).to(torch.bfloat16)
+    lens = torch.tensor(cfg.seq_lens, dtype=torch.int32)
+    for b in range(B):
+        k[b, :, lens[b]:] = float("nan")
+        v[b, :, lens[b]:] = float("nan")
+    run_case(cfg, inputs={"q": q, "k_cache": k, "v_cache": v, "seq_lens": lens})
