@@ -106,8 +106,8 @@ int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
  *   out           device fp32 [batch, n_heads, latent_dim]  (latent space)
  *   lse           device fp32 [batch, n_heads]
  * Score of head h at token t: scale * (q_latent[h] . latent_t + q_rope[h] . rope_t).
- * Precondition: |q_latent| and |latent_cache| values stay within the fp16 range
- * (65504); the value product runs in fp16 on the tensor cores.
+ * Every bf16 value is accepted as is (no narrower intermediate format): the weights
+ * enter the value product as a bf16 high part plus a bf16 remainder.
  */
 int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
                       const uint16_t *latent_cache, const uint16_t *rope_cache,

@@ -131,6 +131,15 @@ __device__ __forceinline__ float bf16_round(float x) {
     return __bfloat162float(__float2bfloat16_rn(x));
 }
 
+// Splits two fp32 weights into bf16 high parts (the top 16 bits, i.e. truncated: no
+// conversion instruction) and bf16 remainders (rounded); hi + lo carries ~16
+// significant bits of each weight.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+    hi = __byte_perm(ua, ub, 0x7632);
+    lo = pack_bf16x2(a - __uint_as_float(ua & 0xffff0000u), b - __uint_as_float(ub & 0xffff0000u));
+}
+
 // 2^x with the hardware approximation (flushes subnormal results to zero).
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;

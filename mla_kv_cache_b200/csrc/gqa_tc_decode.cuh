@@ -20,7 +20,8 @@
 // Per 128-token tile (one CTA per SM, persistent, stream-K over tiles, schedule.cuh):
 //   producer (warp 0)   TMA loads of the K and V tiles (two 128-byte-swizzled boxes of
 //                       [128 tokens x 64] each) into a 3-stage ring; the unit's query
-//                       block once per piece.  No multicast.
+//                       block once per piece, double-buffered when it has <= 32 heads.
+//                       No multicast.
 //   MMA (warp 1)        the score product of the next tile (8 MMAs 128 x N x 16) into one
 //                       of two TMEM score buffers, then the value product of this tile
 //                       (16 MMAs 128 x 64 x 16) into O^T; completion by tcgen05.commit.
@@ -56,8 +57,7 @@ constexpr int NST = 3;                    // pipeline stages
 constexpr int CHUNK = TILE * 128;         // one [128 tokens x 64] bf16 box: 16 KB
 constexpr int KV_BYTES = 2 * CHUNK;       // a K or V tile: 32 KB
 constexpr int STAGE = 2 * KV_BYTES;       // K then V: 64 KB
-constexpr int QCHUNK = HB * 128;          // [64 heads x 64] bf16 box: 8 KB
-constexpr int QBUF = 2 * QCHUNK;          // the unit's query block: 16 KB
+constexpr int QREGION = 2 * HB * 128;     // query blocks: 16 KB (one of 64 heads or two of <= 32)
 constexpr int NTHREADS = 192;             // producer, MMA, 4 softmax warps
 constexpr int NSOFT = 128;
 constexpr uint32_t TM_S = 0;              // two 64-column score buffers
@@ -67,7 +67,7 @@ constexpr float RESCALE_LOG2 = 8.f;
 
 constexpr int OFF_ST = 0;
 constexpr int OFF_Q = OFF_ST + NST * STAGE;        // 196608
-constexpr int OFF_RED = OFF_Q + QBUF;              // [3][4][64] fp32: tile slots 0/1, piece end
+constexpr int OFF_RED = OFF_Q + QREGION;              // [3][4][64] fp32: tile slots 0/1, piece end
 constexpr int OFF_MS = OFF_RED + 3 * 4 * HB * 4;   // [2][64] running max per head
 constexpr int OFF_AS = OFF_MS + 2 * HB * 4;        // [2][64] rescale factor per head
 constexpr int OFF_NF = OFF_AS + 2 * HB * 4;        // [2][64] bytes: head rescaled this tile
@@ -80,8 +80,8 @@ constexpr int smem_bytes(int B) { return 1024 + OFF_PREFIX + (B + 1) * 4; }
 
 struct Bars {
     uint64_t full[NST], empty[NST];
-    uint64_t qfull;       // the unit's query block landed
-    uint64_t qempty;      // every score MMA of the piece has read it
+    uint64_t qfull[2];    // a query block landed (buffer = piece % NQB)
+    uint64_t qempty[2];   // every score MMA of that piece has read it
     uint64_t sready[2];   // scores of a tile in TMEM buffer (tile & 1)
     uint64_t sfree[2];    // the softmax threads have read that buffer
     uint64_t pready[2];   // P^T written (and O^T rescaled): the value product may run
@@ -97,6 +97,11 @@ struct Cfg {
     static constexpr int NQ = NR < 16 ? 16 : NR;           // score-product N (and columns read)
     static constexpr int RW = NR >= 32 ? NR / 32 : 1;      // values a lane holds after the reduction
     static constexpr int LPH = NR >= 32 ? 1 : 32 / NR;     // lanes holding the same head after it
+    static constexpr int QCHUNK = NQ * 128;                // [NQ heads x 64] bf16 box
+    static constexpr int QBLOCK = 2 * QCHUNK;              // one query block (head_dim 128)
+    // query buffers: two when they fit, so that the next piece's block loads while the
+    // current piece still reads its own
+    static constexpr int NQB = 2 * QBLOCK <= QREGION ? 2 : 1;
 };
 
 struct Ctx {
@@ -168,8 +173,10 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[NQ]) 
     }
 }
 // ------------------------------------------------------------------ producer (warp 0, lane 0)
+template <int NR>
 __device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *kmap, const CUtensorMap *vmap,
                                          const CUtensorMap *qmap, const Ctx &c) {
+    using C = Cfg<NR>;
     Bars *bars = c.bars;
     const uint64_t pol = l2_policy_evict_first();
     int k = 0, pi = 0;
@@ -180,14 +187,16 @@ __device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *
         const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
         const int j = pc.i / p.n_hb, hb = pc.i % p.n_hb;
         const int z = pc.b * p.n_kv + j;
-        if (pi > 0 && !mbar_wait(&bars->qempty, (uint32_t)(pi - 1) & 1u, FLAG_EMPTY_WAIT, c.abort_flag)) {
+        const int qb = pi % C::NQB, qu = pi / C::NQB;
+        if (qu > 0 && !mbar_wait(&bars->qempty[qb], (uint32_t)(qu - 1) & 1u, FLAG_EMPTY_WAIT, c.abort_flag)) {
             ok = false;
             break;
         }
-        mbar_arrive_expect_tx(&bars->qfull, QBUF);
+        mbar_arrive_expect_tx(&bars->qfull[qb], C::QBLOCK);
         const int qrow = j * p.g + hb * HB;
-        tma_load_3d(c.smem + OFF_Q, qmap, &bars->qfull, 0, qrow, pc.b, pol);
-        tma_load_3d(c.smem + OFF_Q + QCHUNK, qmap, &bars->qfull, 64, qrow, pc.b, pol);
+        uint8_t *qdst = c.smem + OFF_Q + qb * C::QBLOCK;
+        tma_load_3d(qdst, qmap, &bars->qfull[qb], 0, qrow, pc.b, pol);
+        tma_load_3d(qdst + C::QCHUNK, qmap, &bars->qfull[qb], 64, qrow, pc.b, pol);
         for (int lt = pc.lt0; lt < pc.lt1; ++lt, ++k) {
             const int s = k % NST;
             const uint32_t ph = (uint32_t)(k / NST) & 1u;
@@ -205,7 +214,8 @@ __device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *
         // Let every copy already issued land before the CTA can exit.
         for (int kk = (k > NST ? k - NST : 0); kk < k; ++kk)
             mbar_wait_sleep(&bars->full[kk % NST], (uint32_t)(kk / NST) & 1u, FLAG_FULL_WAIT, nullptr);
-        if (pi > 0) mbar_wait_sleep(&bars->qfull, (uint32_t)(pi - 1) & 1u, FLAG_FULL_WAIT, nullptr);
+        for (int pp = (pi > C::NQB ? pi - C::NQB : 0); pp < pi; ++pp)
+            mbar_wait_sleep(&bars->qfull[pp % C::NQB], (uint32_t)(pp / C::NQB) & 1u, FLAG_FULL_WAIT, nullptr);
     }
 }
 
@@ -213,17 +223,18 @@ __device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *
 // Score product of tile kt into TMEM buffer (kt & 1).  The caller has seen the tile
 // land and the buffer freed.
 template <int NR>
-__device__ __forceinline__ void issue_scores(const Ctx &c, int kt) {
+__device__ __forceinline__ void issue_scores(const Ctx &c, int kt, int qbuf) {
+    using C = Cfg<NR>;
     const int s = kt % NST, sb = kt & 1;
     tc_fence_after();
     constexpr uint32_t idesc = idesc_f16_major(128, Cfg<NR>::NQ, 1, 1, 0, 0);
     const uint32_t st = smem_u32(c.smem + OFF_ST + s * STAGE);
-    const uint32_t qb = smem_u32(c.smem + OFF_Q);
+    const uint32_t qb = smem_u32(c.smem + OFF_Q + qbuf * C::QBLOCK);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t blk = kk >> 2, in = (kk & 3) * 32;
         const uint64_t a = smem_desc_sw128(st + blk * CHUNK + in, 16, 1024);
-        const uint64_t b = smem_desc_sw128(qb + blk * QCHUNK + in, 16, 1024);
+        const uint64_t b = smem_desc_sw128(qb + blk * C::QCHUNK + in, 16, 1024);
         umma_ss(c.tmem + TM_S + 64 * sb, a, b, idesc, kk > 0 ? 1u : 0u);
     }
     umma_commit(&c.bars->sready[sb]);
@@ -263,7 +274,8 @@ __device__ __forceinline__ void mma_issuer(const GqaParams &p, const Ctx &c) {
         const Piece pc = piece_at(c.s_prefix, p.B, c.U, pos, c.p1, c.p0);
         pos = pc.ustart + pc.lt1;
         const int nt = pc.lt1 - pc.lt0;
-        if (!mbar_wait(&bars->qfull, (uint32_t)pi & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
+        const int qb = pi % Cfg<NR>::NQB, qu = pi / Cfg<NR>::NQB;
+        if (!mbar_wait(&bars->qfull[qb], (uint32_t)qu & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
         int nq = 0, nv = 0;
         long long idle_since = clock64();
         while (nv < nt) {
@@ -272,9 +284,9 @@ __device__ __forceinline__ void mma_issuer(const GqaParams &p, const Ctx &c) {
                 const int kt = k + nq;
                 if (mbar_test(&bars->full[kt % NST], (uint32_t)(kt / NST) & 1u) &&
                     (kt < 2 || mbar_test(&bars->sfree[kt & 1], (uint32_t)((kt >> 1) - 1) & 1u))) {
-                    issue_scores<NR>(c, kt);
+                    issue_scores<NR>(c, kt, qb);
                     ++nq;
-                    if (nq == nt) umma_commit(&bars->qempty);
+                    if (nq == nt) umma_commit(&bars->qempty[qb]);
                     progressed = true;
                 }
             }
@@ -409,9 +421,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                     const float b = fast_exp2(sc[h + 1] - mh[2 * e + 1]);
                     l_part[h] += a;
                     l_part[h + 1] += b;
-                    const float ah = bf16_round(a), bh = bf16_round(b);
-                    hw[e] = pack_bf16x2(ah, bh);
-                    lw[e] = pack_bf16x2(a - ah, b - bh);
+                    split_bf16x2(a, b, hw[e], lw[e]);
                 }
                 const int slot = (cc ^ (r & 7)) << 4;
                 *reinterpret_cast<uint4 *>(hrow + slot) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
@@ -512,8 +522,10 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
-        mbar_init(&bars->qfull, 1);
-        mbar_init(&bars->qempty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->qfull[i], 1);
+            mbar_init(&bars->qempty[i], 1);
+        }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->sready[i], 1);
             mbar_init(&bars->sfree[i], NSOFT);
@@ -560,7 +572,7 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
 
     if (c.p0 < total) {
         if (warp == 0) {
-            if (lane == 0) producer(p, &kmap, &vmap, &qmap, c);
+            if (lane == 0) producer<NR>(p, &kmap, &vmap, &qmap, c);
         } else if (warp == 1) {
             if (lane == 0) mma_issuer<NR>(p, c);
         } else {

@@ -424,7 +424,9 @@ int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
     if (tc) {
-        st = make_map_3d(&qmap, q, head_dim, n_q_heads, batch, 64, gqatc::HB, CU_TENSOR_MAP_SWIZZLE_128B);
+        // box rows = the score product's N for this group size (query heads per block)
+        const uint32_t q_rows = g > 32 ? 64 : g > 16 ? 32 : 16;
+        st = make_map_3d(&qmap, q, head_dim, n_q_heads, batch, 64, q_rows, CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != KVATTN_OK) return st;
     }
 

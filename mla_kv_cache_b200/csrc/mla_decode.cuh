@@ -1,5 +1,5 @@
 // mla_decode.cuh -- absorbed multi-head latent attention decode (latent 512 + RoPE 64)
-// on sm_100a tensor cores (tcgen05, accumulators in tensor memory).
+// on sm_100a tensor cores (tcgen05, accumulators and operands in tensor memory).
 //
 // What it computes ("Attention variants: MQA, GQA, and MLA", section "MLA: cache a
 // latent, not the keys and values"): with the key up-projection folded into the query,
@@ -10,35 +10,41 @@
 // whose first 512 elements are also the value.
 //
 // Why a CTA pair.  The fp32 accumulator of 128 heads x 512 latent columns is 256 KB,
-// all of one SM's tensor memory, and the 128 x 576 query alone is 144 KB of shared
-// memory.  A 2-CTA cluster therefore splits the latent columns: CTA r holds columns
-// [256r, 256r + 256) of every cached row (CTA 0 also the 64 RoPE columns), the matching
-// query columns, and the output accumulator O_r = P * C[:, 256r..] (128 x 256 fp32,
-// 256 TMEM columns).  Each CTA computes partial scores over its part of the 576-wide
-// contraction and ships them to the other CTA with st.async (distributed shared memory,
-// completion counted on the receiver's mbarrier); both CTAs then add the two partials
-// in the same order and run the identical online softmax for all 128 heads, so P, the
-// rescale factors and the row sums never have to cross the pair.  Every cached byte is
-// loaded from HBM once and every MMA is a full-rate M = 128 tcgen05.mma.
+// all of one SM's tensor memory.  A 2-CTA cluster therefore splits the latent columns:
+// CTA r holds columns [256r, 256r + 256) of every cached row (CTA 0 also the 64 RoPE
+// columns) and the accumulator O_r = P * C[:, 256r..] (128 x 256 fp32, 256 TMEM columns).
+// Each CTA computes partial scores over its part of the 576-wide contraction and stores
+// them into the other CTA's shared memory (distributed shared memory; each sending
+// thread then arrives with release semantics on the receiver's mbarrier); both CTAs add the two partials in the same order and run
+// the identical online softmax, so P, the rescale factors and the row sums never cross
+// the pair.  Every cached byte is loaded from HBM once; every MMA is M = 128.
+//
+// Tensor memory of a CTA (512 columns): O_r [0, 256), the partial scores S_r of one
+// tile [256, 320), the latent part of Q_r as bf16 pairs [320, 448), and P of one tile
+// [448, 512): its bf16 high part (32 columns, the top 16 bits of each fp32 weight) and
+// bf16 remainder (32 columns).  The
+// value product runs twice, O_r += P_hi C_r + P_lo C_r, so the weights keep ~16
+// significant bits while the cache stays in its bf16 form (no conversion pass).
 //
 // Per 64-token tile and CTA:
 //   TMA (warp 0)       4 (CTA 0: 5) 128-byte-swizzled boxes [64 tokens x 64 columns]
-//                      into a 2-stage ring; the query block once per piece.
-//   MMA (warp 1)       S_r = Q_r C_r^T: 16 (20) kind::f16 bf16 MMAs 128x64x16 into TMEM;
-//                      later O_r += P C_r: 4 kind::f16 fp16 MMAs 128x256x16 (C_r read
-//                      MN-major from the same tile).  Completion via tcgen05.commit.
-//   convert (warps 2-3) once the score MMAs have read the tile, the 256 latent columns
-//                      are converted in place from bf16 to fp16 for the value product.
-//   softmax (warps 4-11) 8 warps = 2 per TMEM lane quadrant, each thread one head row
-//                      and 32 of the 64 token columns: send the partial scores, add the
-//                      peer's, mask, take the running max (rescaling O only when the max
-//                      grows by more than 2^8), write P = 2^(s - m) in fp16, keep the
-//                      row sum.
-// P and the value tile are fp16 (11 significant bits) so that the weights of a sharp
-// softmax over a few tokens stay within the library's tolerance; this is why the latent
-// values must lie in the fp16 range.  At the end of a piece every thread normalises its
-// 128 output columns from TMEM and writes the final result or the worker's partial for
-// the split combine.
+//                      into a 3-stage ring; CTA 0 also the q_rope block once per piece.
+//   MMA (warp 1)       S_r = Q_r C_r^T: 16 MMAs 128x64x16 with A from TMEM (CTA 0: 4 more
+//                      with the RoPE query from shared memory); O_r += P C_r: 8 MMAs
+//                      128x256x16 with A = P from TMEM and C_r read MN-major from the same
+//                      swizzled tile.  It issues whichever product is ready.
+//   softmax (warps 2-9) two groups of four warps (one per TMEM lane quadrant) take the
+//                      tiles in turn, so one group's exchange and exponentials overlap
+//                      the other's.  A thread owns one head row of its group's tiles: it
+//                      reads the row's 64 partial scores, sends them to the peer, adds the
+//                      peer's, masks, and takes the tile maximum.  The running max is
+//                      handed from group to group through shared memory (the only serial
+//                      step); it moves lazily, only when a tile's maximum exceeds it by
+//                      more than 2^8, and then this row of O_r is rescaled in TMEM.  The
+//                      thread writes P = 2^(s - m) into TMEM and keeps its group's row sum.
+// At the end of a piece the two groups merge their row sums, and each normalises half
+// of the row's 256 output columns from TMEM and writes the final result or the worker's
+// partial for the split combine.
 #pragma once
 #include "common.cuh"
 #include "schedule.cuh"
@@ -52,42 +58,44 @@ constexpr int HR = 128;                  // head rows (MMA M)
 constexpr int NCH = 5;                   // 64-column chunks per stage slot (CTA 0 uses 5)
 constexpr int NST = 3;                   // pipeline stages
 constexpr int CHUNK_T = TILE * 128;      // one [64 tokens x 64 cols] bf16 box: 8 KB
-constexpr int CHUNK_Q = HR * 128;        // one [128 heads x 64 cols] box: 16 KB
 constexpr int STAGE = NCH * CHUNK_T;     // 40 KB
-constexpr int PBUF = HR * 128;           // P: [128 heads x 64 tokens] fp16: 16 KB
-constexpr int NTHREADS = 384;
+constexpr int QROPE = HR * 128;          // q_rope block [128 heads x 64] bf16: 16 KB
+constexpr int NTHREADS = 320;            // producer, MMA, two softmax groups of 4 warps
+constexpr int NGROUP = 128;              // threads per softmax group
 constexpr int MAX_BATCH = 1024;
 constexpr uint32_t TM_O = 0;             // TMEM columns [0, 256): O_r
-constexpr uint32_t TM_S = 256;           // TMEM columns [256, 320): partial scores
-constexpr uint32_t TM_Q = 320;           // TMEM columns [320, 480): Q_r (bf16 pairs)
+constexpr uint32_t TM_S = 256;           // [256, 320): partial scores of one tile
+constexpr uint32_t TM_Q = 320;           // [320, 448): latent part of Q_r (bf16 pairs)
+constexpr uint32_t TM_P = 448;           // [448, 480): P high part, [480, 512): remainder
 constexpr uint32_t TM_COLS = 512;
 constexpr float RESCALE_LOG2 = 8.f;      // rescale O only when the row max grows by > 2^8
 constexpr uint32_t RECV_BYTES = HR * TILE * 4;   // the peer's partial scores of one tile
 
 constexpr int OFF_ST = 0;
-constexpr int OFF_P = OFF_ST + NST * STAGE;              // 163840
-constexpr int OFF_RECV = OFF_P + PBUF;                   // the peer's partials: [128 heads][64] fp32
-constexpr int OFF_SEND = OFF_RECV + (int)RECV_BYTES;     // this CTA's partials, same layout
-constexpr int OFF_XCH = OFF_SEND + (int)RECV_BYTES;      // [2][128][2] fp32
-constexpr int OFF_BARS = OFF_XCH + 2 * HR * 2 * 4;       // 215040
-constexpr int OFF_TMEMPTR = OFF_BARS + 256;              // 215296
+constexpr int OFF_QROPE = OFF_ST + NST * STAGE;          // 122880
+constexpr int OFF_RECV = OFF_QROPE + QROPE;              // 139264: two [128 heads][64] fp32
+constexpr int OFF_MREF = OFF_RECV + 2 * (int)RECV_BYTES; // 204800: [2][128] running max
+constexpr int OFF_LX = OFF_MREF + 2 * HR * 4;            // [2][128] row sums of the groups
+constexpr int OFF_BARS = OFF_LX + 2 * HR * 4;            // 206848
+constexpr int OFF_TMEMPTR = OFF_BARS + 256;
 constexpr int OFF_ABORT = OFF_TMEMPTR + 16;
-constexpr int OFF_PREFIX = OFF_ABORT + 16;               // 215328
+constexpr int OFF_PREFIX = OFF_ABORT + 16;
 constexpr int smem_bytes(int B) { return 1024 + OFF_PREFIX + (B + 1) * 4; }
 
 struct Bars {
-    uint64_t full[NST], empty[NST], qkdone[NST], cvt[NST];
-    uint64_t qready;      // Q_r written into TMEM (softmax warps)
-    uint64_t qempty;      // every score MMA of the piece has read Q_r
-    uint64_t sready, sfree;
-    uint64_t recv_full;   // the peer's partial scores landed (tx-counted)
-    uint64_t recv_free;   // the peer has read the partial scores this CTA sent it
-    uint64_t send_ready;  // this CTA's partial scores are in the send buffer
-    uint64_t send_free;   // the bulk copy has finished reading the send buffer
-    uint64_t oready[2];   // P written and O rescaled; PV may run
-    uint64_t odone;       // PV done (also: P buffer free)
-    uint64_t ofree;       // epilogue read O
-    uint64_t pair[4];     // the two threads of a head row, per lane quadrant
+    uint64_t full[NST], empty[NST];
+    uint64_t qready;       // latent part of Q_r written into TMEM (both groups)
+    uint64_t qrope_full;   // q_rope block landed in shared memory (TMA, CTA 0)
+    uint64_t qempty;       // every score MMA of the piece has read Q
+    uint64_t sready[2];    // partial scores of a tile (parity) in TMEM
+    uint64_t sfree;        // the tile's group has read them
+    uint64_t recv_full[2]; // the peer's partial scores of a tile of group g landed (its 128 rows)
+    uint64_t recv_free[2]; // the peer has read what this CTA sent into its buffer g
+    uint64_t hand[2];      // running max of a tile (parity) published
+    uint64_t pready;       // P of a tile in TMEM and O rescaled: the value product may run
+    uint64_t odone[2];     // value product of a tile (parity) finished
+    uint64_t ofree;        // the epilogue has read O
+    uint64_t lx;           // the groups' row sums exchanged (end of a piece)
 };
 static_assert(sizeof(Bars) <= 256, "barrier block overflows its slot");
 
@@ -136,10 +144,19 @@ __device__ __forceinline__ void producer(const MlaParams &p, const MlaMaps &m, c
         const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
         pos = pc.ustart + pc.lt1;
         const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
+        if (c.r == 0) {
+            // the RoPE part of this sequence's queries (the score MMAs read it from here)
+            if (pi > 0 && !mbar_wait(&bars->qempty, (uint32_t)(pi - 1) & 1u, FLAG_EMPTY_WAIT, c.abort_flag)) {
+                ok = false;
+                break;
+            }
+            mbar_arrive_expect_tx(&bars->qrope_full, QROPE);
+            tma_load_3d(c.smem + OFF_QROPE, &m.qrope, &bars->qrope_full, 0, 0, pc.b, pol);
+        }
         for (int lt = pc.lt0; lt < pc.lt1; ++lt, ++k) {
             const int s = k % NST;
             const uint32_t ph = (uint32_t)(k / NST) & 1u;
-            if (!mbar_wait_sleep(&bars->empty[s], ph ^ 1u, FLAG_EMPTY_WAIT, c.abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&bars->empty[s], ph ^ 1u, FLAG_EMPTY_WAIT, c.abort_flag)) { ok = false; break; }
             mbar_arrive_expect_tx(&bars->full[s], nch * CHUNK_T);
             const int y = min(lt * TILE, len - TILE);
             uint8_t *st = c.smem + OFF_ST + s * STAGE;
@@ -152,130 +169,120 @@ __device__ __forceinline__ void producer(const MlaParams &p, const MlaMaps &m, c
         // Let every copy already issued land before the CTA can exit.
         for (int kk = (k > NST ? k - NST : 0); kk < k; ++kk)
             mbar_wait_sleep(&bars->full[kk % NST], (uint32_t)(kk / NST) & 1u, FLAG_FULL_WAIT, nullptr);
+        if (c.r == 0 && pi > 0) mbar_wait_sleep(&bars->qrope_full, (uint32_t)(pi - 1) & 1u, FLAG_FULL_WAIT, nullptr);
     }
 }
 
 // ------------------------------------------------------------------ MMA issuer (warp 1, lane 0)
-__device__ __forceinline__ bool issue_scores(const Ctx &c, int kt, int nch, uint32_t st_base) {
-    Bars *bars = c.bars;
+// Partial scores of tile kt: latent chunks with A = Q_r from TMEM, the RoPE chunk (CTA 0)
+// with A = q_rope from shared memory.  The caller has seen the tile land and S freed.
+__device__ __forceinline__ void issue_scores(const Ctx &c, int kt) {
     const int s = kt % NST;
-    if (!mbar_wait_sleep(&bars->full[s], (uint32_t)(kt / NST) & 1u, FLAG_FULL_WAIT, c.abort_flag)) return false;
-    if (kt > 0 && !mbar_wait_sleep(&bars->sfree, (uint32_t)(kt - 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)) return false;
     tc_fence_after();
     constexpr uint32_t idesc = idesc_f16(128, TILE, 1, 1, 0);
-    for (int ch = 0; ch < nch; ++ch)
+    const uint32_t st = smem_u32(c.smem + OFF_ST + s * STAGE);
+    for (int ch = 0; ch < 4; ++ch)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t b = smem_desc_sw128(st_base + s * STAGE + ch * CHUNK_T + kk * 32, 16, 1024);
-            umma_ts(c.tmem + TM_S, c.tmem + TM_Q + ch * 32 + kk * 8, b, idesc, (ch | kk) != 0);
+            const uint64_t bd = smem_desc_sw128(st + ch * CHUNK_T + kk * 32, 16, 1024);
+            umma_ts(c.tmem + TM_S, c.tmem + TM_Q + ch * 32 + kk * 8, bd, idesc, (ch | kk) != 0);
         }
-    umma_commit(&bars->sready);
-    umma_commit(&bars->qkdone[s]);
-    return true;
+    if (c.r == 0) {
+        const uint32_t qr = smem_u32(c.smem + OFF_QROPE);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = smem_desc_sw128(qr + kk * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(st + 4 * CHUNK_T + kk * 32, 16, 1024);
+            umma_ss(c.tmem + TM_S, ad, bd, idesc, 1u);
+        }
+    }
+    umma_commit(&c.bars->sready[kt & 1]);
 }
 
+// O_r += P C_r for tile kt: 4 token blocks of 16, high part then remainder of P.
+__device__ __forceinline__ void issue_values(const Ctx &c, int kt, bool first) {
+    const int s = kt % NST;
+    tc_fence_after();
+    constexpr uint32_t idesc = idesc_f16(128, 256, 1, 1, 1);
+    const uint32_t st = smem_u32(c.smem + OFF_ST + s * STAGE);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t bd = smem_desc_sw128(st + kk * 2048, CHUNK_T, 1024);
+        umma_ts(c.tmem + TM_O, c.tmem + TM_P + kk * 8, bd, idesc, (!first || kk > 0) ? 1u : 0u);
+        umma_ts(c.tmem + TM_O, c.tmem + TM_P + 32 + kk * 8, bd, idesc, 1u);
+    }
+    umma_commit(&c.bars->empty[s]);
+    umma_commit(&c.bars->odone[kt & 1]);
+}
+
+// Issues the value product of the oldest scored tile (P written; at a piece start, O
+// read out) or the score product of the next tile (tile landed, the previous tile's
+// scores read), whichever is ready -- the value product first, it is on the softmax
+// groups' critical path -- never blocking on one while the other could go.
+// Idle time is bounded like every other wait.
 __device__ __forceinline__ void mma_issuer(const MlaParams &p, const Ctx &c) {
     Bars *bars = c.bars;
-    const int nch = c.r == 0 ? 5 : 4;
-    const uint32_t st_base = smem_u32(c.smem + OFF_ST);
-    const uint32_t p_base = smem_u32(c.smem + OFF_P);
-    constexpr uint32_t idesc_pv = idesc_f16(128, 256, 0, 0, 1);
     int k = 0, pi = 0;
     for (long long pos = c.p0; pos < c.p1; ++pi) {
         const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
         pos = pc.ustart + pc.lt1;
         const int nt = pc.lt1 - pc.lt0;
-        if (!mbar_wait_sleep(&bars->qready, (uint32_t)pi & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
-        tc_fence_after();
-        if (!issue_scores(c, k, nch, st_base)) return;
-        for (int t = 0; t < nt; ++t) {
-            const int kt = k + t;
-            if (t + 1 < nt) {
-                if (!issue_scores(c, kt + 1, nch, st_base)) return;
-            } else {
-                umma_commit(&bars->qempty);      // every score MMA of this piece has read Q
-            }
-            const int s = kt % NST, pb = kt & 1;
-            if (!mbar_wait_sleep(&bars->cvt[s], (uint32_t)(kt / NST) & 1u, FLAG_MMA_WAIT, c.abort_flag)) return;
-            if (!mbar_wait_sleep(&bars->oready[pb], (uint32_t)(kt >> 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)) return;
-            if (t == 0 && pi > 0 &&
-                !mbar_wait_sleep(&bars->ofree, (uint32_t)(pi - 1) & 1u, FLAG_MMA_WAIT, c.abort_flag))
-                return;
-            tc_fence_after();
-            fence_proxy_async_smem();
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t a = smem_desc_sw128(p_base + kk * 32, 16, 1024);
-                const uint64_t b = smem_desc_sw128(st_base + s * STAGE + kk * 2048, CHUNK_T, 1024);
-                umma_ss(c.tmem + TM_O, a, b, idesc_pv, (t > 0 || kk > 0) ? 1u : 0u);
-            }
-            umma_commit(&bars->empty[s]);
-            umma_commit(&bars->odone);
-        }
-        k += nt;
-    }
-}
-
-// ------------------------------------------------------------------ converters (warps 2-3)
-__device__ __forceinline__ void converter(const MlaParams &p, const Ctx &c, int ctid) {
-    Bars *bars = c.bars;
-    int k = 0;
-    for (long long pos = c.p0; pos < c.p1;) {
-        const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
-        pos = pc.ustart + pc.lt1;
-        for (int lt = pc.lt0; lt < pc.lt1; ++lt, ++k) {
-            const int s = k % NST;
-            if (!mbar_wait_sleep(&bars->qkdone[s], (uint32_t)(k / NST) & 1u, FLAG_MMA_WAIT, c.abort_flag)) return;
-            uint4 *base = reinterpret_cast<uint4 *>(c.smem + OFF_ST + s * STAGE);
-            // the four latent chunks (the value columns): 4 x 8 KB = 2048 16-byte units,
-            // four independent loads in flight per thread
-            for (int u0 = ctid; u0 < 4 * CHUNK_T / 16; u0 += 4 * 64) {
-                uint4 v[4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) v[r] = base[u0 + 64 * r];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    uint32_t w[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float lo = __uint_as_float(w[i] << 16);
-                        const float hi = __uint_as_float(w[i] & 0xffff0000u);
-                        __half2 h2 = __floats2half2_rn(lo, hi);
-                        w[i] = *reinterpret_cast<uint32_t *>(&h2);
-                    }
-                    base[u0 + 64 * r] = make_uint4(w[0], w[1], w[2], w[3]);
+        if (!mbar_wait(&bars->qready, (uint32_t)pi & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
+        if (c.r == 0 && !mbar_wait(&bars->qrope_full, (uint32_t)pi & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
+        int nq = 0, nv = 0;
+        long long idle_since = clock64();
+        while (nv < nt) {
+            bool progressed = false;
+            if (nv < nq) {
+                const int kt = k + nv;
+                if (mbar_test(&bars->pready, (uint32_t)kt & 1u) &&
+                    (nv > 0 || pi == 0 || mbar_test(&bars->ofree, (uint32_t)(pi - 1) & 1u))) {
+                    issue_values(c, kt, nv == 0);
+                    ++nv;
+                    progressed = true;
                 }
             }
-            fence_proxy_async_smem();
-            mbar_arrive(&bars->cvt[s]);
+            if (nq < nt && nq < nv + NST) {
+                const int kt = k + nq;
+                if (mbar_test(&bars->full[kt % NST], (uint32_t)(kt / NST) & 1u) &&
+                    (kt == 0 || mbar_test(&bars->sfree, (uint32_t)(kt - 1) & 1u))) {
+                    issue_scores(c, kt);
+                    ++nq;
+                    if (nq == nt) umma_commit(&bars->qempty);   // the piece's last score MMAs
+                    progressed = true;
+                }
+            }
+            if (progressed) {
+                idle_since = clock64();
+            } else {
+                if (*c.abort_flag) return;
+                if (clock64() - idle_since > kWaitLimitCycles) {
+                    atomicOr(&g_device_flags, FLAG_MMA_WAIT);
+                    *c.abort_flag = 1;
+                    return;
+                }
+            }
         }
+        k += nt;
     }
 }
 
 // 16-byte chunk slot of chunk j (columns 4j..4j+3) in row h of a receive buffer.
 __device__ __forceinline__ int recv_chunk(int j, int h) { return j ^ (h & 7); }
 
-// ------------------------------------------------------------------ softmax (warps 4-11)
+// ------------------------------------------------------------------ softmax (warps 2-9)
 __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, int warp, int lane) {
     Bars *bars = c.bars;
-    const int q = warp & 3;
-    const int half = (warp - 4) >> 2;
-    const int h = 32 * q + lane;
-    const bool armer = (warp == 4 && lane == 0);
+    const int g = (warp - 2) >> 2;              // group: takes the tiles k with k % 2 == g
+    const int q = warp & 3;                     // TMEM lane quadrant
+    const int h = 32 * q + lane;                // head row
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    const float *recv = reinterpret_cast<const float *>(c.smem + OFF_RECV);
-    float *xch = reinterpret_cast<float *>(c.smem + OFF_XCH);
-    // Send / receive buffers: row h holds 16 chunks of 16 bytes (64 fp32 scores), chunk
-    // index XOR (row % 8), so a warp's 32 rows spread over all banks.  The whole send
-    // buffer travels to the peer's receive buffer in one bulk copy per tile.
-    uint8_t *send_row = c.smem + OFF_SEND + h * TILE * 4;
-    const uint32_t peer_recv_buf = map_to_rank(smem_u32(c.smem + OFF_RECV), c.peer);
-    const uint32_t send_buf = smem_u32(c.smem + OFF_SEND);
-    const uint32_t peer_recv_full = map_to_rank(smem_u32(&bars->recv_full), c.peer);
-    (void)peer_recv_full;
-    const uint32_t peer_recv_free = map_to_rank(smem_u32(&bars->recv_free), c.peer);
-    uint8_t *prow = c.smem + OFF_P + h * 128;
-    uint32_t pair_uses = 0;
+    const float *recv = reinterpret_cast<const float *>(c.smem + OFF_RECV + g * RECV_BYTES) + h * TILE;
+    const uint32_t peer_recv = map_to_rank(smem_u32(c.smem + OFF_RECV + g * RECV_BYTES), c.peer) + h * TILE * 4;
+    const uint32_t peer_recv_full = map_to_rank(smem_u32(&bars->recv_full[g]), c.peer);
+    const uint32_t peer_recv_free = map_to_rank(smem_u32(&bars->recv_free[g]), c.peer);
+    float *mref = reinterpret_cast<float *>(c.smem + OFF_MREF);
+    float *lx = reinterpret_cast<float *>(c.smem + OFF_LX);
 
     int k = 0, pi = 0;
     for (long long pos = c.p0; pos < c.p1; ++pi) {
@@ -283,170 +290,155 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         pos = pc.ustart + pc.lt1;
         const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
         const int nt = pc.lt1 - pc.lt0;
-        // ---- Q_r of this sequence into TMEM (lane h = head h; bf16 pairs per column):
-        //      CTA 0 holds latent columns 0..255 and the 64 RoPE columns (160 words),
-        //      CTA 1 latent columns 256..511 (128 words).  Half 0 writes words [0, 96),
-        //      half 1 the rest, 32 words per tcgen05.st.
-        if (pi > 0 && !warp_all(mbar_wait_sleep(&bars->qempty, (uint32_t)(pi - 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
+        // ---- latent part of Q_r into TMEM (lane h = head h; bf16 pairs per column):
+        //      128 words per row, group g writes words [64g, 64g + 64)
+        if (pi > 0 && !warp_all(mbar_spin<false>(&bars->qempty, (uint32_t)(pi - 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
             return;
         {
-            const int nwords = c.r == 0 ? 160 : 128;
-            const int w0 = half == 0 ? 0 : 96, w1 = half == 0 ? 96 : nwords;
             const bool real = h < p.H;
             const uint32_t *ql = reinterpret_cast<const uint32_t *>(p.q_latent) +
-                                 ((size_t)pc.b * p.H + (real ? h : 0)) * 256 + 128 * c.r;
-            const uint32_t *qr = reinterpret_cast<const uint32_t *>(p.q_rope) +
-                                 ((size_t)pc.b * p.H + (real ? h : 0)) * 32;
+                                 ((size_t)pc.b * p.H + (real ? h : 0)) * 256 + 128 * c.r + 64 * g;
             tc_fence_after();
-            for (int w = w0; w < w1; w += 32) {
+#pragma unroll
+            for (int w = 0; w < 64; w += 32) {
                 uint32_t v[32];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const int word = w + 4 * j;
                     uint4 x = make_uint4(0, 0, 0, 0);
-                    if (real) x = word < 128 ? __ldg(reinterpret_cast<const uint4 *>(ql + word))
-                                             : __ldg(reinterpret_cast<const uint4 *>(qr + (word - 128)));
+                    if (real) x = __ldg(reinterpret_cast<const uint4 *>(ql + w + 4 * j));
                     v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
                 }
-                tmem_st32(c.tmem + lane_base + TM_Q + w, v);
+                tmem_st32(c.tmem + lane_base + TM_Q + 64 * g + w, v);
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->qready);
         }
-        float m_ref = -INFINITY;
-        float l_part = 0.f;
-        for (int t = 0; t < nt; ++t, ++k) {
+        float m_last = -INFINITY;     // reference of this group's row sum
+        float l_g = 0.f;              // this group's row sum (tiles of the piece it took)
+        const int k0 = k;
+        for (int t = (g - k0) & 1; t < nt; t += 2) {
+            const int kt = k0 + t;
             const int lt = pc.lt0 + t;
             const int y = min(lt * TILE, len - TILE);
             const int tok_lo = lt * TILE - y, tok_hi = min((lt + 1) * TILE, len) - y;
-            // ---- this CTA's partial scores
-            if (!warp_all(mbar_wait_sleep(&bars->sready, (uint32_t)k & 1u, FLAG_MMA_WAIT, c.abort_flag))) return;
+            // ---- this CTA's partial scores of the row
+            // (one barrier per group: the group of tile kt + 1 may start waiting while the
+            // scores of tile kt are still being computed)
+            if (!warp_all(mbar_spin<false>(&bars->sready[g], (uint32_t)(kt >> 1) & 1u, FLAG_MMA_WAIT, c.abort_flag))) return;
             tc_fence_after();
-            uint32_t sv[32];
-            tmem_ld32(c.tmem + lane_base + TM_S + 32 * half, sv);
-            tmem_wait_ld();
+            uint32_t sv[64];
+            {
+                uint32_t a[32], b[32];
+                tmem_ld32(c.tmem + lane_base + TM_S, a);
+                tmem_ld32(c.tmem + lane_base + TM_S + 32, b);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) { sv[j] = a[j]; sv[32 + j] = b[j]; }
+            }
             tc_fence_before();
             mbar_arrive(&bars->sfree);
-            // ---- stage them in the send buffer (free once the previous bulk copy has read it;
-            //      the issuing thread checks that here, off the previous tile's critical path)
-            if (armer && k > 0) {
-                bulk_wait_read_all();
-                mbar_arrive(&bars->send_free);
-            }
-            if (k > 0 && !warp_all(mbar_wait_sleep(&bars->send_free, (uint32_t)(k - 1) & 1u, FLAG_PEER_WAIT,
-                                                   c.abort_flag)))
+            // ---- to the peer (its buffer g must be free: it has read tile kt - 2)
+            if (kt >= 2 && !warp_all(mbar_spin<true>(&bars->recv_free[g], (uint32_t)((kt >> 1) - 1) & 1u,
+                                                       FLAG_PEER_WAIT, c.abort_flag)))
                 return;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                *reinterpret_cast<uint4 *>(send_row + recv_chunk(8 * half + j, h) * 16) =
-                    make_uint4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
-            fence_proxy_async_smem();
-            mbar_arrive(&bars->send_ready);
-            if (armer) {
-                // one bulk copy of all 128 rows into the peer, once the peer has read the last one
-                bool ok = mbar_wait_sleep(&bars->send_ready, (uint32_t)k & 1u, FLAG_FULL_WAIT, c.abort_flag);
-                if (ok && k > 0)
-                    ok = mbar_wait_cluster(&bars->recv_free, (uint32_t)(k - 1) & 1u, FLAG_PEER_WAIT, c.abort_flag);
-                if (ok) {
-                    bulk_copy_to_peer(peer_recv_buf, send_buf, RECV_BYTES, peer_recv_full);
-                    bulk_commit_group();
-                }
-            }
-            // ---- the peer's partial scores of this tile (one arrival + RECV_BYTES per phase)
-            if (armer) mbar_arrive_expect_tx(&bars->recv_full, RECV_BYTES);
-            if (!warp_all(mbar_wait_cluster(&bars->recv_full, (uint32_t)k & 1u, FLAG_PEER_WAIT, c.abort_flag)))
+            for (int j = 0; j < 16; ++j)
+                st_cluster_v4(peer_recv + (uint32_t)(recv_chunk(j, h) * 16), sv[4 * j], sv[4 * j + 1], sv[4 * j + 2],
+                              sv[4 * j + 3]);
+            mbar_arrive_cluster(peer_recv_full);   // release: the stores above are visible first
+            // ---- the peer's partial scores; both CTAs add (own + peer) in the same order
+            if (!warp_all(mbar_spin<true>(&bars->recv_full[g], (uint32_t)(kt >> 1) & 1u, FLAG_PEER_WAIT,
+                                            c.abort_flag)))
                 return;
-            float s[32];
-            const float4 *src = reinterpret_cast<const float4 *>(recv + h * TILE);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float4 v = src[recv_chunk(8 * half + j, h)];
-                // both CTAs add (own + peer); fp32 addition commutes, so the sums match
-                s[4 * j + 0] = __uint_as_float(sv[4 * j + 0]) + v.x;
-                s[4 * j + 1] = __uint_as_float(sv[4 * j + 1]) + v.y;
-                s[4 * j + 2] = __uint_as_float(sv[4 * j + 2]) + v.z;
-                s[4 * j + 3] = __uint_as_float(sv[4 * j + 3]) + v.w;
-            }
+            // scores in place (as float bits) from here on
             float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int row = 32 * half + j;
-                s[j] = (row >= tok_lo && row < tok_hi) ? s[j] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, s[j]);
-            }
-            // the received values are consumed (mx depends on all of them): the peer may
-            // overwrite its slice of this buffer now
-            mbar_arrive_cluster_relaxed(peer_recv_free);
-            // row max over both halves of the tile (the other half lives in warp q +/- 4)
-            float *slot = xch + (pair_uses & 1u) * (HR * 2);
-            slot[h * 2 + half] = mx;
-            mbar_arrive(&bars->pair[q]);
-            if (!warp_all(mbar_wait_sleep(&bars->pair[q], pair_uses & 1u, FLAG_FULL_WAIT, c.abort_flag))) return;
-            ++pair_uses;
-            mx = fmaxf(mx, slot[h * 2 + (half ^ 1)]);
-            float alpha = 1.f;
-            bool rescale = false;
-            if (t == 0) {
-                m_ref = mx;
-            } else if (mx > m_ref + RESCALE_LOG2) {
-                alpha = fast_exp2(m_ref - mx);
-                m_ref = mx;
-                rescale = true;
-            }
-            float ls = 0.f;
-            uint32_t ph[16];
-#pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const float a = fast_exp2(s[2 * j] - m_ref);
-                const float b = fast_exp2(s[2 * j + 1] - m_ref);
-                __half2 h2 = __floats2half2_rn(a, b);
-                ph[j] = *reinterpret_cast<uint32_t *>(&h2);
-                ls += a + b;
-            }
-            l_part = (t == 0) ? ls : (rescale ? l_part * alpha + ls : l_part + ls);
-            // ---- the previous value product has finished with P and with O
-            const bool need = rescale;
-            if (k > 0 && !warp_all(mbar_wait_sleep(&bars->odone, (uint32_t)(k - 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
-                return;
+                const float4 v = reinterpret_cast<const float4 *>(recv)[recv_chunk(j, h)];
+                const float pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int chunk = 4 * half + j;                  // tokens 8*chunk .. +7
-                *reinterpret_cast<uint4 *>(prow + ((chunk ^ (h & 7)) << 4)) =
-                    make_uint4(ph[4 * j], ph[4 * j + 1], ph[4 * j + 2], ph[4 * j + 3]);
+                for (int e = 0; e < 4; ++e) {
+                    const int col = 4 * j + e;
+                    float x = (__uint_as_float(sv[col]) + pv[e]) * p.scale_log2;
+                    x = (col >= tok_lo && col < tok_hi) ? x : -INFINITY;
+                    sv[col] = __float_as_uint(x);
+                    mx = fmaxf(mx, x);
+                }
             }
-            fence_proxy_async_smem();
-            // ---- rescale this row of O_r (tcgen05.ld/st are warp-collective: the whole warp
-            //      takes the branch when any row needs it, with factor 1 for the others)
-            if (__any_sync(0xffffffffu, need)) {
-                tc_fence_after();
-                const float f = need ? alpha : 1.f;
+            // the received values are consumed (mx depends on all of them)
+            mbar_arrive_cluster_relaxed(peer_recv_free);
+            // ---- running max, handed on from the previous tile's group
+            float m_prev = -INFINITY;
+            if (kt > 0) {
+                if (!warp_all(mbar_spin<false>(&bars->hand[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u, FLAG_FULL_WAIT,
+                                        c.abort_flag)))
+                    return;
+                if (t > 0) m_prev = mref[((kt - 1) & 1) * HR + h];
+            }
+            const float m_new = (t == 0 || mx > m_prev + RESCALE_LOG2) ? mx : m_prev;
+            mref[(kt & 1) * HR + h] = m_new;
+            mbar_arrive(&bars->hand[kt & 1]);
+            const bool rescale = t > 0 && m_new != m_prev;
+            const float alpha = rescale ? fast_exp2(m_prev - m_new) : 1.f;
+            // ---- weights, in two halves of 32 tokens; P goes into TMEM once the previous
+            //      value product is done with it (and with O)
+            l_g *= fast_exp2(m_last - m_new);      // 0 while this group has no tile yet
+            m_last = m_new;
+            float ls = 0.f;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const uint32_t addr = c.tmem + lane_base + TM_O + 128 * half + 32 * cc;
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t hw[16], lw[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float a = fast_exp2(__uint_as_float(sv[32 * hf + 2 * j]) - m_new);
+                    const float b = fast_exp2(__uint_as_float(sv[32 * hf + 2 * j + 1]) - m_new);
+                    ls += a + b;
+                    split_bf16x2(a, b, hw[j], lw[j]);
+                }
+                if (hf == 0) {
+                    if (kt > 0 && !warp_all(mbar_spin<false>(&bars->odone[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u,
+                                                      FLAG_MMA_WAIT, c.abort_flag)))
+                        return;
+                    tc_fence_after();
+                }
+                tmem_st16(c.tmem + lane_base + TM_P + 16 * hf, hw);
+                tmem_st16(c.tmem + lane_base + TM_P + 32 + 16 * hf, lw);
+            }
+            l_g += ls;
+            // rescale this row of O_r (tcgen05.ld/st are warp-collective: the whole warp
+            // takes the branch when any row needs it, with factor 1 for the others)
+            if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint32_t addr = c.tmem + lane_base + TM_O + 32 * cc;
                     uint32_t ov[32];
                     tmem_ld32(addr, ov);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * f);
+                    for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
                     tmem_st32(addr, ov);
                 }
-                tmem_wait_st();
             }
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars->oready[k & 1]);
+            mbar_arrive(&bars->pready);
         }
-        // ---- end of the piece: normaliser, lse, output
-        if (!warp_all(mbar_wait_sleep(&bars->odone, (uint32_t)(k - 1) & 1u, FLAG_MMA_WAIT, c.abort_flag))) return;
-        tc_fence_after();
-        float *slot = xch + (pair_uses & 1u) * (HR * 2);
-        slot[h * 2 + half] = l_part;
-        mbar_arrive(&bars->pair[q]);
-        if (!warp_all(mbar_wait_sleep(&bars->pair[q], pair_uses & 1u, FLAG_FULL_WAIT, c.abort_flag))) return;
-        ++pair_uses;
-        const float l = l_part + slot[h * 2 + (half ^ 1)];
-        const float lse_v = l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        k = k0 + nt;
+        // ---- end of the piece: merge the groups' row sums, normalise, write
+        const int klast = k - 1;
+        if (!warp_all(mbar_spin<false>(&bars->hand[klast & 1], (uint32_t)(klast >> 1) & 1u, FLAG_FULL_WAIT, c.abort_flag)))
+            return;
+        const float m_fin = mref[(klast & 1) * HR + h];
+        lx[g * HR + h] = l_g * fast_exp2(m_last - m_fin);
+        mbar_arrive(&bars->lx);
+        if (!warp_all(mbar_spin<false>(&bars->lx, (uint32_t)pi & 1u, FLAG_FULL_WAIT, c.abort_flag))) return;
+        const float l = lx[h] + lx[HR + h];
+        const float lse_v = l > 0.f ? (m_fin + __log2f(l)) * 0.69314718055994531f : -INFINITY;
         const float inv = l > 0.f ? 1.f / l : 0.f;
+        if (!warp_all(mbar_spin<false>(&bars->odone[klast & 1], (uint32_t)(klast >> 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
+            return;
+        tc_fence_after();
         // The TMEM reads are warp-collective (every lane, padded head rows included);
         // only the stores are limited to the real heads.
         const bool real = h < p.H;
@@ -455,11 +447,11 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             dst = p.out + ((size_t)pc.b * p.H + (real ? h : 0)) * 512;
         else
             dst = p.ws_o + (((size_t)c.worker * 2 + pc.slot) * HR + h) * 512;
-        dst += 256 * c.r + 128 * half;
+        dst += 256 * c.r + 128 * g;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
             uint32_t ov[32];
-            tmem_ld32(c.tmem + lane_base + TM_O + 128 * half + 32 * cc, ov);
+            tmem_ld32(c.tmem + lane_base + TM_O + 128 * g + 32 * cc, ov);
             tmem_wait_ld();
             if (real) {
                 float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * cc);
@@ -469,7 +461,7 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
                                         __uint_as_float(ov[4 * j + 2]) * inv, __uint_as_float(ov[4 * j + 3]) * inv);
             }
         }
-        if (real && c.r == 0 && half == 0) {
+        if (real && c.r == 0 && g == 0) {
             if (pc.whole)
                 p.lse[(size_t)pc.b * p.H + h] = lse_v;
             else
@@ -498,22 +490,21 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
         for (int s = 0; s < NST; ++s) {
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1);
-            mbar_init(&bars->qkdone[s], 1);
-            mbar_init(&bars->cvt[s], 64);
         }
-        mbar_init(&bars->qready, 256);
+        mbar_init(&bars->qready, 2 * NGROUP);
+        mbar_init(&bars->qrope_full, 1);
         mbar_init(&bars->qempty, 1);
-        mbar_init(&bars->sready, 1);
-        mbar_init(&bars->sfree, 256);
-        mbar_init(&bars->recv_full, 1);
-        mbar_init(&bars->recv_free, 256);
-        mbar_init(&bars->send_ready, 256);
-        mbar_init(&bars->send_free, 1);
-        mbar_init(&bars->oready[0], 256);
-        mbar_init(&bars->oready[1], 256);
-        mbar_init(&bars->odone, 1);
-        mbar_init(&bars->ofree, 256);
-        for (int i = 0; i < 4; ++i) mbar_init(&bars->pair[i], 64);
+        mbar_init(&bars->sfree, NGROUP);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->sready[i], 1);
+            mbar_init(&bars->recv_full[i], NGROUP);
+            mbar_init(&bars->recv_free[i], NGROUP);
+            mbar_init(&bars->hand[i], NGROUP);
+            mbar_init(&bars->odone[i], 1);
+        }
+        mbar_init(&bars->pready, NGROUP);
+        mbar_init(&bars->ofree, 2 * NGROUP);
+        mbar_init(&bars->lx, 2 * NGROUP);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -525,7 +516,6 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&maps.lat);
         prefetch_tensormap(&maps.rope);
-        prefetch_tensormap(&maps.qlat);
         prefetch_tensormap(&maps.qrope);
     }
     tc_fence_before();
@@ -558,14 +548,11 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
             if (lane == 0) producer(p, maps, c);
         } else if (warp == 1) {
             if (lane == 0) mma_issuer(p, c);
-        } else if (warp < 4) {
-            converter(p, c, tid - 64);
         } else {
             softmax_warps(p, c, warp, lane);
         }
     }
 
-    if (warp == 4 && lane == 0) bulk_wait_read_all();   // the last send has left this CTA
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -117,6 +117,44 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Bounded wait that polls with the non-blocking test_wait (no suspension, so the
+// thread sees the phase complete at once); cluster = acquire at cluster scope, for
+// barriers that receive remote arrivals or transaction bytes.
+template <bool kCluster>
+__device__ __forceinline__ bool mbar_spin(uint64_t *bar, uint32_t parity, unsigned int flag, volatile int *abort) {
+    const uint32_t a = smem_u32(bar);
+    auto test = [&]() -> bool {
+        uint32_t ok;
+        if (kCluster)
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(ok)
+                : "r"(a), "r"(parity)
+                : "memory");
+        else
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                "selp.u32 %0, 1, 0, p;\n\t}"
+                : "=r"(ok)
+                : "r"(a), "r"(parity)
+                : "memory");
+        return ok != 0;
+    };
+    if (test()) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (test()) return true;
+        if (abort != nullptr && *abort) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            atomicOr(&g_device_flags, flag);
+            if (abort != nullptr) *abort = 1;
+            return false;
+        }
+    }
+}
 // Bounded wait (CTA scope) that sleeps between tries.
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, unsigned int flag,
                                                 volatile int *abort) {
