@@ -33,7 +33,7 @@
 //                      with the RoPE query from shared memory); O_r += P C_r: 8 MMAs
 //                      128x256x16 with A = P from TMEM and C_r read MN-major from the same
 //                      swizzled tile.  It issues whichever product is ready.
-//   softmax (warps 2-9) two groups of four warps (one per TMEM lane quadrant) take the
+//   softmax (warps 4-11) two warpgroups (one per TMEM lane quadrant) take the
 //                      tiles in turn, so one group's exchange and exponentials overlap
 //                      the other's.  A thread owns one head row of its group's tiles: it
 //                      reads the row's 64 partial scores, sends them to the peer, adds the
@@ -60,7 +60,9 @@ constexpr int NST = 3;                   // pipeline stages
 constexpr int CHUNK_T = TILE * 128;      // one [64 tokens x 64 cols] bf16 box: 8 KB
 constexpr int STAGE = NCH * CHUNK_T;     // 40 KB
 constexpr int QROPE = HR * 128;          // q_rope block [128 heads x 64] bf16: 16 KB
-constexpr int NTHREADS = 320;            // producer, MMA, two softmax groups of 4 warps
+constexpr int NTHREADS = 384;            // warpgroup 0: producer, MMA (2 idle warps); 1, 2: softmax groups
+constexpr int REGS_WG0 = 96;             // registers per thread after reallocation: warpgroup 0
+constexpr int REGS_SOFTMAX = 200;        //   softmax warpgroups (128 x 96 + 256 x 200 <= 384 x 168)
 constexpr int NGROUP = 128;              // threads per softmax group
 constexpr int MAX_BATCH = 1024;
 constexpr uint32_t TM_O = 0;             // TMEM columns [0, 256): O_r
@@ -270,10 +272,10 @@ __device__ __forceinline__ void mma_issuer(const MlaParams &p, const Ctx &c) {
 // 16-byte chunk slot of chunk j (columns 4j..4j+3) in row h of a receive buffer.
 __device__ __forceinline__ int recv_chunk(int j, int h) { return j ^ (h & 7); }
 
-// ------------------------------------------------------------------ softmax (warps 2-9)
+// ------------------------------------------------------------------ softmax (warps 4-11)
 __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, int warp, int lane) {
     Bars *bars = c.bars;
-    const int g = (warp - 2) >> 2;              // group: takes the tiles k with k % 2 == g
+    const int g = (warp - 4) >> 2;              // group: takes the tiles k with k % 2 == g
     const int q = warp & 3;                     // TMEM lane quadrant
     const int h = 32 * q + lane;                // head row
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
@@ -351,21 +353,38 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             if (!warp_all(mbar_spin<true>(&bars->recv_full[g], (uint32_t)(kt >> 1) & 1u, FLAG_PEER_WAIT,
                                             c.abort_flag)))
                 return;
-            // scores in place (as float bits) from here on
+            // raw scores (own + peer, unscaled) in place from here on; only a tile with
+            // rows outside the sequence needs the mask
             float mx = -INFINITY;
+            const bool full = tok_lo == 0 && tok_hi == TILE;
+            if (full) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float4 v = reinterpret_cast<const float4 *>(recv)[recv_chunk(j, h)];
-                const float pv[4] = {v.x, v.y, v.z, v.w};
+                for (int j = 0; j < 16; ++j) {
+                    const float4 v = reinterpret_cast<const float4 *>(recv)[recv_chunk(j, h)];
+                    const float pv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int col = 4 * j + e;
-                    float x = (__uint_as_float(sv[col]) + pv[e]) * p.scale_log2;
-                    x = (col >= tok_lo && col < tok_hi) ? x : -INFINITY;
-                    sv[col] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
+                    for (int e = 0; e < 4; ++e) {
+                        const float x = __uint_as_float(sv[4 * j + e]) + pv[e];
+                        sv[4 * j + e] = __float_as_uint(x);
+                        mx = fmaxf(mx, x);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float4 v = reinterpret_cast<const float4 *>(recv)[recv_chunk(j, h)];
+                    const float pv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int col = 4 * j + e;
+                        float x = __uint_as_float(sv[col]) + pv[e];
+                        x = (col >= tok_lo && col < tok_hi) ? x : -INFINITY;
+                        sv[col] = __float_as_uint(x);
+                        mx = fmaxf(mx, x);
+                    }
                 }
             }
+            mx *= p.scale_log2;     // the scale is positive: max of the scaled scores
             // the received values are consumed (mx depends on all of them)
             mbar_arrive_cluster_relaxed(peer_recv_free);
             // ---- running max, handed on from the previous tile's group
@@ -391,8 +410,8 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
                 uint32_t hw[16], lw[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float a = fast_exp2(__uint_as_float(sv[32 * hf + 2 * j]) - m_new);
-                    const float b = fast_exp2(__uint_as_float(sv[32 * hf + 2 * j + 1]) - m_new);
+                    const float a = fast_exp2(fmaf(__uint_as_float(sv[32 * hf + 2 * j]), p.scale_log2, -m_new));
+                    const float b = fast_exp2(fmaf(__uint_as_float(sv[32 * hf + 2 * j + 1]), p.scale_log2, -m_new));
                     ls += a + b;
                     split_bf16x2(a, b, hw[j], lw[j]);
                 }
@@ -543,14 +562,15 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
     c.p0 = (long long)c.worker * W;
     c.p1 = (c.p0 + W < total) ? c.p0 + W : total;
 
-    if (c.p0 < total) {
-        if (warp == 0) {
-            if (lane == 0) producer(p, maps, c);
-        } else if (warp == 1) {
-            if (lane == 0) mma_issuer(p, c);
-        } else {
-            softmax_warps(p, c, warp, lane);
+    if (warp < 4) {
+        regs_dec<REGS_WG0>();
+        if (c.p0 < total) {
+            if (warp == 0 && lane == 0) producer(p, maps, c);
+            if (warp == 1 && lane == 0) mma_issuer(p, c);
         }
+    } else {
+        regs_inc<REGS_SOFTMAX>();
+        if (c.p0 < total) softmax_warps(p, c, warp, lane);
     }
 
     tc_fence_before();

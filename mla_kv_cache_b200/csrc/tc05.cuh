@@ -21,6 +21,13 @@ namespace kvattn {
 // instructions (tcgen05.ld/st, ldmatrix, mma.sync) must never split on an abort.
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok) != 0; }
 
+// Register reallocation between warpgroups (every warp of a warpgroup executes the same
+// one).  The counts must keep the block within the registers it was launched with.
+template <int N>
+__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
 // ---------------------------------------------------------------- cluster
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
