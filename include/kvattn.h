@@ -115,6 +115,48 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
                       int latent_dim, int rope_dim, float scale, float *out, float *lse,
                       void *stream);
 
+/*
+ * The step either side of the decode: rotary position embedding (RoPE) of the new
+ * token's query and key, and the append of its key and value to the cache at its
+ * position.  The pages rotate queries and keys before they meet the cache and write the
+ * new token to the cache before attending ("Attention variants: MQA, GQA, and MLA",
+ * section "MLA: cache a latent, not the keys and values"); the rotation itself is the
+ * textbook one: pair i of a head_dim-wide vector at position p turns by the angle
+ * p * rope_base^(-2i / head_dim), the pairs being (2i, 2i+1) when interleaved != 0 and
+ * (i, i + head_dim/2) otherwise.  The angle is formed in fp64; results are rounded to
+ * bf16 once.
+ *   q          device bf16 [batch, n_q_heads, head_dim]: rotated in place
+ *   k_new      device bf16 [batch, n_kv_heads, head_dim]: the new token's keys (not
+ *              rotated); their rotation goes to k_cache[b, j, positions[b], :]
+ *   v_new      device bf16 [batch, n_kv_heads, head_dim]: copied to
+ *              v_cache[b, j, positions[b], :]
+ *   positions  device int32 [batch]: the new token's position (its index in the cache).
+ *              A position outside [0, max_seq_len) writes nothing into the caches (q is
+ *              still rotated with it).  The caller's seq_lens for the following decode
+ *              are positions + 1.
+ *   k_cache, v_cache  device bf16 [batch, n_kv_heads, max_seq_len, head_dim]
+ *   head_dim   even, <= 1024;  rope_base > 0 and finite (e.g. 10000)
+ * Errors as for kvattn_gqa_decode; q and the caches must not overlap each other or the
+ * inputs.  Asynchronous on `stream`.
+ */
+int kvattn_rope_append(uint16_t *q, const uint16_t *k_new, const uint16_t *v_new,
+                       const int32_t *positions, uint16_t *k_cache, uint16_t *v_cache,
+                       int max_seq_len, int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                       float rope_base, int interleaved, void *stream);
+
+/*
+ * The same for absorbed MLA: q_rope [batch, n_heads, rope_dim] is rotated in place, the
+ * new token's decoupled rotary key rope_new [batch, rope_dim] is rotated into
+ * rope_cache[b, positions[b], :], and its latent latent_new [batch, latent_dim] is
+ * copied (unrotated: the latent carries no position) into latent_cache[b, positions[b], :]
+ * ("Attention variants: MQA, GQA, and MLA", section "MLA: cache a latent, not the keys
+ * and values").  latent_dim and rope_dim even; the rest as for kvattn_rope_append.
+ */
+int kvattn_mla_rope_append(uint16_t *q_rope, const uint16_t *latent_new, const uint16_t *rope_new,
+                           const int32_t *positions, uint16_t *latent_cache, uint16_t *rope_cache,
+                           int max_seq_len, int batch, int n_heads, int latent_dim, int rope_dim,
+                           float rope_base, int interleaved, void *stream);
+
 /* Human-readable name of a kvattn_status value (static string, never NULL). */
 const char *kvattn_status_string(int status);
 

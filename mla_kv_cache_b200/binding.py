@@ -37,6 +37,13 @@ _SIGNATURES = {
                                                  ctypes.c_int, ctypes.c_int, ctypes.c_float,
                                                  ctypes.c_void_p, ctypes.c_void_p,
                                                  ctypes.c_void_p]),
+    "kvattn_rope_append": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, _c_u16p, _c_u16p,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
+    "kvattn_mla_rope_append": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, _c_u16p,
+                                              _c_u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                              ctypes.c_void_p]),
     "kvattn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvattn_last_error_detail": (ctypes.c_char_p, []),
     "kvattn_version": (ctypes.c_int, []),
@@ -223,3 +230,46 @@ def kvattn_debug_set_workers(workers, min_tiles=0):
 def kvattn_debug_set_gqa_kernel(which):
     """0: built-in choice, 1: warp-level MMA kernel, 2: tcgen05 kernel."""
     lib().kvattn_debug_set_gqa_kernel(int(which))
+
+
+def kvattn_rope_append(q, k_new, v_new, positions, k_cache, v_cache, rope_base=10000.0,
+                       interleaved=False, stream=None):
+    """Rotary embedding of the new token + cache append (include/kvattn.h,
+    kvattn_rope_append): q [B, n_q, d] is rotated in place; the rotated k_new
+    [B, n_kv, d] and v_new go to the caches [B, n_kv, T, d] at positions [B] (int32)."""
+    import torch
+    B, n_q, d = q.shape
+    n_kv, T = k_cache.shape[1], k_cache.shape[2]
+    _check(q, "q", torch.bfloat16)
+    _check(k_new, "k_new", torch.bfloat16, (B, n_kv, d))
+    _check(v_new, "v_new", torch.bfloat16, (B, n_kv, d))
+    _check(positions, "positions", torch.int32, (B,))
+    _check(k_cache, "k_cache", torch.bfloat16, (B, n_kv, T, d))
+    _check(v_cache, "v_cache", torch.bfloat16, (B, n_kv, T, d))
+    st = lib().kvattn_rope_append(q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), positions.data_ptr(),
+                                  k_cache.data_ptr(), v_cache.data_ptr(), T, B, n_q, n_kv, d,
+                                  float(rope_base), int(bool(interleaved)), _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_rope_append")
+
+
+def kvattn_mla_rope_append(q_rope, latent_new, rope_new, positions, latent_cache, rope_cache,
+                           rope_base=10000.0, interleaved=False, stream=None):
+    """MLA variant (include/kvattn.h, kvattn_mla_rope_append): q_rope [B, H, r] rotated in
+    place; rope_new [B, r] rotated into rope_cache [B, T, r], latent_new [B, c] copied into
+    latent_cache [B, T, c], both at positions [B]."""
+    import torch
+    B, H, r = q_rope.shape
+    T, c = latent_cache.shape[1], latent_cache.shape[2]
+    _check(q_rope, "q_rope", torch.bfloat16)
+    _check(latent_new, "latent_new", torch.bfloat16, (B, c))
+    _check(rope_new, "rope_new", torch.bfloat16, (B, r))
+    _check(positions, "positions", torch.int32, (B,))
+    _check(latent_cache, "latent_cache", torch.bfloat16, (B, T, c))
+    _check(rope_cache, "rope_cache", torch.bfloat16, (B, T, r))
+    st = lib().kvattn_mla_rope_append(q_rope.data_ptr(), latent_new.data_ptr(), rope_new.data_ptr(),
+                                      positions.data_ptr(), latent_cache.data_ptr(), rope_cache.data_ptr(),
+                                      T, B, H, c, r, float(rope_base), int(bool(interleaved)),
+                                      _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_mla_rope_append")

@@ -56,6 +56,8 @@ def load(mutant=0, out_dir=None):
         lib.kvo_gqa_decode.restype = ci
         lib.kvo_mla_decode.argtypes = [dp, dp, dp, dp, ip, ci, ci, ci, ci, ci, cd, dp, dp]
         lib.kvo_mla_decode.restype = ci
+        lib.kvo_rope.argtypes = [dp, ci, ci, ip, cd, ci, dp]
+        lib.kvo_rope.restype = ci
         lib.kvo_num_threads.restype = ci
         lib.kvo_mutant.restype = ci
         _LIBS[key] = lib
@@ -172,3 +174,24 @@ def mla_decode(q_latent, q_rope, latent_cache, rope_cache, seq_lens, scale, batc
         outs.append(o[0])
         lses.append(l[0])
     return np.stack(outs), np.stack(lses)
+
+
+def rope_f64(x, positions, base, interleaved, lib=None):
+    """Rotary embedding of the last axis of x (fp64 result, same shape).  positions
+    holds one position per vector, broadcast over x's leading axes (e.g. [B] for x of
+    shape [B, heads, d]: every head of sequence b at positions[b])."""
+    lib = lib or load()
+    xx = _f64(x)
+    d = xx.shape[-1]
+    lead = xx.shape[:-1]
+    pos = np.ascontiguousarray(np.broadcast_to(
+        np.asarray(positions, dtype=np.int32).reshape(
+            np.asarray(positions).shape + (1,) * (len(lead) - np.asarray(positions).ndim)),
+        lead).reshape(-1))
+    flat = xx.reshape(-1, d)
+    out = np.empty_like(flat)
+    st = lib.kvo_rope(_ptr(flat, ctypes.c_double), flat.shape[0], d, _ptr(pos, ctypes.c_int32),
+                      float(base), int(bool(interleaved)), _ptr(out, ctypes.c_double))
+    if st != 0:
+        raise ValueError("kvo_rope: bad arguments")
+    return out.reshape(xx.shape)

@@ -194,6 +194,49 @@ int kvo_mla_decode(const double *q_lat, const double *q_rope, const double *lat,
     return failed ? -2 : 0;
 }
 
+/*
+ * Rotary position embedding of vectors (the new token's query and key before they
+ * meet the cache).  The pages name RoPE -- applied to queries and keys upstream of the
+ * attention ("Attention variants: MQA, GQA, and MLA", section "MLA: cache a latent, not
+ * the keys and values": the decoupled rotary key cached alongside the latent) -- but do
+ * not write its formula, so this is the textbook rotation of feature pairs: for a
+ * vector x of even length d at position p, pair i (i = 0 .. d/2 - 1) turns by the angle
+ *     theta_i = p * base^(-2i / d)
+ *     x'_a = x_a cos(theta_i) - x_b sin(theta_i)
+ *     x'_b = x_a sin(theta_i) + x_b cos(theta_i)
+ * with (a, b) = (2i, 2i + 1) for interleaved pairs and (i, i + d/2) for split halves.
+ * n vectors of length d in x (row r at position pos[r]); out may alias x.
+ */
+int kvo_rope(const double *x, int n, int d, const int32_t *pos, double base, int interleaved,
+             double *out) {
+    if (d <= 0 || (d & 1) || base <= 0.0) return 1;
+    const int half = d / 2;
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < n; ++r) {
+        const double *xr = x + (size_t)r * d;
+        double *yr = out + (size_t)r * d;
+        for (int i = 0; i < half; ++i) {
+#if KVO_MUTANT == 8
+            const double freq = pow(base, -(double)i / (double)d);   /* planted mistake: exponent i/d */
+#else
+            const double freq = pow(base, -2.0 * (double)i / (double)d);
+#endif
+            const double theta = (double)pos[r] * freq;
+            const int a = interleaved ? 2 * i : i;
+            const int b = interleaved ? 2 * i + 1 : i + half;
+            const double xa = xr[a], xb = xr[b];
+#if KVO_MUTANT == 7
+            yr[a] = xa * cos(theta) + xb * sin(theta);                 /* planted mistake: sign */
+            yr[b] = -xa * sin(theta) + xb * cos(theta);
+#else
+            yr[a] = xa * cos(theta) - xb * sin(theta);
+            yr[b] = xa * sin(theta) + xb * cos(theta);
+#endif
+        }
+    }
+    return 0;
+}
+
 /* Number of OpenMP threads a parallel region of this library uses. */
 int kvo_num_threads(void) {
     int n = 1;

@@ -267,9 +267,65 @@ def pin_mla_without_rope_is_mqa(lib):
     assert np.allclose(o1, o2, atol=1e-14) and np.allclose(l1, l2, atol=1e-13)
 
 
+# --------------------------------------------------------------------------------------
+# Rotary position embedding (the textbook rotation of feature pairs; the pages name RoPE
+# without its formula).  Pinned to mathematics, not to a retyped formula: position 0 is
+# the identity, the angles of tiny cases are worked by hand (d = 2: one pair turning by
+# p radians when base is anything, d = 4: the second pair turns by p / sqrt(base)),
+# rotations keep every pair's length and compose (p then p' equals p + p'), the score
+# of a rotated query and key depends only on the positions' difference, and the two
+# pair layouts differ by a fixed permutation of the features.
+# --------------------------------------------------------------------------------------
+def pin_rope_identity_and_hand_cases(lib):
+    r = _rng(31)
+    x = r.standard_normal((5, 8))
+    for inter in (0, 1):
+        assert np.array_equal(oracle.rope_f64(x, np.zeros(5, np.int32), 10000.0, inter, lib=lib), x)
+    # d = 2: (1, 0) at position p -> (cos p, sin p); (0, 1) -> (-sin p, cos p)
+    for p in (1, 2, 7):
+        y = oracle.rope_f64(np.array([[1.0, 0.0], [0.0, 1.0]]), [p, p], 10000.0, 1, lib=lib)
+        assert np.allclose(y, [[math.cos(p), math.sin(p)], [-math.sin(p), math.cos(p)]], atol=1e-15), p
+    # d = 4, base 100: pair 0 turns by p, pair 1 by p / 10
+    p = 3
+    y = oracle.rope_f64(np.array([[0.0, 0.0, 1.0, 0.0]]), [p], 100.0, 1, lib=lib)
+    assert np.allclose(y, [[0.0, 0.0, math.cos(0.3), math.sin(0.3)]], atol=1e-15)
+    y = oracle.rope_f64(np.array([[0.0, 1.0, 0.0, 0.0]]), [p], 100.0, 0, lib=lib)   # halves: pair 1 = (1, 3)
+    assert np.allclose(y, [[0.0, math.cos(0.3), 0.0, math.sin(0.3)]], atol=1e-15)
+
+
+def pin_rope_invariants(lib):
+    r = _rng(32)
+    d = 16
+    x = r.standard_normal((6, d))
+    pos = np.array([0, 1, 5, 100, 4095, 32767], np.int32)
+    for inter in (0, 1):
+        y = oracle.rope_f64(x, pos, 10000.0, inter, lib=lib)
+        pairs = (lambda z: np.stack([z[:, 0::2], z[:, 1::2]], -1)) if inter else \
+                (lambda z: np.stack([z[:, : d // 2], z[:, d // 2:]], -1))
+        assert np.allclose(np.linalg.norm(pairs(y), axis=-1), np.linalg.norm(pairs(x), axis=-1), atol=1e-12)
+        # composition
+        a, b = np.array([3] * 6, np.int32), np.array([11] * 6, np.int32)
+        twice = oracle.rope_f64(oracle.rope_f64(x, a, 10000.0, inter, lib=lib), b, 10000.0, inter, lib=lib)
+        assert np.allclose(twice, oracle.rope_f64(x, a + b, 10000.0, inter, lib=lib), atol=1e-12)
+        # relative position: <R_m q, R_n k> == <R_{m-n} q, k>
+        q, k = r.standard_normal(d), r.standard_normal(d)
+        for m, n in [(7, 2), (300, 299), (1000, 10)]:
+            lhs = oracle.rope_f64(q[None], [m], 10000.0, inter, lib=lib)[0] @ \
+                oracle.rope_f64(k[None], [n], 10000.0, inter, lib=lib)[0]
+            rhs = oracle.rope_f64(q[None], [m - n], 10000.0, inter, lib=lib)[0] @ k
+            assert abs(lhs - rhs) < 1e-9 * (1 + abs(rhs)), (m, n)
+    # layouts: interleaved == halves under the permutation that interleaves the halves
+    perm = np.empty(d, dtype=np.int64)
+    perm[0::2] = np.arange(d // 2)
+    perm[1::2] = np.arange(d // 2) + d // 2
+    yi = oracle.rope_f64(x[:, perm], pos, 10000.0, 1, lib=lib)
+    yh = oracle.rope_f64(x, pos, 10000.0, 0, lib=lib)
+    assert np.allclose(yi, yh[:, perm], atol=1e-12)
+
+
 ALL_PINS = [
     pin_gqa_equals_mha_on_repeated_kv, pin_sdpa_enable_gqa, pin_closed_forms,
     pin_empty_sequence, pin_brute_force_tiny, pin_split_merge, pin_permutation_invariance,
     pin_scale_equivariance, pin_mla_absorbed_equals_explicit, pin_mla_matches_sdpa,
-    pin_mla_without_rope_is_mqa,
+    pin_mla_without_rope_is_mqa, pin_rope_identity_and_hand_cases, pin_rope_invariants,
 ]

@@ -124,6 +124,49 @@ def test_mla_rejects_bad_arguments(lib, kw, expected):
     assert call_mla(lib, mla_args(**kw)) == expected
 
 
+def rope_args(**kw):
+    args = dict(q=A, kn=2 * A, vn=3 * A, pos=4 * A, kc=5 * A, vc=7 * A, T=1024, B=2, nq=8, nkv=2, d=128,
+                base=10000.0, inter=0, stream=None)
+    args.update(kw)
+    return args
+
+
+def call_rope(lib, a):
+    return lib.kvattn_rope_append(a["q"], a["kn"], a["vn"], a["pos"], a["kc"], a["vc"], a["T"], a["B"],
+                                  a["nq"], a["nkv"], a["d"], a["base"], a["inter"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(q=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(pos=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(vc=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(B=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(nq=8, nkv=3), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(base=0.0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(base=float("nan")), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(d=127), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(d=2048), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(kc=5 * A + 4), kb.KVATTN_ERR_MISALIGNED),
+    (dict(q=5 * A), kb.KVATTN_ERR_INVALID_ARG),            # q overlaps the K cache
+    (dict(kn=7 * A + 64), kb.KVATTN_ERR_INVALID_ARG),      # the new key lies inside the V cache
+])
+def test_rope_append_rejects_bad_arguments(lib, kw, expected):
+    assert call_rope(lib, rope_args(**kw)) == expected
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(dr=63), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(lat=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(rope=4 * A + 2), kb.KVATTN_ERR_MISALIGNED),
+])
+def test_mla_rope_append_rejects_bad_arguments(lib, kw, expected):
+    a = dict(qr=A, ln=2 * A, rn=3 * A, pos=4 * A, lat=5 * A, rope=7 * A, T=1024, B=2, H=128, dc=512, dr=64)
+    a.update(kw)
+    st = lib.kvattn_mla_rope_append(a["qr"], a["ln"], a["rn"], a["pos"], a["lat"], a["rope"], a["T"], a["B"],
+                                    a["H"], a["dc"], a["dr"], 10000.0, 0, None)
+    assert st == expected
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     q = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
