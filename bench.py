@@ -212,13 +212,53 @@ def dist_barrier():
 
 
 # ----------------------------------------------------------------------------- GPU arm
+PAGED = 0   # --paged: rows per page of a paged cache layout (0: contiguous cache)
+
+
+def to_pages(cache, page_size, seq_axis, perm):
+    """A contiguous cache [B, ..., T, ...] (T at seq_axis) laid out as a shuffled pool of
+    pages: page b * M + lp of the natural order goes to slot perm[b * M + lp]."""
+    B, T = cache.shape[0], cache.shape[seq_axis]
+    M = T // page_size
+    if seq_axis == 2:    # [B, n_kv, T, d] -> [B * M, n_kv, S, d]
+        pages = cache.view(B, cache.shape[1], M, page_size, cache.shape[3]).permute(0, 2, 1, 3, 4)
+        pages = pages.reshape(B * M, cache.shape[1], page_size, cache.shape[3])
+    else:                # [B, T, c] -> [B * M, S, c]
+        pages = cache.view(B * M, page_size, cache.shape[2])
+    pool = torch.empty_like(pages)
+    pool[perm] = pages
+    return pool
+
+
 def device_inputs(cfg, seed):
     x = wl.make_inputs(cfg, seed=seed)
-    return x, {k: v.cuda() for k, v in x.items()}
+    d = {k: v.cuda() for k, v in x.items()}
+    if PAGED:
+        T = cfg.max_seq_len
+        if T % PAGED:
+            raise ValueError(f"--paged {PAGED} does not divide the cache capacity {T}")
+        M = T // PAGED
+        g = torch.Generator().manual_seed(seed + 17)
+        perm = torch.randperm(cfg.batch * M, generator=g).cuda()
+        d["block_table"] = perm.view(cfg.batch, M).to(torch.int32).contiguous()
+        names = ("latent_cache", "rope_cache") if isinstance(cfg, wl.MLAConfig) else ("k_cache", "v_cache")
+        axis = 1 if isinstance(cfg, wl.MLAConfig) else 2
+        for n in names:
+            d[n + "_pages"] = to_pages(d.pop(n), PAGED, axis, perm)
+        torch.cuda.empty_cache()
+    return x, d
 
 
 def make_call(cfg, d, out, lse, stream):
     from mla_kv_cache_b200 import binding as kb
+    if PAGED:
+        if isinstance(cfg, wl.MLAConfig):
+            return lambda: kb.kvattn_mla_decode_paged(d["q_latent"], d["q_rope"], d["latent_cache_pages"],
+                                                      d["rope_cache_pages"], d["block_table"], d["seq_lens"],
+                                                      cfg.scale, out=out, lse=lse, stream=stream)
+        return lambda: kb.kvattn_gqa_decode_paged(d["q"], d["k_cache_pages"], d["v_cache_pages"],
+                                                  d["block_table"], d["seq_lens"], cfg.scale, out=out,
+                                                  lse=lse, stream=stream)
     if isinstance(cfg, wl.MLAConfig):
         return lambda: kb.kvattn_mla_decode(d["q_latent"], d["q_rope"], d["latent_cache"],
                                             d["rope_cache"], d["seq_lens"], cfg.scale, out=out,
@@ -404,6 +444,8 @@ def gpu_arm(args):
         "data": "synthetic (seeded N(0,1) bf16, shapes of the workload)",
         "config": {"workload": args.config, **workload_fields(head_cfg),
                    "bytes_per_step": nb["total"],
+                   "cache_layout": f"paged: {PAGED}-row pages in a shuffled pool, block table" if PAGED
+                   else "contiguous [B, n_kv, T, d]",
                    "l2": "flushed before every timed step (256 MiB device write + read-back, outside the timed interval)",
                    "parallelism": f"replicas x{world}: one independent batch per GPU, no collective"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -486,7 +528,12 @@ def main():
     ap.add_argument("--no-extra-configs", action="store_true")
     ap.add_argument("--cpu-sample-s", type=float, default=10.0)
     ap.add_argument("--ref-sequences", type=int, default=2)
+    ap.add_argument("--paged", type=int, default=0, metavar="PAGE_SIZE",
+                    help="time the paged-cache entry points, the cache cut into pages of this "
+                         "many rows (a multiple of 64) and shuffled over a pool")
     args = ap.parse_args()
+    global PAGED
+    PAGED = args.paged
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -116,6 +116,41 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
                       void *stream);
 
 /*
+ * kvattn_gqa_decode over a paged KV cache: the cache is a pool of pages and each
+ * sequence lists its pages in a block table (the serving-engine layout the pages name,
+ * "Attention variants: MQA, GQA, and MLA", section "Against the real libraries": vLLM's
+ * PagedAttention).  Token t of sequence b lives in page block_table[b][t / page_size],
+ * row t % page_size.
+ *   k_pages, v_pages  device bf16 [num_pages, n_kv_heads, page_size, head_dim]
+ *   block_table       device int32 [batch, max_pages_per_seq]: physical page of each
+ *                     logical page; entries past a sequence's last page are not read.
+ *                     Every entry that is read must lie in [0, num_pages).
+ *   seq_lens          device int32 [batch], 0 <= len <= max_pages_per_seq * page_size
+ *   page_size         a multiple of 64 (the tensor-core kernel for groups of >= 4 heads
+ *                     runs when it is a multiple of 128; otherwise the warp-level kernel)
+ * Everything else, the results and the errors are those of kvattn_gqa_decode.  Rows
+ * of a sequence's last page past its length are never read.
+ */
+int kvattn_gqa_decode_paged(const uint16_t *q, const uint16_t *k_pages, const uint16_t *v_pages,
+                            const int32_t *block_table, const int32_t *seq_lens, int num_pages,
+                            int page_size, int max_pages_per_seq, int batch, int n_q_heads,
+                            int n_kv_heads, int head_dim, float scale, float *out, float *lse,
+                            void *stream);
+
+/*
+ * kvattn_mla_decode over a paged latent cache: latent_pages [num_pages, page_size,
+ * latent_dim] and rope_pages [num_pages, page_size, rope_dim] bf16, block_table and
+ * seq_lens as for kvattn_gqa_decode_paged; page_size a multiple of 64.  Everything else
+ * as for kvattn_mla_decode.
+ */
+int kvattn_mla_decode_paged(const uint16_t *q_latent, const uint16_t *q_rope,
+                            const uint16_t *latent_pages, const uint16_t *rope_pages,
+                            const int32_t *block_table, const int32_t *seq_lens, int num_pages,
+                            int page_size, int max_pages_per_seq, int batch, int n_heads,
+                            int latent_dim, int rope_dim, float scale, float *out, float *lse,
+                            void *stream);
+
+/*
  * The step either side of the decode: rotary position embedding (RoPE) of the new
  * token's query and key, and the append of its key and value to the cache at its
  * position.  The pages rotate queries and keys before they meet the cache and write the

@@ -37,6 +37,15 @@ _SIGNATURES = {
                                                  ctypes.c_int, ctypes.c_int, ctypes.c_float,
                                                  ctypes.c_void_p, ctypes.c_void_p,
                                                  ctypes.c_void_p]),
+    "kvattn_gqa_decode_paged": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "kvattn_mla_decode_paged": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p]),
     "kvattn_rope_append": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, _c_u16p, _c_u16p,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
@@ -273,3 +282,62 @@ def kvattn_mla_rope_append(q_rope, latent_new, rope_new, positions, latent_cache
                                       _stream_handle(stream))
     if st != KVATTN_OK:
         raise KvattnError(st, "kvattn_mla_rope_append")
+
+
+def kvattn_gqa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale, out=None, lse=None,
+                            stream=None):
+    """GQA decode over a paged cache (include/kvattn.h, kvattn_gqa_decode_paged):
+    k_pages / v_pages [num_pages, n_kv, page_size, d] bf16, block_table [B, max_pages]
+    int32, seq_lens [B] int32.  Returns (out [B, n_q, d] fp32, lse [B, n_q] fp32)."""
+    import torch
+    B, n_q, d = q.shape
+    P, n_kv, S = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    M = block_table.shape[1]
+    _check(q, "q", torch.bfloat16)
+    _check(k_pages, "k_pages", torch.bfloat16, (P, n_kv, S, d))
+    _check(v_pages, "v_pages", torch.bfloat16, (P, n_kv, S, d))
+    _check(block_table, "block_table", torch.int32, (B, M))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, n_q, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, n_q), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, (B, n_q, d))
+    _check(lse, "lse", torch.float32, (B, n_q))
+    st = lib().kvattn_gqa_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                       block_table.data_ptr(), seq_lens.data_ptr(), P, S, M, B, n_q, n_kv,
+                                       d, float(scale), out.data_ptr(), lse.data_ptr(),
+                                       _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_gqa_decode_paged")
+    return out, lse
+
+
+def kvattn_mla_decode_paged(q_latent, q_rope, latent_pages, rope_pages, block_table, seq_lens, scale,
+                            out=None, lse=None, stream=None):
+    """MLA decode over a paged cache (include/kvattn.h, kvattn_mla_decode_paged):
+    latent_pages [P, page_size, 512], rope_pages [P, page_size, 64] bf16."""
+    import torch
+    B, H, dc = q_latent.shape
+    dr = q_rope.shape[2]
+    P, S = latent_pages.shape[0], latent_pages.shape[1]
+    M = block_table.shape[1]
+    _check(q_latent, "q_latent", torch.bfloat16)
+    _check(q_rope, "q_rope", torch.bfloat16, (B, H, dr))
+    _check(latent_pages, "latent_pages", torch.bfloat16, (P, S, dc))
+    _check(rope_pages, "rope_pages", torch.bfloat16, (P, S, dr))
+    _check(block_table, "block_table", torch.int32, (B, M))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, H, dc), dtype=torch.float32, device=q_latent.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q_latent.device)
+    _check(out, "out", torch.float32, (B, H, dc))
+    _check(lse, "lse", torch.float32, (B, H))
+    st = lib().kvattn_mla_decode_paged(q_latent.data_ptr(), q_rope.data_ptr(), latent_pages.data_ptr(),
+                                       rope_pages.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(), P,
+                                       S, M, B, H, dc, dr, float(scale), out.data_ptr(), lse.data_ptr(),
+                                       _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_mla_decode_paged")
+    return out, lse

@@ -40,6 +40,9 @@ struct GqaParams {
     int workers;                // gridDim.x
     int min_tiles;
     float scale_log2;           // scale * log2(e)
+    const int32_t *block_table; // [B, max_pages] physical pages (paged cache); null: contiguous
+    int max_pages;              // block-table columns
+    int page_size;              // rows per page (T_max when contiguous)
 };
 
 template <int D, int MT>
@@ -135,13 +138,14 @@ gqa_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap,
             const Piece pc = piece_at(s_prefix, p.B, U, pos, p1, p0);
             const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
             const int j = pc.i / p.n_hb;
-            const int z = pc.b * p.n_kv + j;
             for (int lt = pc.lt0; lt < pc.lt1; ++lt, ++k) {
                 const int stage = k % C::NST;
                 const uint32_t ph = (uint32_t)(k / C::NST) & 1u;
                 if (!mbar_wait(&empty[stage], ph ^ 1u, FLAG_EMPTY_WAIT, abort_flag)) { ok = false; break; }
                 mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-                const int y = min(lt * C::TILE, len - C::TILE);
+                const TileSrc src = tile_source(p.block_table, p.max_pages, p.page_size, pc.b, lt, C::TILE, len);
+                const int y = src.y;
+                const int z = src.page * p.n_kv + j;
                 uint8_t *kt = smem + stage * C::STAGE_BYTES;
                 uint8_t *vt = kt + C::KV_TILE_BYTES;
 #pragma unroll

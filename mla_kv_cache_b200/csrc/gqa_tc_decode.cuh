@@ -186,7 +186,6 @@ __device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *
         pos = pc.ustart + pc.lt1;
         const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
         const int j = pc.i / p.n_hb, hb = pc.i % p.n_hb;
-        const int z = pc.b * p.n_kv + j;
         const int qb = pi % C::NQB, qu = pi / C::NQB;
         if (qu > 0 && !mbar_wait(&bars->qempty[qb], (uint32_t)(qu - 1) & 1u, FLAG_EMPTY_WAIT, c.abort_flag)) {
             ok = false;
@@ -202,7 +201,9 @@ __device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *
             const uint32_t ph = (uint32_t)(k / NST) & 1u;
             if (!mbar_wait(&bars->empty[s], ph ^ 1u, FLAG_EMPTY_WAIT, c.abort_flag)) { ok = false; break; }
             mbar_arrive_expect_tx(&bars->full[s], STAGE);
-            const int y = min(lt * TILE, len - TILE);
+            const TileSrc src = tile_source(p.block_table, p.max_pages, p.page_size, pc.b, lt, TILE, len);
+            const int y = src.y;
+            const int z = src.page * p.n_kv + j;
             uint8_t *st = c.smem + OFF_ST + s * STAGE;
             tma_load_3d(st, kmap, &bars->full[s], 0, y, z, pol);
             tma_load_3d(st + CHUNK, kmap, &bars->full[s], 64, y, z, pol);

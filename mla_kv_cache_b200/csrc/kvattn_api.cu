@@ -371,57 +371,44 @@ bool use_tc_kernel(int head_dim, int g, int batch, const DeviceState *dev) {
     return possible && g >= 4;
 }
 
-}  // namespace
+// A K/V cache as the decode kernels see it: pages of page_size rows per (page, KV head);
+// a contiguous cache is one page per sequence (page_size = capacity, no block table).
+struct GqaCache {
+    const uint16_t *k, *v;
+    const int32_t *block_table;   // [batch, max_pages] or null (contiguous)
+    int capacity;                 // rows addressable per sequence (seq_lens are clamped to it)
+    int page_size;
+    int max_pages;
+    long long pages;              // pages in the pool (contiguous: batch)
+};
 
-extern "C" {
-
-int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
-                      const int32_t *seq_lens, int max_seq_len, int batch, int n_q_heads,
-                      int n_kv_heads, int head_dim, float scale, float *out, float *lse,
-                      void *stream) {
-    if (!q || !k_cache || !v_cache || !seq_lens || !out || !lse) return KVATTN_ERR_INVALID_ARG;
-    if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || max_seq_len <= 0)
-        return KVATTN_ERR_INVALID_ARG;
-    if (n_q_heads % n_kv_heads != 0) return KVATTN_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
-    if (head_dim != 64 && head_dim != 128) return KVATTN_ERR_UNSUPPORTED;
-    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
-    if ((long long)batch * n_kv_heads * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seq_lens) ||
-        !aligned16(out) || !aligned16(lse))
-        return KVATTN_ERR_MISALIGNED;
-    const size_t q_bytes = (size_t)batch * n_q_heads * head_dim * 2;
-    const size_t kv_bytes = (size_t)batch * n_kv_heads * max_seq_len * head_dim * 2;
-    const size_t out_bytes = (size_t)batch * n_q_heads * head_dim * 4;
-    const size_t lse_bytes = (size_t)batch * n_q_heads * 4;
-    const void *ins[4] = {q, k_cache, v_cache, seq_lens};
-    const size_t in_sz[4] = {q_bytes, kv_bytes, kv_bytes, (size_t)batch * 4};
-    for (int i = 0; i < 4; ++i)
-        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
-            return KVATTN_ERR_INVALID_ARG;
-    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
-
+int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq_lens, int batch,
+                    int n_q_heads, int n_kv_heads, int head_dim, float scale, float *out, float *lse,
+                    void *stream) {
     DeviceState *dev = nullptr;
     int st = device_state(&dev);
     if (st != KVATTN_OK) return st;
 
     const int g = n_q_heads / n_kv_heads;
-    if (g_gqa_kernel == 2 && !use_tc_kernel(head_dim, g, batch, dev)) {
-        snprintf(t_detail, sizeof(t_detail), "tcgen05 GQA kernel needs head_dim 128 and batch <= %d",
+    // a paged cache needs pages made of whole 128-token tiles for the tcgen05 kernel
+    const bool tiles_fit = cache.block_table == nullptr || cache.page_size % gqatc::TILE == 0;
+    if (g_gqa_kernel == 2 && !(tiles_fit && use_tc_kernel(head_dim, g, batch, dev))) {
+        snprintf(t_detail, sizeof(t_detail),
+                 "tcgen05 GQA kernel needs head_dim 128, batch <= %d and pages of multiples of 128 rows",
                  (dev->max_smem_optin - gqatc::smem_bytes(0)) / 4);
         return KVATTN_ERR_UNSUPPORTED;
     }
-    const bool tc = use_tc_kernel(head_dim, g, batch, dev);
+    const bool tc = tiles_fit && use_tc_kernel(head_dim, g, batch, dev);
     const int MT = g <= 16 ? 1 : 2;
     const int heads = tc ? gqatc::HB : 16 * MT;
     const int n_hb = (g + heads - 1) / heads;
     const uint32_t box_rows = tc ? gqatc::TILE : 64;
 
     CUtensorMap kmap, vmap, qmap;
-    st = make_map_3d(&kmap, k_cache, head_dim, max_seq_len, (uint64_t)batch * n_kv_heads, 64, box_rows,
+    st = make_map_3d(&kmap, cache.k, head_dim, cache.page_size, (uint64_t)cache.pages * n_kv_heads, 64, box_rows,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
-    st = make_map_3d(&vmap, v_cache, head_dim, max_seq_len, (uint64_t)batch * n_kv_heads, 64, box_rows,
+    st = make_map_3d(&vmap, cache.v, head_dim, cache.page_size, (uint64_t)cache.pages * n_kv_heads, 64, box_rows,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
     if (tc) {
@@ -439,10 +426,13 @@ int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
     p.B = batch;
     p.n_q = n_q_heads;
     p.n_kv = n_kv_heads;
-    p.T_max = max_seq_len;
+    p.T_max = cache.capacity;
     p.g = g;
     p.n_hb = n_hb;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.block_table = cache.block_table;
+    p.max_pages = cache.max_pages;
+    p.page_size = cache.page_size;
     const int U = n_kv_heads * n_hb;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (tc) {
@@ -456,44 +446,29 @@ int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
     return MT == 1 ? run_gqa<64, 1>(p, kmap, vmap, dev, U, s) : run_gqa<64, 2>(p, kmap, vmap, dev, U, s);
 }
 
-int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
-                      const uint16_t *latent_cache, const uint16_t *rope_cache,
-                      const int32_t *seq_lens, int max_seq_len, int batch, int n_heads,
-                      int latent_dim, int rope_dim, float scale, float *out, float *lse,
-                      void *stream) {
-    if (!q_latent || !q_rope || !latent_cache || !rope_cache || !seq_lens || !out || !lse)
-        return KVATTN_ERR_INVALID_ARG;
-    if (batch <= 0 || n_heads <= 0 || max_seq_len <= 0 || latent_dim <= 0 || rope_dim < 0)
-        return KVATTN_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
-    if (latent_dim != 512 || rope_dim != 64 || n_heads > 128) return KVATTN_ERR_UNSUPPORTED;
-    if (batch > mla::MAX_BATCH) return KVATTN_ERR_UNSUPPORTED;
-    if ((long long)batch * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
-    if (!aligned16(q_latent) || !aligned16(q_rope) || !aligned16(latent_cache) ||
-        !aligned16(rope_cache) || !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
-        return KVATTN_ERR_MISALIGNED;
-    const size_t ql_bytes = (size_t)batch * n_heads * latent_dim * 2;
-    const size_t qr_bytes = (size_t)batch * n_heads * rope_dim * 2;
-    const size_t lat_bytes = (size_t)batch * max_seq_len * latent_dim * 2;
-    const size_t rope_bytes = (size_t)batch * max_seq_len * rope_dim * 2;
-    const size_t out_bytes = (size_t)batch * n_heads * latent_dim * 4;
-    const size_t lse_bytes = (size_t)batch * n_heads * 4;
-    const void *ins[5] = {q_latent, q_rope, latent_cache, rope_cache, seq_lens};
-    const size_t in_sz[5] = {ql_bytes, qr_bytes, lat_bytes, rope_bytes, (size_t)batch * 4};
-    for (int i = 0; i < 5; ++i)
-        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
-            return KVATTN_ERR_INVALID_ARG;
-    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+// A latent + rotary-key cache as the MLA kernel sees it (pages of page_size rows; a
+// contiguous cache is one page per sequence).
+struct MlaCache {
+    const uint16_t *lat, *rope;
+    const int32_t *block_table;   // [batch, max_pages] or null (contiguous)
+    int capacity;
+    int page_size;
+    int max_pages;
+    long long pages;
+};
 
+int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaCache &cache,
+                    const int32_t *seq_lens, int batch, int n_heads, float scale, float *out, float *lse,
+                    void *stream) {
     DeviceState *dev = nullptr;
     int st = device_state(&dev);
     if (st != KVATTN_OK) return st;
 
     MlaMaps maps;
-    st = make_map_3d(&maps.lat, latent_cache, 512, max_seq_len, batch, 64, mla::TILE,
+    st = make_map_3d(&maps.lat, cache.lat, 512, cache.page_size, (uint64_t)cache.pages, 64, mla::TILE,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
-    st = make_map_3d(&maps.rope, rope_cache, 64, max_seq_len, batch, 64, mla::TILE,
+    st = make_map_3d(&maps.rope, cache.rope, 64, cache.page_size, (uint64_t)cache.pages, 64, mla::TILE,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
     st = make_map_3d(&maps.qlat, q_latent, 512, n_heads, batch, 64, mla::HR, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -509,7 +484,10 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
     p.lse = lse;
     p.B = batch;
     p.H = n_heads;
-    p.T_max = max_seq_len;
+    p.T_max = cache.capacity;
+    p.block_table = cache.block_table;
+    p.max_pages = cache.max_pages;
+    p.page_size = cache.page_size;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     const int smem = mla::smem_bytes(batch);
     if (smem > dev->max_smem_optin) {
@@ -541,7 +519,7 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
         }
         dev->mla_clusters = n < dev->sms / 2 ? n : dev->sms / 2;
     }
-    const long long max_tiles = (long long)batch * ((max_seq_len + mla::TILE - 1) / mla::TILE);
+    const long long max_tiles = (long long)batch * ((cache.capacity + mla::TILE - 1) / mla::TILE);
     p.min_tiles = g_force_min_tiles > 0 ? g_force_min_tiles : 4;
     long long workers = g_force_workers > 0 ? g_force_workers : dev->mla_clusters;
     const long long by_size = (max_tiles + p.min_tiles - 1) / p.min_tiles;
@@ -584,7 +562,145 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
     cp.workers = p.workers;
     cp.min_tiles = p.min_tiles;
     return launch_combine(512, cp, batch, n_heads, s,
-                          combine_warps((max_seq_len + mla::TILE - 1) / mla::TILE, max_tiles, p.workers));
+                          combine_warps((cache.capacity + mla::TILE - 1) / mla::TILE, max_tiles, p.workers));
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                      const int32_t *seq_lens, int max_seq_len, int batch, int n_q_heads,
+                      int n_kv_heads, int head_dim, float scale, float *out, float *lse,
+                      void *stream) {
+    if (!q || !k_cache || !v_cache || !seq_lens || !out || !lse) return KVATTN_ERR_INVALID_ARG;
+    if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || max_seq_len <= 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if (n_q_heads % n_kv_heads != 0) return KVATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return KVATTN_ERR_UNSUPPORTED;
+    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
+    if ((long long)batch * n_kv_heads * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seq_lens) ||
+        !aligned16(out) || !aligned16(lse))
+        return KVATTN_ERR_MISALIGNED;
+    const size_t q_bytes = (size_t)batch * n_q_heads * head_dim * 2;
+    const size_t kv_bytes = (size_t)batch * n_kv_heads * max_seq_len * head_dim * 2;
+    const size_t out_bytes = (size_t)batch * n_q_heads * head_dim * 4;
+    const size_t lse_bytes = (size_t)batch * n_q_heads * 4;
+    const void *ins[4] = {q, k_cache, v_cache, seq_lens};
+    const size_t in_sz[4] = {q_bytes, kv_bytes, kv_bytes, (size_t)batch * 4};
+    for (int i = 0; i < 4; ++i)
+        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
+            return KVATTN_ERR_INVALID_ARG;
+    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+    const GqaCache cache{k_cache, v_cache, nullptr, max_seq_len, max_seq_len, 1, batch};
+    return gqa_decode_impl(q, cache, seq_lens, batch, n_q_heads, n_kv_heads, head_dim, scale, out, lse, stream);
+}
+
+int kvattn_gqa_decode_paged(const uint16_t *q, const uint16_t *k_pages, const uint16_t *v_pages,
+                            const int32_t *block_table, const int32_t *seq_lens, int num_pages,
+                            int page_size, int max_pages_per_seq, int batch, int n_q_heads,
+                            int n_kv_heads, int head_dim, float scale, float *out, float *lse,
+                            void *stream) {
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out || !lse) return KVATTN_ERR_INVALID_ARG;
+    if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || num_pages <= 0 || page_size <= 0 ||
+        max_pages_per_seq <= 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if (n_q_heads % n_kv_heads != 0) return KVATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return KVATTN_ERR_UNSUPPORTED;
+    if (page_size % 64 != 0) return KVATTN_ERR_UNSUPPORTED;
+    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
+    if ((long long)num_pages * n_kv_heads * page_size >= (1ll << 31) ||
+        (long long)max_pages_per_seq * page_size >= (1ll << 31))
+        return KVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(block_table) ||
+        !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
+        return KVATTN_ERR_MISALIGNED;
+    const size_t q_bytes = (size_t)batch * n_q_heads * head_dim * 2;
+    const size_t kv_bytes = (size_t)num_pages * n_kv_heads * page_size * head_dim * 2;
+    const size_t out_bytes = (size_t)batch * n_q_heads * head_dim * 4;
+    const size_t lse_bytes = (size_t)batch * n_q_heads * 4;
+    const void *ins[5] = {q, k_pages, v_pages, seq_lens, block_table};
+    const size_t in_sz[5] = {q_bytes, kv_bytes, kv_bytes, (size_t)batch * 4,
+                             (size_t)batch * max_pages_per_seq * 4};
+    for (int i = 0; i < 5; ++i)
+        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
+            return KVATTN_ERR_INVALID_ARG;
+    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+    const GqaCache cache{k_pages, v_pages, block_table, max_pages_per_seq * page_size, page_size,
+                         max_pages_per_seq, num_pages};
+    return gqa_decode_impl(q, cache, seq_lens, batch, n_q_heads, n_kv_heads, head_dim, scale, out, lse, stream);
+}
+
+int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
+                      const uint16_t *latent_cache, const uint16_t *rope_cache,
+                      const int32_t *seq_lens, int max_seq_len, int batch, int n_heads,
+                      int latent_dim, int rope_dim, float scale, float *out, float *lse,
+                      void *stream) {
+    if (!q_latent || !q_rope || !latent_cache || !rope_cache || !seq_lens || !out || !lse)
+        return KVATTN_ERR_INVALID_ARG;
+    if (batch <= 0 || n_heads <= 0 || max_seq_len <= 0 || latent_dim <= 0 || rope_dim < 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
+    if (latent_dim != 512 || rope_dim != 64 || n_heads > 128) return KVATTN_ERR_UNSUPPORTED;
+    if (batch > mla::MAX_BATCH) return KVATTN_ERR_UNSUPPORTED;
+    if ((long long)batch * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q_latent) || !aligned16(q_rope) || !aligned16(latent_cache) ||
+        !aligned16(rope_cache) || !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
+        return KVATTN_ERR_MISALIGNED;
+    const size_t ql_bytes = (size_t)batch * n_heads * latent_dim * 2;
+    const size_t qr_bytes = (size_t)batch * n_heads * rope_dim * 2;
+    const size_t lat_bytes = (size_t)batch * max_seq_len * latent_dim * 2;
+    const size_t rope_bytes = (size_t)batch * max_seq_len * rope_dim * 2;
+    const size_t out_bytes = (size_t)batch * n_heads * latent_dim * 4;
+    const size_t lse_bytes = (size_t)batch * n_heads * 4;
+    const void *ins[5] = {q_latent, q_rope, latent_cache, rope_cache, seq_lens};
+    const size_t in_sz[5] = {ql_bytes, qr_bytes, lat_bytes, rope_bytes, (size_t)batch * 4};
+    for (int i = 0; i < 5; ++i)
+        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
+            return KVATTN_ERR_INVALID_ARG;
+    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+
+    const MlaCache cache{latent_cache, rope_cache, nullptr, max_seq_len, max_seq_len, 1, batch};
+    return mla_decode_impl(q_latent, q_rope, cache, seq_lens, batch, n_heads, scale, out, lse, stream);
+}
+
+int kvattn_mla_decode_paged(const uint16_t *q_latent, const uint16_t *q_rope, const uint16_t *latent_pages,
+                            const uint16_t *rope_pages, const int32_t *block_table, const int32_t *seq_lens,
+                            int num_pages, int page_size, int max_pages_per_seq, int batch, int n_heads,
+                            int latent_dim, int rope_dim, float scale, float *out, float *lse, void *stream) {
+    if (!q_latent || !q_rope || !latent_pages || !rope_pages || !block_table || !seq_lens || !out || !lse)
+        return KVATTN_ERR_INVALID_ARG;
+    if (batch <= 0 || n_heads <= 0 || num_pages <= 0 || page_size <= 0 || max_pages_per_seq <= 0 ||
+        latent_dim <= 0 || rope_dim < 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
+    if (latent_dim != 512 || rope_dim != 64 || n_heads > 128) return KVATTN_ERR_UNSUPPORTED;
+    if (page_size % mla::TILE != 0) return KVATTN_ERR_UNSUPPORTED;
+    if (batch > mla::MAX_BATCH) return KVATTN_ERR_UNSUPPORTED;
+    if ((long long)num_pages * page_size >= (1ll << 31) || (long long)max_pages_per_seq * page_size >= (1ll << 31))
+        return KVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q_latent) || !aligned16(q_rope) || !aligned16(latent_pages) || !aligned16(rope_pages) ||
+        !aligned16(block_table) || !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
+        return KVATTN_ERR_MISALIGNED;
+    const size_t ql_bytes = (size_t)batch * n_heads * latent_dim * 2;
+    const size_t qr_bytes = (size_t)batch * n_heads * rope_dim * 2;
+    const size_t lat_bytes = (size_t)num_pages * page_size * latent_dim * 2;
+    const size_t rope_bytes = (size_t)num_pages * page_size * rope_dim * 2;
+    const size_t out_bytes = (size_t)batch * n_heads * latent_dim * 4;
+    const size_t lse_bytes = (size_t)batch * n_heads * 4;
+    const void *ins[6] = {q_latent, q_rope, latent_pages, rope_pages, seq_lens, block_table};
+    const size_t in_sz[6] = {ql_bytes, qr_bytes, lat_bytes, rope_bytes, (size_t)batch * 4,
+                             (size_t)batch * max_pages_per_seq * 4};
+    for (int i = 0; i < 6; ++i)
+        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
+            return KVATTN_ERR_INVALID_ARG;
+    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+    const MlaCache cache{latent_pages, rope_pages, block_table, max_pages_per_seq * page_size, page_size,
+                         max_pages_per_seq, num_pages};
+    return mla_decode_impl(q_latent, q_rope, cache, seq_lens, batch, n_heads, scale, out, lse, stream);
 }
 
 const char *kvattn_status_string(int status) {
@@ -913,6 +1029,9 @@ extern "C" int kvattn_gqa_decode_noalloc(const uint16_t *q, const uint16_t *k_ca
     p.g = g;
     p.n_hb = n_hb;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.block_table = nullptr;           // contiguous cache: one page per sequence
+    p.max_pages = 1;
+    p.page_size = max_seq_len;
     const int U = n_kv_heads * n_hb;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (head_dim == 128)

@@ -116,6 +116,9 @@ struct MlaParams {
     int workers;       // clusters
     int min_tiles;
     float scale_log2;
+    const int32_t *block_table; // [B, max_pages] physical pages (paged cache); null: contiguous
+    int max_pages;              // block-table columns
+    int page_size;              // rows per page (T_max when contiguous)
 };
 
 struct MlaMaps {
@@ -160,11 +163,12 @@ __device__ __forceinline__ void producer(const MlaParams &p, const MlaMaps &m, c
             const uint32_t ph = (uint32_t)(k / NST) & 1u;
             if (!mbar_wait(&bars->empty[s], ph ^ 1u, FLAG_EMPTY_WAIT, c.abort_flag)) { ok = false; break; }
             mbar_arrive_expect_tx(&bars->full[s], nch * CHUNK_T);
-            const int y = min(lt * TILE, len - TILE);
+            const TileSrc src = tile_source(p.block_table, p.max_pages, p.page_size, pc.b, lt, TILE, len);
             uint8_t *st = c.smem + OFF_ST + s * STAGE;
             for (int ch = 0; ch < 4; ++ch)
-                tma_load_3d(st + ch * CHUNK_T, &m.lat, &bars->full[s], 256 * (int)c.r + 64 * ch, y, pc.b, pol);
-            if (c.r == 0) tma_load_3d(st + 4 * CHUNK_T, &m.rope, &bars->full[s], 0, y, pc.b, pol);
+                tma_load_3d(st + ch * CHUNK_T, &m.lat, &bars->full[s], 256 * (int)c.r + 64 * ch, src.y, src.page,
+                            pol);
+            if (c.r == 0) tma_load_3d(st + 4 * CHUNK_T, &m.rope, &bars->full[s], 0, src.y, src.page, pol);
         }
     }
     if (!ok) {

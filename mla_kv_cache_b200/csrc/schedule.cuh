@@ -81,6 +81,28 @@ __device__ __forceinline__ Piece piece_at(const int *s_prefix, int B, int U, lon
     return pc;
 }
 
+// Where the TMA finds tile lt of sequence b.  The cache is a sequence of pages of
+// page_size rows (a contiguous cache is one page per sequence, page_size = its capacity,
+// page = b); a tile never straddles two pages (page_size is a multiple of the tile).
+// The last tile of a sequence is loaded shifted back inside its page so that it ends at
+// the sequence's last row: its first rows then repeat rows of the previous tile, or lie
+// before the page (a negative row, zero-filled by the TMA unit), and the consumers mask
+// them (tile rows below TILE - valid).  No load touches a row at or past the length.
+struct TileSrc {
+    int y;      // first row inside the page
+    int page;   // physical page
+};
+__device__ __forceinline__ TileSrc tile_source(const int32_t *block_table, int max_pages, int page_size,
+                                               int b, int lt, int tile, int len) {
+    const int tok0 = lt * tile;
+    const int lp = tok0 / page_size;
+    const int valid = min(tile, len - tok0);
+    TileSrc s;
+    s.y = tok0 - lp * page_size + valid - tile;
+    s.page = block_table != nullptr ? __ldg(block_table + (size_t)b * max_pages + lp) : b;
+    return s;
+}
+
 // Tiles per worker, identical on every CTA and in the combine kernel.
 __device__ __forceinline__ long long tiles_per_worker(long long total, int workers, int min_tiles) {
     long long w = (total + workers - 1) / workers;

@@ -167,6 +167,43 @@ def test_mla_rope_append_rejects_bad_arguments(lib, kw, expected):
     assert st == expected
 
 
+@pytest.mark.parametrize("kw,expected", [
+    (dict(table=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(P=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(S=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(M=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(S=16), kb.KVATTN_ERR_UNSUPPORTED),       # pages must hold whole 64-row tiles
+    (dict(S=96), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(d=96), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(table=6 * A + 4), kb.KVATTN_ERR_MISALIGNED),
+    (dict(out=7 * A + 32), kb.KVATTN_ERR_INVALID_ARG),    # output overlaps the block table
+])
+def test_gqa_paged_rejects_bad_arguments(lib, kw, expected):
+    a = dict(q=A, k=2 * A, v=3 * A, table=6 * A, lens=5 * A, P=64, S=128, M=8, B=2, nq=8, nkv=2, d=128,
+             scale=0.088, out=7 * A, lse=8 * A)
+    a.update(kw)
+    if kw.get("out") == 7 * A + 32:
+        a["table"] = 7 * A
+    st = lib.kvattn_gqa_decode_paged(a["q"], a["k"], a["v"], a["table"], a["lens"], a["P"], a["S"], a["M"],
+                                     a["B"], a["nq"], a["nkv"], a["d"], a["scale"], a["out"], a["lse"], None)
+    assert st == expected
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(S=32), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(dc=256), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(table=0), kb.KVATTN_ERR_INVALID_ARG),
+])
+def test_mla_paged_rejects_bad_arguments(lib, kw, expected):
+    a = dict(ql=A, qr=2 * A, lat=3 * A, rope=4 * A, table=5 * A, lens=6 * A, P=64, S=64, M=8, B=2, H=128,
+             dc=512, dr=64, out=7 * A, lse=8 * A)
+    a.update(kw)
+    st = lib.kvattn_mla_decode_paged(a["ql"], a["qr"], a["lat"], a["rope"], a["table"], a["lens"], a["P"],
+                                     a["S"], a["M"], a["B"], a["H"], a["dc"], a["dr"], 0.0722, a["out"],
+                                     a["lse"], None)
+    assert st == expected
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     q = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
