@@ -56,6 +56,8 @@ def load(mutant=0, out_dir=None):
         lib.kvo_gqa_decode.restype = ci
         lib.kvo_mla_decode.argtypes = [dp, dp, dp, dp, ip, ci, ci, ci, ci, ci, cd, dp, dp]
         lib.kvo_mla_decode.restype = ci
+        lib.kvo_gqa_decode_multi.argtypes = [dp, dp, dp, ip, ci, ci, ci, ci, ci, ci, cd, ci, dp, dp]
+        lib.kvo_gqa_decode_multi.restype = ci
         lib.kvo_rope.argtypes = [dp, ci, ci, ip, cd, ci, dp]
         lib.kvo_rope.restype = ci
         lib.kvo_num_threads.restype = ci
@@ -195,3 +197,37 @@ def rope_f64(x, positions, base, interleaved, lib=None):
     if st != 0:
         raise ValueError("kvo_rope: bad arguments")
     return out.reshape(xx.shape)
+
+
+def gqa_decode_multi_f64(q, k, v, seq_lens, scale, window=0, lib=None):
+    """Multi-token decode on fp64 arrays: q [B, L, n_q, d], k / v [B, n_kv, T, d];
+    returns (out [B, L, n_q, d], lse [B, L, n_q])."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, L, n_q, d = q.shape
+    n_kv, T = k.shape[1], k.shape[2]
+    lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    out = np.zeros((B, L, n_q, d))
+    lse = np.zeros((B, L, n_q))
+    st = lib.kvo_gqa_decode_multi(_ptr(q, ctypes.c_double), _ptr(k, ctypes.c_double), _ptr(v, ctypes.c_double),
+                                  _ptr(lens, ctypes.c_int32), B, L, n_q, n_kv, d, T, float(scale), int(window),
+                                  _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if st != 0:
+        raise RuntimeError(f"kvo_gqa_decode_multi failed ({st})")
+    return out, lse
+
+
+def gqa_decode_multi(q, k_cache, v_cache, seq_lens, scale, window=0, lib=None):
+    """Multi-token decode on the bf16 (or any float) tensors, one sequence at a time so
+    only the touched rows are converted to fp64."""
+    B = q.shape[0]
+    lens = [int(x) for x in (seq_lens.tolist() if hasattr(seq_lens, "tolist") else seq_lens)]
+    outs, lses = [], []
+    for b in range(B):
+        T = max(0, min(lens[b], k_cache.shape[2]))
+        n = max(T, 1)
+        o, l = gqa_decode_multi_f64(q[b:b + 1], k_cache[b:b + 1, :, :n], v_cache[b:b + 1, :, :n],
+                                    [T], scale, window, lib=lib)
+        outs.append(o[0])
+        lses.append(l[0])
+    return np.stack(outs), np.stack(lses)

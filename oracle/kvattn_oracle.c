@@ -135,6 +135,85 @@ int kvo_gqa_decode(const double *q, const double *k, const double *v,
 }
 
 /*
+ * Several new tokens per sequence (multi-token decode, e.g. verifying drafted tokens),
+ * optionally with a sliding window.
+ *   q    [B, L, n_q, d]     the L newest tokens' queries, oldest first
+ *   k, v [B, n_kv, T_max, d] the cache, which already holds those L tokens at positions
+ *                           seq_lens[b] - L .. seq_lens[b] - 1
+ *   out  [B, L, n_q, d],  lse [B, L, n_q]
+ * Query i sits at position p = seq_lens[b] - L + i and attends to the cached positions
+ * t <= p (the causal mask of "Attention variants: MQA, GQA, and MLA", section
+ * "Implementation, twice": a query never sees later tokens) and, when window > 0, only
+ * to the last `window` of them, p - window < t (the sliding window named in
+ * "Grouped-Query Attention: Fewer KV Heads, Same Quality", section on modern
+ * architectures, Mistral 7B).  A query with no visible position (p < 0) gets out = 0,
+ * lse = -inf.  Each query is the plain softmax of the single-token routine over its
+ * visible positions, in the same three passes.
+ */
+int kvo_gqa_decode_multi(const double *q, const double *k, const double *v, const int32_t *seq_lens,
+                         int B, int L, int n_q, int n_kv, int d, int T_max, double scale, int window,
+                         double *out, double *lse) {
+    if (B < 0 || L <= 0 || n_q <= 0 || n_kv <= 0 || d <= 0 || T_max < 0 || n_q % n_kv != 0 || window < 0)
+        return -1;
+    int failed = 0;
+#pragma omp parallel for collapse(3) schedule(dynamic)
+    for (int b = 0; b < B; ++b) {
+        for (int i = 0; i < L; ++i) {
+            for (int h = 0; h < n_q; ++h) {
+                int T = seq_lens[b];
+                if (T < 0) T = 0;
+                if (T > T_max) T = T_max;
+                const int pos = T - L + i;
+#if KVO_MUTANT == 9
+                const int hi = pos;                 /* planted mistake: the query's own position hidden */
+#else
+                const int hi = pos + 1;             /* visible: t < hi */
+#endif
+#if KVO_MUTANT == 10
+                const int lo = window > 0 ? (hi - window - 1 > 0 ? hi - window - 1 : 0) : 0;  /* planted: window + 1 */
+#else
+                const int lo = window > 0 ? (hi - window > 0 ? hi - window : 0) : 0;
+#endif
+                const int j = kv_head_of(h, n_q, n_kv);
+                const double *qh = q + (((size_t)b * L + i) * n_q + h) * d;
+                const double *kb = k + ((size_t)b * n_kv + j) * (size_t)T_max * d;
+                const double *vb = v + ((size_t)b * n_kv + j) * (size_t)T_max * d;
+                double *oh = out + (((size_t)b * L + i) * n_q + h) * d;
+                double *lh = lse + ((size_t)b * L + i) * n_q + h;
+                for (int e = 0; e < d; ++e) oh[e] = 0.0;
+                if (hi <= lo) {
+                    *lh = -INFINITY;
+                    continue;
+                }
+                const int n = hi - lo;
+                double *s = (double *)malloc(sizeof(double) * (size_t)n);
+                if (!s) {
+#pragma omp atomic write
+                    failed = 1;
+                    continue;
+                }
+                for (int t = 0; t < n; ++t) {
+                    double acc = 0.0;
+                    for (int e = 0; e < d; ++e) acc += qh[e] * kb[(size_t)(lo + t) * d + e];
+                    s[t] = scale * acc;
+                }
+                double m = s[0];
+                for (int t = 1; t < n; ++t) if (s[t] > m) m = s[t];
+                double l = 0.0;
+                for (int t = 0; t < n; ++t) l += exp(s[t] - m);
+                for (int t = 0; t < n; ++t) {
+                    const double w = exp(s[t] - m) / l;
+                    for (int e = 0; e < d; ++e) oh[e] += w * vb[(size_t)(lo + t) * d + e];
+                }
+                *lh = m + log(l);
+                free(s);
+            }
+        }
+    }
+    return failed ? -2 : 0;
+}
+
+/*
  * Absorbed MLA decode.
  *   q_lat  [B, H, d_c]      query already multiplied by W_UK (latent space)
  *   q_rope [B, H, d_r]      rotated decoupled-RoPE query part

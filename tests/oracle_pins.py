@@ -323,9 +323,79 @@ def pin_rope_invariants(lib):
     assert np.allclose(yi, yh[:, perm], atol=1e-12)
 
 
+# --------------------------------------------------------------------------------------
+# Several new tokens per sequence with the causal mask ("Attention variants: MQA, GQA,
+# and MLA", "Implementation, twice") and an optional sliding window.  Pinned to PyTorch
+# SDPA in fp64 with an explicit boolean mask (the library routine the pages use), to
+# the single-token routine on each query's visible slice, and to closed forms: a
+# window of one token returns that token's value; a query before the cache's start
+# sees nothing.
+# --------------------------------------------------------------------------------------
+def _multi_case(seed, B=3, L=4, n_q=8, n_kv=2, d=16, T=20):
+    r = _rng(seed)
+    q = r.standard_normal((B, L, n_q, d))
+    k = r.standard_normal((B, n_kv, T, d))
+    v = r.standard_normal((B, n_kv, T, d))
+    return q, k, v
+
+
+def pin_multi_token_sdpa(lib):
+    q, k, v = _multi_case(41)
+    B, L, n_q, d = q.shape
+    n_kv, T = k.shape[1], k.shape[2]
+    lens = np.array([20, 9, 4], np.int32)
+    for window in (0, 1, 3, 6, 50):
+        out, lse = oracle.gqa_decode_multi_f64(q, k, v, lens, 0.37, window=window, lib=lib)
+        for b in range(B):
+            n = int(lens[b])
+            qt = torch.from_numpy(q[b]).permute(1, 0, 2)[None]              # [1, n_q, L, d]
+            kt = torch.from_numpy(k[b, :, :n])[None]
+            vt = torch.from_numpy(v[b, :, :n])[None]
+            pos = torch.arange(n - L, n)[:, None]
+            t = torch.arange(n)[None, :]
+            vis = t <= pos
+            if window > 0:
+                vis &= t > pos - window
+            ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=vis, scale=0.37, enable_gqa=True)
+            assert np.allclose(out[b], ref[0].permute(1, 0, 2).numpy(), atol=1e-12), (b, window)
+            s = torch.einsum("hld,htd->hlt", qt[0], kt[0].repeat_interleave(n_q // n_kv, 0)) * 0.37
+            s = s.masked_fill(~vis[None], float("-inf"))
+            assert np.allclose(lse[b], torch.logsumexp(s, -1).permute(1, 0).numpy(), atol=1e-12), (b, window)
+
+
+def pin_multi_token_reductions(lib):
+    q, k, v = _multi_case(42, B=2, L=3)
+    lens = np.array([11, 6], np.int32)
+    L, n_q = q.shape[1], q.shape[2]
+    g = n_q // k.shape[1]
+    for window in (0, 4):
+        out, lse = oracle.gqa_decode_multi_f64(q, k, v, lens, 0.5, window=window, lib=lib)
+        for b in range(2):
+            for i in range(L):
+                pos = int(lens[b]) - L + i
+                lo = max(0, pos + 1 - window) if window else 0
+                # each query equals the single-token routine over its visible slice
+                o1, l1 = oracle.gqa_decode_f64(q[b:b + 1, i], k[b:b + 1, :, lo:pos + 1], v[b:b + 1, :, lo:pos + 1],
+                                               np.array([pos + 1 - lo], np.int32), 0.5, lib=lib)
+                assert np.allclose(out[b, i], o1[0], atol=1e-14) and np.allclose(lse[b, i], l1[0], atol=1e-13)
+    # window 1: the query sees only its own token
+    out, lse = oracle.gqa_decode_multi_f64(q, k, v, lens, 0.5, window=1, lib=lib)
+    for b in range(2):
+        for i in range(L):
+            pos = int(lens[b]) - L + i
+            for h in range(n_q):
+                assert np.allclose(out[b, i, h], v[b, h // g, pos], atol=1e-15)
+                assert abs(lse[b, i, h] - 0.5 * q[b, i, h] @ k[b, h // g, pos]) < 1e-12
+    # queries before the cache's first position see nothing
+    out, lse = oracle.gqa_decode_multi_f64(q, k, v, np.array([2, 0], np.int32), 0.5, lib=lib)
+    assert np.all(np.isneginf(lse[0, 0])) and np.all(out[0, 0] == 0) and np.all(np.isfinite(lse[0, 1:]))
+    assert np.all(np.isneginf(lse[1])) and np.all(out[1] == 0)
+
+
 ALL_PINS = [
     pin_gqa_equals_mha_on_repeated_kv, pin_sdpa_enable_gqa, pin_closed_forms,
     pin_empty_sequence, pin_brute_force_tiny, pin_split_merge, pin_permutation_invariance,
     pin_scale_equivariance, pin_mla_absorbed_equals_explicit, pin_mla_matches_sdpa,
     pin_mla_without_rope_is_mqa, pin_rope_identity_and_hand_cases, pin_rope_invariants,
+    pin_multi_token_sdpa, pin_multi_token_reductions,
 ]

@@ -1,7 +1,8 @@
 """Plant one mistake at a time in the oracle (CPU builds with -DKVO_MUTANT=n) and show
 that the pins catch each one: a strided group index, a dropped scale, a base-2 lse, a
 dropped RoPE term, values read from the key cache, a dropped last position, a flipped
-rotary sine, a halved rotary frequency exponent."""
+rotary sine, a halved rotary frequency exponent, a multi-token query that cannot see its
+own position, a sliding window one token too wide."""
 import pytest
 
 import oracle
@@ -9,7 +10,8 @@ from tests import oracle_pins
 
 MUTANTS = {1: "strided group index", 2: "scale dropped", 3: "base-2 log-sum-exp",
            4: "MLA RoPE score term dropped", 5: "values read from K", 6: "last position dropped",
-           7: "rotary sine sign flipped", 8: "rotary frequency exponent halved"}
+           7: "rotary sine sign flipped", 8: "rotary frequency exponent halved",
+           9: "multi-token: own position hidden", 10: "multi-token: window one too wide"}
 
 
 @pytest.mark.parametrize("mutant", sorted(MUTANTS), ids=lambda m: MUTANTS[m])
