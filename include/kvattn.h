@@ -116,6 +116,30 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
                       void *stream);
 
 /*
+ * Several new tokens per sequence in one call (multi-token decode: verifying drafted
+ * tokens, or a short prompt continuation), with the causal mask of "Attention variants:
+ * MQA, GQA, and MLA", section "Implementation, twice" (a query never sees a later
+ * token), and optionally a sliding window (the Mistral-style window named in
+ * "Grouped-Query Attention: Fewer KV Heads, Same Quality").
+ *   q         device bf16 [batch, q_len, n_q_heads, head_dim]: the q_len newest tokens'
+ *             queries, oldest first
+ *   k_cache, v_cache, seq_lens, max_seq_len: as for kvattn_gqa_decode; the cache already
+ *             holds the q_len new tokens at positions seq_lens[b] - q_len .. seq_lens[b] - 1
+ *   window    0: no window; w > 0: query i, at position p = seq_lens[b] - q_len + i,
+ *             attends to positions p - w < t <= p only (its last w tokens, itself included);
+ *             otherwise to all t <= p.  Tiles wholly before the earliest visible position
+ *             are not read.
+ *   out       device fp32 [batch, q_len, n_q_heads, head_dim];  lse fp32 [batch, q_len, n_q_heads]
+ * A query with no visible position (p < 0) gets out = 0 and lse = -inf.  q_len == 1 and
+ * window == 0 is exactly kvattn_gqa_decode.  Otherwise head_dim must be 128 and
+ * (n_q_heads / n_kv_heads) * q_len <= 64 (KVATTN_ERR_UNSUPPORTED if not).
+ */
+int kvattn_gqa_decode_multi(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                            const int32_t *seq_lens, int max_seq_len, int batch, int q_len,
+                            int n_q_heads, int n_kv_heads, int head_dim, float scale, int window,
+                            float *out, float *lse, void *stream);
+
+/*
  * kvattn_gqa_decode over a paged KV cache: the cache is a pool of pages and each
  * sequence lists its pages in a block table (the serving-engine layout the pages name,
  * "Attention variants: MQA, GQA, and MLA", section "Against the real libraries": vLLM's

@@ -37,6 +37,10 @@ _SIGNATURES = {
                                                  ctypes.c_int, ctypes.c_int, ctypes.c_float,
                                                  ctypes.c_void_p, ctypes.c_void_p,
                                                  ctypes.c_void_p]),
+    "kvattn_gqa_decode_multi": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_void_p]),
     "kvattn_gqa_decode_paged": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, ctypes.c_void_p,
                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
@@ -340,4 +344,29 @@ def kvattn_mla_decode_paged(q_latent, q_rope, latent_pages, rope_pages, block_ta
                                        _stream_handle(stream))
     if st != KVATTN_OK:
         raise KvattnError(st, "kvattn_mla_decode_paged")
+    return out, lse
+
+
+def kvattn_gqa_decode_multi(q, k_cache, v_cache, seq_lens, scale, window=0, out=None, lse=None, stream=None):
+    """Multi-token decode (include/kvattn.h, kvattn_gqa_decode_multi): q [B, L, n_q, d]
+    bf16, caches [B, n_kv, T, d] bf16 holding the L new tokens at the end of each
+    sequence.  Returns (out [B, L, n_q, d] fp32, lse [B, L, n_q] fp32)."""
+    import torch
+    B, L, n_q, d = q.shape
+    n_kv, T = k_cache.shape[1], k_cache.shape[2]
+    _check(q, "q", torch.bfloat16)
+    _check(k_cache, "k_cache", torch.bfloat16, (B, n_kv, T, d))
+    _check(v_cache, "v_cache", torch.bfloat16, (B, n_kv, T, d))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, L, n_q, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, L, n_q), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, (B, L, n_q, d))
+    _check(lse, "lse", torch.float32, (B, L, n_q))
+    st = lib().kvattn_gqa_decode_multi(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seq_lens.data_ptr(),
+                                       T, B, L, n_q, n_kv, d, float(scale), int(window), out.data_ptr(),
+                                       lse.data_ptr(), _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_gqa_decode_multi")
     return out, lse

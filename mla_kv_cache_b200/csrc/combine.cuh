@@ -38,6 +38,8 @@ struct CombineParams {
     int tile;              // tokens per tile of the decode kernel
     int workers;           // decode workers (CTAs or CTA pairs)
     int min_tiles;         // the decode kernel's minimum tiles per worker
+    int q_len;             // new tokens per sequence (rows of a unit: q_len x g)
+    int window;            // sliding window (0: none)
 };
 
 // D columns, D / 32 floats per lane; NW warps share the partials of one output row.
@@ -54,16 +56,19 @@ __global__ void __launch_bounds__(NW * 32) combine_kernel(const CombineParams p)
     const int i = u % p.units_per_seq;
     const int j = i / p.n_hb;
     const int hb = i % p.n_hb;
-    const int hg = hb * p.heads_per_unit + r;
-    if (hg >= p.g) return;
-    const size_t gh = (size_t)b * p.n_q + (size_t)j * p.g + hg;
+    // row of the unit: query position qi and head hg of the group (qi-major)
+    const int vr = hb * p.heads_per_unit + r;
+    if (vr >= p.g * p.q_len) return;
+    const int qi = vr / p.g, hg = vr - qi * p.g;
+    const size_t gh = ((size_t)b * p.q_len + qi) * p.n_q + (size_t)j * p.g + hg;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int col = lane * VEC;
 
     // ---- the work split, from seq_lens (an input: readable before the decode grid ends)
     int before = 0, all = 0;
     for (int x = threadIdx.x; x < p.B; x += blockDim.x) {
-        const int t = tiles_of(clamp_len(__ldg(p.seq_lens + x), p.T_max), p.tile);
+        const int lx = clamp_len(__ldg(p.seq_lens + x), p.T_max);
+        const int t = tiles_of(lx - active_start(lx, p.q_len, p.window), p.tile);
         all += t;
         if (x < b) before += t;
     }
@@ -79,7 +84,8 @@ __global__ void __launch_bounds__(NW * 32) combine_kernel(const CombineParams p)
     all = 0;
 #pragma unroll
     for (int w = 0; w < kCombineWarps; ++w) { before += s_sum[0][w]; all += s_sum[1][w]; }
-    const int n_tiles = tiles_of(clamp_len(__ldg(p.seq_lens + b), p.T_max), p.tile);
+    const int len_b = clamp_len(__ldg(p.seq_lens + b), p.T_max);
+    const int n_tiles = tiles_of(len_b - active_start(len_b, p.q_len, p.window), p.tile);
     const long long W = tiles_per_worker((long long)all * p.units_per_seq, p.workers, p.min_tiles);
     if (n_tiles == 0) {
         // nothing of this unit was touched by the decode kernel
@@ -153,10 +159,12 @@ __global__ void __launch_bounds__(NW * 32) combine_kernel(const CombineParams p)
 #pragma unroll
         for (int v = 0; v < VEC; ++v) res[v] += s_acc[w][col + v] * f;
     }
-    const float inv = 1.f / tot;
+    // a row may have no visible position in any partial (a new token before the cache's
+    // start): out 0, lse -inf
+    const float inv = tot > 0.f ? 1.f / tot : 0.f;
 #pragma unroll
     for (int v = 0; v < VEC; ++v) p.out[gh * D + col + v] = res[v] * inv;
-    if (lane == 0) p.lse[gh] = M + __logf(tot);
+    if (lane == 0) p.lse[gh] = tot > 0.f ? M + __logf(tot) : -INFINITY;
 }
 
 }  // namespace kvattn

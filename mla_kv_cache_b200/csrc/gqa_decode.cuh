@@ -43,6 +43,8 @@ struct GqaParams {
     const int32_t *block_table; // [B, max_pages] physical pages (paged cache); null: contiguous
     int max_pages;              // block-table columns
     int page_size;              // rows per page (T_max when contiguous)
+    int q_len;                  // new tokens per sequence (1: single-token decode)
+    int window;                 // sliding window in tokens (0: none)
 };
 
 template <int D, int MT>

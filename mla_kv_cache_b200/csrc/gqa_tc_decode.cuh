@@ -191,17 +191,27 @@ __device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *
             ok = false;
             break;
         }
-        mbar_arrive_expect_tx(&bars->qfull[qb], C::QBLOCK);
         const int qrow = j * p.g + hb * HB;
         uint8_t *qdst = c.smem + OFF_Q + qb * C::QBLOCK;
-        tma_load_3d(qdst, qmap, &bars->qfull[qb], 0, qrow, pc.b, pol);
-        tma_load_3d(qdst + C::QCHUNK, qmap, &bars->qfull[qb], 64, qrow, pc.b, pol);
+        if (p.q_len == 1) {
+            mbar_arrive_expect_tx(&bars->qfull[qb], C::QBLOCK);
+            tma_load_3d(qdst, qmap, &bars->qfull[qb], 0, qrow, pc.b, pol);
+            tma_load_3d(qdst + C::QCHUNK, qmap, &bars->qfull[qb], 64, qrow, pc.b, pol);
+        } else {
+            // several new tokens: rows (position qi, head h) = the g heads of the group at
+            // each of the q_len positions, qi-major (a 4-D box of q[B, q_len, n_q, d])
+            const uint32_t bytes = 2u * (uint32_t)(p.g * p.q_len) * 128u;
+            mbar_arrive_expect_tx(&bars->qfull[qb], bytes);
+            tma_load_4d(qdst, qmap, &bars->qfull[qb], 0, j * p.g, 0, pc.b, pol);
+            tma_load_4d(qdst + C::QCHUNK, qmap, &bars->qfull[qb], 64, j * p.g, 0, pc.b, pol);
+        }
+        const int start = active_start(len, p.q_len, p.window);
         for (int lt = pc.lt0; lt < pc.lt1; ++lt, ++k) {
             const int s = k % NST;
             const uint32_t ph = (uint32_t)(k / NST) & 1u;
             if (!mbar_wait(&bars->empty[s], ph ^ 1u, FLAG_EMPTY_WAIT, c.abort_flag)) { ok = false; break; }
             mbar_arrive_expect_tx(&bars->full[s], STAGE);
-            const TileSrc src = tile_source(p.block_table, p.max_pages, p.page_size, pc.b, lt, TILE, len);
+            const TileSrc src = tile_source(p.block_table, p.max_pages, p.page_size, pc.b, lt, TILE, len, start);
             const int y = src.y;
             const int z = src.page * p.n_kv + j;
             uint8_t *st = c.smem + OFF_ST + s * STAGE;
@@ -345,6 +355,9 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
         const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
         const int j = pc.i / p.n_hb, hb = pc.i % p.n_hb;
         const int nt = pc.lt1 - pc.lt0;
+        const int start = active_start(len, p.q_len, p.window);
+        // columns of one query position (the group's heads); all columns of the unit
+        const uint64_t group_bits = p.g >= 64 ? ~0ull : ((1ull << p.g) - 1ull);
         float m_own = -INFINITY;              // running max of head st_id (owner threads)
         float l_part[NR];
 #pragma unroll
@@ -354,8 +367,25 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
             const int kt = k + t;
             const int s = kt % NST, sb = kt & 1;
             const int lt = pc.lt0 + t;
-            const int y = min(lt * TILE, len - TILE);
-            const int tok_lo = lt * TILE - y, tok_hi = min((lt + 1) * TILE, len) - y;
+            // tile row r holds position y + r (the last tile is shifted back to end at len;
+            // its rows before tok0 belong to the previous tile)
+            const int tok0 = start + lt * TILE;
+            const int y = min(tok0, len - TILE);
+            const int posr = y + r;
+            // the columns (query position qi, head) that may see this token: query qi sits
+            // at len - q_len + qi and sees [that + 1 - window, that] (causal, windowed)
+            uint64_t vis = 0;
+            if (posr >= tok0 && posr < len) {
+                if (p.q_len == 1) {
+                    vis = group_bits;
+                } else {
+                    for (int qi = 0; qi < p.q_len; ++qi) {
+                        const int hi = len - p.q_len + qi + 1;
+                        const int lo = p.window > 0 ? hi - p.window : 0;
+                        if (posr < hi && posr >= lo) vis |= group_bits << (qi * p.g);
+                    }
+                }
+            }
             // ---- this token's scores
             if (!warp_all(mbar_wait(&bars->sready[sb], (uint32_t)(kt >> 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
                 return;
@@ -365,11 +395,10 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bars->sfree[sb]);
-            const bool valid = r >= tok_lo && r < tok_hi;
             float sc[NR], v[NR];
 #pragma unroll
             for (int h = 0; h < NR; ++h) {
-                sc[h] = valid ? __uint_as_float(sv[h]) * p.scale_log2 : -INFINITY;
+                sc[h] = ((vis >> h) & 1ull) ? __uint_as_float(sv[h]) * p.scale_log2 : -INFINITY;
                 v[h] = sc[h];
             }
             // ---- per-head maximum over the tile's 128 tokens
@@ -414,7 +443,10 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                 uint32_t hw[4], lw[4];
                 const float4 m0 = *reinterpret_cast<const float4 *>(ms + sb * HB + 8 * cc);
                 const float4 m1 = *reinterpret_cast<const float4 *>(ms + sb * HB + 8 * cc + 4);
-                const float mh[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                // (a column with no visible token so far has max -inf; its weights are 0)
+                float mh[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mh[e] = mh[e] == -INFINITY ? 0.f : mh[e];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int h = 8 * cc + 2 * e;
@@ -466,9 +498,15 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
         warp_xreduce<NR, false>(v, lane);
         store_reduced<NR>(red + (2 * 4 + q) * HB, v, lane);
         if (!grp_sync()) return;
-        const int h_real = min(HB, p.g - hb * HB);
-        const size_t head0 = (size_t)pc.b * p.n_q + (size_t)j * p.g + (size_t)hb * HB;
+        // columns of the unit: (query position qi, head h of the group), qi-major; output
+        // row of column cc in out [B, q_len, n_q, d] / lse [B, q_len, n_q]
+        const int h_real = min(HB, p.g * p.q_len - hb * HB);
         const size_t part = ((size_t)blockIdx.x * 2 + pc.slot) * HB;
+        auto out_row = [&](int cc) -> size_t {
+            const int vr = hb * HB + cc;
+            const int qi = vr / p.g;
+            return ((size_t)pc.b * p.q_len + qi) * p.n_q + (size_t)j * p.g + (vr - qi * p.g);
+        };
         if (st_id < NR) {
             const float l = red[(8 + 0) * HB + st_id] + red[(8 + 1) * HB + st_id] + red[(8 + 2) * HB + st_id] +
                             red[(8 + 3) * HB + st_id];
@@ -476,7 +514,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
             const float lse_v = l > 0.f ? (m_own + __log2f(l)) * 0.69314718055994531f : -INFINITY;
             if (st_id < h_real) {
                 if (pc.whole)
-                    p.lse[head0 + st_id] = lse_v;
+                    p.lse[out_row(st_id)] = lse_v;
                 else
                     p.ws_lse[part + st_id] = lse_v;
             }
@@ -486,15 +524,19 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
         if (!warp_all(mbar_wait(&bars->odone[klast & 1], (uint32_t)(klast >> 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
             return;
         tc_fence_after();
-        float *dst = pc.whole ? p.out + head0 * D : p.ws_o + part * D;
 #pragma unroll
         for (int c0 = 0; c0 < NQ; c0 += 16) {
             uint32_t ov[16];
             tmem_ld16(c.tmem + lane_base + TM_O + c0, ov);
             tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < 16; ++h)
-                if (c0 + h < NR && c0 + h < h_real) dst[(size_t)(c0 + h) * D + r] = __uint_as_float(ov[h]) * linv[c0 + h];
+            for (int h = 0; h < 16; ++h) {
+                const int cc = c0 + h;
+                if (cc < NR && cc < h_real) {
+                    float *dst = pc.whole ? p.out + out_row(cc) * D : p.ws_o + (part + cc) * D;
+                    dst[r] = __uint_as_float(ov[h]) * linv[cc];
+                }
+            }
         }
         tc_fence_before();
         mbar_arrive(&bars->ofree);
@@ -542,7 +584,11 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
         tmem_alloc(smem_u32(tmem_ptr), TM_COLS);
         tmem_relinquish();
     }
-    if (warp == 2) build_tile_prefix(p.seq_lens, p.B, p.T_max, TILE, s_prefix, lane);
+    if (warp == 2) build_tile_prefix(p.seq_lens, p.B, p.T_max, TILE, s_prefix, lane, p.q_len, p.window);
+    // query buffers start zeroed: rows a unit's block does not fill stay finite
+    for (int i = tid; i < QREGION / 16; i += NTHREADS)
+        reinterpret_cast<uint4 *>(smem + OFF_Q)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);

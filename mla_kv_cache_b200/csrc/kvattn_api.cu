@@ -175,6 +175,29 @@ int encode_map_3d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t di
     return KVATTN_OK;
 }
 
+// 4-D bf16 tensor [dim3][dim2][dim1][dim0] (dim0 fastest, densely packed), box
+// {box0, box1, box2, 1}.  Not cached (used once per call).
+int make_map_4d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint64_t dim3,
+                uint32_t box0, uint32_t box1, uint32_t box2, CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) {
+        snprintf(t_detail, sizeof(t_detail), "cuTensorMapEncodeTiled unavailable");
+        return KVATTN_ERR_CUDA;
+    }
+    cuuint64_t dims[4] = {dim0, dim1, dim2, dim3};
+    cuuint64_t strides[3] = {dim0 * 2, dim0 * dim1 * 2, dim0 * dim1 * dim2 * 2};
+    cuuint32_t box[4] = {box0, box1, box2, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(t_detail, sizeof(t_detail), "cuTensorMapEncodeTiled (4-D) failed (%d)", (int)r);
+        return KVATTN_ERR_CUDA;
+    }
+    return KVATTN_OK;
+}
+
 // Raises a kernel's dynamic shared-memory limit once per device (the largest request
 // seen so far is kept).
 cudaError_t set_smem_limit(const void *kern, DeviceState *dev, int smem) {
@@ -294,6 +317,8 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
     cp.tile = C::TILE;
     cp.workers = p.workers;
     cp.min_tiles = p.min_tiles;
+    cp.q_len = 1;
+    cp.window = 0;
     const int rows = p.g < C::HEADS ? p.g : C::HEADS;
     return launch_combine(D, cp, p.B * units_per_seq, rows, stream,
                           combine_warps((p.T_max + C::TILE - 1) / C::TILE, max_tiles, p.workers));
@@ -356,7 +381,9 @@ int run_gqa_tc(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap
     cp.tile = gqatc::TILE;
     cp.workers = p.workers;
     cp.min_tiles = p.min_tiles;
-    const int rows = p.g < gqatc::HB ? p.g : gqatc::HB;
+    cp.q_len = p.q_len;
+    cp.window = p.window;
+    const int rows = p.g * p.q_len < gqatc::HB ? p.g * p.q_len : gqatc::HB;
     return launch_combine(gqatc::D, cp, p.B * units_per_seq, rows, stream,
                           combine_warps((p.T_max + gqatc::TILE - 1) / gqatc::TILE, max_tiles, p.workers));
 }
@@ -384,7 +411,7 @@ struct GqaCache {
 
 int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq_lens, int batch,
                     int n_q_heads, int n_kv_heads, int head_dim, float scale, float *out, float *lse,
-                    void *stream) {
+                    void *stream, int q_len = 1, int window = 0) {
     DeviceState *dev = nullptr;
     int st = device_state(&dev);
     if (st != KVATTN_OK) return st;
@@ -398,10 +425,19 @@ int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq
                  (dev->max_smem_optin - gqatc::smem_bytes(0)) / 4);
         return KVATTN_ERR_UNSUPPORTED;
     }
-    const bool tc = tiles_fit && use_tc_kernel(head_dim, g, batch, dev);
+    // several new tokens, or a window: the tcgen05 kernel, whose score columns are the
+    // (position, head) pairs of a group
+    const bool multi = q_len > 1 || window > 0;
+    if (multi && !(tiles_fit && head_dim == 128 && gqatc::smem_bytes(batch) <= dev->max_smem_optin &&
+                   g * q_len <= gqatc::HB)) {
+        snprintf(t_detail, sizeof(t_detail), "multi-token decode needs head_dim 128 and g * q_len <= %d",
+                 gqatc::HB);
+        return KVATTN_ERR_UNSUPPORTED;
+    }
+    const bool tc = multi || (tiles_fit && use_tc_kernel(head_dim, g, batch, dev));
     const int MT = g <= 16 ? 1 : 2;
     const int heads = tc ? gqatc::HB : 16 * MT;
-    const int n_hb = (g + heads - 1) / heads;
+    const int n_hb = (g * q_len + heads - 1) / heads;
     const uint32_t box_rows = tc ? gqatc::TILE : 64;
 
     CUtensorMap kmap, vmap, qmap;
@@ -411,10 +447,15 @@ int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq
     st = make_map_3d(&vmap, cache.v, head_dim, cache.page_size, (uint64_t)cache.pages * n_kv_heads, 64, box_rows,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
-    if (tc) {
+    const int gl = g * q_len;    // score columns of a unit
+    if (tc && q_len == 1) {
         // box rows = the score product's N for this group size (query heads per block)
         const uint32_t q_rows = g > 32 ? 64 : g > 16 ? 32 : 16;
         st = make_map_3d(&qmap, q, head_dim, n_q_heads, batch, 64, q_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != KVATTN_OK) return st;
+    } else if (tc) {
+        // q [B, q_len, n_q, d]: box of the group's g heads at all q_len positions
+        st = make_map_4d(&qmap, q, head_dim, n_q_heads, q_len, batch, 64, g, q_len, CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != KVATTN_OK) return st;
     }
 
@@ -433,12 +474,14 @@ int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq
     p.block_table = cache.block_table;
     p.max_pages = cache.max_pages;
     p.page_size = cache.page_size;
+    p.q_len = q_len;
+    p.window = window;
     const int U = n_kv_heads * n_hb;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (tc) {
-        if (g > 32) return run_gqa_tc<64>(p, kmap, vmap, qmap, dev, U, s);
-        if (g > 16) return run_gqa_tc<32>(p, kmap, vmap, qmap, dev, U, s);
-        if (g > 8) return run_gqa_tc<16>(p, kmap, vmap, qmap, dev, U, s);
+        if (gl > 32) return run_gqa_tc<64>(p, kmap, vmap, qmap, dev, U, s);
+        if (gl > 16) return run_gqa_tc<32>(p, kmap, vmap, qmap, dev, U, s);
+        if (gl > 8) return run_gqa_tc<16>(p, kmap, vmap, qmap, dev, U, s);
         return run_gqa_tc<8>(p, kmap, vmap, qmap, dev, U, s);
     }
     if (head_dim == 128)
@@ -561,6 +604,8 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
     cp.tile = mla::TILE;
     cp.workers = p.workers;
     cp.min_tiles = p.min_tiles;
+    cp.q_len = 1;
+    cp.window = 0;
     return launch_combine(512, cp, batch, n_heads, s,
                           combine_warps((cache.capacity + mla::TILE - 1) / mla::TILE, max_tiles, p.workers));
 }
@@ -632,6 +677,38 @@ int kvattn_gqa_decode_paged(const uint16_t *q, const uint16_t *k_pages, const ui
     const GqaCache cache{k_pages, v_pages, block_table, max_pages_per_seq * page_size, page_size,
                          max_pages_per_seq, num_pages};
     return gqa_decode_impl(q, cache, seq_lens, batch, n_q_heads, n_kv_heads, head_dim, scale, out, lse, stream);
+}
+
+int kvattn_gqa_decode_multi(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                            const int32_t *seq_lens, int max_seq_len, int batch, int q_len, int n_q_heads,
+                            int n_kv_heads, int head_dim, float scale, int window, float *out, float *lse,
+                            void *stream) {
+    if (!q || !k_cache || !v_cache || !seq_lens || !out || !lse) return KVATTN_ERR_INVALID_ARG;
+    if (batch <= 0 || q_len <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || max_seq_len <= 0 || window < 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if (n_q_heads % n_kv_heads != 0) return KVATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return KVATTN_ERR_UNSUPPORTED;
+    if ((q_len > 1 || window > 0) && (head_dim != 128 || (n_q_heads / n_kv_heads) * q_len > gqatc::HB))
+        return KVATTN_ERR_UNSUPPORTED;
+    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
+    if ((long long)batch * n_kv_heads * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seq_lens) ||
+        !aligned16(out) || !aligned16(lse))
+        return KVATTN_ERR_MISALIGNED;
+    const size_t q_bytes = (size_t)batch * q_len * n_q_heads * head_dim * 2;
+    const size_t kv_bytes = (size_t)batch * n_kv_heads * max_seq_len * head_dim * 2;
+    const size_t out_bytes = (size_t)batch * q_len * n_q_heads * head_dim * 4;
+    const size_t lse_bytes = (size_t)batch * q_len * n_q_heads * 4;
+    const void *ins[4] = {q, k_cache, v_cache, seq_lens};
+    const size_t in_sz[4] = {q_bytes, kv_bytes, kv_bytes, (size_t)batch * 4};
+    for (int i = 0; i < 4; ++i)
+        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
+            return KVATTN_ERR_INVALID_ARG;
+    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+    const GqaCache cache{k_cache, v_cache, nullptr, max_seq_len, max_seq_len, 1, batch};
+    return gqa_decode_impl(q, cache, seq_lens, batch, n_q_heads, n_kv_heads, head_dim, scale, out, lse, stream,
+                           q_len, window);
 }
 
 int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
@@ -963,6 +1040,8 @@ int run_gqa_noalloc(const GqaParams &base, const CUtensorMap &kmap, const CUtens
     cp.tile = C::TILE;
     cp.workers = p.workers;
     cp.min_tiles = p.min_tiles;
+    cp.q_len = 1;
+    cp.window = 0;
     const int rows = p.g < C::HEADS ? p.g : C::HEADS;
     return launch_combine(D, cp, p.B * units_per_seq, rows, stream,
                           combine_warps((p.T_max + C::TILE - 1) / C::TILE, max_tiles, p.workers));
@@ -1032,6 +1111,8 @@ extern "C" int kvattn_gqa_decode_noalloc(const uint16_t *q, const uint16_t *k_ca
     p.block_table = nullptr;           // contiguous cache: one page per sequence
     p.max_pages = 1;
     p.page_size = max_seq_len;
+    p.q_len = 1;
+    p.window = 0;
     const int U = n_kv_heads * n_hb;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (head_dim == 128)

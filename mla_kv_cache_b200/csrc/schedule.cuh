@@ -36,15 +36,30 @@ __device__ __forceinline__ int clamp_len(int len, int T_max) {
     return len < 0 ? 0 : (len > T_max ? T_max : len);
 }
 
+// First cached position any query of a sequence of length len can see: 0, unless the
+// L newest tokens attend through a sliding window of `window` tokens (window > 0), in
+// which case the oldest of them, at position len - L, sees back to len - L + 1 - window.
+// The tiles of a sequence cover [active_start, len).
+__device__ __forceinline__ int active_start(int len, int q_len, int window) {
+    if (window <= 0) return 0;
+    const int s = len - q_len + 1 - window;
+    return s > 0 ? s : 0;
+}
+
 // Warp 0 of the block fills s_prefix[0..B] with the exclusive prefix of tiles per
-// sequence.  The caller synchronises the block afterwards.
+// sequence (tiles of its active range).  The caller synchronises the block afterwards.
 __device__ __forceinline__ void build_tile_prefix(const int32_t *seq_lens, int B, int T_max,
-                                                  int tile, int *s_prefix, int lane) {
+                                                  int tile, int *s_prefix, int lane, int q_len = 1,
+                                                  int window = 0) {
     int running = 0;
     if (lane == 0) s_prefix[0] = 0;
     for (int base = 0; base < B; base += 32) {
         const int idx = base + lane;
-        int v = idx < B ? tiles_of(clamp_len(__ldg(seq_lens + idx), T_max), tile) : 0;
+        int v = 0;
+        if (idx < B) {
+            const int len = clamp_len(__ldg(seq_lens + idx), T_max);
+            v = tiles_of(len - active_start(len, q_len, window), tile);
+        }
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int n = __shfl_up_sync(0xffffffffu, v, off);
@@ -81,7 +96,9 @@ __device__ __forceinline__ Piece piece_at(const int *s_prefix, int B, int U, lon
     return pc;
 }
 
-// Where the TMA finds tile lt of sequence b.  The cache is a sequence of pages of
+// Where the TMA finds tile lt of sequence b (the tile starting at position start +
+// lt * tile; start is the active range's first position, a page boundary or 0 for a
+// paged cache).  The cache is a sequence of pages of
 // page_size rows (a contiguous cache is one page per sequence, page_size = its capacity,
 // page = b); a tile never straddles two pages (page_size is a multiple of the tile).
 // The last tile of a sequence is loaded shifted back inside its page so that it ends at
@@ -93,8 +110,8 @@ struct TileSrc {
     int page;   // physical page
 };
 __device__ __forceinline__ TileSrc tile_source(const int32_t *block_table, int max_pages, int page_size,
-                                               int b, int lt, int tile, int len) {
-    const int tok0 = lt * tile;
+                                               int b, int lt, int tile, int len, int start = 0) {
+    const int tok0 = start + lt * tile;
     const int lp = tok0 / page_size;
     const int valid = min(tile, len - tok0);
     TileSrc s;

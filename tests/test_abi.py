@@ -204,6 +204,24 @@ def test_mla_paged_rejects_bad_arguments(lib, kw, expected):
     assert st == expected
 
 
+@pytest.mark.parametrize("kw,expected", [
+    (dict(L=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(window=-1), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(L=2, nq=64, nkv=1), kb.KVATTN_ERR_UNSUPPORTED),   # 64 heads x 2 positions > 64 columns
+    (dict(L=2, d=64), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(window=5, d=64), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(q=A + 4), kb.KVATTN_ERR_MISALIGNED),
+    (dict(out=A + 16), kb.KVATTN_ERR_INVALID_ARG),          # output overlaps q
+])
+def test_gqa_multi_rejects_bad_arguments(lib, kw, expected):
+    a = dict(q=A, k=2 * A, v=3 * A, lens=4 * A, T=4096, B=2, L=4, nq=32, nkv=8, d=128, window=0,
+             out=5 * A, lse=6 * A)
+    a.update(kw)
+    st = lib.kvattn_gqa_decode_multi(a["q"], a["k"], a["v"], a["lens"], a["T"], a["B"], a["L"], a["nq"], a["nkv"],
+                                     a["d"], 0.088, a["window"], a["out"], a["lse"], None)
+    assert st == expected
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     q = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
