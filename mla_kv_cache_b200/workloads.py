@@ -142,6 +142,41 @@ def make_gqa_inputs(cfg: GQAConfig, seed: int = 0, poison_tail: bool = False):
     return {"q": q, "k_cache": k, "v_cache": v, "seq_lens": lens}
 
 
+def quantize_e4m3(x, seq_lens=None, seq_axis=2):
+    """Synthesises an fp8 (E4M3) cache from a bf16 one: scale = max|x| / 448 (float32),
+    codes = the nearest E4M3 values of x / scale (PyTorch's conversion).  Rows past
+    seq_lens[b] (NaN in a poisoned cache) get the NaN code.  Returns (codes as a
+    float8_e4m3fn tensor, scale)."""
+    finite = x[~torch.isnan(x)] if torch.isnan(x).any() else x
+    amax = float(finite.abs().max().float()) if finite.numel() else 1.0
+    scale = float(torch.tensor(amax / 448.0 if amax > 0 else 1.0, dtype=torch.float32))
+    codes = torch.empty(x.shape, dtype=torch.float8_e4m3fn)
+    s32 = torch.tensor(scale, dtype=torch.float32)
+    for b in range(x.shape[0]):
+        xb = x[b].float() / s32
+        codes[b] = xb.clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+    if seq_lens is not None:
+        raw = codes.view(torch.uint8)
+        for b, n in enumerate(seq_lens.tolist()):
+            idx = [b] + [slice(None)] * (x.dim() - 1)
+            idx[seq_axis] = slice(int(n), None)
+            raw[tuple(idx)] = 0x7F
+    return codes, scale
+
+
+def make_gqa_inputs_fp8(cfg: GQAConfig, seed: int = 0, poison_tail: bool = False):
+    """The bf16 workload of make_gqa_inputs (same draws), with its caches stored as
+    E4M3 codes and one float scale per cache tensor.  Returns dict(q, k_cache, v_cache,
+    seq_lens, k_scale, v_scale); the caches are float8_e4m3fn tensors."""
+    x = make_gqa_inputs(cfg, seed, poison_tail=False)
+    lens = x["seq_lens"] if poison_tail else None
+    k8, ks = quantize_e4m3(x["k_cache"], lens)
+    del x["k_cache"]
+    v8, vs = quantize_e4m3(x["v_cache"], lens)
+    del x["v_cache"]
+    return {"q": x["q"], "k_cache": k8, "v_cache": v8, "seq_lens": x["seq_lens"], "k_scale": ks, "v_scale": vs}
+
+
 def make_mla_inputs(cfg: MLAConfig, seed: int = 0, poison_tail: bool = False):
     """Returns dict(q_latent, q_rope, latent_cache, rope_cache, seq_lens) (CPU tensors)."""
     g = torch.Generator().manual_seed(seed)

@@ -61,6 +61,15 @@ def load(mutant=0, out_dir=None):
         lib.kvo_rope.argtypes = [dp, ci, ci, ip, cd, ci, dp]
         lib.kvo_rope.restype = ci
         lib.kvo_num_threads.restype = ci
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        lib.kvo_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.kvo_e4m3_value.restype = cd
+        lib.kvo_e4m3_dequant.argtypes = [u8p, ctypes.c_longlong, cd, dp]
+        lib.kvo_e4m3_dequant.restype = ci
+        lib.kvo_e4m3_code.argtypes = [ctypes.c_float]
+        lib.kvo_e4m3_code.restype = ctypes.c_uint8
+        lib.kvo_e4m3_quant.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_longlong, ctypes.c_float, u8p]
+        lib.kvo_e4m3_quant.restype = ci
         lib.kvo_mutant.restype = ci
         _LIBS[key] = lib
         return lib
@@ -228,6 +237,71 @@ def gqa_decode_multi(q, k_cache, v_cache, seq_lens, scale, window=0, lib=None):
         n = max(T, 1)
         o, l = gqa_decode_multi_f64(q[b:b + 1], k_cache[b:b + 1, :, :n], v_cache[b:b + 1, :, :n],
                                     [T], scale, window, lib=lib)
+        outs.append(o[0])
+        lses.append(l[0])
+    return np.stack(outs), np.stack(lses)
+
+
+def _codes(x):
+    """E4M3 codes as a contiguous uint8 array (torch float8_e4m3fn / uint8 tensor, or array)."""
+    if hasattr(x, "detach"):
+        import torch
+        x = x.detach().to("cpu")
+        if x.dtype != torch.uint8:
+            x = x.view(torch.uint8)
+        x = x.numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.uint8))
+
+
+def e4m3_value(code, lib=None):
+    """Value of one E4M3 code (fp64)."""
+    return float((lib or load()).kvo_e4m3_value(int(code) & 0xFF))
+
+
+def e4m3_dequant(codes, scale, lib=None):
+    """Dequantised cache: value(code) * scale, fp64, same shape."""
+    lib = lib or load()
+    c = _codes(codes)
+    out = np.empty(c.shape, dtype=np.float64)
+    st = lib.kvo_e4m3_dequant(_ptr(c, ctypes.c_uint8), c.size, float(scale), _ptr(out, ctypes.c_double))
+    if st != 0:
+        raise ValueError("kvo_e4m3_dequant: bad arguments")
+    return out
+
+
+def e4m3_quant(x, scale, lib=None):
+    """E4M3 codes of float32(x) / float32(scale) (ties to even, saturated), uint8."""
+    lib = lib or load()
+    xf = x.detach().to("cpu").float().numpy() if hasattr(x, "detach") else np.asarray(x, dtype=np.float32)
+    xf = np.ascontiguousarray(xf, dtype=np.float32)
+    out = np.empty(xf.shape, dtype=np.uint8)
+    st = lib.kvo_e4m3_quant(_ptr(xf, ctypes.c_float), xf.size, float(np.float32(scale)), _ptr(out, ctypes.c_uint8))
+    if st != 0:
+        raise ValueError("kvo_e4m3_quant: bad arguments")
+    return out
+
+
+def gqa_decode_fp8(q, k_codes, v_codes, seq_lens, scale, k_scale, v_scale, window=0, lib=None):
+    """Decode over an E4M3 cache: attention on the dequantised keys value(k) * k_scale and
+    values value(v) * v_scale.  q [B, n_q, d] (single token: returns out [B, n_q, d],
+    lse [B, n_q]) or [B, L, n_q, d] (L new tokens, causal, optional window: returns
+    [B, L, n_q, d], [B, L, n_q]).  Caches [B, n_kv, T_max, d] of codes; only the first
+    seq_lens[b] rows of each sequence are read."""
+    lib = lib or load()
+    lens = _lens(seq_lens)
+    kc, vc = _codes(k_codes), _codes(v_codes)
+    T_max = kc.shape[2]
+    multi = len(q.shape) == 4
+    outs, lses = [], []
+    for b in range(q.shape[0]):
+        T = int(min(max(int(lens[b]), 0), T_max))
+        n = max(T, 1)
+        kb = e4m3_dequant(kc[b:b + 1, :, :n], k_scale, lib=lib)
+        vb = e4m3_dequant(vc[b:b + 1, :, :n], v_scale, lib=lib)
+        if multi:
+            o, l = gqa_decode_multi_f64(q[b:b + 1], kb, vb, [T], scale, window, lib=lib)
+        else:
+            o, l = gqa_decode_f64(q[b:b + 1], kb, vb, np.array([T], dtype=np.int32), scale, lib=lib)
         outs.append(o[0])
         lses.append(l[0])
     return np.stack(outs), np.stack(lses)

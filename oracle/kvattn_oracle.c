@@ -316,6 +316,79 @@ int kvo_rope(const double *x, int n, int d, const int32_t *pos, double base, int
     return 0;
 }
 
+/*
+ * Quantised (fp8) KV cache.  The pages list quantised caches among what the libraries
+ * build around the attention module ("Attention variants: MQA, GQA, and MLA", section
+ * "Against the real libraries"); stored in 8 bits, the cache a decode step reads halves.
+ * They fix no format.  Reading: the 8-bit floating-point format
+ * E4M3 (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0
+ * holds the subnormals m * 2^-9; no infinities; S.1111.111 is the only NaN, so the
+ * largest finite magnitude is 1.75 * 2^8 = 448), with one float scale per cache tensor:
+ * the cached value is  code_value * scale.
+ */
+
+/* Value of one E4M3 code, from the format's definition. */
+double kvo_e4m3_value(uint8_t c) {
+    const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+#if KVO_MUTANT == 11
+    if (e == 0) mag = ldexp(1.0 + m / 8.0, -6);       /* planted mistake: no subnormals */
+#else
+    if (e == 0) mag = ldexp((double)m, -9);           /* subnormal: m/8 * 2^(1-7) */
+#endif
+#if KVO_MUTANT == 12
+    else mag = ldexp(1.0 + m / 8.0, e - 8);           /* planted mistake: bias 8 */
+#else
+    else mag = ldexp(1.0 + m / 8.0, e - 7);
+#endif
+    return sign ? -mag : mag;
+}
+
+/* out[i] = value(in[i]) * scale (the dequantised cache), n codes. */
+int kvo_e4m3_dequant(const uint8_t *in, long long n, double scale, double *out) {
+    if (n < 0) return 1;
+#pragma omp parallel for schedule(static)
+    for (long long i = 0; i < n; ++i) out[i] = kvo_e4m3_value(in[i]) * scale;
+    return 0;
+}
+
+/* Nearest E4M3 code to the float x, ties to the even code, magnitudes past the largest
+ * finite value saturated to +-448; NaN gives the NaN code.  (Quantising a value for the
+ * cache: the caller has already divided it by the tensor's scale in float.) */
+uint8_t kvo_e4m3_code(float x) {
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    const double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal range: spacing 2^-9; m = 8 is the smallest normal, code 0x08 */
+        const double m = rint(a / ldexp(1.0, -9));   /* round half to even (default mode) */
+        return sign | (uint8_t)m;
+    }
+    int e = (int)floor(log2(a));
+    if (ldexp(1.0, e) > a) --e;                        /* guard log2 rounding */
+    if (ldexp(1.0, e + 1) <= a) ++e;
+#if KVO_MUTANT == 13
+    double n = floor(a / ldexp(1.0, e - 3) + 0.5);     /* planted mistake: ties away from zero */
+#else
+    double n = rint(a / ldexp(1.0, e - 3));            /* 8 .. 16 steps of 2^(e-3) */
+#endif
+    if (n >= 16.0) { n = 8.0; ++e; }
+    if (e > 8 || (e == 8 && n > 14.0)) return sign | 0x7E;
+    return sign | (uint8_t)(((e + 7) << 3) | ((int)n - 8));
+}
+
+/* codes[i] = kvo_e4m3_code(x[i] / scale), the division in float. */
+int kvo_e4m3_quant(const float *x, long long n, float scale, uint8_t *codes) {
+    if (n < 0 || !(scale > 0.0f)) return 1;
+    for (long long i = 0; i < n; ++i) {
+        const float y = x[i] / scale;
+        codes[i] = kvo_e4m3_code(y);
+    }
+    return 0;
+}
+
 /* Number of OpenMP threads a parallel region of this library uses. */
 int kvo_num_threads(void) {
     int n = 1;

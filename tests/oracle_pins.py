@@ -392,10 +392,96 @@ def pin_multi_token_reductions(lib):
     assert np.all(np.isneginf(lse[1])) and np.all(out[1] == 0)
 
 
+# --------------------------------------------------------------------------------------
+# Quantised (fp8) cache ("Attention variants: MQA, GQA, and MLA", section "Against the
+# real libraries": quantised caches).  The codes follow the E4M3 format's definition:
+# hand-worked values, every code against PyTorch's float8_e4m3fn conversion, the
+# encoder's ties and saturation by hand, and the fp8 decode equal to the (separately
+# pinned) decode over caches dequantised by PyTorch.
+# --------------------------------------------------------------------------------------
+E4M3_BY_HAND = {
+    0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x0F: 1.875 * 2.0 ** -6,
+    0x30: 0.5, 0x38: 1.0, 0x39: 1.125, 0x3F: 1.875, 0x40: 2.0, 0x78: 256.0, 0x7E: 448.0,
+    0x80: -0.0, 0xB8: -1.0, 0xFE: -448.0,
+}
+
+
+def pin_e4m3_codes(lib):
+    for c, v in E4M3_BY_HAND.items():
+        got = oracle.e4m3_value(c, lib=lib)
+        assert got == v and math.copysign(1.0, got) == math.copysign(1.0, v), (hex(c), got, v)
+    assert math.isnan(oracle.e4m3_value(0x7F, lib=lib)) and math.isnan(oracle.e4m3_value(0xFF, lib=lib))
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.e4m3_dequant(codes, 1.0, lib=lib)
+    same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+    assert same.all(), np.nonzero(~same)
+
+
+def pin_e4m3_encoder(lib):
+    finite = [c for c in range(256) if c not in (0x7F, 0xFF)]
+    # every finite value encodes to its own code
+    vals = np.array([oracle.e4m3_value(c, lib=lib) for c in finite], np.float32)
+    assert (oracle.e4m3_quant(vals, 1.0, lib=lib) == np.array(finite, np.uint8)).all()
+    # midpoints between neighbours go to the even code; saturation; NaN
+    hand = {1.0625: 0x38, 1.1875: 0x3A, 3 * 2.0 ** -10: 0x02, 2.0 ** -10: 0x00, 1.5 * 2.0 ** -9: 0x02,
+            440.0: 0x7E, 448.0: 0x7E, 449.0: 0x7E, 1e30: 0x7E, -1e30: 0xFE, -1.0625: 0xB8, 17.0: 0x58, 19.0: 0x5A}
+    for x, c in hand.items():
+        got = int(oracle.e4m3_quant(np.array([x], np.float32), 1.0, lib=lib)[0])
+        assert got == c, (x, hex(got), hex(c))
+    assert int(oracle.e4m3_quant(np.array([np.nan], np.float32), 1.0, lib=lib)[0]) == 0x7F
+    # in range, against PyTorch's round-to-nearest-even conversion
+    x = torch.from_numpy(_rng(51).standard_normal(20000).astype(np.float32) * 60.0)
+    x = x[x.abs() < 448]
+    assert (oracle.e4m3_quant(x, 1.0, lib=lib) == x.to(torch.float8_e4m3fn).view(torch.uint8).numpy()).all()
+    # the division by the scale is taken in float
+    s = np.float32(0.0371)
+    y = (x.numpy() / s).astype(np.float32)
+    y = np.clip(y, -447, 447)
+    xs = (torch.from_numpy(y) * torch.tensor(float(s))).numpy()
+    want = torch.from_numpy((xs / s).astype(np.float32)).clamp(-448, 448).to(torch.float8_e4m3fn)
+    assert (oracle.e4m3_quant(xs, s, lib=lib) == want.view(torch.uint8).numpy()).all()
+
+
+def _fp8_case(seed, B=2, n_q=8, n_kv=2, d=16, T=15):
+    r = _rng(seed)
+    q = r.standard_normal((B, n_q, d))
+    codes = r.integers(0, 256, size=(2, B, n_kv, T, d), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3C      # no NaN codes
+    return q, codes[0], codes[1]
+
+
+def _torch_dequant(codes, s):
+    return torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy() * s
+
+
+def pin_fp8_decode_on_dequantised_cache(lib):
+    q, kc, vc = _fp8_case(52)
+    lens = np.array([15, 6], np.int32)
+    for ks, vs in ((0.125, 4.0), (0.0371, 0.0213), (1.0, 1.0)):
+        out, lse = oracle.gqa_decode_fp8(q, kc, vc, lens, 0.3, ks, vs, lib=lib)
+        ro, rl = oracle.gqa_decode_f64(q, _torch_dequant(kc, ks), _torch_dequant(vc, vs), lens, 0.3, lib=lib)
+        assert np.allclose(out, ro, rtol=1e-13, atol=1e-13) and np.allclose(lse, rl, rtol=1e-13, atol=1e-13), (ks, vs)
+    # the value scale scales the output and leaves lse alone; the key scale is a score scale
+    o1, l1 = oracle.gqa_decode_fp8(q, kc, vc, lens, 0.3, 0.5, 1.0, lib=lib)
+    o2, l2 = oracle.gqa_decode_fp8(q, kc, vc, lens, 0.3, 0.5, 8.0, lib=lib)
+    assert np.allclose(o2, 8.0 * o1, rtol=1e-13, atol=1e-13) and np.array_equal(l1, l2)
+    o3, l3 = oracle.gqa_decode_fp8(q, kc, vc, lens, 0.15, 1.0, 1.0, lib=lib)
+    assert np.allclose(o1, o3, rtol=1e-13, atol=1e-13) and np.allclose(l1, l3, rtol=1e-13, atol=1e-13)
+    # several new tokens: the multi-token oracle on the dequantised cache
+    r = _rng(53)
+    qm = r.standard_normal((2, 3, 8, 16))
+    out, lse = oracle.gqa_decode_fp8(qm, kc, vc, lens, 0.3, 0.25, 2.0, window=4, lib=lib)
+    ro, rl = oracle.gqa_decode_multi_f64(qm, _torch_dequant(kc, 0.25), _torch_dequant(vc, 2.0), lens, 0.3,
+                                         window=4, lib=lib)
+    assert np.allclose(out, ro, atol=1e-13) and np.allclose(lse, rl, atol=1e-13)
+
+
 ALL_PINS = [
     pin_gqa_equals_mha_on_repeated_kv, pin_sdpa_enable_gqa, pin_closed_forms,
     pin_empty_sequence, pin_brute_force_tiny, pin_split_merge, pin_permutation_invariance,
     pin_scale_equivariance, pin_mla_absorbed_equals_explicit, pin_mla_matches_sdpa,
     pin_mla_without_rope_is_mqa, pin_rope_identity_and_hand_cases, pin_rope_invariants,
-    pin_multi_token_sdpa, pin_multi_token_reductions,
+    pin_multi_token_sdpa, pin_multi_token_reductions, pin_e4m3_codes, pin_e4m3_encoder,
+    pin_fp8_decode_on_dequantised_cache,
 ]
