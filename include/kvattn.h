@@ -140,6 +140,43 @@ int kvattn_gqa_decode_multi(const uint16_t *q, const uint16_t *k_cache, const ui
                             float *out, float *lse, void *stream);
 
 /*
+ * Decode over a quantised (fp8) KV cache.  The pages list quantised caches among what the
+ * libraries build around the attention module ("Attention variants: MQA, GQA, and MLA",
+ * section "Against the real libraries"); at one byte per cached value the cache a decode
+ * step reads halves.  The format is E4M3 (1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits; largest finite magnitude 448; codes 0x7F / 0xFF are NaN) with one
+ * float scale per cache tensor: the cached key is value(code) * k_scale, the value
+ * value(code) * v_scale.  The result is attention on those dequantised values, as
+ * kvattn_gqa_decode_multi computes it (q_len = 1, window = 0: kvattn_gqa_decode).
+ *   q           device bf16 [batch, q_len, n_q_heads, head_dim]
+ *   k_cache, v_cache  device E4M3 codes (one byte each)
+ *               [batch, n_kv_heads, max_seq_len, head_dim]
+ *   k_scale, v_scale  finite, > 0
+ *   out, lse    device fp32 [batch, q_len, n_q_heads, head_dim], [batch, q_len, n_q_heads]
+ * head_dim must be 128 and (n_q_heads / n_kv_heads) * q_len <= 64 (else
+ * KVATTN_ERR_UNSUPPORTED); everything else as for kvattn_gqa_decode_multi.  The query
+ * and the softmax weights enter the tensor-core products as two E4M3 parts each (~8
+ * significant bits), the codes exactly; accumulation is fp32.  Codes past a sequence's
+ * length are never read.
+ */
+int kvattn_gqa_decode_fp8(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                          const int32_t *seq_lens, int max_seq_len, int batch, int q_len,
+                          int n_q_heads, int n_kv_heads, int head_dim, float scale, float k_scale,
+                          float v_scale, int window, float *out, float *lse, void *stream);
+
+/*
+ * kvattn_gqa_decode_fp8 for one new token per sequence over a paged E4M3 cache:
+ * k_pages, v_pages [num_pages, n_kv_heads, page_size, head_dim] codes, block_table and
+ * seq_lens as for kvattn_gqa_decode_paged, page_size a multiple of 128; q [batch,
+ * n_q_heads, head_dim] bf16, out [batch, n_q_heads, head_dim], lse [batch, n_q_heads].
+ */
+int kvattn_gqa_decode_fp8_paged(const uint16_t *q, const uint8_t *k_pages, const uint8_t *v_pages,
+                                const int32_t *block_table, const int32_t *seq_lens, int num_pages,
+                                int page_size, int max_pages_per_seq, int batch, int n_q_heads,
+                                int n_kv_heads, int head_dim, float scale, float k_scale, float v_scale,
+                                float *out, float *lse, void *stream);
+
+/*
  * kvattn_gqa_decode over a paged KV cache: the cache is a pool of pages and each
  * sequence lists its pages in a block table (the serving-engine layout the pages name,
  * "Attention variants: MQA, GQA, and MLA", section "Against the real libraries": vLLM's

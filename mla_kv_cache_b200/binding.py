@@ -41,6 +41,15 @@ _SIGNATURES = {
                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_void_p,
                                                ctypes.c_void_p, ctypes.c_void_p]),
+    "kvattn_gqa_decode_fp8": (ctypes.c_int, [_c_u16p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                             ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "kvattn_gqa_decode_fp8_paged": (ctypes.c_int, [_c_u16p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                   ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "kvattn_gqa_decode_paged": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, ctypes.c_void_p,
                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
@@ -314,6 +323,73 @@ def kvattn_gqa_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale, o
                                        _stream_handle(stream))
     if st != KVATTN_OK:
         raise KvattnError(st, "kvattn_gqa_decode_paged")
+    return out, lse
+
+
+def _check_e4m3(t, name, shape):
+    """An E4M3 cache: float8_e4m3fn or uint8 codes."""
+    import torch
+    if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise ValueError(f"{name} must be float8_e4m3fn (or uint8 codes), got {t.dtype}")
+    _check(t, name, t.dtype, shape)
+
+
+def kvattn_gqa_decode_fp8(q, k_cache, v_cache, seq_lens, scale, k_scale, v_scale, window=0, out=None, lse=None,
+                          stream=None):
+    """Decode over an E4M3 cache (include/kvattn.h, kvattn_gqa_decode_fp8): q [B, n_q, d]
+    (one new token) or [B, L, n_q, d] bf16, caches [B, n_kv, T, d] float8_e4m3fn (or
+    uint8 codes), value = code * k_scale / v_scale.  Returns (out, lse) shaped like q
+    without / with its L axis, fp32."""
+    import torch
+    single = q.dim() == 3
+    q4 = q.unsqueeze(1) if single else q
+    B, L, n_q, d = q4.shape
+    n_kv, T = k_cache.shape[1], k_cache.shape[2]
+    _check(q4, "q", torch.bfloat16)
+    _check_e4m3(k_cache, "k_cache", (B, n_kv, T, d))
+    _check_e4m3(v_cache, "v_cache", (B, n_kv, T, d))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    shape_o, shape_l = ((B, n_q, d), (B, n_q)) if single else ((B, L, n_q, d), (B, L, n_q))
+    if out is None:
+        out = torch.empty(shape_o, dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty(shape_l, dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, shape_o)
+    _check(lse, "lse", torch.float32, shape_l)
+    st = lib().kvattn_gqa_decode_fp8(q4.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seq_lens.data_ptr(),
+                                     T, B, L, n_q, n_kv, d, float(scale), float(k_scale), float(v_scale),
+                                     int(window), out.data_ptr(), lse.data_ptr(), _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_gqa_decode_fp8")
+    return out, lse
+
+
+def kvattn_gqa_decode_fp8_paged(q, k_pages, v_pages, block_table, seq_lens, scale, k_scale, v_scale, out=None,
+                                lse=None, stream=None):
+    """kvattn_gqa_decode_fp8 over a paged E4M3 cache (include/kvattn.h,
+    kvattn_gqa_decode_fp8_paged): k_pages / v_pages [num_pages, n_kv, page_size, d]
+    codes, block_table [B, max_pages] int32.  Returns (out [B, n_q, d], lse [B, n_q])."""
+    import torch
+    B, n_q, d = q.shape
+    P, n_kv, S = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    M = block_table.shape[1]
+    _check(q, "q", torch.bfloat16)
+    _check_e4m3(k_pages, "k_pages", (P, n_kv, S, d))
+    _check_e4m3(v_pages, "v_pages", (P, n_kv, S, d))
+    _check(block_table, "block_table", torch.int32, (B, M))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, n_q, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, n_q), dtype=torch.float32, device=q.device)
+    _check(out, "out", torch.float32, (B, n_q, d))
+    _check(lse, "lse", torch.float32, (B, n_q))
+    st = lib().kvattn_gqa_decode_fp8_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                           block_table.data_ptr(), seq_lens.data_ptr(), P, S, M, B, n_q, n_kv, d,
+                                           float(scale), float(k_scale), float(v_scale), out.data_ptr(),
+                                           lse.data_ptr(), _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_gqa_decode_fp8_paged")
     return out, lse
 
 

@@ -45,6 +45,7 @@ struct GqaParams {
     int page_size;              // rows per page (T_max when contiguous)
     int q_len;                  // new tokens per sequence (1: single-token decode)
     int window;                 // sliding window in tokens (0: none)
+    float k_scale, v_scale;     // E4M3 cache: value = code * scale (1 for a bf16 cache)
 };
 
 template <int D, int MT>

@@ -35,6 +35,20 @@
 //                       weights keep ~16 significant bits.  The running max moves lazily:
 //                       only when a head's tile maximum exceeds it by more than 2^8, and
 //                       then that head's column of O^T and its row sums are rescaled.
+// E4M3 cache (KV8).  A tile of K or V is one 128-byte-swizzled box of [128 tokens x 128
+// codes]; the ring holds six 32 KB stages.  Both products run as kind::f8f6f4 MMAs on
+// E4M3 operands straight from the TMA'd tiles, so nothing is converted per tile:
+//   - the query block is split, once per piece and in place by the MMA warp, into an
+//     E4M3 high part and an E4M3 remainder after scaling by 2^e (the block's largest
+//     magnitude lands in [128, 256)); K times both parts, summed in the accumulator,
+//     is K times the query to ~8 significant bits.  The score scale folds in the key
+//     scale and 2^-e;
+//   - P^T is written as an E4M3 high part and remainder of 64 * 2^(s - m) (the running
+//     max moves once a head's tile maximum exceeds it by 2^2, so the weights stay in
+//     E4M3's range), in the plain (unswizzled) MN-major layout: 16 heads x 128 tokens
+//     per 2 KB block, one 16-byte row per token;
+//   - V^T is the V tile read MN-major (128 dimensions = one 128-byte row per token);
+//     the value scale and 1/64 fold into the final 1 / row sum.
 // Each thread keeps its token slot's partial row sums per head; at the end of a piece
 // they are reduced the same way and every thread writes its output dimension of every
 // head (final output, or the worker's partial for the split combine).
@@ -53,35 +67,49 @@ namespace gqatc {
 constexpr int TILE = 128;                 // tokens per tile = MMA M
 constexpr int D = 128;                    // head dimension
 constexpr int HB = 64;                    // query heads per unit (value-product N)
-constexpr int NST = 3;                    // pipeline stages
-constexpr int CHUNK = TILE * 128;         // one [128 tokens x 64] bf16 box: 16 KB
-constexpr int KV_BYTES = 2 * CHUNK;       // a K or V tile: 32 KB
-constexpr int STAGE = 2 * KV_BYTES;       // K then V: 64 KB
+constexpr int CHUNK = TILE * 128;         // one [128 tokens x 128 bytes] box: 16 KB
+constexpr int RING = 12 * CHUNK;          // the stage ring: 192 KB
 constexpr int QREGION = 2 * HB * 128;     // query blocks: 16 KB (one of 64 heads or two of <= 32)
 constexpr int NTHREADS = 192;             // producer, MMA, 4 softmax warps
 constexpr int NSOFT = 128;
 constexpr uint32_t TM_S = 0;              // two 64-column score buffers
 constexpr uint32_t TM_O = 128;            // O^T: 64 columns
 constexpr uint32_t TM_COLS = 256;
-constexpr float RESCALE_LOG2 = 8.f;
+constexpr int NST_MAX = 6;
+constexpr int P8_LO = 8192;               // E4M3 P^T: remainder after the high part (K half of a stage)
+constexpr float P8_LOG2 = 6.f;            // E4M3 P^T holds 2^6 * 2^(s - m)
+
+// Per cache type: bf16 (a tile is two [128 x 64] boxes, 3 stages of 64 KB) or E4M3
+// (one [128 x 128] box, 6 stages of 32 KB).
+template <bool KV8>
+struct Kv {
+    static constexpr int KV_BYTES = KV8 ? CHUNK : 2 * CHUNK;     // a K or V tile
+    static constexpr int STAGE = 2 * KV_BYTES;                   // K then V
+    static constexpr int NST = RING / STAGE;
+    // the running max moves when a head's tile maximum exceeds it by 2^RESCALE
+    static constexpr float RESCALE = KV8 ? 2.f : 8.f;
+    static_assert(NST <= NST_MAX, "stage barriers");
+};
 
 constexpr int OFF_ST = 0;
-constexpr int OFF_Q = OFF_ST + NST * STAGE;        // 196608
+constexpr int OFF_Q = OFF_ST + RING;               // 196608
 constexpr int OFF_RED = OFF_Q + QREGION;              // [3][4][64] fp32: tile slots 0/1, piece end
 constexpr int OFF_MS = OFF_RED + 3 * 4 * HB * 4;   // [2][64] running max per head
 constexpr int OFF_AS = OFF_MS + 2 * HB * 4;        // [2][64] rescale factor per head
 constexpr int OFF_NF = OFF_AS + 2 * HB * 4;        // [2][64] bytes: head rescaled this tile
 constexpr int OFF_LINV = OFF_NF + 2 * HB;          // [64] 1 / row sum
-constexpr int OFF_BARS = OFF_LINV + HB * 4;
+constexpr int OFF_QS = OFF_LINV + HB * 4;          // [2] fp32: 2^-e of each E4M3 query buffer
+constexpr int OFF_BARS = OFF_QS + 16;
 constexpr int OFF_TMEMPTR = OFF_BARS + 256;
 constexpr int OFF_ABORT = OFF_TMEMPTR + 16;
 constexpr int OFF_PREFIX = OFF_ABORT + 16;
 constexpr int smem_bytes(int B) { return 1024 + OFF_PREFIX + (B + 1) * 4; }
 
 struct Bars {
-    uint64_t full[NST], empty[NST];
+    uint64_t full[NST_MAX], empty[NST_MAX];
     uint64_t qfull[2];    // a query block landed (buffer = piece % NQB)
     uint64_t qempty[2];   // every score MMA of that piece has read it
+    uint64_t qconv[2];    // E4M3 cache: the MMA warp has split that block (and its 2^-e)
     uint64_t sready[2];   // scores of a tile in TMEM buffer (tile & 1)
     uint64_t sfree[2];    // the softmax threads have read that buffer
     uint64_t pready[2];   // P^T written (and O^T rescaled): the value product may run
@@ -173,10 +201,12 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[NQ]) 
     }
 }
 // ------------------------------------------------------------------ producer (warp 0, lane 0)
-template <int NR>
+template <int NR, bool KV8>
 __device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *kmap, const CUtensorMap *vmap,
                                          const CUtensorMap *qmap, const Ctx &c) {
     using C = Cfg<NR>;
+    using L = Kv<KV8>;
+    constexpr int NST = L::NST;
     Bars *bars = c.bars;
     const uint64_t pol = l2_policy_evict_first();
     int k = 0, pi = 0;
@@ -210,15 +240,21 @@ __device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *
             const int s = k % NST;
             const uint32_t ph = (uint32_t)(k / NST) & 1u;
             if (!mbar_wait(&bars->empty[s], ph ^ 1u, FLAG_EMPTY_WAIT, c.abort_flag)) { ok = false; break; }
-            mbar_arrive_expect_tx(&bars->full[s], STAGE);
+            mbar_arrive_expect_tx(&bars->full[s], L::STAGE);
             const TileSrc src = tile_source(p.block_table, p.max_pages, p.page_size, pc.b, lt, TILE, len, start);
             const int y = src.y;
             const int z = src.page * p.n_kv + j;
-            uint8_t *st = c.smem + OFF_ST + s * STAGE;
-            tma_load_3d(st, kmap, &bars->full[s], 0, y, z, pol);
-            tma_load_3d(st + CHUNK, kmap, &bars->full[s], 64, y, z, pol);
-            tma_load_3d(st + KV_BYTES, vmap, &bars->full[s], 0, y, z, pol);
-            tma_load_3d(st + KV_BYTES + CHUNK, vmap, &bars->full[s], 64, y, z, pol);
+            uint8_t *st = c.smem + OFF_ST + s * L::STAGE;
+            if constexpr (KV8) {
+                // one 128-byte box per tile (the map sees a row as 64 two-byte elements)
+                tma_load_3d(st, kmap, &bars->full[s], 0, y, z, pol);
+                tma_load_3d(st + L::KV_BYTES, vmap, &bars->full[s], 0, y, z, pol);
+            } else {
+                tma_load_3d(st, kmap, &bars->full[s], 0, y, z, pol);
+                tma_load_3d(st + CHUNK, kmap, &bars->full[s], 64, y, z, pol);
+                tma_load_3d(st + L::KV_BYTES, vmap, &bars->full[s], 0, y, z, pol);
+                tma_load_3d(st + L::KV_BYTES + CHUNK, vmap, &bars->full[s], 64, y, z, pol);
+            }
         }
     }
     if (!ok) {
@@ -230,42 +266,161 @@ __device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *
     }
 }
 
+// ------------------------------------------------------------------ E4M3 query split (warp 1)
+// Two bf16 values (one 32-bit word) as float.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// E4M3 high part and remainder of two values (already scaled into E4M3's range): the
+// pair goes through f16 (exact for the 8-bit bf16 significands scaled by a power of
+// two), the high part is the nearest E4M3 pair, the remainder the nearest E4M3 pair
+// to what is left (exact in f16).  Element order is kept (x in the low byte).
+__device__ __forceinline__ void split_e4m3x2(float x, float y, uint16_t &hi, uint16_t &lo) {
+    const __half2 h = __floats2half2_rn(x, y);
+    const __half2_raw hr = h;
+    hi = __nv_cvt_halfraw2_to_fp8x2(hr, __NV_SATFINITE, __NV_E4M3);
+    const __half2 back = __half2(__nv_cvt_fp8x2_to_halfraw2(hi, __NV_E4M3));
+    const __half2_raw rr = __hsub2(h, back);
+    lo = __nv_cvt_halfraw2_to_fp8x2(rr, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Splits the bf16 query block at qbase (two 128-byte-swizzled [NQ x 64] boxes) in place
+// into two E4M3 blocks of [NQ x 128] in the same swizzle: the high parts where the first
+// box was, the remainders where the second was.  Every value is first multiplied by
+// 2^e, e chosen so that the block's largest magnitude lands in [128, 256).  Run by the
+// 32 lanes of one warp; returns 2^-e.  Row h of both boxes holds only row h's data, so
+// rows are independent: lanes take eight rows at a time (four lanes a row, 32
+// dimensions each), read everything they need, meet, then write.
+template <int NQ>
+__device__ __forceinline__ float split_query_e4m3(uint8_t *qbase, int lane) {
+    constexpr int QCHUNK = NQ * 128;
+    float amax = 0.f;
+    const uint4 *src = reinterpret_cast<const uint4 *>(qbase);
+    for (int i = lane; i < 2 * QCHUNK / 16; i += 32) {
+        const uint4 u = src[i];
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[t])), fabsf(bf16_hi(w[t]))));
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    int e = 0;
+    if (amax > 0.f && amax <= 3.0e38f) {
+        int x;
+        frexpf(amax, &x);                 // amax in [2^(x-1), 2^x)
+        e = min(max(8 - x, -126), 126);
+    }
+    const float up = __int_as_float((127 + e) << 23);
+    const float down = __int_as_float((127 - e) << 23);
+    const int m = lane & 3;               // dimensions 32m .. 32m + 31
+    const int chunk = m >> 1;             // in bf16 box m / 2, 16-byte units 4 (m & 1) .. + 3
+#pragma unroll 1
+    for (int g0 = 0; g0 < NQ; g0 += 8) {
+        const int h = g0 + (lane >> 2);
+        const int sw = h & 7;
+        const uint8_t *row = qbase + chunk * QCHUNK + h * 128;
+        uint4 in[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) in[j] = *reinterpret_cast<const uint4 *>(row + (((4 * (m & 1) + j) ^ sw) << 4));
+        __syncwarp();
+        uint32_t hw[8], lw[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t w[4] = {in[j].x, in[j].y, in[j].z, in[j].w};
+#pragma unroll
+            for (int t = 0; t < 4; t += 2) {
+                uint16_t h0, l0, h1, l1;
+                split_e4m3x2(bf16_lo(w[t]) * up, bf16_hi(w[t]) * up, h0, l0);
+                split_e4m3x2(bf16_lo(w[t + 1]) * up, bf16_hi(w[t + 1]) * up, h1, l1);
+                hw[2 * j + t / 2] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                lw[2 * j + t / 2] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+            }
+        }
+        // E4M3 16-byte units 2m and 2m + 1 of row h (dimensions 32m .. 32m + 31)
+        uint8_t *hrow = qbase + h * 128;
+        uint8_t *lrow = qbase + QCHUNK + h * 128;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int slot = ((2 * m + u) ^ sw) << 4;
+            *reinterpret_cast<uint4 *>(hrow + slot) = make_uint4(hw[4 * u], hw[4 * u + 1], hw[4 * u + 2], hw[4 * u + 3]);
+            *reinterpret_cast<uint4 *>(lrow + slot) = make_uint4(lw[4 * u], lw[4 * u + 1], lw[4 * u + 2], lw[4 * u + 3]);
+        }
+        __syncwarp();
+    }
+    return down;
+}
+
 // ------------------------------------------------------------------ MMA issuer (warp 1, lane 0)
 // Score product of tile kt into TMEM buffer (kt & 1).  The caller has seen the tile
 // land and the buffer freed.
-template <int NR>
+template <int NR, bool KV8>
 __device__ __forceinline__ void issue_scores(const Ctx &c, int kt, int qbuf) {
     using C = Cfg<NR>;
-    const int s = kt % NST, sb = kt & 1;
+    using L = Kv<KV8>;
+    const int s = kt % L::NST, sb = kt & 1;
     tc_fence_after();
-    constexpr uint32_t idesc = idesc_f16_major(128, Cfg<NR>::NQ, 1, 1, 0, 0);
-    const uint32_t st = smem_u32(c.smem + OFF_ST + s * STAGE);
+    const uint32_t st = smem_u32(c.smem + OFF_ST + s * L::STAGE);
     const uint32_t qb = smem_u32(c.smem + OFF_Q + qbuf * C::QBLOCK);
+    if constexpr (KV8) {
+        // K (E4M3, [128 tokens x 128], K-major) times the query's high part, then its
+        // remainder: 4 + 4 MMAs of K = 32
+        constexpr uint32_t idesc = idesc_e4m3(128, Cfg<NR>::NQ, 0, 0);
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t blk = kk >> 2, in = (kk & 3) * 32;
-        const uint64_t a = smem_desc_sw128(st + blk * CHUNK + in, 16, 1024);
-        const uint64_t b = smem_desc_sw128(qb + blk * C::QCHUNK + in, 16, 1024);
-        umma_ss(c.tmem + TM_S + 64 * sb, a, b, idesc, kk > 0 ? 1u : 0u);
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+            for (int kk = 0; kk < D / 32; ++kk) {
+                const uint64_t a = smem_desc_sw128(st + kk * 32, 16, 1024);
+                const uint64_t b = smem_desc_sw128(qb + part * C::QCHUNK + kk * 32, 16, 1024);
+                umma_ss_f8(c.tmem + TM_S + 64 * sb, a, b, idesc, (part | kk) ? 1u : 0u);
+            }
+        }
+    } else {
+        constexpr uint32_t idesc = idesc_f16_major(128, Cfg<NR>::NQ, 1, 1, 0, 0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t blk = kk >> 2, in = (kk & 3) * 32;
+            const uint64_t a = smem_desc_sw128(st + blk * CHUNK + in, 16, 1024);
+            const uint64_t b = smem_desc_sw128(qb + blk * C::QCHUNK + in, 16, 1024);
+            umma_ss(c.tmem + TM_S + 64 * sb, a, b, idesc, kk > 0 ? 1u : 0u);
+        }
     }
     umma_commit(&c.bars->sready[sb]);
 }
 
 // Value product of tile kt into O^T (first = the piece's first tile: overwrite).
+template <int NR, bool KV8>
 __device__ __forceinline__ void issue_values(const Ctx &c, int kt, bool first) {
-    const int s = kt % NST;
-    constexpr uint32_t idesc_pv = idesc_f16_major(128, HB, 1, 1, 1, 1);
+    using L = Kv<KV8>;
+    const int s = kt % L::NST;
     tc_fence_after();
-    const uint32_t st = smem_u32(c.smem + OFF_ST + s * STAGE);
+    const uint32_t st = smem_u32(c.smem + OFF_ST + s * L::STAGE);
+    if constexpr (KV8) {
+        // V^T: M = 128 dimensions (one 128-byte row per token, MN-major), K = 32 tokens;
+        // P^T: N = NQ heads in 16-head blocks 2 KB apart, 16 bytes per token (plain
+        // MN-major: 8-token core matrices 128 bytes apart)
+        constexpr int NQ = Cfg<NR>::NQ;
+        constexpr uint32_t idesc_pv = idesc_e4m3(128, NQ, 1, 1);
 #pragma unroll
-    for (int kk = 0; kk < TILE / 16; ++kk) {
-        // V^T: M = 128 dimensions in two 64-wide blocks 16 KB apart, K = 16 tokens
-        const uint64_t a = smem_desc_sw128(st + KV_BYTES + kk * 2048, CHUNK, 1024);
-        // P^T high part and remainder (in the K half of the stage): N = 64 heads
-        const uint64_t bh = smem_desc_sw128(st + kk * 2048, CHUNK, 1024);
-        const uint64_t bl = smem_desc_sw128(st + CHUNK + kk * 2048, CHUNK, 1024);
-        umma_ss(c.tmem + TM_O, a, bh, idesc_pv, (!first || kk > 0) ? 1u : 0u);
-        umma_ss(c.tmem + TM_O, a, bl, idesc_pv, 1u);
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+            for (int kk = 0; kk < TILE / 32; ++kk) {
+                const uint64_t a = smem_desc_sw128(st + L::KV_BYTES + kk * 4096, CHUNK, 1024);
+                const uint64_t b = smem_desc_plain(st + part * P8_LO + kk * 512, 128, 2048);
+                umma_ss_f8(c.tmem + TM_O, a, b, idesc_pv, (!first || part || kk) ? 1u : 0u);
+            }
+        }
+    } else {
+        constexpr uint32_t idesc_pv = idesc_f16_major(128, HB, 1, 1, 1, 1);
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk) {
+            // V^T: M = 128 dimensions in two 64-wide blocks 16 KB apart, K = 16 tokens
+            const uint64_t a = smem_desc_sw128(st + L::KV_BYTES + kk * 2048, CHUNK, 1024);
+            // P^T high part and remainder (in the K half of the stage): N = 64 heads
+            const uint64_t bh = smem_desc_sw128(st + kk * 2048, CHUNK, 1024);
+            const uint64_t bl = smem_desc_sw128(st + CHUNK + kk * 2048, CHUNK, 1024);
+            umma_ss(c.tmem + TM_O, a, bh, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+            umma_ss(c.tmem + TM_O, a, bl, idesc_pv, 1u);
+        }
     }
     umma_commit(&c.bars->empty[s]);
     umma_commit(&c.bars->odone[kt & 1]);
@@ -276,9 +431,13 @@ __device__ __forceinline__ void issue_values(const Ctx &c, int kt, bool first) {
 // product (P^T written; at a piece start, O^T read out) may run and issues whatever is
 // ready.  Score products run at most two tiles ahead of value products -- the order a
 // blocking loop would give -- which keeps every tested barrier within one phase of the
-// tested parity.  Idle time is bounded like every other wait.
-template <int NR>
-__device__ __forceinline__ void mma_issuer(const GqaParams &p, const Ctx &c) {
+// tested parity.  Idle time is bounded like every other wait.  The whole warp runs the
+// loop over pieces (with an E4M3 cache its 32 lanes split each query block); lane 0
+// alone issues.
+template <int NR, bool KV8>
+__device__ __forceinline__ void mma_issuer(const GqaParams &p, const Ctx &c, int lane) {
+    using L = Kv<KV8>;
+    constexpr int NST = L::NST;
     Bars *bars = c.bars;
     int k = 0, pi = 0;
     for (long long pos = c.p0; pos < c.p1; ++pi) {
@@ -286,50 +445,64 @@ __device__ __forceinline__ void mma_issuer(const GqaParams &p, const Ctx &c) {
         pos = pc.ustart + pc.lt1;
         const int nt = pc.lt1 - pc.lt0;
         const int qb = pi % Cfg<NR>::NQB, qu = pi / Cfg<NR>::NQB;
-        if (!mbar_wait(&bars->qfull[qb], (uint32_t)qu & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
-        int nq = 0, nv = 0;
-        long long idle_since = clock64();
-        while (nv < nt) {
-            bool progressed = false;
-            if (nq < nt && nq < nv + 2) {
-                const int kt = k + nq;
-                if (mbar_test(&bars->full[kt % NST], (uint32_t)(kt / NST) & 1u) &&
-                    (kt < 2 || mbar_test(&bars->sfree[kt & 1], (uint32_t)((kt >> 1) - 1) & 1u))) {
-                    issue_scores<NR>(c, kt, qb);
-                    ++nq;
-                    if (nq == nt) umma_commit(&bars->qempty[qb]);
-                    progressed = true;
+        if (!warp_all(mbar_wait(&bars->qfull[qb], (uint32_t)qu & 1u, FLAG_FULL_WAIT, c.abort_flag))) return;
+        if constexpr (KV8) {
+            const float down = split_query_e4m3<Cfg<NR>::NQ>(c.smem + OFF_Q + qb * Cfg<NR>::QBLOCK, lane);
+            if (lane == 0) reinterpret_cast<float *>(c.smem + OFF_QS)[qb] = down;
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->qconv[qb]);
+            __syncwarp();
+        }
+        int failed = 0;
+        if (lane == 0) {
+            int nq = 0, nv = 0;
+            long long idle_since = clock64();
+            while (nv < nt) {
+                bool progressed = false;
+                if (nq < nt && nq < nv + 2) {
+                    const int kt = k + nq;
+                    if (mbar_test(&bars->full[kt % NST], (uint32_t)(kt / NST) & 1u) &&
+                        (kt < 2 || mbar_test(&bars->sfree[kt & 1], (uint32_t)((kt >> 1) - 1) & 1u))) {
+                        issue_scores<NR, KV8>(c, kt, qb);
+                        ++nq;
+                        if (nq == nt) umma_commit(&bars->qempty[qb]);
+                        progressed = true;
+                    }
                 }
-            }
-            if (nv < nq) {
-                const int kt = k + nv;
-                if (mbar_test(&bars->pready[kt & 1], (uint32_t)(kt >> 1) & 1u) &&
-                    (nv > 0 || pi == 0 || mbar_test(&bars->ofree, (uint32_t)(pi - 1) & 1u))) {
-                    issue_values(c, kt, nv == 0);
-                    ++nv;
-                    progressed = true;
+                if (nv < nq) {
+                    const int kt = k + nv;
+                    if (mbar_test(&bars->pready[kt & 1], (uint32_t)(kt >> 1) & 1u) &&
+                        (nv > 0 || pi == 0 || mbar_test(&bars->ofree, (uint32_t)(pi - 1) & 1u))) {
+                        issue_values<NR, KV8>(c, kt, nv == 0);
+                        ++nv;
+                        progressed = true;
+                    }
                 }
-            }
-            if (progressed) {
-                idle_since = clock64();
-            } else {
-                if (*c.abort_flag) return;
-                if (clock64() - idle_since > kWaitLimitCycles) {
-                    atomicOr(&g_device_flags, FLAG_MMA_WAIT);
-                    *c.abort_flag = 1;
-                    return;
+                if (progressed) {
+                    idle_since = clock64();
+                } else {
+                    if (*c.abort_flag) { failed = 1; break; }
+                    if (clock64() - idle_since > kWaitLimitCycles) {
+                        atomicOr(&g_device_flags, FLAG_MMA_WAIT);
+                        *c.abort_flag = 1;
+                        failed = 1;
+                        break;
+                    }
                 }
             }
         }
+        if (__shfl_sync(0xffffffffu, failed, 0)) return;
         k += nt;
     }
 }
 
 // ------------------------------------------------------------------ softmax (warps 2-5)
-template <int NR>
+template <int NR, bool KV8>
 __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, int warp, int lane) {
     using C = Cfg<NR>;
+    using L = Kv<KV8>;
     constexpr int NQ = C::NQ;
+    constexpr int NST = L::NST;
     Bars *bars = c.bars;
     const int q = warp & 3;               // TMEM lane quadrant
     const int r = 32 * q + lane;          // token row of a tile / output dimension
@@ -358,6 +531,14 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
         const int start = active_start(len, p.q_len, p.window);
         // columns of one query position (the group's heads); all columns of the unit
         const uint64_t group_bits = p.g >= 64 ? ~0ull : ((1ull << p.g) - 1ull);
+        // score scale (log2 units); with an E4M3 cache also the key scale and the 2^-e
+        // of the split query block
+        float cs = p.scale_log2;
+        if constexpr (KV8) {
+            const int qb = pi % C::NQB, qu = pi / C::NQB;
+            if (!warp_all(mbar_wait(&bars->qconv[qb], (uint32_t)qu & 1u, FLAG_MMA_WAIT, c.abort_flag))) return;
+            cs *= p.k_scale * reinterpret_cast<const float *>(c.smem + OFF_QS)[qb];
+        }
         float m_own = -INFINITY;              // running max of head st_id (owner threads)
         float l_part[NR];
 #pragma unroll
@@ -398,7 +579,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
             float sc[NR], v[NR];
 #pragma unroll
             for (int h = 0; h < NR; ++h) {
-                sc[h] = ((vis >> h) & 1ull) ? __uint_as_float(sv[h]) * p.scale_log2 : -INFINITY;
+                sc[h] = ((vis >> h) & 1ull) ? __uint_as_float(sv[h]) * cs : -INFINITY;
                 v[h] = sc[h];
             }
             // ---- per-head maximum over the tile's 128 tokens
@@ -412,7 +593,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                 uint8_t need = 0;
                 if (t == 0) {
                     m_own = tm;
-                } else if (tm > m_own + RESCALE_LOG2) {
+                } else if (tm > m_own + L::RESCALE) {
                     alpha = fast_exp2(m_own - tm);
                     m_own = tm;
                     need = 1;
@@ -435,7 +616,35 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                     l_part[h] *= x.x; l_part[h + 1] *= x.y; l_part[h + 2] *= x.z; l_part[h + 3] *= x.w;
                 }
             }
-            uint8_t *st = c.smem + OFF_ST + s * STAGE;
+            uint8_t *st = c.smem + OFF_ST + s * L::STAGE;
+            if constexpr (KV8) {
+                // 16 heads per 16-byte row of a 2 KB block; heads past NR are zero
+#pragma unroll
+                for (int cb = 0; cb < NQ / 16; ++cb) {
+                    uint32_t hw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int h = 16 * cb + 4 * e;
+                        if (h < NR) {
+                            float a[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const float mu = ms[sb * HB + h + u];
+                                // 2^6 * 2^(s - m), summed in the same units
+                                a[u] = fast_exp2(sc[h + u] - (mu == -INFINITY ? 0.f : mu) + P8_LOG2);
+                                l_part[h + u] += a[u];
+                            }
+                            uint16_t h0, l0, h1, l1;
+                            split_e4m3x2(a[0], a[1], h0, l0);
+                            split_e4m3x2(a[2], a[3], h1, l1);
+                            hw[e] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                            lw[e] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                        }
+                    }
+                    *reinterpret_cast<uint4 *>(st + cb * 2048 + r * 16) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4 *>(st + P8_LO + cb * 2048 + r * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                }
+            } else {
             uint8_t *hrow = st + r * 128;
             uint8_t *lrow = st + CHUNK + r * 128;
 #pragma unroll
@@ -459,6 +668,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                 const int slot = (cc ^ (r & 7)) << 4;
                 *reinterpret_cast<uint4 *>(hrow + slot) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
                 *reinterpret_cast<uint4 *>(lrow + slot) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
             }
             fence_proxy_async_smem();
             // ---- rescale the affected heads' columns of O^T (after the previous value product)
@@ -510,8 +720,10 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
         if (st_id < NR) {
             const float l = red[(8 + 0) * HB + st_id] + red[(8 + 1) * HB + st_id] + red[(8 + 2) * HB + st_id] +
                             red[(8 + 3) * HB + st_id];
-            linv[st_id] = l > 0.f ? 1.f / l : 0.f;
-            const float lse_v = l > 0.f ? (m_own + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+            // (E4M3 cache: l and O^T both carry 2^6; the value scale enters here)
+            linv[st_id] = l > 0.f ? (KV8 ? p.v_scale : 1.f) / l : 0.f;
+            const float lse_v =
+                l > 0.f ? (m_own + __log2f(l) - (KV8 ? P8_LOG2 : 0.f)) * 0.69314718055994531f : -INFINITY;
             if (st_id < h_real) {
                 if (pc.whole)
                     p.lse[out_row(st_id)] = lse_v;
@@ -545,7 +757,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
 
 }  // namespace gqatc
 
-template <int NR>
+template <int NR, bool KV8>
 __global__ void __launch_bounds__(gqatc::NTHREADS, 1)
 gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
@@ -561,13 +773,14 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
     const int U = p.n_kv * p.n_hb;
 
     if (tid == 0) {
-        for (int s = 0; s < NST; ++s) {
+        for (int s = 0; s < Kv<KV8>::NST; ++s) {
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->qfull[i], 1);
             mbar_init(&bars->qempty[i], 1);
+            mbar_init(&bars->qconv[i], 32);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->sready[i], 1);
@@ -619,11 +832,11 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
 
     if (c.p0 < total) {
         if (warp == 0) {
-            if (lane == 0) producer<NR>(p, &kmap, &vmap, &qmap, c);
+            if (lane == 0) producer<NR, KV8>(p, &kmap, &vmap, &qmap, c);
         } else if (warp == 1) {
-            if (lane == 0) mma_issuer<NR>(p, c);
+            mma_issuer<NR, KV8>(p, c, lane);
         } else {
-            softmax_warps<NR>(p, c, warp, lane);
+            softmax_warps<NR, KV8>(p, c, warp, lane);
         }
     }
 

@@ -326,7 +326,7 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
 
 // The tcgen05 kernel (gqa_tc_decode.cuh): tokens on the MMA rows, up to 64 query heads
 // per unit, NR head columns processed.
-template <int NR>
+template <int NR, bool KV8>
 int run_gqa_tc(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &vmap,
                const CUtensorMap &qmap, DeviceState *dev, int units_per_seq, cudaStream_t stream) {
     GqaParams p = base;
@@ -357,7 +357,7 @@ int run_gqa_tc(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap
     p.ws_lse = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes);
     p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes + lse_bytes);
 
-    auto kern = gqa_tc_decode_kernel<NR>;
+    auto kern = gqa_tc_decode_kernel<NR, KV8>;
     cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), dev, smem);
     if (e != cudaSuccess) return fail_cuda(e, "cudaFuncSetAttribute(gqa tc)");
     kern<<<p.workers, gqatc::NTHREADS, smem, stream>>>(p, kmap, vmap, qmap);
@@ -401,12 +401,14 @@ bool use_tc_kernel(int head_dim, int g, int batch, const DeviceState *dev) {
 // A K/V cache as the decode kernels see it: pages of page_size rows per (page, KV head);
 // a contiguous cache is one page per sequence (page_size = capacity, no block table).
 struct GqaCache {
-    const uint16_t *k, *v;
+    const void *k, *v;
     const int32_t *block_table;   // [batch, max_pages] or null (contiguous)
     int capacity;                 // rows addressable per sequence (seq_lens are clamped to it)
     int page_size;
     int max_pages;
     long long pages;              // pages in the pool (contiguous: batch)
+    bool e4m3 = false;            // E4M3 codes (value = code * scale) instead of bf16
+    float k_scale = 1.f, v_scale = 1.f;
 };
 
 int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq_lens, int batch,
@@ -434,17 +436,27 @@ int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq
                  gqatc::HB);
         return KVATTN_ERR_UNSUPPORTED;
     }
-    const bool tc = multi || (tiles_fit && use_tc_kernel(head_dim, g, batch, dev));
+    // an E4M3 cache: the tcgen05 kernel (8-bit MMAs straight from the tiles)
+    if (cache.e4m3 && (g_gqa_kernel == 1 || !(tiles_fit && head_dim == 128 && g * q_len <= gqatc::HB &&
+                                              gqatc::smem_bytes(batch) <= dev->max_smem_optin))) {
+        snprintf(t_detail, sizeof(t_detail), "E4M3 cache needs head_dim 128, g * q_len <= %d and pages of "
+                 "multiples of 128 rows", gqatc::HB);
+        return KVATTN_ERR_UNSUPPORTED;
+    }
+    const bool tc = multi || cache.e4m3 || (tiles_fit && use_tc_kernel(head_dim, g, batch, dev));
     const int MT = g <= 16 ? 1 : 2;
     const int heads = tc ? gqatc::HB : 16 * MT;
     const int n_hb = (g * q_len + heads - 1) / heads;
     const uint32_t box_rows = tc ? gqatc::TILE : 64;
 
+    // (an E4M3 row of head_dim codes is mapped as head_dim / 2 two-byte elements: the TMA
+    // moves bytes, and its zero fill is zero codes)
+    const uint64_t row_elems = cache.e4m3 ? (uint64_t)head_dim / 2 : (uint64_t)head_dim;
     CUtensorMap kmap, vmap, qmap;
-    st = make_map_3d(&kmap, cache.k, head_dim, cache.page_size, (uint64_t)cache.pages * n_kv_heads, 64, box_rows,
+    st = make_map_3d(&kmap, cache.k, row_elems, cache.page_size, (uint64_t)cache.pages * n_kv_heads, 64, box_rows,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
-    st = make_map_3d(&vmap, cache.v, head_dim, cache.page_size, (uint64_t)cache.pages * n_kv_heads, 64, box_rows,
+    st = make_map_3d(&vmap, cache.v, row_elems, cache.page_size, (uint64_t)cache.pages * n_kv_heads, 64, box_rows,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
     const int gl = g * q_len;    // score columns of a unit
@@ -476,13 +488,21 @@ int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq
     p.page_size = cache.page_size;
     p.q_len = q_len;
     p.window = window;
+    p.k_scale = cache.k_scale;
+    p.v_scale = cache.v_scale;
     const int U = n_kv_heads * n_hb;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tc && cache.e4m3) {
+        if (gl > 32) return run_gqa_tc<64, true>(p, kmap, vmap, qmap, dev, U, s);
+        if (gl > 16) return run_gqa_tc<32, true>(p, kmap, vmap, qmap, dev, U, s);
+        if (gl > 8) return run_gqa_tc<16, true>(p, kmap, vmap, qmap, dev, U, s);
+        return run_gqa_tc<8, true>(p, kmap, vmap, qmap, dev, U, s);
+    }
     if (tc) {
-        if (gl > 32) return run_gqa_tc<64>(p, kmap, vmap, qmap, dev, U, s);
-        if (gl > 16) return run_gqa_tc<32>(p, kmap, vmap, qmap, dev, U, s);
-        if (gl > 8) return run_gqa_tc<16>(p, kmap, vmap, qmap, dev, U, s);
-        return run_gqa_tc<8>(p, kmap, vmap, qmap, dev, U, s);
+        if (gl > 32) return run_gqa_tc<64, false>(p, kmap, vmap, qmap, dev, U, s);
+        if (gl > 16) return run_gqa_tc<32, false>(p, kmap, vmap, qmap, dev, U, s);
+        if (gl > 8) return run_gqa_tc<16, false>(p, kmap, vmap, qmap, dev, U, s);
+        return run_gqa_tc<8, false>(p, kmap, vmap, qmap, dev, U, s);
     }
     if (head_dim == 128)
         return MT == 1 ? run_gqa<128, 1>(p, kmap, vmap, dev, U, s) : run_gqa<128, 2>(p, kmap, vmap, dev, U, s);
@@ -709,6 +729,80 @@ int kvattn_gqa_decode_multi(const uint16_t *q, const uint16_t *k_cache, const ui
     const GqaCache cache{k_cache, v_cache, nullptr, max_seq_len, max_seq_len, 1, batch};
     return gqa_decode_impl(q, cache, seq_lens, batch, n_q_heads, n_kv_heads, head_dim, scale, out, lse, stream,
                            q_len, window);
+}
+
+int kvattn_gqa_decode_fp8(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                          const int32_t *seq_lens, int max_seq_len, int batch, int q_len, int n_q_heads,
+                          int n_kv_heads, int head_dim, float scale, float k_scale, float v_scale, int window,
+                          float *out, float *lse, void *stream) {
+    if (!q || !k_cache || !v_cache || !seq_lens || !out || !lse) return KVATTN_ERR_INVALID_ARG;
+    if (batch <= 0 || q_len <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || max_seq_len <= 0 || window < 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if (n_q_heads % n_kv_heads != 0) return KVATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) ||
+        !(v_scale > 0.f))
+        return KVATTN_ERR_INVALID_ARG;
+    if (head_dim != 128 || (n_q_heads / n_kv_heads) * q_len > gqatc::HB) return KVATTN_ERR_UNSUPPORTED;
+    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
+    if ((long long)batch * n_kv_heads * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seq_lens) ||
+        !aligned16(out) || !aligned16(lse))
+        return KVATTN_ERR_MISALIGNED;
+    const size_t q_bytes = (size_t)batch * q_len * n_q_heads * head_dim * 2;
+    const size_t kv_bytes = (size_t)batch * n_kv_heads * max_seq_len * head_dim;
+    const size_t out_bytes = (size_t)batch * q_len * n_q_heads * head_dim * 4;
+    const size_t lse_bytes = (size_t)batch * q_len * n_q_heads * 4;
+    const void *ins[4] = {q, k_cache, v_cache, seq_lens};
+    const size_t in_sz[4] = {q_bytes, kv_bytes, kv_bytes, (size_t)batch * 4};
+    for (int i = 0; i < 4; ++i)
+        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
+            return KVATTN_ERR_INVALID_ARG;
+    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+    GqaCache cache{k_cache, v_cache, nullptr, max_seq_len, max_seq_len, 1, batch};
+    cache.e4m3 = true;
+    cache.k_scale = k_scale;
+    cache.v_scale = v_scale;
+    return gqa_decode_impl(q, cache, seq_lens, batch, n_q_heads, n_kv_heads, head_dim, scale, out, lse, stream,
+                           q_len, window);
+}
+
+int kvattn_gqa_decode_fp8_paged(const uint16_t *q, const uint8_t *k_pages, const uint8_t *v_pages,
+                                const int32_t *block_table, const int32_t *seq_lens, int num_pages, int page_size,
+                                int max_pages_per_seq, int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                                float scale, float k_scale, float v_scale, float *out, float *lse, void *stream) {
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out || !lse) return KVATTN_ERR_INVALID_ARG;
+    if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || num_pages <= 0 || page_size <= 0 ||
+        max_pages_per_seq <= 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if (n_q_heads % n_kv_heads != 0) return KVATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || !std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) ||
+        !(v_scale > 0.f))
+        return KVATTN_ERR_INVALID_ARG;
+    if (head_dim != 128 || n_q_heads / n_kv_heads > gqatc::HB || page_size % gqatc::TILE != 0)
+        return KVATTN_ERR_UNSUPPORTED;
+    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
+    if ((long long)num_pages * n_kv_heads * page_size >= (1ll << 31) ||
+        (long long)max_pages_per_seq * page_size >= (1ll << 31))
+        return KVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(block_table) ||
+        !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
+        return KVATTN_ERR_MISALIGNED;
+    const size_t q_bytes = (size_t)batch * n_q_heads * head_dim * 2;
+    const size_t kv_bytes = (size_t)num_pages * n_kv_heads * page_size * head_dim;
+    const size_t out_bytes = (size_t)batch * n_q_heads * head_dim * 4;
+    const size_t lse_bytes = (size_t)batch * n_q_heads * 4;
+    const void *ins[5] = {q, k_pages, v_pages, seq_lens, block_table};
+    const size_t in_sz[5] = {q_bytes, kv_bytes, kv_bytes, (size_t)batch * 4, (size_t)batch * max_pages_per_seq * 4};
+    for (int i = 0; i < 5; ++i)
+        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
+            return KVATTN_ERR_INVALID_ARG;
+    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+    GqaCache cache{k_pages, v_pages, block_table, max_pages_per_seq * page_size, page_size, max_pages_per_seq,
+                   num_pages};
+    cache.e4m3 = true;
+    cache.k_scale = k_scale;
+    cache.v_scale = v_scale;
+    return gqa_decode_impl(q, cache, seq_lens, batch, n_q_heads, n_kv_heads, head_dim, scale, out, lse, stream);
 }
 
 int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,

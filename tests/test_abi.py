@@ -222,6 +222,44 @@ def test_gqa_multi_rejects_bad_arguments(lib, kw, expected):
     assert st == expected
 
 
+@pytest.mark.parametrize("kw,expected", [
+    (dict(d=64), kb.KVATTN_ERR_UNSUPPORTED),                 # E4M3 path: head_dim 128 only
+    (dict(L=3, nq=64, nkv=2), kb.KVATTN_ERR_UNSUPPORTED),    # 32 heads x 3 positions > 64 columns
+    (dict(ks=0.0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(vs=-1.0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(ks=float("inf")), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(vs=float("nan")), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(window=-2), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(k=2 * A + 8), kb.KVATTN_ERR_MISALIGNED),
+    (dict(out=2 * A + 64), kb.KVATTN_ERR_INVALID_ARG),      # output inside the key cache
+    (dict(k=0), kb.KVATTN_ERR_INVALID_ARG),
+])
+def test_gqa_fp8_rejects_bad_arguments(lib, kw, expected):
+    a = dict(q=A, k=2 * A, v=3 * A, lens=4 * A, T=4096, B=2, L=1, nq=32, nkv=8, d=128, ks=0.01, vs=0.02,
+             window=0, out=5 * A, lse=6 * A)
+    a.update(kw)
+    st = lib.kvattn_gqa_decode_fp8(a["q"], a["k"], a["v"], a["lens"], a["T"], a["B"], a["L"], a["nq"], a["nkv"],
+                                   a["d"], 0.088, a["ks"], a["vs"], a["window"], a["out"], a["lse"], None)
+    assert st == expected
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(S=64), kb.KVATTN_ERR_UNSUPPORTED),                 # pages of whole 128-token tiles
+    (dict(d=64), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(table=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(ks=0.0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(table=6 * A + 4), kb.KVATTN_ERR_MISALIGNED),
+])
+def test_gqa_fp8_paged_rejects_bad_arguments(lib, kw, expected):
+    a = dict(q=A, k=2 * A, v=3 * A, table=6 * A, lens=5 * A, P=64, S=128, M=8, B=2, nq=8, nkv=2, d=128,
+             ks=0.01, vs=0.02, out=7 * A, lse=8 * A)
+    a.update(kw)
+    st = lib.kvattn_gqa_decode_fp8_paged(a["q"], a["k"], a["v"], a["table"], a["lens"], a["P"], a["S"], a["M"],
+                                         a["B"], a["nq"], a["nkv"], a["d"], 0.088, a["ks"], a["vs"], a["out"],
+                                         a["lse"], None)
+    assert st == expected
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     q = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
