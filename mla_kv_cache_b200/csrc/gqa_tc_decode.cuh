@@ -72,11 +72,8 @@ constexpr int RING = 12 * CHUNK;          // the stage ring: 192 KB
 constexpr int QREGION = 2 * HB * 128;     // query blocks: 16 KB (one of 64 heads or two of <= 32)
 constexpr int NTHREADS = 192;             // producer, MMA, 4 softmax warps
 constexpr int NSOFT = 128;
-constexpr uint32_t TM_S = 0;              // two 64-column score buffers
-constexpr uint32_t TM_O = 128;            // O^T: 64 columns
-constexpr uint32_t TM_COLS = 256;
+constexpr uint32_t TM_S = 0;              // two score buffers
 constexpr int NST_MAX = 6;
-constexpr int P8_LO = 8192;               // E4M3 P^T: remainder after the high part (K half of a stage)
 constexpr float P8_LOG2 = 6.f;            // E4M3 P^T holds 2^6 * 2^(s - m)
 
 // Per cache type: bf16 (a tile is two [128 x 64] boxes, 3 stages of 64 KB) or E4M3
@@ -88,6 +85,12 @@ struct Kv {
     static constexpr int NST = RING / STAGE;
     // the running max moves when a head's tile maximum exceeds it by 2^RESCALE
     static constexpr float RESCALE = KV8 ? 2.f : 8.f;
+    // tensor memory: two score buffers (E4M3: the query's high-part and remainder
+    // products side by side, 2 x NQ columns each), then O^T as two halves -- the value
+    // product of the weights' high part and of their remainder -- summed at the end
+    static constexpr uint32_t S_STRIDE = KV8 ? 128 : 64;
+    static constexpr uint32_t TM_O = 2 * S_STRIDE;
+    static constexpr uint32_t TM_COLS = KV8 ? 512 : 256;
     static_assert(NST <= NST_MAX, "stage barriers");
 };
 
@@ -183,6 +186,15 @@ __device__ __forceinline__ void store_reduced(float *row, const float (&v)[NR], 
     } else {
         if ((lane & (C::LPH - 1)) == 0) row[lane / C::LPH] = v[0];
     }
+}
+
+// One arrival per warp on a barrier the softmax warps share (initialised with a count of
+// warps): the lanes meet first, so every lane's earlier writes and fences are ordered
+// before lane 0's arrival, which releases them.  (128 single-thread arrivals on one
+// barrier word cost several hundred cycles per barrier.)
+__device__ __forceinline__ void warp_arrive(uint64_t *bar, int lane) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
 }
 
 // NQ consecutive TMEM columns of this thread's lane.
@@ -362,17 +374,16 @@ __device__ __forceinline__ void issue_scores(const Ctx &c, int kt, int qbuf) {
     const uint32_t st = smem_u32(c.smem + OFF_ST + s * L::STAGE);
     const uint32_t qb = smem_u32(c.smem + OFF_Q + qbuf * C::QBLOCK);
     if constexpr (KV8) {
-        // K (E4M3, [128 tokens x 128], K-major) times the query's high part, then its
-        // remainder: 4 + 4 MMAs of K = 32
-        constexpr uint32_t idesc = idesc_e4m3(128, Cfg<NR>::NQ, 0, 0);
+        // K (E4M3, [128 tokens x 128], K-major) times the query's high part and its
+        // remainder at once: the two blocks are consecutive 128-byte rows, so N = 2 NQ
+        // and the tile is read once (4 MMAs of K = 32); TMEM columns [0, NQ) get the
+        // high-part scores, [NQ, 2 NQ) the remainder's
+        constexpr uint32_t idesc = idesc_e4m3(128, 2 * Cfg<NR>::NQ, 0, 0);
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-#pragma unroll
-            for (int kk = 0; kk < D / 32; ++kk) {
-                const uint64_t a = smem_desc_sw128(st + kk * 32, 16, 1024);
-                const uint64_t b = smem_desc_sw128(qb + part * C::QCHUNK + kk * 32, 16, 1024);
-                umma_ss_f8(c.tmem + TM_S + 64 * sb, a, b, idesc, (part | kk) ? 1u : 0u);
-            }
+        for (int kk = 0; kk < D / 32; ++kk) {
+            const uint64_t a = smem_desc_sw128(st + kk * 32, 16, 1024);
+            const uint64_t b = smem_desc_sw128(qb + kk * 32, 16, 1024);
+            umma_ss_f8(c.tmem + TM_S + L::S_STRIDE * sb, a, b, idesc, kk ? 1u : 0u);
         }
     } else {
         constexpr uint32_t idesc = idesc_f16_major(128, Cfg<NR>::NQ, 1, 1, 0, 0);
@@ -381,7 +392,7 @@ __device__ __forceinline__ void issue_scores(const Ctx &c, int kt, int qbuf) {
             const uint32_t blk = kk >> 2, in = (kk & 3) * 32;
             const uint64_t a = smem_desc_sw128(st + blk * CHUNK + in, 16, 1024);
             const uint64_t b = smem_desc_sw128(qb + blk * C::QCHUNK + in, 16, 1024);
-            umma_ss(c.tmem + TM_S + 64 * sb, a, b, idesc, kk > 0 ? 1u : 0u);
+            umma_ss(c.tmem + TM_S + L::S_STRIDE * sb, a, b, idesc, kk > 0 ? 1u : 0u);
         }
     }
     umma_commit(&c.bars->sready[sb]);
@@ -396,30 +407,27 @@ __device__ __forceinline__ void issue_values(const Ctx &c, int kt, bool first) {
     const uint32_t st = smem_u32(c.smem + OFF_ST + s * L::STAGE);
     if constexpr (KV8) {
         // V^T: M = 128 dimensions (one 128-byte row per token, MN-major), K = 32 tokens;
-        // P^T: N = NQ heads in 16-head blocks 2 KB apart, 16 bytes per token (plain
-        // MN-major: 8-token core matrices 128 bytes apart)
+        // P^T: N = 2 NQ columns -- the high parts' 16-head blocks, then the remainders',
+        // 2 KB apart, 16 bytes per token (plain MN-major: 8-token core matrices 128
+        // bytes apart); the tile is read once (4 MMAs)
         constexpr int NQ = Cfg<NR>::NQ;
-        constexpr uint32_t idesc_pv = idesc_e4m3(128, NQ, 1, 1);
+        constexpr uint32_t idesc_pv = idesc_e4m3(128, 2 * NQ, 1, 1);
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-#pragma unroll
-            for (int kk = 0; kk < TILE / 32; ++kk) {
-                const uint64_t a = smem_desc_sw128(st + L::KV_BYTES + kk * 4096, CHUNK, 1024);
-                const uint64_t b = smem_desc_plain(st + part * P8_LO + kk * 512, 128, 2048);
-                umma_ss_f8(c.tmem + TM_O, a, b, idesc_pv, (!first || part || kk) ? 1u : 0u);
-            }
+        for (int kk = 0; kk < TILE / 32; ++kk) {
+            const uint64_t a = smem_desc_sw128(st + L::KV_BYTES + kk * 4096, CHUNK, 1024);
+            const uint64_t b = smem_desc_plain(st + kk * 512, 128, 2048);
+            umma_ss_f8(c.tmem + L::TM_O, a, b, idesc_pv, (!first || kk) ? 1u : 0u);
         }
     } else {
-        constexpr uint32_t idesc_pv = idesc_f16_major(128, HB, 1, 1, 1, 1);
+        constexpr uint32_t idesc_pv = idesc_f16_major(128, 2 * HB, 1, 1, 1, 1);
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk) {
             // V^T: M = 128 dimensions in two 64-wide blocks 16 KB apart, K = 16 tokens
             const uint64_t a = smem_desc_sw128(st + L::KV_BYTES + kk * 2048, CHUNK, 1024);
-            // P^T high part and remainder (in the K half of the stage): N = 64 heads
-            const uint64_t bh = smem_desc_sw128(st + kk * 2048, CHUNK, 1024);
-            const uint64_t bl = smem_desc_sw128(st + CHUNK + kk * 2048, CHUNK, 1024);
-            umma_ss(c.tmem + TM_O, a, bh, idesc_pv, (!first || kk > 0) ? 1u : 0u);
-            umma_ss(c.tmem + TM_O, a, bl, idesc_pv, 1u);
+            // P^T (in the K half of the stage): N = 128 columns, the high part's 64 heads
+            // and the remainder's 64, two 64-wide blocks 16 KB apart; the tile is read once
+            const uint64_t b = smem_desc_sw128(st + kk * 2048, CHUNK, 1024);
+            umma_ss(c.tmem + L::TM_O, a, b, idesc_pv, (!first || kk > 0) ? 1u : 0u);
         }
     }
     umma_commit(&c.bars->empty[s]);
@@ -503,6 +511,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
     using L = Kv<KV8>;
     constexpr int NQ = C::NQ;
     constexpr int NST = L::NST;
+    constexpr uint32_t O_LO = KV8 ? NQ : HB;     // column of O^T's remainder half
     Bars *bars = c.bars;
     const int q = warp & 3;               // TMEM lane quadrant
     const int r = 32 * q + lane;          // token row of a tile / output dimension
@@ -515,7 +524,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
     float *linv = reinterpret_cast<float *>(c.smem + OFF_LINV);
     uint32_t grp_uses = 0;
     auto grp_sync = [&]() -> bool {
-        mbar_arrive(&bars->grp);
+        warp_arrive(&bars->grp, lane);
         const bool ok = mbar_wait(&bars->grp, grp_uses & 1u, FLAG_FULL_WAIT, c.abort_flag);
         ++grp_uses;
         return warp_all(ok);
@@ -572,10 +581,24 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                 return;
             tc_fence_after();
             uint32_t sv[NQ];
-            tmem_ld_cols<NQ>(c.tmem + lane_base + TM_S + 64 * sb, sv);
-            tmem_wait_ld();
+            if constexpr (KV8) {
+                // high-part and remainder scores, added (16 columns at a time)
+#pragma unroll
+                for (int c0 = 0; c0 < NQ; c0 += 16) {
+                    uint32_t a16[16], b16[16];
+                    tmem_ld16(c.tmem + lane_base + TM_S + L::S_STRIDE * sb + c0, a16);
+                    tmem_ld16(c.tmem + lane_base + TM_S + L::S_STRIDE * sb + NQ + c0, b16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        sv[c0 + i] = __float_as_uint(__uint_as_float(a16[i]) + __uint_as_float(b16[i]));
+                }
+            } else {
+                tmem_ld_cols<NQ>(c.tmem + lane_base + TM_S + L::S_STRIDE * sb, sv);
+                tmem_wait_ld();
+            }
             tc_fence_before();
-            mbar_arrive(&bars->sfree[sb]);
+            warp_arrive(&bars->sfree[sb], lane);
             float sc[NR], v[NR];
 #pragma unroll
             for (int h = 0; h < NR; ++h) {
@@ -618,7 +641,8 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
             }
             uint8_t *st = c.smem + OFF_ST + s * L::STAGE;
             if constexpr (KV8) {
-                // 16 heads per 16-byte row of a 2 KB block; heads past NR are zero
+                // 16 heads per 16-byte row of a 2 KB block, the remainders' blocks after the
+                // high parts' (NQ / 16 blocks each); heads past NR are zero
 #pragma unroll
                 for (int cb = 0; cb < NQ / 16; ++cb) {
                     uint32_t hw[4] = {0u, 0u, 0u, 0u}, lw[4] = {0u, 0u, 0u, 0u};
@@ -642,7 +666,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                         }
                     }
                     *reinterpret_cast<uint4 *>(st + cb * 2048 + r * 16) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                    *reinterpret_cast<uint4 *>(st + P8_LO + cb * 2048 + r * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                    *reinterpret_cast<uint4 *>(st + NQ * 128 + cb * 2048 + r * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
                 }
             } else {
             uint8_t *hrow = st + r * 128;
@@ -678,26 +702,30 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                     return;
                 tc_fence_after();
 #pragma unroll
-                for (int c0 = 0; c0 < NQ; c0 += 16) {
-                    uint32_t ov[16];
-                    tmem_ld16(c.tmem + lane_base + TM_O + c0, ov);
-                    tmem_wait_ld();
+                for (int half = 0; half < 2; ++half) {
 #pragma unroll
-                    for (int h = 0; h < 16; h += 4) {
-                        if (c0 + h < NR) {
-                            const float4 x = *reinterpret_cast<const float4 *>(as_t + c0 + h);
-                            ov[h] = __float_as_uint(__uint_as_float(ov[h]) * x.x);
-                            ov[h + 1] = __float_as_uint(__uint_as_float(ov[h + 1]) * x.y);
-                            ov[h + 2] = __float_as_uint(__uint_as_float(ov[h + 2]) * x.z);
-                            ov[h + 3] = __float_as_uint(__uint_as_float(ov[h + 3]) * x.w);
+                    for (int c0 = 0; c0 < NQ; c0 += 16) {
+                        const uint32_t col = L::TM_O + half * O_LO + c0;
+                        uint32_t ov[16];
+                        tmem_ld16(c.tmem + lane_base + col, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int h = 0; h < 16; h += 4) {
+                            if (c0 + h < NR) {
+                                const float4 x = *reinterpret_cast<const float4 *>(as_t + c0 + h);
+                                ov[h] = __float_as_uint(__uint_as_float(ov[h]) * x.x);
+                                ov[h + 1] = __float_as_uint(__uint_as_float(ov[h + 1]) * x.y);
+                                ov[h + 2] = __float_as_uint(__uint_as_float(ov[h + 2]) * x.z);
+                                ov[h + 3] = __float_as_uint(__uint_as_float(ov[h + 3]) * x.w);
+                            }
                         }
+                        tmem_st16(c.tmem + lane_base + col, ov);
                     }
-                    tmem_st16(c.tmem + lane_base + TM_O + c0, ov);
                 }
                 tmem_wait_st();
             }
             tc_fence_before();
-            mbar_arrive(&bars->pready[sb]);
+            warp_arrive(&bars->pready[sb], lane);
         }
         k += nt;
 
@@ -738,20 +766,21 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
         tc_fence_after();
 #pragma unroll
         for (int c0 = 0; c0 < NQ; c0 += 16) {
-            uint32_t ov[16];
-            tmem_ld16(c.tmem + lane_base + TM_O + c0, ov);
+            uint32_t ov[16], ol[16];
+            tmem_ld16(c.tmem + lane_base + L::TM_O + c0, ov);
+            tmem_ld16(c.tmem + lane_base + L::TM_O + O_LO + c0, ol);
             tmem_wait_ld();
 #pragma unroll
             for (int h = 0; h < 16; ++h) {
                 const int cc = c0 + h;
                 if (cc < NR && cc < h_real) {
                     float *dst = pc.whole ? p.out + out_row(cc) * D : p.ws_o + (part + cc) * D;
-                    dst[r] = __uint_as_float(ov[h]) * linv[cc];
+                    dst[r] = (__uint_as_float(ov[h]) + __uint_as_float(ol[h])) * linv[cc];
                 }
             }
         }
         tc_fence_before();
-        mbar_arrive(&bars->ofree);
+        warp_arrive(&bars->ofree, lane);
     }
 }
 
@@ -784,17 +813,17 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->sready[i], 1);
-            mbar_init(&bars->sfree[i], NSOFT);
-            mbar_init(&bars->pready[i], NSOFT);
+            mbar_init(&bars->sfree[i], NSOFT / 32);
+            mbar_init(&bars->pready[i], NSOFT / 32);
             mbar_init(&bars->odone[i], 1);
         }
-        mbar_init(&bars->ofree, NSOFT);
-        mbar_init(&bars->grp, NSOFT);
+        mbar_init(&bars->ofree, NSOFT / 32);
+        mbar_init(&bars->grp, NSOFT / 32);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_ptr), TM_COLS);
+        tmem_alloc(smem_u32(tmem_ptr), Kv<KV8>::TM_COLS);
         tmem_relinquish();
     }
     if (warp == 2) build_tile_prefix(p.seq_lens, p.B, p.T_max, TILE, s_prefix, lane, p.q_len, p.window);
@@ -844,7 +873,7 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(c.tmem, TM_COLS);
+        tmem_dealloc(c.tmem, Kv<KV8>::TM_COLS);
     }
 }
 
