@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvattn|reference]
                     [--config NAME] [--no-extra-configs] [--cpu-sample-s S]
+                    [--paged PAGE_SIZE] [--kv-dtype bf16|e4m3] [--q-len L] [--window W]
 
 A step is one library call covering every sequence of one layer's decode step for the
 workload (all of its query heads, out and lse complete, split-KV combine included).
@@ -17,7 +18,10 @@ maximum over ranks and the value is the bytes of all ranks over that time.
 
 Metric: decode-attention time per step, bytes per second and fraction of the measured
 HBM peak.  Bytes per step are the algorithmic minimum: q + the touched K/V (or latent +
-RoPE) cache rows + fp32 out + fp32 lse.
+RoPE) cache rows + fp32 out + fp32 lse.  Variants of the GQA workloads: an E4M3 cache
+(--kv-dtype e4m3, one byte per cached value), L new tokens per sequence with the causal
+mask (--q-len) and a sliding window (--window: only the rows some query can see are
+touched).
 """
 import argparse
 import json
@@ -42,6 +46,35 @@ FALLBACK_BF16_TFLOPS = 1590.0
 HOST_HIDE_CYCLES = 200_000      # ~0.1 ms of GPU spin before each timed step
 
 
+# ----------------------------------------------------------------------------- variants
+PAGED = 0   # --paged: rows per page of a paged cache layout (0: contiguous cache)
+KV8 = False  # --kv-dtype e4m3: E4M3 cache codes, one scale per tensor
+QLEN = 1    # --q-len: new tokens per sequence (causal among them)
+WINDOW = 0  # --window: sliding window in tokens (0: none)
+
+
+def variant_suffix():
+    return (("_e4m3" if KV8 else "") + (f"_L{QLEN}" if QLEN > 1 else "") +
+            (f"_w{WINDOW}" if WINDOW else "") + (f"_paged{PAGED}" if PAGED else ""))
+
+
+def active_rows(n):
+    """Rows of a sequence of n cached tokens that some query can see."""
+    if WINDOW <= 0:
+        return n
+    return n - max(0, n - QLEN + 1 - WINDOW)
+
+
+def visible_pairs(n):
+    """(query, cached row) pairs that take part in attention for one head of a sequence."""
+    tot = 0
+    for i in range(QLEN):
+        hi = n - QLEN + i + 1
+        lo = max(0, hi - WINDOW) if WINDOW > 0 else 0
+        tot += max(0, hi - lo)
+    return tot
+
+
 # ----------------------------------------------------------------------------- bytes / flops
 def step_bytes(cfg, lens):
     """Algorithmic bytes of one step: q + touched cache rows + out (fp32) + lse (fp32)."""
@@ -52,19 +85,23 @@ def step_bytes(cfg, lens):
         out = cfg.batch * cfg.n_heads * cfg.latent_dim * 4
         lse = cfg.batch * cfg.n_heads * 4
     else:
-        q = cfg.batch * cfg.n_q_heads * cfg.head_dim * 2
-        kv = 2 * sum(lens) * cfg.n_kv_heads * cfg.head_dim * 2
-        out = cfg.batch * cfg.n_q_heads * cfg.head_dim * 4
-        lse = cfg.batch * cfg.n_q_heads * 4
+        q = QLEN * cfg.batch * cfg.n_q_heads * cfg.head_dim * 2
+        kv = 2 * sum(active_rows(n) for n in lens) * cfg.n_kv_heads * cfg.head_dim * (1 if KV8 else 2)
+        out = QLEN * cfg.batch * cfg.n_q_heads * cfg.head_dim * 4
+        lse = QLEN * cfg.batch * cfg.n_q_heads * 4
     return {"total": q + kv + out + lse, "kv": kv, "q": q, "out": out + lse}
 
 
 def step_flops(cfg, lens):
     """Algorithmic flops: 2 per multiply-add of the score and the value products."""
-    T = sum(min(max(int(x), 0), cfg.max_seq_len) for x in lens)
+    lens = [min(max(int(x), 0), cfg.max_seq_len) for x in lens]
     if isinstance(cfg, wl.MLAConfig):
-        return T * cfg.n_heads * 2 * ((cfg.latent_dim + cfg.rope_dim) + cfg.latent_dim)
-    return T * cfg.n_q_heads * 4 * cfg.head_dim
+        return sum(lens) * cfg.n_heads * 2 * ((cfg.latent_dim + cfg.rope_dim) + cfg.latent_dim)
+    return sum(visible_pairs(n) for n in lens) * cfg.n_q_heads * 4 * cfg.head_dim
+
+
+def variant_fields():
+    return {"kv_dtype": "e4m3 (one scale per tensor)" if KV8 else "bf16", "q_len": QLEN, "window": WINDOW}
 
 
 def workload_fields(cfg):
@@ -212,7 +249,6 @@ def dist_barrier():
 
 
 # ----------------------------------------------------------------------------- GPU arm
-PAGED = 0   # --paged: rows per page of a paged cache layout (0: contiguous cache)
 
 
 def to_pages(cache, page_size, seq_axis, perm):
@@ -230,9 +266,27 @@ def to_pages(cache, page_size, seq_axis, perm):
     return pool
 
 
+def host_inputs(cfg, seed):
+    """The workload's seeded inputs (CPU) with the variant applied."""
+    if (KV8 or QLEN > 1 or WINDOW) and isinstance(cfg, wl.MLAConfig):
+        raise ValueError("E4M3 cache, several new tokens and windows: GQA workloads only")
+    x = wl.make_gqa_inputs_fp8(cfg, seed=seed) if KV8 else wl.make_inputs(cfg, seed=seed)
+    if QLEN > 1:
+        g = torch.Generator().manual_seed(seed + 29)
+        x["q"] = torch.randn((cfg.batch, QLEN, cfg.n_q_heads, cfg.head_dim), generator=g).to(torch.bfloat16)
+    elif WINDOW and not KV8:
+        x["q"] = x["q"][:, None].contiguous()     # the multi-token entry point's layout, L = 1
+    return x
+
+
+def q4d():
+    """The variant's query carries an L axis (and so do out and lse)."""
+    return QLEN > 1 or (WINDOW > 0 and not KV8)
+
+
 def device_inputs(cfg, seed):
-    x = wl.make_inputs(cfg, seed=seed)
-    d = {k: v.cuda() for k, v in x.items()}
+    x = host_inputs(cfg, seed)
+    d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
     if PAGED:
         T = cfg.max_seq_len
         if T % PAGED:
@@ -251,6 +305,21 @@ def device_inputs(cfg, seed):
 
 def make_call(cfg, d, out, lse, stream):
     from mla_kv_cache_b200 import binding as kb
+    if KV8 and PAGED:
+        if QLEN > 1 or WINDOW:
+            raise ValueError("the paged E4M3 entry point takes one new token and no window")
+        return lambda: kb.kvattn_gqa_decode_fp8_paged(d["q"], d["k_cache_pages"], d["v_cache_pages"],
+                                                      d["block_table"], d["seq_lens"], cfg.scale, d["k_scale"],
+                                                      d["v_scale"], out=out, lse=lse, stream=stream)
+    if KV8:
+        return lambda: kb.kvattn_gqa_decode_fp8(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], cfg.scale,
+                                                d["k_scale"], d["v_scale"], window=WINDOW, out=out, lse=lse,
+                                                stream=stream)
+    if QLEN > 1 or WINDOW:
+        if PAGED:
+            raise ValueError("the paged entry points take one new token and no window")
+        return lambda: kb.kvattn_gqa_decode_multi(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], cfg.scale,
+                                                  window=WINDOW, out=out, lse=lse, stream=stream)
     if PAGED:
         if isinstance(cfg, wl.MLAConfig):
             return lambda: kb.kvattn_mla_decode_paged(d["q_latent"], d["q_rope"], d["latent_cache_pages"],
@@ -270,7 +339,29 @@ def make_call(cfg, d, out, lse, stream):
 def out_shapes(cfg):
     if isinstance(cfg, wl.MLAConfig):
         return (cfg.batch, cfg.n_heads, cfg.latent_dim), (cfg.batch, cfg.n_heads)
+    if q4d():
+        return (cfg.batch, QLEN, cfg.n_q_heads, cfg.head_dim), (cfg.batch, QLEN, cfg.n_q_heads)
     return (cfg.batch, cfg.n_q_heads, cfg.head_dim), (cfg.batch, cfg.n_q_heads)
+
+
+def oracle_step(cfg, x, ids):
+    """The oracle on sequences `ids` of the workload (variant applied)."""
+    import oracle
+    if isinstance(cfg, wl.MLAConfig):
+        return oracle.mla_decode(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"],
+                                 x["seq_lens"], cfg.scale, batch_ids=ids)
+    if KV8:
+        for b in ids:
+            oracle.gqa_decode_fp8(x["q"][b:b + 1], x["k_cache"][b:b + 1], x["v_cache"][b:b + 1],
+                                  x["seq_lens"][b:b + 1], cfg.scale, x["k_scale"], x["v_scale"], window=WINDOW)
+        return None
+    if QLEN > 1 or WINDOW:
+        q = x["q"] if x["q"].dim() == 4 else x["q"][:, None]
+        for b in ids:
+            oracle.gqa_decode_multi(q[b:b + 1], x["k_cache"][b:b + 1], x["v_cache"][b:b + 1],
+                                    x["seq_lens"][b:b + 1], cfg.scale, window=WINDOW)
+        return None
+    return oracle.gqa_decode(x["q"], x["k_cache"], x["v_cache"], x["seq_lens"], cfg.scale, batch_ids=ids)
 
 
 def flush_l2(buf):
@@ -343,12 +434,7 @@ def cpu_baseline(cfg, x, budget_s):
     done, t_used = [], 0.0
     t0 = time.perf_counter()
     for b in order:
-        if isinstance(cfg, wl.MLAConfig):
-            oracle.mla_decode(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"],
-                              x["seq_lens"], cfg.scale, batch_ids=[b])
-        else:
-            oracle.gqa_decode(x["q"], x["k_cache"], x["v_cache"], x["seq_lens"], cfg.scale,
-                              batch_ids=[b])
+        oracle_step(cfg, x, [b])
         done.append(b)
         t_used = time.perf_counter() - t0
         if t_used >= budget_s:
@@ -359,7 +445,7 @@ def cpu_baseline(cfg, x, budget_s):
     return {"value": nbytes / t_used / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": f"{len(done)} of {cfg.batch} sequences of {cfg.name} (all their heads), "
-                      f"{t_used:.1f} s of fp64 CPU work incl. exact bf16->fp64 conversion; "
+                      f"{t_used:.1f} s of fp64 CPU work incl. exact conversion to fp64; "
                       f"bytes scaled by the sample's share of tokens",
             "us_per_step_extrapolated": t_used * 1e6 * sum(lens) / max(sum(sample_lens), 1)}
 
@@ -436,13 +522,15 @@ def gpu_arm(args):
     e2e_times, h2d, d2h = time_e2e(head_cfg, d, stream, max(args.steps // 10, 20), args.warmup, flush)
     e2e_ms = dist_max(sum(e2e_times) / len(e2e_times))
     achieved = nb["total"] / (ms * 1e-3) / 1e9
-    traffic = recorded_traffic(args.config)
+    traffic = recorded_traffic(args.config + variant_suffix())
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "us_per_step": ms * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16, shapes of the workload)",
-        "config": {"workload": args.config, **workload_fields(head_cfg),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 operands, fp32 accumulate" if KV8 else "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, shapes of the workload" +
+                ("; cache stored as E4M3 codes, scale = max|x| / 448)" if KV8 else ")"),
+        "config": {"workload": args.config + variant_suffix(), **workload_fields(head_cfg), **variant_fields(),
                    "bytes_per_step": nb["total"],
                    "cache_layout": f"paged: {PAGED}-row pages in a shuffled pool, block table" if PAGED
                    else "contiguous [B, n_kv, T, d]",
@@ -475,7 +563,7 @@ def reference_arm(args):
         return
     import oracle
     cfg = wl.CONFIGS[args.config]
-    x = wl.make_inputs(cfg, seed=0)
+    x = host_inputs(cfg, seed=0)
     lens = x["seq_lens"].tolist()
     nb = step_bytes(cfg, lens)
     per_step_seqs = max(1, min(cfg.batch, args.ref_sequences))
@@ -483,12 +571,7 @@ def reference_arm(args):
     for s in range(args.warmup + args.steps):
         ids = [(s * per_step_seqs + i) % cfg.batch for i in range(per_step_seqs)]
         t0 = time.perf_counter()
-        if isinstance(cfg, wl.MLAConfig):
-            oracle.mla_decode(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"],
-                              x["seq_lens"], cfg.scale, batch_ids=ids)
-        else:
-            oracle.gqa_decode(x["q"], x["k_cache"], x["v_cache"], x["seq_lens"], cfg.scale,
-                              batch_ids=ids)
+        oracle_step(cfg, x, ids)
         dt = time.perf_counter() - t0
         if s >= args.warmup:
             times.append(dt)
@@ -501,7 +584,8 @@ def reference_arm(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16, shapes of the workload)",
-        "config": {"workload": args.config, "bytes_per_step": nb["total"]},
+        "config": {"workload": args.config + variant_suffix(), **variant_fields(),
+                   "bytes_per_step": nb["total"]},
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(),
                          "kind": "oracle",
                          "sample": f"{per_step_seqs} of {cfg.batch} sequences per step (all heads), "
@@ -531,9 +615,18 @@ def main():
     ap.add_argument("--paged", type=int, default=0, metavar="PAGE_SIZE",
                     help="time the paged-cache entry points, the cache cut into pages of this "
                          "many rows (a multiple of 64) and shuffled over a pool")
+    ap.add_argument("--kv-dtype", default="bf16", choices=["bf16", "e4m3"],
+                    help="cache storage: bf16, or E4M3 codes with one scale per tensor (GQA workloads)")
+    ap.add_argument("--q-len", type=int, default=1, help="new tokens per sequence (causal among them)")
+    ap.add_argument("--window", type=int, default=0, help="sliding window in tokens (0: none)")
     args = ap.parse_args()
-    global PAGED
+    global PAGED, KV8, QLEN, WINDOW
     PAGED = args.paged
+    KV8 = args.kv_dtype == "e4m3"
+    QLEN = args.q_len
+    WINDOW = args.window
+    if QLEN < 1 or WINDOW < 0:
+        ap.error("--q-len must be >= 1 and --window >= 0")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
