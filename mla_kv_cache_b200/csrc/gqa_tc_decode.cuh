@@ -70,8 +70,7 @@ constexpr int HB = 64;                    // query heads per unit (value-product
 constexpr int CHUNK = TILE * 128;         // one [128 tokens x 128 bytes] box: 16 KB
 constexpr int RING = 12 * CHUNK;          // the stage ring: 192 KB
 constexpr int QREGION = 2 * HB * 128;     // query blocks: 16 KB (one of 64 heads or two of <= 32)
-constexpr int NTHREADS = 192;             // producer, MMA, 4 softmax warps
-constexpr int NSOFT = 128;
+constexpr int NTHREADS_MAX = 320;         // producer, MMA, up to two groups of 4 softmax warps
 constexpr uint32_t TM_S = 0;              // two score buffers
 constexpr int NST_MAX = 6;
 constexpr float P8_LOG2 = 6.f;            // E4M3 P^T holds 2^6 * 2^(s - m)
@@ -96,11 +95,14 @@ struct Kv {
 
 constexpr int OFF_ST = 0;
 constexpr int OFF_Q = OFF_ST + RING;               // 196608
-constexpr int OFF_RED = OFF_Q + QREGION;              // [3][4][64] fp32: tile slots 0/1, piece end
-constexpr int OFF_MS = OFF_RED + 3 * 4 * HB * 4;   // [2][64] running max per head
-constexpr int OFF_AS = OFF_MS + 2 * HB * 4;        // [2][64] rescale factor per head
-constexpr int OFF_NF = OFF_AS + 2 * HB * 4;        // [2][64] bytes: head rescaled this tile
-constexpr int OFF_LINV = OFF_NF + 2 * HB;          // [64] 1 / row sum
+constexpr int OFF_RED = OFF_Q + QREGION;              // [4][4][64] fp32: tile maxima of groups 0/1, piece-end sums
+constexpr int OFF_MS = OFF_RED + 4 * 4 * HB * 4;   // [2][64] running max after a group's latest tile
+constexpr int OFF_ASO = OFF_MS + 2 * HB * 4;       // [2][64] rescale of O^T since the previous tile
+constexpr int OFF_ASL = OFF_ASO + 2 * HB * 4;      // [2][64] rescale of a group's row sums
+constexpr int OFF_NFO = OFF_ASL + 2 * HB * 4;      // [2][64] bytes: O^T column rescaled this tile
+constexpr int OFF_NFL = OFF_NFO + 2 * HB;          // [2][64] bytes: row sum rescaled this tile
+constexpr int OFF_MFIN = OFF_NFL + 2 * HB;         // [2][64] each group's last max (piece end)
+constexpr int OFF_LINV = OFF_MFIN + 2 * HB * 4;    // [64] 1 / row sum
 constexpr int OFF_QS = OFF_LINV + HB * 4;          // [2] fp32: 2^-e of each E4M3 query buffer
 constexpr int OFF_BARS = OFF_QS + 16;
 constexpr int OFF_TMEMPTR = OFF_BARS + 256;
@@ -118,7 +120,9 @@ struct Bars {
     uint64_t pready[2];   // P^T written (and O^T rescaled): the value product may run
     uint64_t odone[2];    // value product of a tile (parity tile & 1) finished
     uint64_t ofree;       // the epilogue has read O^T
-    uint64_t grp;         // barrier of the 128 softmax threads
+    uint64_t grp[2];      // barrier of a softmax group's four warps
+    uint64_t hand[2];     // running max after a tile of group g published (two groups)
+    uint64_t all;         // barrier of every softmax warp (piece end)
 };
 static_assert(sizeof(Bars) <= 256, "barrier block overflows its slot");
 
@@ -133,6 +137,11 @@ struct Cfg {
     // query buffers: two when they fit, so that the next piece's block loads while the
     // current piece still reads its own
     static constexpr int NQB = 2 * QBLOCK <= QREGION ? 2 : 1;
+    // softmax groups: two, taking alternate tiles, for 16 and 32 columns (where one
+    // group's per-tile work paces the kernel); one for 8 columns (the data's arrival
+    // paces it, measured) and for 64 (a thread's registers do not allow 320 threads)
+    static constexpr int NG = (NR == 16 || NR == 32) ? 2 : 1;
+    static constexpr int NTHREADS = 64 + 128 * NG;
 };
 
 struct Ctx {
@@ -504,29 +513,49 @@ __device__ __forceinline__ void mma_issuer(const GqaParams &p, const Ctx &c, int
     }
 }
 
-// ------------------------------------------------------------------ softmax (warps 2-5)
+// ------------------------------------------------------------------ softmax (warps 2 ..)
+// NG groups of four warps (one thread per TMEM lane each).  With two groups, group g
+// takes the tiles kt with kt % 2 == g (and the score buffer g), so one group's tile
+// overlaps the other's; the running max of each column is handed from group to group
+// through shared memory (ms[g]) and the hand[g] barriers -- the one serial step.  Each
+// group keeps its own row sums, relative to the max it last used; at the end of a piece
+// they are merged at the final max.  O^T is rescaled, in tile order, by the factor
+// between consecutive tiles' maxima.
 template <int NR, bool KV8>
 __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, int warp, int lane) {
     using C = Cfg<NR>;
     using L = Kv<KV8>;
     constexpr int NQ = C::NQ;
     constexpr int NST = L::NST;
+    constexpr int NG = C::NG;
+    constexpr int NOWN = (NR + 31) / 32;            // warps holding owner threads
     constexpr uint32_t O_LO = KV8 ? NQ : HB;     // column of O^T's remainder half
     Bars *bars = c.bars;
+    const int g = (warp - 2) >> 2;        // group
+    const int wg = (warp - 2) & 3;        // warp within the group
     const int q = warp & 3;               // TMEM lane quadrant
     const int r = 32 * q + lane;          // token row of a tile / output dimension
-    const int st_id = (warp - 2) * 32 + lane;
+    const int st_id = wg * 32 + lane;     // owner index (column) within the group
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     float *red = reinterpret_cast<float *>(c.smem + OFF_RED);
     float *ms = reinterpret_cast<float *>(c.smem + OFF_MS);
-    float *as = reinterpret_cast<float *>(c.smem + OFF_AS);
-    uint8_t *nf = c.smem + OFF_NF;
+    float *aso = reinterpret_cast<float *>(c.smem + OFF_ASO);
+    float *asl = reinterpret_cast<float *>(c.smem + OFF_ASL);
+    uint8_t *nfo = c.smem + OFF_NFO;
+    uint8_t *nfl = c.smem + OFF_NFL;
+    float *mfin = reinterpret_cast<float *>(c.smem + OFF_MFIN);
     float *linv = reinterpret_cast<float *>(c.smem + OFF_LINV);
-    uint32_t grp_uses = 0;
+    uint32_t grp_uses = 0, all_uses = 0;
     auto grp_sync = [&]() -> bool {
-        warp_arrive(&bars->grp, lane);
-        const bool ok = mbar_wait(&bars->grp, grp_uses & 1u, FLAG_FULL_WAIT, c.abort_flag);
+        warp_arrive(&bars->grp[g], lane);
+        const bool ok = mbar_wait(&bars->grp[g], grp_uses & 1u, FLAG_FULL_WAIT, c.abort_flag);
         ++grp_uses;
+        return warp_all(ok);
+    };
+    auto all_sync = [&]() -> bool {
+        warp_arrive(&bars->all, lane);
+        const bool ok = mbar_wait(&bars->all, all_uses & 1u, FLAG_FULL_WAIT, c.abort_flag);
+        ++all_uses;
         return warp_all(ok);
     };
 
@@ -548,12 +577,12 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
             if (!warp_all(mbar_wait(&bars->qconv[qb], (uint32_t)qu & 1u, FLAG_MMA_WAIT, c.abort_flag))) return;
             cs *= p.k_scale * reinterpret_cast<const float *>(c.smem + OFF_QS)[qb];
         }
-        float m_own = -INFINITY;              // running max of head st_id (owner threads)
+        float m_own = -INFINITY;              // max of column st_id this group last used (owners)
         float l_part[NR];
 #pragma unroll
         for (int h = 0; h < NR; ++h) l_part[h] = 0.f;
 
-        for (int t = 0; t < nt; ++t) {
+        for (int t = NG == 1 ? 0 : ((g - k) & 1); t < nt; t += NG) {
             const int kt = k + t;
             const int s = kt % NST, sb = kt & 1;
             const int lt = pc.lt0 + t;
@@ -605,40 +634,52 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                 sc[h] = ((vis >> h) & 1ull) ? __uint_as_float(sv[h]) * cs : -INFINITY;
                 v[h] = sc[h];
             }
-            // ---- per-head maximum over the tile's 128 tokens
+            // ---- per-column maximum over the tile's 128 tokens
             warp_xreduce<NR, true>(v, lane);
-            store_reduced<NR>(red + (sb * 4 + q) * HB, v, lane);
+            store_reduced<NR>(red + (g * 4 + q) * HB, v, lane);
             if (!grp_sync()) return;
+            // ---- owners: the running max after this tile (from the previous tile's, which
+            //      the other group handed over), the rescale of O^T since the previous
+            //      tile and of this group's row sums since its own previous tile
             if (st_id < NR) {
-                const float tm = fmaxf(fmaxf(red[(sb * 4 + 0) * HB + st_id], red[(sb * 4 + 1) * HB + st_id]),
-                                       fmaxf(red[(sb * 4 + 2) * HB + st_id], red[(sb * 4 + 3) * HB + st_id]));
-                float alpha = 1.f;
-                uint8_t need = 0;
-                if (t == 0) {
-                    m_own = tm;
-                } else if (tm > m_own + L::RESCALE) {
-                    alpha = fast_exp2(m_own - tm);
-                    m_own = tm;
-                    need = 1;
+                const float tm = fmaxf(fmaxf(red[(g * 4 + 0) * HB + st_id], red[(g * 4 + 1) * HB + st_id]),
+                                       fmaxf(red[(g * 4 + 2) * HB + st_id], red[(g * 4 + 3) * HB + st_id]));
+                float m_prev = m_own;
+                if (NG == 2 && t > 0) {
+                    if (!mbar_wait(&bars->hand[g ^ 1], (uint32_t)((kt - 1) >> 1) & 1u, FLAG_FULL_WAIT, c.abort_flag))
+                        m_prev = -INFINITY;   // (abandoned: the group's next wait fails too)
+                    else
+                        m_prev = ms[(g ^ 1) * HB + st_id];
                 }
-                ms[sb * HB + st_id] = m_own;
-                as[sb * HB + st_id] = alpha;
-                nf[sb * HB + st_id] = need;
+                const float m_new = (t == 0 || tm > m_prev + L::RESCALE) ? tm : m_prev;
+                const bool need_o = t > 0 && m_new != m_prev;
+                const bool need_l = m_own != m_new && m_own != -INFINITY;
+                ms[g * HB + st_id] = m_new;
+                aso[g * HB + st_id] = need_o ? fast_exp2(m_prev - m_new) : 1.f;
+                asl[g * HB + st_id] = need_l ? fast_exp2(m_own - m_new) : 1.f;
+                nfo[g * HB + st_id] = need_o;
+                nfl[g * HB + st_id] = need_l;
+                m_own = m_new;
             }
+            if (NG == 2 && wg < NOWN) warp_arrive(&bars->hand[g], lane);
             if (!grp_sync()) return;
+            if (*c.abort_flag) return;
             // ---- weights: P^T row r, high part and remainder, into the stage's K half
-            uint32_t anyw = 0;
+            uint32_t any_o = 0, any_l = 0;
 #pragma unroll
-            for (int h = 0; h < NR; h += 4) anyw |= *reinterpret_cast<const uint32_t *>(nf + sb * HB + h);
-            const bool rescale = anyw != 0;     // the same for every thread
-            const float *as_t = as + sb * HB;
-            if (rescale) {
+            for (int h = 0; h < NR; h += 4) {
+                any_o |= *reinterpret_cast<const uint32_t *>(nfo + g * HB + h);
+                any_l |= *reinterpret_cast<const uint32_t *>(nfl + g * HB + h);
+            }
+            if (any_l != 0) {
+                const float *a = asl + g * HB;
 #pragma unroll
                 for (int h = 0; h < NR; h += 4) {
-                    const float4 x = *reinterpret_cast<const float4 *>(as_t + h);
+                    const float4 x = *reinterpret_cast<const float4 *>(a + h);
                     l_part[h] *= x.x; l_part[h + 1] *= x.y; l_part[h + 2] *= x.z; l_part[h + 3] *= x.w;
                 }
             }
+            const float *msg = ms + g * HB;
             uint8_t *st = c.smem + OFF_ST + s * L::STAGE;
             if constexpr (KV8) {
                 // 16 heads per 16-byte row of a 2 KB block, the remainders' blocks after the
@@ -653,7 +694,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                             float a[4];
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
-                                const float mu = ms[sb * HB + h + u];
+                                const float mu = msg[h + u];
                                 // 2^6 * 2^(s - m), summed in the same units
                                 a[u] = fast_exp2(sc[h + u] - (mu == -INFINITY ? 0.f : mu) + P8_LOG2);
                                 l_part[h + u] += a[u];
@@ -669,38 +710,39 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                     *reinterpret_cast<uint4 *>(st + NQ * 128 + cb * 2048 + r * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
                 }
             } else {
-            uint8_t *hrow = st + r * 128;
-            uint8_t *lrow = st + CHUNK + r * 128;
+                uint8_t *hrow = st + r * 128;
+                uint8_t *lrow = st + CHUNK + r * 128;
 #pragma unroll
-            for (int cc = 0; cc < NR / 8; ++cc) {
-                uint32_t hw[4], lw[4];
-                const float4 m0 = *reinterpret_cast<const float4 *>(ms + sb * HB + 8 * cc);
-                const float4 m1 = *reinterpret_cast<const float4 *>(ms + sb * HB + 8 * cc + 4);
-                // (a column with no visible token so far has max -inf; its weights are 0)
-                float mh[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                for (int cc = 0; cc < NR / 8; ++cc) {
+                    uint32_t hw[4], lw[4];
+                    const float4 m0 = *reinterpret_cast<const float4 *>(msg + 8 * cc);
+                    const float4 m1 = *reinterpret_cast<const float4 *>(msg + 8 * cc + 4);
+                    // (a column with no visible token so far has max -inf; its weights are 0)
+                    float mh[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) mh[e] = mh[e] == -INFINITY ? 0.f : mh[e];
+                    for (int e = 0; e < 8; ++e) mh[e] = mh[e] == -INFINITY ? 0.f : mh[e];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int h = 8 * cc + 2 * e;
-                    const float a = fast_exp2(sc[h] - mh[2 * e]);
-                    const float b = fast_exp2(sc[h + 1] - mh[2 * e + 1]);
-                    l_part[h] += a;
-                    l_part[h + 1] += b;
-                    split_bf16x2(a, b, hw[e], lw[e]);
+                    for (int e = 0; e < 4; ++e) {
+                        const int h = 8 * cc + 2 * e;
+                        const float a = fast_exp2(sc[h] - mh[2 * e]);
+                        const float b = fast_exp2(sc[h + 1] - mh[2 * e + 1]);
+                        l_part[h] += a;
+                        l_part[h + 1] += b;
+                        split_bf16x2(a, b, hw[e], lw[e]);
+                    }
+                    const int slot = (cc ^ (r & 7)) << 4;
+                    *reinterpret_cast<uint4 *>(hrow + slot) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4 *>(lrow + slot) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
                 }
-                const int slot = (cc ^ (r & 7)) << 4;
-                *reinterpret_cast<uint4 *>(hrow + slot) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4 *>(lrow + slot) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            }
             }
             fence_proxy_async_smem();
-            // ---- rescale the affected heads' columns of O^T (after the previous value product)
-            if (rescale) {
+            // ---- rescale the affected columns of O^T (after the previous tile's value product)
+            if (any_o != 0) {
                 if (!warp_all(mbar_wait(&bars->odone[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u, FLAG_MMA_WAIT,
                                         c.abort_flag)))
                     return;
                 tc_fence_after();
+                const float *a = aso + g * HB;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -712,7 +754,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
 #pragma unroll
                         for (int h = 0; h < 16; h += 4) {
                             if (c0 + h < NR) {
-                                const float4 x = *reinterpret_cast<const float4 *>(as_t + c0 + h);
+                                const float4 x = *reinterpret_cast<const float4 *>(a + c0 + h);
                                 ov[h] = __float_as_uint(__uint_as_float(ov[h]) * x.x);
                                 ov[h + 1] = __float_as_uint(__uint_as_float(ov[h + 1]) * x.y);
                                 ov[h + 2] = __float_as_uint(__uint_as_float(ov[h + 2]) * x.z);
@@ -729,13 +771,14 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
         }
         k += nt;
 
-        // ---- end of the piece: row sums, lse, output
+        // ---- end of the piece: the groups' row sums (merged at the final max), lse, output
         float v[NR];
 #pragma unroll
         for (int h = 0; h < NR; ++h) v[h] = l_part[h];
         warp_xreduce<NR, false>(v, lane);
-        store_reduced<NR>(red + (2 * 4 + q) * HB, v, lane);
-        if (!grp_sync()) return;
+        store_reduced<NR>(red + ((2 + g) * 4 + q) * HB, v, lane);
+        if (st_id < NR) mfin[g * HB + st_id] = m_own;
+        if (!all_sync()) return;
         // columns of the unit: (query position qi, head h of the group), qi-major; output
         // row of column cc in out [B, q_len, n_q, d] / lse [B, q_len, n_q]
         const int h_real = min(HB, p.g * p.q_len - hb * HB);
@@ -745,13 +788,22 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
             const int qi = vr / p.g;
             return ((size_t)pc.b * p.q_len + qi) * p.n_q + (size_t)j * p.g + (vr - qi * p.g);
         };
-        if (st_id < NR) {
-            const float l = red[(8 + 0) * HB + st_id] + red[(8 + 1) * HB + st_id] + red[(8 + 2) * HB + st_id] +
-                            red[(8 + 3) * HB + st_id];
+        if (g == 0 && st_id < NR) {
+            float M = -INFINITY, l = 0.f, lg[NG], mg[NG];
+#pragma unroll
+            for (int x = 0; x < NG; ++x) {
+                lg[x] = red[((2 + x) * 4 + 0) * HB + st_id] + red[((2 + x) * 4 + 1) * HB + st_id] +
+                        red[((2 + x) * 4 + 2) * HB + st_id] + red[((2 + x) * 4 + 3) * HB + st_id];
+                mg[x] = mfin[x * HB + st_id];
+                M = fmaxf(M, mg[x]);
+            }
+#pragma unroll
+            for (int x = 0; x < NG; ++x)
+                if (lg[x] > 0.f) l += mg[x] == M ? lg[x] : lg[x] * fast_exp2(mg[x] - M);
             // (E4M3 cache: l and O^T both carry 2^6; the value scale enters here)
             linv[st_id] = l > 0.f ? (KV8 ? p.v_scale : 1.f) / l : 0.f;
             const float lse_v =
-                l > 0.f ? (m_own + __log2f(l) - (KV8 ? P8_LOG2 : 0.f)) * 0.69314718055994531f : -INFINITY;
+                l > 0.f ? (M + __log2f(l) - (KV8 ? P8_LOG2 : 0.f)) * 0.69314718055994531f : -INFINITY;
             if (st_id < h_real) {
                 if (pc.whole)
                     p.lse[out_row(st_id)] = lse_v;
@@ -759,13 +811,15 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                     p.ws_lse[part + st_id] = lse_v;
             }
         }
-        if (!grp_sync()) return;
+        if (!all_sync()) return;
         const int klast = k - 1;
         if (!warp_all(mbar_wait(&bars->odone[klast & 1], (uint32_t)(klast >> 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
             return;
         tc_fence_after();
+        // 16-column chunks of O^T, taken by the groups in turn
 #pragma unroll
         for (int c0 = 0; c0 < NQ; c0 += 16) {
+            if ((c0 / 16) % NG != g) continue;
             uint32_t ov[16], ol[16];
             tmem_ld16(c.tmem + lane_base + L::TM_O + c0, ov);
             tmem_ld16(c.tmem + lane_base + L::TM_O + O_LO + c0, ol);
@@ -787,7 +841,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
 }  // namespace gqatc
 
 template <int NR, bool KV8>
-__global__ void __launch_bounds__(gqatc::NTHREADS, 1)
+__global__ void __launch_bounds__(gqatc::Cfg<NR>::NTHREADS, 1)
 gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
     using namespace gqatc;
@@ -811,14 +865,17 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
             mbar_init(&bars->qempty[i], 1);
             mbar_init(&bars->qconv[i], 32);
         }
+        constexpr int NG = Cfg<NR>::NG;
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->sready[i], 1);
-            mbar_init(&bars->sfree[i], NSOFT / 32);
-            mbar_init(&bars->pready[i], NSOFT / 32);
+            mbar_init(&bars->sfree[i], 4);        // the four warps of the tile's group
+            mbar_init(&bars->pready[i], 4);
             mbar_init(&bars->odone[i], 1);
+            mbar_init(&bars->grp[i], 4);
+            mbar_init(&bars->hand[i], (NR + 31) / 32);   // the group's warps holding owners
         }
-        mbar_init(&bars->ofree, NSOFT / 32);
-        mbar_init(&bars->grp, NSOFT / 32);
+        mbar_init(&bars->ofree, 4 * NG);
+        mbar_init(&bars->all, 4 * NG);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -828,7 +885,7 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
     }
     if (warp == 2) build_tile_prefix(p.seq_lens, p.B, p.T_max, TILE, s_prefix, lane, p.q_len, p.window);
     // query buffers start zeroed: rows a unit's block does not fill stay finite
-    for (int i = tid; i < QREGION / 16; i += NTHREADS)
+    for (int i = tid; i < QREGION / 16; i += Cfg<NR>::NTHREADS)
         reinterpret_cast<uint4 *>(smem + OFF_Q)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
     if (warp == 0 && lane == 0) {
@@ -852,7 +909,7 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
     if (blockIdx.x == 0) {
         MetaView mv = meta_view(p.ws_meta);
         if (tid == 0) { mv.w_total[0] = W; mv.w_total[1] = total; }
-        for (int i = tid; i <= p.B; i += NTHREADS) mv.prefix[i] = s_prefix[i];
+        for (int i = tid; i <= p.B; i += Cfg<NR>::NTHREADS) mv.prefix[i] = s_prefix[i];
     }
     // The combine kernel may be scheduled now; it waits for this grid to finish.
     pdl_launch_dependents();
