@@ -13,9 +13,10 @@
 // all of one SM's tensor memory.  A 2-CTA cluster therefore splits the latent columns:
 // CTA r holds columns [256r, 256r + 256) of every cached row (CTA 0 also the 64 RoPE
 // columns) and the accumulator O_r = P * C[:, 256r..] (128 x 256 fp32, 256 TMEM columns).
-// Each CTA computes partial scores over its part of the 576-wide contraction and stores
-// them into the other CTA's shared memory (distributed shared memory; each sending
-// thread then arrives with release semantics on the receiver's mbarrier); both CTAs add the two partials in the same order and run
+// Each CTA computes partial scores over its part of the 576-wide contraction, stages
+// them in a local send buffer, and one bulk copy per tile (distributed shared memory,
+// issued by warp 2) moves them into the other CTA's receive buffer, completing its
+// mbarrier's transaction count; both CTAs add the two partials in the same order and run
 // the identical online softmax, so P, the rescale factors and the row sums never cross
 // the pair.  Every cached byte is loaded from HBM once; every MMA is M = 128.
 //
@@ -29,6 +30,7 @@
 // Per 64-token tile and CTA:
 //   TMA (warp 0)       4 (CTA 0: 5) 128-byte-swizzled boxes [64 tokens x 64 columns]
 //                      into a 3-stage ring; CTA 0 also the q_rope block once per piece.
+//   send (warp 2)      one bulk copy per tile of the staged partial scores to the peer.
 //   MMA (warp 1)       S_r = Q_r C_r^T: 16 MMAs 128x64x16 with A from TMEM (CTA 0: 4 more
 //                      with the RoPE query from shared memory); O_r += P C_r: 8 MMAs
 //                      128x256x16 with A = P from TMEM and C_r read MN-major from the same
@@ -60,7 +62,7 @@ constexpr int NST = 3;                   // pipeline stages
 constexpr int CHUNK_T = TILE * 128;      // one [64 tokens x 64 cols] bf16 box: 8 KB
 constexpr int STAGE = NCH * CHUNK_T;     // 40 KB
 constexpr int QROPE = HR * 128;          // q_rope block [128 heads x 64] bf16: 16 KB
-constexpr int NTHREADS = 384;            // warpgroup 0: producer, MMA (2 idle warps); 1, 2: softmax groups
+constexpr int NTHREADS = 384;            // warpgroup 0: producer, MMA, sender (1 idle warp); 1, 2: softmax groups
 constexpr int REGS_WG0 = 96;             // registers per thread after reallocation: warpgroup 0
 constexpr int REGS_SOFTMAX = 200;        //   softmax warpgroups (128 x 96 + 256 x 200 <= 384 x 168)
 constexpr int NGROUP = 128;              // threads per softmax group
@@ -75,12 +77,13 @@ constexpr uint32_t RECV_BYTES = HR * TILE * 4;   // the peer's partial scores of
 
 constexpr int OFF_ST = 0;
 constexpr int OFF_QROPE = OFF_ST + NST * STAGE;          // 122880
-constexpr int OFF_RECV = OFF_QROPE + QROPE;              // 139264: two [128 heads][64] fp32
+constexpr int OFF_RECV = OFF_QROPE + QROPE;              // 139264: [128 heads][64] fp32 from the peer
+constexpr int OFF_SEND = OFF_RECV + (int)RECV_BYTES;     // 172032: [128 heads][64] fp32 to the peer
 constexpr int OFF_MREF = OFF_RECV + 2 * (int)RECV_BYTES; // 204800: [2][128] running max
 constexpr int OFF_LX = OFF_MREF + 2 * HR * 4;            // [2][128] row sums of the groups
 constexpr int OFF_BARS = OFF_LX + 2 * HR * 4;            // 206848
 constexpr int OFF_TMEMPTR = OFF_BARS + 256;
-constexpr int OFF_ABORT = OFF_TMEMPTR + 16;
+constexpr int OFF_ABORT = OFF_TMEMPTR + 16;     // abort flag; +8: tiles whose send buffer the sender has read
 constexpr int OFF_PREFIX = OFF_ABORT + 16;
 constexpr int smem_bytes(int B) { return 1024 + OFF_PREFIX + (B + 1) * 4; }
 
@@ -91,8 +94,9 @@ struct Bars {
     uint64_t qempty;       // every score MMA of the piece has read Q
     uint64_t sready[2];    // partial scores of a tile (parity) in TMEM
     uint64_t sfree;        // the tile's group has read them
-    uint64_t recv_full[2]; // the peer's partial scores of a tile of group g landed (its 128 rows)
-    uint64_t recv_free[2]; // the peer has read what this CTA sent into its buffer g
+    uint64_t recv_full[2]; // the peer's partial scores of a tile of group g landed (armed by g)
+    uint64_t peer_rfree;   // the peer has consumed the tile this CTA last sent (4 remote arrivals)
+    uint64_t staged;       // a tile's partial scores written into the send buffer (4 warps)
     uint64_t hand[2];      // running max of a tile (parity) published
     uint64_t pready;       // P of a tile in TMEM and O rescaled: the value product may run
     uint64_t odone[2];     // value product of a tile (parity) finished
@@ -273,6 +277,62 @@ __device__ __forceinline__ void mma_issuer(const MlaParams &p, const Ctx &c) {
     }
 }
 
+// Monotone count of tiles whose send buffer the bulk copy has read (a counter, not an
+// mbarrier: the two groups wait on it for alternate tiles, so a phase parity could be
+// two phases behind one of them).
+__device__ __forceinline__ void publish_count(int *cnt, int v) {
+    asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(cnt)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int read_count(const int *cnt) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(cnt)) : "memory");
+    return v;
+}
+// Bounded wait until the count reaches `target`.
+__device__ __forceinline__ bool wait_count(const int *cnt, int target, unsigned int flag, volatile int *abort) {
+    if (read_count(cnt) >= target) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (read_count(cnt) >= target) return true;
+        if (abort != nullptr && *abort) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            atomicOr(&g_device_flags, flag);
+            if (abort != nullptr) *abort = 1;
+            return false;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ sender (warp 2, lane 0)
+// Ships each tile's partial scores to the peer: once the tile's group has staged them in
+// the send buffer and the peer has consumed the previous tile, one bulk copy moves the
+// 32 KB into the peer's receive buffer and completes the transaction count of the
+// peer's recv_full barrier of the tile's group; the send buffer is released (the count)
+// as soon as the copy has read it.  (Per-thread remote stores of the same bytes took
+// ~2.8 us per tile.)
+__device__ __forceinline__ void sender(const MlaParams &p, const Ctx &c) {
+    Bars *bars = c.bars;
+    const uint32_t src = smem_u32(c.smem + OFF_SEND);
+    const uint32_t dst = map_to_rank(smem_u32(c.smem + OFF_RECV), c.peer);
+    const uint32_t dst_bar0 = map_to_rank(smem_u32(&bars->recv_full[0]), c.peer);
+    const uint32_t dst_bar1 = map_to_rank(smem_u32(&bars->recv_full[1]), c.peer);
+    int *sent = reinterpret_cast<int *>(c.smem + OFF_ABORT + 8);
+    int k = 0;
+    for (long long pos = c.p0; pos < c.p1;) {
+        const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
+        pos = pc.ustart + pc.lt1;
+        for (int t = 0; t < pc.lt1 - pc.lt0; ++t, ++k) {
+            if (!mbar_wait(&bars->staged, (uint32_t)k & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
+            if (k > 0 && !mbar_wait_cluster(&bars->peer_rfree, (uint32_t)(k - 1) & 1u, FLAG_PEER_WAIT, c.abort_flag))
+                return;
+            bulk_copy_to_peer(dst, src, RECV_BYTES, (k & 1) ? dst_bar1 : dst_bar0);
+            bulk_commit_group();
+            bulk_wait_read_all();
+            publish_count(sent, k + 1);
+        }
+    }
+}
+
 // 16-byte chunk slot of chunk j (columns 4j..4j+3) in row h of a receive buffer.
 __device__ __forceinline__ int recv_chunk(int j, int h) { return j ^ (h & 7); }
 
@@ -283,10 +343,9 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
     const int q = warp & 3;                     // TMEM lane quadrant
     const int h = 32 * q + lane;                // head row
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    const float *recv = reinterpret_cast<const float *>(c.smem + OFF_RECV + g * RECV_BYTES) + h * TILE;
-    const uint32_t peer_recv = map_to_rank(smem_u32(c.smem + OFF_RECV + g * RECV_BYTES), c.peer) + h * TILE * 4;
-    const uint32_t peer_recv_full = map_to_rank(smem_u32(&bars->recv_full[g]), c.peer);
-    const uint32_t peer_recv_free = map_to_rank(smem_u32(&bars->recv_free[g]), c.peer);
+    const float *recv = reinterpret_cast<const float *>(c.smem + OFF_RECV) + h * TILE;
+    uint8_t *send = c.smem + OFF_SEND + h * TILE * 4;
+    const uint32_t peer_rfree = map_to_rank(smem_u32(&bars->peer_rfree), c.peer);
     float *mref = reinterpret_cast<float *>(c.smem + OFF_MREF);
     float *lx = reinterpret_cast<float *>(c.smem + OFF_LX);
 
@@ -344,53 +403,52 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             }
             tc_fence_before();
             mbar_arrive(&bars->sfree);
-            // ---- to the peer (its buffer g must be free: it has read tile kt - 2)
-            if (kt >= 2 && !warp_all(mbar_spin<true>(&bars->recv_free[g], (uint32_t)((kt >> 1) - 1) & 1u,
-                                                       FLAG_PEER_WAIT, c.abort_flag)))
+            // ---- to the peer: into the send buffer (free once the previous tile's copy has
+            //      read it), same row layout as the peer's receive buffer; the sender thread
+            //      ships it
+            if (kt >= 1 && !warp_all(wait_count(reinterpret_cast<const int *>(c.smem + OFF_ABORT + 8), kt,
+                                                  FLAG_PEER_WAIT, c.abort_flag)))
                 return;
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-                st_cluster_v4(peer_recv + (uint32_t)(recv_chunk(j, h) * 16), sv[4 * j], sv[4 * j + 1], sv[4 * j + 2],
-                              sv[4 * j + 3]);
-            mbar_arrive_cluster(peer_recv_full);   // release: the stores above are visible first
+                *reinterpret_cast<uint4 *>(send + recv_chunk(j, h) * 16) =
+                    make_uint4(sv[4 * j], sv[4 * j + 1], sv[4 * j + 2], sv[4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->staged);
             // ---- the peer's partial scores; both CTAs add (own + peer) in the same order
             if (!warp_all(mbar_spin<true>(&bars->recv_full[g], (uint32_t)(kt >> 1) & 1u, FLAG_PEER_WAIT,
                                             c.abort_flag)))
                 return;
-            // raw scores (own + peer, unscaled) in place from here on; only a tile with
-            // rows outside the sequence needs the mask
+            // arm this group's next tile (kt + 2): its phase of recv_full[g] is the next one
+            if (h == 0) mbar_arrive_expect_tx(&bars->recv_full[g], RECV_BYTES);
+            // raw scores (own + peer, unscaled) in place from here on
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float4 v = reinterpret_cast<const float4 *>(recv)[recv_chunk(j, h)];
+                sv[4 * j] = __float_as_uint(__uint_as_float(sv[4 * j]) + v.x);
+                sv[4 * j + 1] = __float_as_uint(__uint_as_float(sv[4 * j + 1]) + v.y);
+                sv[4 * j + 2] = __float_as_uint(__uint_as_float(sv[4 * j + 2]) + v.z);
+                sv[4 * j + 3] = __float_as_uint(__uint_as_float(sv[4 * j + 3]) + v.w);
+            }
+            // the received values are in registers (the adds above consumed them, and
+            // instructions issue in order): the peer may send the next tile at once
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_relaxed(peer_rfree);
+            // only a tile with rows outside the sequence needs the mask
             float mx = -INFINITY;
-            const bool full = tok_lo == 0 && tok_hi == TILE;
-            if (full) {
+            if (tok_lo == 0 && tok_hi == TILE) {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float4 v = reinterpret_cast<const float4 *>(recv)[recv_chunk(j, h)];
-                    const float pv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float x = __uint_as_float(sv[4 * j + e]) + pv[e];
-                        sv[4 * j + e] = __float_as_uint(x);
-                        mx = fmaxf(mx, x);
-                    }
-                }
+                for (int i = 0; i < 64; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
             } else {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float4 v = reinterpret_cast<const float4 *>(recv)[recv_chunk(j, h)];
-                    const float pv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int col = 4 * j + e;
-                        float x = __uint_as_float(sv[col]) + pv[e];
-                        x = (col >= tok_lo && col < tok_hi) ? x : -INFINITY;
-                        sv[col] = __float_as_uint(x);
-                        mx = fmaxf(mx, x);
-                    }
+                for (int i = 0; i < 64; ++i) {
+                    const float x = (i >= tok_lo && i < tok_hi) ? __uint_as_float(sv[i]) : -INFINITY;
+                    sv[i] = __float_as_uint(x);
+                    mx = fmaxf(mx, x);
                 }
             }
             mx *= p.scale_log2;     // the scale is positive: max of the scaled scores
-            // the received values are consumed (mx depends on all of them)
-            mbar_arrive_cluster_relaxed(peer_recv_free);
             // ---- running max, handed on from the previous tile's group
             float m_prev = -INFINITY;
             if (kt > 0) {
@@ -520,16 +578,21 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
         mbar_init(&bars->sfree, NGROUP);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->sready[i], 1);
-            mbar_init(&bars->recv_full[i], NGROUP);
-            mbar_init(&bars->recv_free[i], NGROUP);
             mbar_init(&bars->hand[i], NGROUP);
             mbar_init(&bars->odone[i], 1);
         }
+        mbar_init(&bars->recv_full[0], 1);
+        mbar_init(&bars->recv_full[1], 1);
+        mbar_init(&bars->peer_rfree, 4);
+        mbar_init(&bars->staged, 4);
         mbar_init(&bars->pready, NGROUP);
         mbar_init(&bars->ofree, 2 * NGROUP);
         mbar_init(&bars->lx, 2 * NGROUP);
         *abort_flag = 0;
+        *reinterpret_cast<int *>(smem + OFF_ABORT + 8) = 0;
         fence_mbar_init();
+        mbar_arrive_expect_tx(&bars->recv_full[0], RECV_BYTES);   // the phases of tiles 0 and 1
+        mbar_arrive_expect_tx(&bars->recv_full[1], RECV_BYTES);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_ptr), TM_COLS);
@@ -571,6 +634,7 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
         if (c.p0 < total) {
             if (warp == 0 && lane == 0) producer(p, maps, c);
             if (warp == 1 && lane == 0) mma_issuer(p, c);
+            if (warp == 2 && lane == 0) sender(p, c);
         }
     } else {
         regs_inc<REGS_SOFTMAX>();
