@@ -241,6 +241,23 @@ int kvattn_rope_append(uint16_t *q, const uint16_t *k_new, const uint16_t *v_new
                        float rope_base, int interleaved, void *stream);
 
 /*
+ * kvattn_rope_append into an E4M3 (fp8) cache, the producer side of
+ * kvattn_gqa_decode_fp8: q is rotated in place (bf16) as above; the new token's rotated
+ * key is stored as E4M3 codes of key / k_scale and its value as codes of value /
+ * v_scale (the quotient taken in fp32, correctly rounded; the nearest code, ties to
+ * even, magnitudes past 448 saturated to +-448, NaN to the NaN code), so that the
+ * cached value is code * scale as the decode reads it.
+ *   k_cache, v_cache  device E4M3 codes [batch, n_kv_heads, max_seq_len, head_dim]
+ *   k_scale, v_scale  finite, > 0 (the scales the cache was quantised with)
+ * Everything else, including positions outside the cache, as for kvattn_rope_append.
+ */
+int kvattn_rope_append_fp8(uint16_t *q, const uint16_t *k_new, const uint16_t *v_new,
+                           const int32_t *positions, uint8_t *k_cache, uint8_t *v_cache,
+                           int max_seq_len, int batch, int n_q_heads, int n_kv_heads, int head_dim,
+                           float rope_base, int interleaved, float k_scale, float v_scale,
+                           void *stream);
+
+/*
  * The same for absorbed MLA: q_rope [batch, n_heads, rope_dim] is rotated in place, the
  * new token's decoupled rotary key rope_new [batch, rope_dim] is rotated into
  * rope_cache[b, positions[b], :], and its latent latent_new [batch, latent_dim] is

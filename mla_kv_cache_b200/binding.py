@@ -62,6 +62,10 @@ _SIGNATURES = {
     "kvattn_rope_append": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, _c_u16p, _c_u16p,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
+    "kvattn_rope_append_fp8": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, ctypes.c_void_p,
+                                              ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                              ctypes.c_float, ctypes.c_float, ctypes.c_void_p]),
     "kvattn_mla_rope_append": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, _c_u16p,
                                               _c_u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
@@ -273,6 +277,28 @@ def kvattn_rope_append(q, k_new, v_new, positions, k_cache, v_cache, rope_base=1
                                   float(rope_base), int(bool(interleaved)), _stream_handle(stream))
     if st != KVATTN_OK:
         raise KvattnError(st, "kvattn_rope_append")
+
+
+def kvattn_rope_append_fp8(q, k_new, v_new, positions, k_cache, v_cache, k_scale, v_scale, rope_base=10000.0,
+                           interleaved=False, stream=None):
+    """kvattn_rope_append into an E4M3 cache (include/kvattn.h, kvattn_rope_append_fp8):
+    q [B, n_q, d] bf16 rotated in place; the rotated k_new and v_new [B, n_kv, d] bf16 are
+    stored as codes of value / scale in the caches [B, n_kv, T, d] (float8_e4m3fn or uint8)
+    at positions [B] (int32)."""
+    import torch
+    B, n_q, d = q.shape
+    n_kv, T = k_cache.shape[1], k_cache.shape[2]
+    _check(q, "q", torch.bfloat16)
+    _check(k_new, "k_new", torch.bfloat16, (B, n_kv, d))
+    _check(v_new, "v_new", torch.bfloat16, (B, n_kv, d))
+    _check(positions, "positions", torch.int32, (B,))
+    _check_e4m3(k_cache, "k_cache", (B, n_kv, T, d))
+    _check_e4m3(v_cache, "v_cache", (B, n_kv, T, d))
+    st = lib().kvattn_rope_append_fp8(q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), positions.data_ptr(),
+                                      k_cache.data_ptr(), v_cache.data_ptr(), T, B, n_q, n_kv, d, float(rope_base),
+                                      int(bool(interleaved)), float(k_scale), float(v_scale), _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_rope_append_fp8")
 
 
 def kvattn_mla_rope_append(q_rope, latent_new, rope_new, positions, latent_cache, rope_cache,

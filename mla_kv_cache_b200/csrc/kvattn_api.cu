@@ -921,7 +921,7 @@ int kvattn_clear_device_flags(void) {
 }
 
 // ---- rotary embedding of the new token + cache append
-static int launch_rope_append(RopeAppendParams &p, cudaStream_t s) {
+static int launch_rope_append(RopeAppendParams &p, cudaStream_t s, bool kv8 = false) {
     DeviceState *dev = nullptr;
     int st = device_state(&dev);
     if (st != KVATTN_OK) return st;
@@ -930,7 +930,10 @@ static int launch_rope_append(RopeAppendParams &p, cudaStream_t s) {
     const long long cap = (long long)dev->sms * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    rope_append_kernel<<<(unsigned)blocks, 256, 0, s>>>(p);
+    if (kv8)
+        rope_append_kernel<true><<<(unsigned)blocks, 256, 0, s>>>(p);
+    else
+        rope_append_kernel<false><<<(unsigned)blocks, 256, 0, s>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e, "rope append launch");
     return KVATTN_OK;
@@ -965,8 +968,8 @@ int kvattn_rope_append(uint16_t *q, const uint16_t *k_new, const uint16_t *v_new
     p.k_new = reinterpret_cast<const __nv_bfloat16 *>(k_new);
     p.v_new = reinterpret_cast<const __nv_bfloat16 *>(v_new);
     p.positions = positions;
-    p.k_cache = reinterpret_cast<__nv_bfloat16 *>(k_cache);
-    p.v_cache = reinterpret_cast<__nv_bfloat16 *>(v_cache);
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
     p.B = batch;
     p.n_q = n_q_heads;
     p.n_kv = n_kv_heads;
@@ -978,6 +981,55 @@ int kvattn_rope_append(uint16_t *q, const uint16_t *k_new, const uint16_t *v_new
     p.n_k_pairs = (long long)batch * n_kv_heads * (head_dim / 2);
     p.n_v_words = (long long)batch * n_kv_heads * (head_dim / 2);
     return launch_rope_append(p, static_cast<cudaStream_t>(stream));
+}
+
+int kvattn_rope_append_fp8(uint16_t *q, const uint16_t *k_new, const uint16_t *v_new, const int32_t *positions,
+                           uint8_t *k_cache, uint8_t *v_cache, int max_seq_len, int batch, int n_q_heads,
+                           int n_kv_heads, int head_dim, float rope_base, int interleaved, float k_scale,
+                           float v_scale, void *stream) {
+    if (!q || !k_new || !v_new || !positions || !k_cache || !v_cache) return KVATTN_ERR_INVALID_ARG;
+    if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || max_seq_len <= 0) return KVATTN_ERR_INVALID_ARG;
+    if (n_q_heads % n_kv_heads != 0) return KVATTN_ERR_INVALID_ARG;
+    if (head_dim <= 0 || (head_dim & 1) || head_dim > 1024) return KVATTN_ERR_UNSUPPORTED;
+    if (!std::isfinite(rope_base) || rope_base <= 0.f) return KVATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f))
+        return KVATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(positions) ||
+        !aligned16(k_cache) || !aligned16(v_cache))
+        return KVATTN_ERR_MISALIGNED;
+    const size_t q_bytes = (size_t)batch * n_q_heads * head_dim * 2;
+    const size_t new_bytes = (size_t)batch * n_kv_heads * head_dim * 2;
+    const size_t cache_bytes = (size_t)batch * n_kv_heads * max_seq_len * head_dim;
+    const void *w[3] = {q, k_cache, v_cache};
+    const size_t wn[3] = {q_bytes, cache_bytes, cache_bytes};
+    const void *r[3] = {k_new, v_new, positions};
+    const size_t rn[3] = {new_bytes, new_bytes, (size_t)batch * 4};
+    for (int i = 0; i < 3; ++i) {
+        for (int j = 0; j < 3; ++j)
+            if (overlaps(w[i], wn[i], r[j], rn[j])) return KVATTN_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 3; ++j)
+            if (overlaps(w[i], wn[i], w[j], wn[j])) return KVATTN_ERR_INVALID_ARG;
+    }
+    RopeAppendParams p = {};
+    p.q = reinterpret_cast<__nv_bfloat16 *>(q);
+    p.k_new = reinterpret_cast<const __nv_bfloat16 *>(k_new);
+    p.v_new = reinterpret_cast<const __nv_bfloat16 *>(v_new);
+    p.positions = positions;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.B = batch;
+    p.n_q = n_q_heads;
+    p.n_kv = n_kv_heads;
+    p.dq = p.dk = p.dv = head_dim;
+    p.T_max = max_seq_len;
+    p.log2_base = std::log2((double)rope_base);
+    p.interleaved = interleaved ? 1 : 0;
+    p.n_q_pairs = (long long)batch * n_q_heads * (head_dim / 2);
+    p.n_k_pairs = (long long)batch * n_kv_heads * (head_dim / 2);
+    p.n_v_words = (long long)batch * n_kv_heads * (head_dim / 2);
+    return launch_rope_append(p, static_cast<cudaStream_t>(stream), true);
 }
 
 int kvattn_mla_rope_append(uint16_t *q_rope, const uint16_t *latent_new, const uint16_t *rope_new,

@@ -14,7 +14,10 @@
 // formed and reduced in fp64 (positions reach tens of thousands of radians, where an
 // fp32 angle would be off by ~1e-3), then the pair is turned in fp32 and rounded to
 // bf16 once.  A position outside [0, T_max) is not written into the cache (the query
-// is still rotated with it).
+// is still rotated with it).  For an E4M3 cache (KV8) the rotated key and the value are
+// divided by their tensor's scale in fp32 (correctly rounded) and stored as the nearest
+// E4M3 codes (ties to even, magnitudes past 448 saturated): the cached value is code *
+// scale, as the decode reads it.
 #pragma once
 #include "common.cuh"
 
@@ -25,8 +28,9 @@ struct RopeAppendParams {
     const __nv_bfloat16 *k_new;    // [B, n_kv, dk]: rotated into k_cache
     const __nv_bfloat16 *v_new;    // [B, n_kv, dv]: copied into v_cache (null: none)
     const int32_t *positions;      // [B]
-    __nv_bfloat16 *k_cache;        // [B, n_kv, T_max, dk]
-    __nv_bfloat16 *v_cache;        // [B, n_kv, T_max, dv]
+    void *k_cache;                 // [B, n_kv, T_max, dk] bf16, or E4M3 codes (KV8)
+    void *v_cache;                 // [B, n_kv, T_max, dv] bf16, or E4M3 codes (KV8)
+    float k_scale, v_scale;        // E4M3 cache: value = code * scale
     int B, n_q, n_kv, dq, dk, dv, T_max;
     double log2_base;
     int interleaved;
@@ -49,6 +53,7 @@ __device__ __forceinline__ void rope_pair(const __nv_bfloat16 *row, int d, int i
     yb = fmaf(xa, sf, xb * cf);
 }
 
+template <bool KV8>
 __global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams p) {
     const long long total = p.n_q_pairs + p.n_k_pairs + p.n_v_words;
     for (long long w = (long long)blockIdx.x * blockDim.x + threadIdx.x; w < total;
@@ -77,9 +82,16 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams
             int ia, ib;
             float ya, yb;
             rope_pair(p.k_new + row * p.dk, p.dk, i, pos, p.log2_base, p.interleaved, ia, ib, ya, yb);
-            __nv_bfloat16 *dst = p.k_cache + (row * p.T_max + pos) * p.dk;
-            dst[ia] = __float2bfloat16_rn(ya);
-            dst[ib] = __float2bfloat16_rn(yb);
+            const long long base = (row * p.T_max + pos) * p.dk;
+            if constexpr (KV8) {
+                uint8_t *dst = static_cast<uint8_t *>(p.k_cache) + base;
+                dst[ia] = __nv_cvt_float_to_fp8(__fdiv_rn(ya, p.k_scale), __NV_SATFINITE, __NV_E4M3);
+                dst[ib] = __nv_cvt_float_to_fp8(__fdiv_rn(yb, p.k_scale), __NV_SATFINITE, __NV_E4M3);
+            } else {
+                __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.k_cache) + base;
+                dst[ia] = __float2bfloat16_rn(ya);
+                dst[ib] = __float2bfloat16_rn(yb);
+            }
         } else {
             // ---- value (or latent): copied into the cache row, one 4-byte word each
             const long long u = w - p.n_q_pairs - p.n_k_pairs;
@@ -90,8 +102,18 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const RopeAppendParams
             const int pos = __ldg(p.positions + b);
             if (pos < 0 || pos >= p.T_max) continue;
             const uint32_t *src = reinterpret_cast<const uint32_t *>(p.v_new + row * p.dv);
-            uint32_t *dst = reinterpret_cast<uint32_t *>(p.v_cache + (row * p.T_max + pos) * p.dv);
-            dst[c] = __ldg(src + c);
+            const long long base = (row * p.T_max + pos) * p.dv;
+            if constexpr (KV8) {
+                // two values: bf16 pair -> two E4M3 codes (element order kept)
+                const uint32_t w2 = __ldg(src + c);
+                const float2 x = make_float2(__fdiv_rn(__uint_as_float(w2 << 16), p.v_scale),
+                                             __fdiv_rn(__uint_as_float(w2 & 0xFFFF0000u), p.v_scale));
+                *reinterpret_cast<__nv_fp8x2_storage_t *>(static_cast<uint8_t *>(p.v_cache) + base + 2 * c) =
+                    __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
+            } else {
+                uint32_t *dst = reinterpret_cast<uint32_t *>(static_cast<__nv_bfloat16 *>(p.v_cache) + base);
+                dst[c] = __ldg(src + c);
+            }
         }
     }
 }

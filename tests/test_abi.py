@@ -260,6 +260,24 @@ def test_gqa_fp8_paged_rejects_bad_arguments(lib, kw, expected):
     assert st == expected
 
 
+@pytest.mark.parametrize("kw,expected", [
+    (dict(ks=0.0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(vs=float("inf")), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(d=7), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(base=-1.0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(kc=2 * A + 4), kb.KVATTN_ERR_MISALIGNED),
+    (dict(vc=4 * A + 64), kb.KVATTN_ERR_INVALID_ARG),       # value cache inside the key cache
+    (dict(q=0), kb.KVATTN_ERR_INVALID_ARG),
+])
+def test_rope_append_fp8_rejects_bad_arguments(lib, kw, expected):
+    a = dict(q=A, kn=6 * A, vn=7 * A, pos=8 * A, kc=4 * A, vc=5 * A, T=1024, B=2, nq=8, nkv=2, d=128,
+             base=10000.0, ks=0.01, vs=0.02)
+    a.update(kw)
+    st = lib.kvattn_rope_append_fp8(a["q"], a["kn"], a["vn"], a["pos"], a["kc"], a["vc"], a["T"], a["B"], a["nq"],
+                                    a["nkv"], a["d"], a["base"], 0, a["ks"], a["vs"], None)
+    assert st == expected
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     q = torch.zeros(1, 8, 64, dtype=torch.bfloat16)

@@ -130,3 +130,73 @@ def test_append_then_decode_matches_oracle():
     ro, rl = oracle.gqa_decode(q_ref, kc, vc, x["seq_lens"], cfg.scale)
     assert_close(out.cpu().numpy(), ro, "step out")
     assert_close(lse.cpu().numpy(), rl, "step lse")
+
+
+def _signed_code(c):
+    """E4M3 codes as signed integers ordered like their values (sign-magnitude -> +-mag)."""
+    c = c.to(torch.int32)
+    mag = c & 0x7F
+    return torch.where((c & 0x80) != 0, -mag, mag)
+
+
+@pytest.mark.parametrize("interleaved", [0, 1], ids=["halves", "interleaved"])
+def test_rope_append_fp8(interleaved):
+    """E4M3 cache: the value's codes are bit-exact against the oracle's encoder (the same
+    fp32 quotient, ties to even); the key's are within one code step of the oracle's
+    encoding of its fp64 rotation rounded to fp32 (the kernel turns the pair in fp32);
+    every other cache row is unchanged."""
+    g = torch.Generator().manual_seed(11)
+    B, n_q, n_kv, d, T = 5, 32, 8, 128, 3000
+    q = _rand((B, n_q, d), g)
+    k_new = _rand((B, n_kv, d), g, 3.0)
+    v_new = _rand((B, n_kv, d), g, 3.0)
+    pos = torch.tensor([0, 2999, 1234, 3000, -5], dtype=torch.int32)
+    ks, vs = 0.0125, 0.00875
+    kc = torch.randint(0, 256, (B, n_kv, T, d), generator=g, dtype=torch.uint8)
+    vc = torch.randint(0, 256, (B, n_kv, T, d), generator=g, dtype=torch.uint8)
+    dq, dkc, dvc = q.cuda(), kc.cuda(), vc.cuda()
+    kb.kvattn_rope_append_fp8(dq, k_new.cuda(), v_new.cuda(), pos.cuda(), dkc, dvc, ks, vs, rope_base=10000.0,
+                              interleaved=interleaved)
+    torch.cuda.synchronize()
+    assert_within_one_ulp(dq, _bf16(oracle.rope_f64(q, pos.numpy(), 10000.0, interleaved)), "q")
+    k_rot = np.asarray(oracle.rope_f64(k_new, pos.numpy(), 10000.0, interleaved), dtype=np.float32)
+    k_codes = torch.from_numpy(oracle.e4m3_quant(k_rot, ks))
+    v_codes = torch.from_numpy(oracle.e4m3_quant(v_new.float().numpy(), vs))
+    kg, vg = dkc.cpu(), dvc.cpu()
+    for b in range(B):
+        p = int(pos[b])
+        ke, ve = kc[b].clone(), vc[b].clone()
+        if 0 <= p < T:
+            diff = (_signed_code(kg[b, :, p]) - _signed_code(k_codes[b])).abs()
+            assert int(diff.max()) <= 1, f"key codes of sequence {b} more than one step apart"
+            assert (diff == 0).float().mean().item() > 0.97, f"key codes of sequence {b}"
+            assert torch.equal(vg[b, :, p], v_codes[b]), f"value codes of sequence {b}"
+            ke[:, p] = kg[b, :, p]
+            ve[:, p] = v_codes[b]
+        assert torch.equal(kg[b], ke) and torch.equal(vg[b], ve), f"other rows of sequence {b} changed"
+
+
+def test_append_fp8_then_decode_matches_oracle():
+    """One decode step into an E4M3 cache end to end: rotate + quantise-append, then the
+    fp8 decode, against the oracle appending its own codes and attending in fp64."""
+    cfg = wl.GQAConfig("step8", 4, 32, 8, 128, 3000, 1.0 / math.sqrt(128.0), seq_lens=(2999, 1, 1500, 64))
+    x = wl.make_gqa_inputs_fp8(cfg, seed=23)
+    g = torch.Generator().manual_seed(24)
+    k_new = _rand((cfg.batch, cfg.n_kv_heads, cfg.head_dim), g)
+    v_new = _rand((cfg.batch, cfg.n_kv_heads, cfg.head_dim), g)
+    pos = (x["seq_lens"] - 1).to(torch.int32)
+    dq, dkc, dvc = x["q"].cuda(), x["k_cache"].cuda(), x["v_cache"].cuda()
+    kb.kvattn_rope_append_fp8(dq, k_new.cuda(), v_new.cuda(), pos.cuda(), dkc, dvc, x["k_scale"], x["v_scale"])
+    out, lse = kb.kvattn_gqa_decode_fp8(dq, dkc, dvc, x["seq_lens"].cuda(), cfg.scale, x["k_scale"], x["v_scale"])
+    torch.cuda.synchronize()
+    q_ref = _bf16(oracle.rope_f64(x["q"], pos.numpy(), 10000.0, 0))
+    k_rot = np.asarray(oracle.rope_f64(k_new, pos.numpy(), 10000.0, 0), dtype=np.float32)
+    k_codes = torch.from_numpy(oracle.e4m3_quant(k_rot, x["k_scale"]))
+    v_codes = torch.from_numpy(oracle.e4m3_quant(v_new.float().numpy(), x["v_scale"]))
+    kc, vc = x["k_cache"].view(torch.uint8).clone(), x["v_cache"].view(torch.uint8).clone()
+    for b in range(cfg.batch):
+        kc[b, :, int(pos[b])] = k_codes[b]
+        vc[b, :, int(pos[b])] = v_codes[b]
+    ro, rl = oracle.gqa_decode_fp8(q_ref, kc, vc, x["seq_lens"], cfg.scale, x["k_scale"], x["v_scale"])
+    assert_close(out.cpu().numpy(), ro, "fp8 step out")
+    assert_close(lse.cpu().numpy(), rl, "fp8 step lse")
