@@ -1,14 +1,14 @@
 // tc05.cuh -- tcgen05 (5th-generation tensor core, tensor memory) and thread-block
 // cluster helpers for sm_100a.
 //
-// Conventions used by the MLA kernel:
+// Conventions used by the tcgen05 kernels (GQA and MLA):
 //  - shared-memory matrix descriptors describe 128-byte-swizzled canonical layouts
 //    (the layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B into 1024-byte aligned
 //    buffers): K-major (rows of 128 bytes, 8-row groups 1024 bytes apart) or MN-major
-//    (128-byte rows along K, 64-element MN blocks `lbo` bytes apart, 8-row K groups
-//    `sbo` bytes apart);
+//    (128-byte rows along K, MN blocks of one 128-byte row `lbo` bytes apart, 8-row K
+//    groups `sbo` bytes apart); or the unswizzled layout (8-row x 16-byte core matrices);
 //  - one thread issues every tcgen05.mma of a CTA (cta_group::1) and signals their
-//    completion with tcgen05.commit on an mbarrier (optionally multicast to the cluster);
+//    completion with tcgen05.commit on an mbarrier of its own CTA;
 //  - TMEM addresses are (lane << 16) | column; a warp may only touch the 32 lanes of its
 //    quadrant (warp_id % 4).
 // No TMA or bulk load in this library uses .multicast::cluster.
@@ -43,22 +43,6 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t ran
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
-}
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-// 16-byte store into another CTA's shared memory that completes `bytes` of the
-// transaction count of the mbarrier at `mbar_cluster_addr` (in that CTA) when it lands.
-__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                            uint32_t mbar_cluster_addr) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                     addr),
-                 "r"(a), "r"(b), "r"(c), "r"(d), "r"(mbar_cluster_addr)
-                 : "memory");
-}
 // Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into another CTA's
 // shared memory (no multicast), completing that many bytes of the transaction count of
 // the mbarrier at `mbar_cluster_addr` in the destination CTA.
@@ -74,10 +58,6 @@ __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bul
 // Waits until every committed bulk copy of this thread has finished reading its source.
 __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// Arrive (release, cluster scope) on an mbarrier given by its shared::cluster address.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 constexpr uint32_t kSuspendHintNsCl = 20000;
 // Relaxed arrive on a (possibly remote) mbarrier: no ordering of this thread's earlier
@@ -197,9 +177,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
 // Generic-proxy writes to shared memory become visible to the async proxy (tensor core).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-    asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- tensor memory
@@ -343,13 +320,4 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
                      smem_u32(bar))
                  : "memory");
 }
-// Same, arriving on the mbarrier at this offset in every CTA of `mask`.
-__device__ __forceinline__ void umma_commit_mc(uint64_t *bar, uint16_t mask) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-            smem_u32(bar)),
-        "h"(mask)
-        : "memory");
-}
-
 }  // namespace kvattn
