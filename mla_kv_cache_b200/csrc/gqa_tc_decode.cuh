@@ -521,7 +521,11 @@ __device__ __forceinline__ void mma_issuer(const GqaParams &p, const Ctx &c, int
 // group keeps its own row sums, relative to the max it last used; at the end of a piece
 // they are merged at the final max.  O^T is rescaled, in tile order, by the factor
 // between consecutive tiles' maxima.
-template <int NR, bool KV8>
+// MULTI: several new tokens or a window (the per-column visibility mask and the
+// (position, head) output rows); without it the kernel keeps the single-token forms --
+// a compile-time split, because the multi-token code in the same kernel costs the
+// single-token MQA workload ~4 us per step (measured) even where it does not run.
+template <int NR, bool KV8, bool MULTI>
 __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, int warp, int lane) {
     using C = Cfg<NR>;
     using L = Kv<KV8>;
@@ -568,7 +572,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
         const int nt = pc.lt1 - pc.lt0;
         const int start = active_start(len, p.q_len, p.window);
         // columns of one query position (the group's heads); all columns of the unit
-        const uint64_t group_bits = p.g >= 64 ? ~0ull : ((1ull << p.g) - 1ull);
+        const uint64_t group_bits = (!MULTI || p.g >= 64) ? ~0ull : ((1ull << p.g) - 1ull);
         // score scale (log2 units); with an E4M3 cache also the key scale and the 2^-e
         // of the split query block
         float cs = p.scale_log2;
@@ -594,10 +598,9 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
             // the columns (query position qi, head) that may see this token: query qi sits
             // at len - q_len + qi and sees [that + 1 - window, that] (causal, windowed)
             uint64_t vis = 0;
-            if (posr >= tok0 && posr < len) {
-                if (p.q_len == 1) {
-                    vis = group_bits;
-                } else {
+            const bool in_tile = posr >= tok0 && posr < len;
+            if constexpr (MULTI) {
+                if (in_tile) {
                     for (int qi = 0; qi < p.q_len; ++qi) {
                         const int hi = len - p.q_len + qi + 1;
                         const int lo = p.window > 0 ? hi - p.window : 0;
@@ -631,7 +634,8 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
             float sc[NR], v[NR];
 #pragma unroll
             for (int h = 0; h < NR; ++h) {
-                sc[h] = ((vis >> h) & 1ull) ? __uint_as_float(sv[h]) * cs : -INFINITY;
+                const bool see = MULTI ? ((vis >> h) & 1ull) != 0 : in_tile;
+                sc[h] = see ? __uint_as_float(sv[h]) * cs : -INFINITY;
                 v[h] = sc[h];
             }
             // ---- per-column maximum over the tile's 128 tokens
@@ -784,6 +788,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
         const int h_real = min(HB, p.g * p.q_len - hb * HB);
         const size_t part = ((size_t)blockIdx.x * 2 + pc.slot) * HB;
         auto out_row = [&](int cc) -> size_t {
+            if constexpr (!MULTI) return (size_t)pc.b * p.n_q + (size_t)j * p.g + (size_t)hb * HB + cc;
             const int vr = hb * HB + cc;
             const int qi = vr / p.g;
             return ((size_t)pc.b * p.q_len + qi) * p.n_q + (size_t)j * p.g + (vr - qi * p.g);
@@ -840,7 +845,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
 
 }  // namespace gqatc
 
-template <int NR, bool KV8>
+template <int NR, bool KV8, bool MULTI>
 __global__ void __launch_bounds__(gqatc::Cfg<NR>::NTHREADS, 1)
 gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
@@ -884,9 +889,11 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
         tmem_relinquish();
     }
     if (warp == 2) build_tile_prefix(p.seq_lens, p.B, p.T_max, TILE, s_prefix, lane, p.q_len, p.window);
-    // query buffers start zeroed: rows a unit's block does not fill stay finite
-    for (int i = tid; i < QREGION / 16; i += Cfg<NR>::NTHREADS)
-        reinterpret_cast<uint4 *>(smem + OFF_Q)[i] = make_uint4(0, 0, 0, 0);
+    // query buffers start zeroed: rows a unit's block does not fill stay finite (a
+    // single-token block is a full box: the TMA fills its rows past the heads with zeros)
+    if constexpr (MULTI)
+        for (int i = tid; i < QREGION / 16; i += Cfg<NR>::NTHREADS)
+            reinterpret_cast<uint4 *>(smem + OFF_Q)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&kmap);
@@ -922,7 +929,7 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
         } else if (warp == 1) {
             mma_issuer<NR, KV8>(p, c, lane);
         } else {
-            softmax_warps<NR, KV8>(p, c, warp, lane);
+            softmax_warps<NR, KV8, MULTI>(p, c, warp, lane);
         }
     }
 

@@ -38,7 +38,7 @@ struct DeviceState {
     struct Func {
         const void *kern;
         int smem;
-    } funcs[16] = {};
+    } funcs[64] = {};
     int n_funcs = 0;
     int mla_clusters = 0;   // co-resident MLA CTA pairs (0: not queried yet)
 };
@@ -357,7 +357,8 @@ int run_gqa_tc(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap
     p.ws_lse = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes);
     p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes + lse_bytes);
 
-    auto kern = gqa_tc_decode_kernel<NR, KV8>;
+    // several new tokens or a window: the instantiation with the visibility mask
+    auto kern = (p.q_len > 1 || p.window > 0) ? gqa_tc_decode_kernel<NR, KV8, true> : gqa_tc_decode_kernel<NR, KV8, false>;
     cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), dev, smem);
     if (e != cudaSuccess) return fail_cuda(e, "cudaFuncSetAttribute(gqa tc)");
     kern<<<p.workers, gqatc::Cfg<NR>::NTHREADS, smem, stream>>>(p, kmap, vmap, qmap);
