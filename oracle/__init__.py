@@ -99,6 +99,13 @@ def _lens(seq_lens):
     return np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
 
 
+def _rows(length, capacity):
+    """Cache rows a sequence of this length attends to: the length clamped to
+    [0, capacity], as the fp64 core clamps it.  The per-sequence wrappers below convert
+    and pass exactly these rows, so a cache position at or past the length is never read."""
+    return int(min(max(int(length), 0), int(capacity)))
+
+
 def gqa_decode_f64(q, k, v, seq_lens, scale, lib=None):
     """GQA/MQA/MHA decode on fp64 arrays.
 
@@ -162,7 +169,7 @@ def gqa_decode(q, k_cache, v_cache, seq_lens, scale, batch_ids=None, lib=None):
     ids = range(q.shape[0]) if batch_ids is None else batch_ids
     outs, lses = [], []
     for b in ids:
-        T = int(min(max(int(lens[b]), 0), T_max))
+        T = _rows(lens[b], T_max)
         o, l = gqa_decode_f64(q[b:b + 1], k_cache[b:b + 1, :, :T], v_cache[b:b + 1, :, :T],
                               np.array([T], dtype=np.int32), scale, lib=lib)
         outs.append(o[0])
@@ -178,7 +185,7 @@ def mla_decode(q_latent, q_rope, latent_cache, rope_cache, seq_lens, scale, batc
     ids = range(q_latent.shape[0]) if batch_ids is None else batch_ids
     outs, lses = [], []
     for b in ids:
-        T = int(min(max(int(lens[b]), 0), T_max))
+        T = _rows(lens[b], T_max)
         o, l = mla_decode_f64(q_latent[b:b + 1], q_rope[b:b + 1], latent_cache[b:b + 1, :T],
                               rope_cache[b:b + 1, :T], np.array([T], dtype=np.int32), scale,
                               lib=lib)
@@ -230,10 +237,10 @@ def gqa_decode_multi(q, k_cache, v_cache, seq_lens, scale, window=0, lib=None):
     """Multi-token decode on the bf16 (or any float) tensors, one sequence at a time so
     only the touched rows are converted to fp64."""
     B = q.shape[0]
-    lens = [int(x) for x in (seq_lens.tolist() if hasattr(seq_lens, "tolist") else seq_lens)]
+    lens = _lens(seq_lens)
     outs, lses = [], []
     for b in range(B):
-        T = max(0, min(lens[b], k_cache.shape[2]))
+        T = _rows(lens[b], k_cache.shape[2])
         n = max(T, 1)
         o, l = gqa_decode_multi_f64(q[b:b + 1], k_cache[b:b + 1, :, :n], v_cache[b:b + 1, :, :n],
                                     [T], scale, window, lib=lib)
@@ -294,7 +301,7 @@ def gqa_decode_fp8(q, k_codes, v_codes, seq_lens, scale, k_scale, v_scale, windo
     multi = len(q.shape) == 4
     outs, lses = [], []
     for b in range(q.shape[0]):
-        T = int(min(max(int(lens[b]), 0), T_max))
+        T = _rows(lens[b], T_max)
         n = max(T, 1)
         kb = e4m3_dequant(kc[b:b + 1, :, :n], k_scale, lib=lib)
         vb = e4m3_dequant(vc[b:b + 1, :, :n], v_scale, lib=lib)
