@@ -112,6 +112,19 @@ def workload_fields(cfg):
             "head_dim": cfg.head_dim, "seq_len": cfg.max_seq_len}
 
 
+def config_fields(name, cfg, nb, world):
+    """The line's "config" object; both arms print the same one for the same workload."""
+    if isinstance(cfg, wl.MLAConfig):
+        layout = "contiguous latent [B, T, 512] + RoPE key [B, T, 64]"
+    else:
+        layout = "contiguous [B, n_kv, T, d]"
+    return {"workload": name + variant_suffix(), **workload_fields(cfg), **variant_fields(),
+            "bytes_per_step": nb["total"],
+            "cache_layout": f"paged: {PAGED}-row pages in a shuffled pool, block table" if PAGED else layout,
+            "l2": "flushed before every timed step (256 MiB device write + read-back, outside the timed interval)",
+            "parallelism": f"replicas x{world}: one independent batch per GPU, no collective"}
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -530,12 +543,7 @@ def gpu_arm(args):
         "dtype": "e4m3 operands, fp32 accumulate" if KV8 else "bf16",
         "data": "synthetic (seeded N(0,1) bf16, shapes of the workload" +
                 ("; cache stored as E4M3 codes, scale = max|x| / 448)" if KV8 else ")"),
-        "config": {"workload": args.config + variant_suffix(), **workload_fields(head_cfg), **variant_fields(),
-                   "bytes_per_step": nb["total"],
-                   "cache_layout": f"paged: {PAGED}-row pages in a shuffled pool, block table" if PAGED
-                   else "contiguous [B, n_kv, T, d]",
-                   "l2": "flushed before every timed step (256 MiB device write + read-back, outside the timed interval)",
-                   "parallelism": f"replicas x{world}: one independent batch per GPU, no collective"},
+        "config": config_fields(args.config, head_cfg, nb, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
                      "peak_source": pk["source"] + " burst copy bandwidth",
@@ -584,8 +592,7 @@ def reference_arm(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) bf16, shapes of the workload)",
-        "config": {"workload": args.config + variant_suffix(), **variant_fields(),
-                   "bytes_per_step": nb["total"]},
+        "config": config_fields(args.config, cfg, nb, world),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(),
                          "kind": "oracle",
                          "sample": f"{per_step_seqs} of {cfg.batch} sequences per step (all heads), "

@@ -315,14 +315,16 @@ void kvattn_debug_set_gqa_kernel(int which);
  * kvattn_gqa_decode without any allocation by the library.  The pages have no
  * counterpart to this call; it exists for callers that must not have a library call
  * cudaMalloc: serving engines that reserve nearly all device memory for their own
- * KV-cache pool, code being recorded into a CUDA graph, and loops that cannot afford
- * cudaMalloc's implicit synchronisation.
- *   Arguments, layouts, results and errors are those of kvattn_gqa_decode.
+ * KV-cache pool (a stray allocation can fail or fragment it), and loops that cannot
+ * afford cudaMalloc's implicit synchronisation.
+ *   Arguments, layouts, results and errors are those of kvattn_gqa_decode; the call
+ *   always runs the warp-level kernel (see kvattn_debug_set_gqa_kernel).
  *   Scratch: a fixed 6 MiB array inside the library, present on every GPU that loads
- *   the library until the process exits.  A plan that needs more (only possible with
- *   kvattn_debug_set_workers forcing many workers) returns KVATTN_ERR_UNSUPPORTED with
- *   the sizes in kvattn_last_error_detail.  It calls no cudaMalloc, cudaFree or other
- *   allocating routine.
+ *   the library until the process exits.  It holds the built-in plan of any batch on a
+ *   device of up to 160 SMs (one worker per SM); a plan that needs more (a larger
+ *   device, or kvattn_debug_set_workers forcing many workers) returns
+ *   KVATTN_ERR_UNSUPPORTED with the sizes in kvattn_last_error_detail.  It calls no
+ *   cudaMalloc, cudaFree or other allocating routine.
  *   The first call on a device looks up the array's device address (once per device,
  *   with that device current); make that first call before any stream capture.
  *   All calls share the one array and it keeps the last call's contents: calls that

@@ -31,6 +31,7 @@ int fail_cuda(cudaError_t e, const char *where) {
 
 struct DeviceState {
     bool init = false;
+    int id = 0;
     int sms = 0;
     int max_smem_optin = 0;
     void *ws = nullptr;
@@ -58,6 +59,7 @@ int device_state(DeviceState **out) {
     }
     DeviceState &s = g_dev[dev];
     if (!s.init) {
+        s.id = dev;
         e = cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return fail_cuda(e, "cudaDeviceGetAttribute(SMs)");
         e = cudaDeviceGetAttribute(&s.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -260,9 +262,66 @@ int launch_combine(int D, const CombineParams &cp, int units, int rows, cudaStre
     return KVATTN_OK;
 }
 
+// ---------------------------------------------------------------------------------------
+// Scratch of kvattn_gqa_decode_noalloc.
+//
+// Some callers cannot let a library call cudaMalloc: a serving engine that reserves
+// almost all of the GPU's memory up front for its paged KV-cache pool (a stray
+// allocation can fail or fragment that pool), and latency-critical loops where the
+// implicit device synchronisation of cudaMalloc / cudaFree is unacceptable.  For them
+// kvattn_gqa_decode_noalloc runs the same warp-level decode and combine kernels as
+// kvattn_gqa_decode, through the same code below, but keeps the split-KV scratch (the
+// published work split and the per-worker partial outputs) in this fixed array, which
+// every GPU that loads the library holds until the process exits.  Its size bounds the
+// plans it accepts: the built-in plan of the warp-level kernel needs the work split
+// (at most 16 + 4 * (4096 + 1) bytes, rounded to 256) plus, per worker (one per SM),
+// two partial slots of 32 head rows x (128 + 1) floats, so the array serves every
+// device of up to kStaticScratchMaxSms SMs (a B200 has 148).
+// ---------------------------------------------------------------------------------------
+constexpr int kStaticScratchMaxSms = 160;
+constexpr size_t kStaticScratchBytes = 6u << 20;   // 6 MiB
+static_assert(((16 + 4 * (4096 + 1) + 255) / 256) * 256 + (size_t)kStaticScratchMaxSms * 2 * 32 * (128 + 1) * 4 +
+                      256 <= kStaticScratchBytes,
+              "the static scratch does not hold the default plan of a device with kStaticScratchMaxSms SMs");
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch, looked up once per device with that device
+// current (a host-side reference to the array is a host stand-in, not a device address).
+void *g_static_scratch_ptr[kMaxDevices] = {};
+
+int static_scratch(int dev, void **ptr) {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if (!g_static_scratch_ptr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(static scratch)");
+        g_static_scratch_ptr[dev] = p;
+    }
+    *ptr = g_static_scratch_ptr[dev];
+    return KVATTN_OK;
+}
+
+// Scratch of a warp-level GQA plan of `bytes`: the per-device workspace (grown with
+// cudaMalloc when needed), or, when fixed_scratch is set, the static array above (plans
+// that do not fit are refused; nothing is allocated).
+int gqa_scratch(DeviceState *dev, size_t bytes, bool fixed_scratch, void **ws) {
+    if (fixed_scratch) {
+        if (bytes > kStaticScratchBytes) {
+            snprintf(t_detail, sizeof(t_detail), "plan needs %zu B of scratch; the static scratch holds %zu B",
+                     bytes, kStaticScratchBytes);
+            return KVATTN_ERR_UNSUPPORTED;
+        }
+        // Nothing in the scratch has to start at zero: the decode kernel writes the work
+        // split and every partial before the combine kernel reads them.
+        return static_scratch(dev->id, ws);
+    }
+    std::lock_guard<std::mutex> lk(g_mutex);
+    return ensure_workspace(dev, bytes, ws);
+}
+
 template <int D, int MT>
 int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &vmap,
-            DeviceState *dev, int units_per_seq, cudaStream_t stream) {
+            DeviceState *dev, int units_per_seq, cudaStream_t stream, bool fixed_scratch) {
     using C = GqaCfg<D, MT>;
     GqaParams p = base;
     const int smem = C::smem_bytes(p.B);
@@ -285,8 +344,7 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
     const size_t lse_bytes = (((size_t)p.workers * 2 * C::HEADS * 4) + 255) & ~size_t(255);
     const size_t o_bytes = (size_t)p.workers * 2 * C::HEADS * D * 4;
     {
-        std::lock_guard<std::mutex> lk(g_mutex);
-        int st = ensure_workspace(dev, meta_bytes + lse_bytes + o_bytes, &ws);
+        int st = gqa_scratch(dev, meta_bytes + lse_bytes + o_bytes, fixed_scratch, &ws);
         if (st != KVATTN_OK) return st;
     }
     p.ws_meta = ws;
@@ -412,9 +470,11 @@ struct GqaCache {
     float k_scale = 1.f, v_scale = 1.f;
 };
 
+// noalloc: the warp-level kernel with its scratch in the static array (one new token,
+// no window, bf16 contiguous cache).
 int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq_lens, int batch,
                     int n_q_heads, int n_kv_heads, int head_dim, float scale, float *out, float *lse,
-                    void *stream, int q_len = 1, int window = 0) {
+                    void *stream, int q_len = 1, int window = 0, bool noalloc = false) {
     DeviceState *dev = nullptr;
     int st = device_state(&dev);
     if (st != KVATTN_OK) return st;
@@ -422,7 +482,7 @@ int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq
     const int g = n_q_heads / n_kv_heads;
     // a paged cache needs pages made of whole 128-token tiles for the tcgen05 kernel
     const bool tiles_fit = cache.block_table == nullptr || cache.page_size % gqatc::TILE == 0;
-    if (g_gqa_kernel == 2 && !(tiles_fit && use_tc_kernel(head_dim, g, batch, dev))) {
+    if (!noalloc && g_gqa_kernel == 2 && !(tiles_fit && use_tc_kernel(head_dim, g, batch, dev))) {
         snprintf(t_detail, sizeof(t_detail),
                  "tcgen05 GQA kernel needs head_dim 128, batch <= %d and pages of multiples of 128 rows",
                  (dev->max_smem_optin - gqatc::smem_bytes(0)) / 4);
@@ -444,7 +504,7 @@ int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq
                  "multiples of 128 rows", gqatc::HB);
         return KVATTN_ERR_UNSUPPORTED;
     }
-    const bool tc = multi || cache.e4m3 || (tiles_fit && use_tc_kernel(head_dim, g, batch, dev));
+    const bool tc = !noalloc && (multi || cache.e4m3 || (tiles_fit && use_tc_kernel(head_dim, g, batch, dev)));
     const int MT = g <= 16 ? 1 : 2;
     const int heads = tc ? gqatc::HB : 16 * MT;
     const int n_hb = (g * q_len + heads - 1) / heads;
@@ -506,8 +566,10 @@ int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq
         return run_gqa_tc<8, false>(p, kmap, vmap, qmap, dev, U, s);
     }
     if (head_dim == 128)
-        return MT == 1 ? run_gqa<128, 1>(p, kmap, vmap, dev, U, s) : run_gqa<128, 2>(p, kmap, vmap, dev, U, s);
-    return MT == 1 ? run_gqa<64, 1>(p, kmap, vmap, dev, U, s) : run_gqa<64, 2>(p, kmap, vmap, dev, U, s);
+        return MT == 1 ? run_gqa<128, 1>(p, kmap, vmap, dev, U, s, noalloc)
+                       : run_gqa<128, 2>(p, kmap, vmap, dev, U, s, noalloc);
+    return MT == 1 ? run_gqa<64, 1>(p, kmap, vmap, dev, U, s, noalloc)
+                   : run_gqa<64, 2>(p, kmap, vmap, dev, U, s, noalloc);
 }
 
 // A latent + rotary-key cache as the MLA kernel sees it (pages of page_size rows; a
@@ -631,14 +693,11 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
                           combine_warps((cache.capacity + mla::TILE - 1) / mla::TILE, max_tiles, p.workers));
 }
 
-}  // namespace
-
-extern "C" {
-
-int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
-                      const int32_t *seq_lens, int max_seq_len, int batch, int n_q_heads,
-                      int n_kv_heads, int head_dim, float scale, float *out, float *lse,
-                      void *stream) {
+// Argument checks of kvattn_gqa_decode (and of kvattn_gqa_decode_noalloc, which takes the
+// same arguments).
+int check_gqa_args(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache, const int32_t *seq_lens,
+                   int max_seq_len, int batch, int n_q_heads, int n_kv_heads, int head_dim, float scale,
+                   const float *out, const float *lse) {
     if (!q || !k_cache || !v_cache || !seq_lens || !out || !lse) return KVATTN_ERR_INVALID_ARG;
     if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || max_seq_len <= 0)
         return KVATTN_ERR_INVALID_ARG;
@@ -660,6 +719,20 @@ int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t
         if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
             return KVATTN_ERR_INVALID_ARG;
     if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+    return KVATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvattn_gqa_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                      const int32_t *seq_lens, int max_seq_len, int batch, int n_q_heads,
+                      int n_kv_heads, int head_dim, float scale, float *out, float *lse,
+                      void *stream) {
+    const int st = check_gqa_args(q, k_cache, v_cache, seq_lens, max_seq_len, batch, n_q_heads, n_kv_heads,
+                                  head_dim, scale, out, lse);
+    if (st != KVATTN_OK) return st;
     const GqaCache cache{k_cache, v_cache, nullptr, max_seq_len, max_seq_len, 1, batch};
     return gqa_decode_impl(q, cache, seq_lens, batch, n_q_heads, n_kv_heads, head_dim, scale, out, lse, stream);
 }
@@ -1091,180 +1164,18 @@ void kvattn_debug_set_gqa_kernel(int which) {
 
 }  // extern "C"
 
-// ---------------------------------------------------------------------------------------
-// Decode without any allocation by the library.
-//
-// Some callers cannot let a library call cudaMalloc: a serving engine that reserves
-// almost all of the GPU's memory up front for its paged KV-cache pool (a stray
-// allocation can fail or fragment that pool), code that records the call into a CUDA
-// graph (cudaMalloc cannot be captured), and latency-critical loops where the implicit
-// device synchronisation of cudaMalloc / cudaFree is unacceptable.  For them
-// kvattn_gqa_decode_noalloc runs the same kernels as kvattn_gqa_decode but keeps its
-// split-KV scratch (the published work split and the per-worker partial outputs) in the
-// fixed array below, which every GPU that loads this library holds until the process
-// exits.  Its size bounds the plans it accepts.
-// ---------------------------------------------------------------------------------------
-static constexpr size_t kStaticScratchBytes = 6u << 20;   // 6 MiB
-static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-namespace {
-
-// Device address of g_static_scratch, looked up once per device with that device
-// current (a host-side reference to the array is a host stand-in, not a device address).
-void *g_static_scratch_ptr[kMaxDevices] = {};
-
-int static_scratch(int dev, void **ptr) {
-    std::lock_guard<std::mutex> lk(g_mutex);
-    if (!g_static_scratch_ptr[dev]) {
-        void *p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess) return fail_cuda(e, "cudaGetSymbolAddress(static scratch)");
-        g_static_scratch_ptr[dev] = p;
-    }
-    *ptr = g_static_scratch_ptr[dev];
-    return KVATTN_OK;
-}
-
-template <int D, int MT>
-int run_gqa_noalloc(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &vmap,
-                    DeviceState *dev, int dev_id, int units_per_seq, cudaStream_t stream) {
-    using C = GqaCfg<D, MT>;
-    GqaParams p = base;
-    const int smem = C::smem_bytes(p.B);
-    if (smem > dev->max_smem_optin) {
-        snprintf(t_detail, sizeof(t_detail), "needs %d B shared memory", smem);
-        return KVATTN_ERR_UNSUPPORTED;
-    }
-    const long long max_tiles =
-        (long long)p.B * units_per_seq * ((p.T_max + C::TILE - 1) / C::TILE);
-    p.min_tiles = g_force_min_tiles > 0 ? g_force_min_tiles : 4;
-    long long workers = g_force_workers > 0 ? g_force_workers : dev->sms;
-    const long long by_size = (max_tiles + p.min_tiles - 1) / p.min_tiles;
-    if (g_force_workers <= 0 && workers > by_size) workers = by_size;
-    if (workers < 1) workers = 1;
-    p.workers = (int)workers;
-
-    const size_t meta_bytes = ((16 + (size_t)(p.B + 1) * 4) + 255) & ~size_t(255);
-    const size_t lse_bytes = (((size_t)p.workers * 2 * C::HEADS * 4) + 255) & ~size_t(255);
-    const size_t o_bytes = (size_t)p.workers * 2 * C::HEADS * D * 4;
-    const size_t need = meta_bytes + lse_bytes + o_bytes;
-    if (need > kStaticScratchBytes) {
-        snprintf(t_detail, sizeof(t_detail),
-                 "plan needs %zu B of scratch; the static scratch holds %zu B", need,
-                 kStaticScratchBytes);
-        return KVATTN_ERR_UNSUPPORTED;
-    }
-    void *ws = nullptr;
-    int st = static_scratch(dev_id, &ws);
-    if (st != KVATTN_OK) return st;
-    // Nothing in the scratch has to start at zero: the decode kernel writes the work
-    // split and every partial before the combine kernel reads them.
-    p.ws_meta = ws;
-    p.ws_lse = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes);
-    p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes + lse_bytes);
-
-    auto kern = gqa_decode_kernel<D, MT>;
-    cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), dev, smem);
-    if (e != cudaSuccess) return fail_cuda(e, "cudaFuncSetAttribute(gqa)");
-    kern<<<p.workers, C::NTHREADS, smem, stream>>>(p, kmap, vmap);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return fail_cuda(e, "gqa decode launch");
-
-    CombineParams cp;
-    cp.seq_lens = p.seq_lens;
-    cp.ws_lse = p.ws_lse;
-    cp.ws_o = p.ws_o;
-    cp.out = p.out;
-    cp.lse = p.lse;
-    cp.B = p.B;
-    cp.n_q = p.n_q;
-    cp.units_per_seq = units_per_seq;
-    cp.heads_per_unit = C::HEADS;
-    cp.n_hb = p.n_hb;
-    cp.n_kv = p.n_kv;
-    cp.g = p.g;
-    cp.T_max = p.T_max;
-    cp.tile = C::TILE;
-    cp.workers = p.workers;
-    cp.min_tiles = p.min_tiles;
-    cp.q_len = 1;
-    cp.window = 0;
-    const int rows = p.g < C::HEADS ? p.g : C::HEADS;
-    return launch_combine(D, cp, p.B * units_per_seq, rows, stream,
-                          combine_warps((p.T_max + C::TILE - 1) / C::TILE, max_tiles, p.workers));
-}
-
-}  // namespace
-
+// Decode without any allocation by the library: kvattn_gqa_decode's checks and code path
+// with the warp-level kernel and the static scratch above.
 extern "C" int kvattn_gqa_decode_noalloc(const uint16_t *q, const uint16_t *k_cache,
                                          const uint16_t *v_cache, const int32_t *seq_lens,
                                          int max_seq_len, int batch, int n_q_heads, int n_kv_heads,
                                          int head_dim, float scale, float *out, float *lse,
                                          void *stream) {
-    if (!q || !k_cache || !v_cache || !seq_lens || !out || !lse) return KVATTN_ERR_INVALID_ARG;
-    if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || max_seq_len <= 0)
-        return KVATTN_ERR_INVALID_ARG;
-    if (n_q_heads % n_kv_heads != 0) return KVATTN_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
-    if (head_dim != 64 && head_dim != 128) return KVATTN_ERR_UNSUPPORTED;
-    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
-    if ((long long)batch * n_kv_heads * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seq_lens) ||
-        !aligned16(out) || !aligned16(lse))
-        return KVATTN_ERR_MISALIGNED;
-    const size_t q_bytes = (size_t)batch * n_q_heads * head_dim * 2;
-    const size_t kv_bytes = (size_t)batch * n_kv_heads * max_seq_len * head_dim * 2;
-    const size_t out_bytes = (size_t)batch * n_q_heads * head_dim * 4;
-    const size_t lse_bytes = (size_t)batch * n_q_heads * 4;
-    const void *ins[4] = {q, k_cache, v_cache, seq_lens};
-    const size_t in_sz[4] = {q_bytes, kv_bytes, kv_bytes, (size_t)batch * 4};
-    for (int i = 0; i < 4; ++i)
-        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
-            return KVATTN_ERR_INVALID_ARG;
-    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
-
-    int dev_id = 0;
-    cudaError_t e = cudaGetDevice(&dev_id);
-    if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
-    DeviceState *dev = nullptr;
-    int st = device_state(&dev);
+    const int st = check_gqa_args(q, k_cache, v_cache, seq_lens, max_seq_len, batch, n_q_heads, n_kv_heads,
+                                  head_dim, scale, out, lse);
     if (st != KVATTN_OK) return st;
-
-    const int g = n_q_heads / n_kv_heads;
-    const int MT = g <= 16 ? 1 : 2;
-    const int heads = 16 * MT;
-    const int n_hb = (g + heads - 1) / heads;
-
-    CUtensorMap kmap, vmap;
-    st = make_map_3d(&kmap, k_cache, head_dim, max_seq_len, (uint64_t)batch * n_kv_heads, 64, 64,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != KVATTN_OK) return st;
-    st = make_map_3d(&vmap, v_cache, head_dim, max_seq_len, (uint64_t)batch * n_kv_heads, 64, 64,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != KVATTN_OK) return st;
-
-    GqaParams p = {};
-    p.q = reinterpret_cast<const __nv_bfloat16 *>(q);
-    p.seq_lens = seq_lens;
-    p.out = out;
-    p.lse = lse;
-    p.B = batch;
-    p.n_q = n_q_heads;
-    p.n_kv = n_kv_heads;
-    p.T_max = max_seq_len;
-    p.g = g;
-    p.n_hb = n_hb;
-    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    p.block_table = nullptr;           // contiguous cache: one page per sequence
-    p.max_pages = 1;
-    p.page_size = max_seq_len;
-    p.q_len = 1;
-    p.window = 0;
-    const int U = n_kv_heads * n_hb;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (head_dim == 128)
-        return MT == 1 ? run_gqa_noalloc<128, 1>(p, kmap, vmap, dev, dev_id, U, s)
-                       : run_gqa_noalloc<128, 2>(p, kmap, vmap, dev, dev_id, U, s);
-    return MT == 1 ? run_gqa_noalloc<64, 1>(p, kmap, vmap, dev, dev_id, U, s)
-                   : run_gqa_noalloc<64, 2>(p, kmap, vmap, dev, dev_id, U, s);
+    const GqaCache cache{k_cache, v_cache, nullptr, max_seq_len, max_seq_len, 1, batch};
+    return gqa_decode_impl(q, cache, seq_lens, batch, n_q_heads, n_kv_heads, head_dim, scale, out, lse, stream,
+                           1, 0, true);
 }

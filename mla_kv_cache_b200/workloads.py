@@ -7,7 +7,7 @@ seeded by the caller (default 0), in a fixed draw order, and rounded once to bf1
 (round to nearest even) after any scaling or offset, so the stored bf16 values are
 the ground truth for both the CUDA path and the oracle.
 
-Draw order for one workload (the recipe the design doc states):
+Draw order for one workload:
   GQA: seq_lens (ragged configs only), q, k, v, then spike positions (spiky configs).
   MLA: seq_lens (ragged configs only), q_latent, q_rope, latent_cache, rope_cache.
 Caches are drawn one sequence at a time (batch-major), so a workload's values do not

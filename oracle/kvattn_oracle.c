@@ -24,7 +24,7 @@
  *   latents c_t (W_UV is applied downstream).  Keys and values are the same
  *   latent vector; the RoPE part enters the score only.
  *
- * Readings where the pages are silent (stated once more in the design doc):
+ * Readings where the pages are silent:
  *   - decode attends to every cached position t < seq_lens[b]; no mask;
  *   - lse is the natural log of sum_t exp(s_t) with s_t already scaled;
  *   - an empty sequence (seq_lens[b] == 0) gives out = 0 and lse = -inf;

@@ -1,9 +1,9 @@
 """kvattn_gqa_decode_noalloc: the decode entry point that allocates nothing.
 
 It is meant for callers that cannot let a library call cudaMalloc: serving engines
-that reserve nearly all device memory for their own KV-cache pool, code recorded into
-a CUDA graph, and loops that cannot afford cudaMalloc's implicit synchronisation.  Its
-scratch is a fixed array inside the library shared by every call.
+that reserve nearly all device memory for their own KV-cache pool, and loops that
+cannot afford cudaMalloc's implicit synchronisation.  Its scratch is a fixed array
+inside the library shared by every call.
 
 The test calls it through the C ABI (ctypes, no Python wrapper) twice in a row on
 different workloads and checks both results against kvattn_gqa_decode's at the
