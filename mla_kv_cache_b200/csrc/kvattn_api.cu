@@ -591,15 +591,15 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
     if (st != KVATTN_OK) return st;
 
     MlaMaps maps;
-    st = make_map_3d(&maps.lat, cache.lat, 512, cache.page_size, (uint64_t)cache.pages, 64, mla::TILE,
+    st = make_map_3d(&maps.lat, cache.lat, 512, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
-    st = make_map_3d(&maps.rope, cache.rope, 64, cache.page_size, (uint64_t)cache.pages, 64, mla::TILE,
+    st = make_map_3d(&maps.rope, cache.rope, 64, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
-    st = make_map_3d(&maps.qlat, q_latent, 512, n_heads, batch, 64, mla::HR, CU_TENSOR_MAP_SWIZZLE_128B);
+    st = make_map_3d(&maps.qlat, q_latent, 512, n_heads, batch, 64, mla::HC, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
-    st = make_map_3d(&maps.qrope, q_rope, 64, n_heads, batch, 64, mla::HR, CU_TENSOR_MAP_SWIZZLE_128B);
+    st = make_map_3d(&maps.qrope, q_rope, 64, n_heads, batch, 64, mla::HC, CU_TENSOR_MAP_SWIZZLE_128B);
     if (st != KVATTN_OK) return st;
 
     MlaParams p = {};
@@ -923,7 +923,7 @@ int kvattn_mla_decode_paged(const uint16_t *q_latent, const uint16_t *q_rope, co
         return KVATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
     if (latent_dim != 512 || rope_dim != 64 || n_heads > 128) return KVATTN_ERR_UNSUPPORTED;
-    if (page_size % mla::TILE != 0) return KVATTN_ERR_UNSUPPORTED;
+    if (page_size % mla::SUB != 0) return KVATTN_ERR_UNSUPPORTED;
     if (batch > mla::MAX_BATCH) return KVATTN_ERR_UNSUPPORTED;
     if ((long long)num_pages * page_size >= (1ll << 31) || (long long)max_pages_per_seq * page_size >= (1ll << 31))
         return KVATTN_ERR_UNSUPPORTED;

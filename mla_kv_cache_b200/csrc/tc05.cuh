@@ -320,4 +320,47 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
                      smem_u32(bar))
                  : "memory");
 }
+
+// ---------------------------------------------------------------- CTA pairs (cta_group::2)
+// A pair MMA spans the two CTAs of a 2-CTA cluster (ranks 0 and 1): one thread of rank 0
+// issues it, each CTA supplies its half of the A rows and of the B columns from its own
+// shared memory at the same addresses, and each CTA's tensor memory receives its half of
+// D.  Every tcgen05 allocation, MMA and commit of such a kernel uses cta_group::2.
+
+// Allocation of tensor-memory columns in both CTAs of the pair: executed by the same
+// warp in each CTA, with the same destination address.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t smem_dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_dst), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T over the pair, issued by one thread of rank 0.
+__device__ __forceinline__ void umma_pair_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Once every pair MMA issued so far by this thread has completed, arrive on the mbarrier
+// at this shared-memory offset in both CTAs of the pair.
+__device__ __forceinline__ void umma_pair_commit_both(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"((uint16_t)3)
+        : "memory");
+}
+// Arrive (release at cluster scope) on an mbarrier given by its shared::cluster address,
+// which may lie in either CTA of the cluster.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 }  // namespace kvattn
