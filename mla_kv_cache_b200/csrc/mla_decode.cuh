@@ -20,10 +20,12 @@
 //
 // Per 128-token tile t0 .. t0+127 (tokens of half h: t0 + 64h ..):
 //   score product S = Q K^T (M = 128 heads, N = 128 tokens, K = 576): A = this CTA's 64
-//     query rows (shared memory, loaded once per sequence: 8 latent chunks + 1 RoPE
-//     chunk of 64 columns), B = the 576-wide key rows of tile half r (CTA r loads the
-//     half its B columns are).  9 chunks x 4 MMAs of K = 16.  In tensor memory, lane m
-//     holds head 64r + m's scores of half 0's tokens, lane 64 + m those of half 1's.
+//     query rows, once per sequence -- latent columns [0, 256) in tensor memory (written
+//     by the softmax threads, each row in lanes m and 64 + m), latent columns [256, 512)
+//     and the RoPE part in shared memory (TMA) --, B = the 576-wide key rows of tile half
+//     r (CTA r loads the half its B columns are).  9 chunks of 64 columns x 4 MMAs of
+//     K = 16.  In tensor memory, lane m holds head 64r + m's scores of half 0's tokens,
+//     lane 64 + m those of half 1's.
 //   value product O += P C (M = 128 heads, N = 256 latent columns per MMA, two MMAs for
 //     the 512 columns, K = 128 tokens): A = this CTA's weights P (shared memory, K-major),
 //     B = the latent columns [256j + 128r, 256j + 128r + 128) of all 128 tokens (MN-major,
@@ -36,17 +38,24 @@
 // values by each CTA for its columns), the second time from L2.
 //
 // Warp roles (256 threads per CTA):
-//   warp 0, one thread   TMA producer (both CTAs): the query block once per sequence, a
-//                        6-slot ring of key chunks (8 KB) and a 4-slot ring of value
-//                        chunk pairs (16 KB); completions signal rank 0's barriers.
-//   warp 1, one thread   MMA issuer (rank 0 only): S of tile k + 1 before O += P C of
-//                        tile k, so the softmax of tile k overlaps the next score product.
-//   warps 4-7            softmax, one thread per tensor-memory lane (head 64r + m, tile
-//                        half h): masks, tile maximum (the two halves of a head meet in
-//                        shared memory), lazy running max (moves only when a tile's
-//                        maximum exceeds it by more than 2^8; then this CTA's rows of O
-//                        are rescaled in tensor memory), weights into shared memory,
-//                        row sums; at the end of a piece the normalised result.
+//   warp 0, one thread   key producer (both CTAs): the shared-memory part of the query
+//                        block once per sequence and a ring of three 24 KB key slots (one
+//                        tile); completions signal rank 0's barriers.
+//   warp 2, one thread   value producer (both CTAs): a ring of two 32 KB value slots (one
+//                        tile), independent of the key stream; its loads hit L2 (the keys'
+//                        latent columns, loaded by the pair moments before).
+// Each slot release is one tcgen05.commit, which costs the issuing thread ~300 cycles
+// (measured, against ~56 for an MMA), so the slots are a few chunks each.
+//   warp 1, one thread   score MMA issuer (rank 0 only), running ahead of the softmax by
+//                        one tile (two score buffers).
+//   warp 3, one thread   value MMA issuer (rank 0 only).
+//   warps 4-11           softmax, two threads per tensor-memory lane (head 64r + m, tile
+//                        half h; 32 score columns each): masks, partial tile maxima (the
+//                        four parts of a head meet in shared memory), lazy running max
+//                        (moves only when a tile's maximum exceeds it by more than 2^8;
+//                        then this CTA's rows of O are rescaled in tensor memory), weights
+//                        into shared memory, row sums; at the end of a piece the
+//                        normalised result.
 // Every wait is bounded; every wait ahead of a warp-collective instruction is made
 // warp-uniform.  No TMA load uses multicast.
 #pragma once
@@ -62,23 +71,29 @@ constexpr int SUB = 64;                  // tokens of a tile half (one CTA's B c
 constexpr int HR = 128;                  // head rows of the pair (M)
 constexpr int HC = 64;                   // head rows of one CTA
 constexpr int CHUNK = SUB * 128;         // one TMA box [64 rows x 64 bf16 columns], 128-byte swizzled: 8 KB
-constexpr int NQC = 9;                   // query chunks: 8 latent + 1 RoPE
-constexpr int NSS = 6;                   // key ring slots (one chunk each)
-constexpr int NPV = 4;                   // value ring slots (two chunks each: 128 latent columns)
-constexpr int NTHREADS = 256;
+constexpr int NQC = 9;                   // query / key chunks of 64 columns: 8 latent + 1 RoPE
+constexpr int NQT = 4;                   // query chunks held in tensor memory (latent columns [0, 256))
+constexpr int NQS = NQC - NQT;           // query chunks in shared memory (latent [256, 512) + RoPE)
+constexpr int NKS = 3;                   // key ring: 3 slots of 3 chunks (192 columns), one tile
+constexpr int NVS = 2;                   // value ring: 2 slots (latent block j: 128 columns of both halves), one tile
+constexpr int KSLOT = 3 * CHUNK;         // 24 KB
+constexpr int VSLOT = 4 * CHUNK;         // 32 KB
+constexpr int NTHREADS = 384;            // warps 0-3: producers and MMA issuers, 4-11: softmax
+constexpr int NSOFT = 8;                 // softmax warps
 constexpr int MAX_BATCH = 1024;
 constexpr float RESCALE_LOG2 = 8.f;      // rescale O only when the row max grows by > 2^8
 constexpr uint32_t TM_O = 0;             // tensor memory columns [0, 256): O (two blocks of 128)
 constexpr uint32_t TM_S = 256;           // [256, 384): the scores of two tiles (64 columns each)
+constexpr uint32_t TM_Q = 384;           // [384, 512): query latent columns [0, 256), bf16 pairs
 constexpr uint32_t TM_COLS = 512;
 
-constexpr int OFF_Q = 0;                               // query chunks [9][64 heads x 128 B]
-constexpr int OFF_P = OFF_Q + NQC * CHUNK;             // weights: high [2 halves], remainder [2 halves]
+constexpr int OFF_Q = 0;                               // query chunks [5][64 heads x 128 B]
+constexpr int OFF_P = OFF_Q + NQS * CHUNK;             // weights of a tile: high h0, h1, remainder h0, h1
 constexpr int OFF_SR = OFF_P + 4 * CHUNK;              // key ring
-constexpr int OFF_PV = OFF_SR + NSS * CHUNK;           // value ring
-constexpr int OFF_MX = OFF_PV + NPV * 2 * CHUNK;       // [2 tiles][2 halves][64] tile maxima
-constexpr int OFF_LX = OFF_MX + 2 * 2 * HC * 4;        // [2 halves][64] row sums
-constexpr int OFF_BARS = OFF_LX + 2 * HC * 4;
+constexpr int OFF_PV = OFF_SR + NKS * KSLOT;           // value ring
+constexpr int OFF_MX = OFF_PV + NVS * VSLOT;           // [2 tiles][4 parts][64] partial tile maxima
+constexpr int OFF_LX = OFF_MX + 2 * 4 * HC * 4;        // [4 parts][64] partial row sums
+constexpr int OFF_BARS = OFF_LX + 4 * HC * 4;
 constexpr int OFF_TMEMPTR = OFF_BARS + 512;
 constexpr int OFF_ABORT = OFF_TMEMPTR + 16;
 constexpr int OFF_PREFIX = OFF_ABORT + 16;
@@ -86,14 +101,21 @@ constexpr int smem_bytes(int B) { return 1024 + OFF_PREFIX + (B + 1) * 4; }
 static_assert(smem_bytes(MAX_BATCH) <= 232448, "shared memory of the MLA kernel exceeds 227 KB");
 
 struct Bars {
-    uint64_t sfull[NSS], sempty[NSS];   // key ring (full: rank 0, both CTAs' bytes; empty: both CTAs)
-    uint64_t vfull[NPV], vempty[NPV];   // value ring
-    uint64_t qfull;                     // query block of both CTAs landed (rank 0)
+    // Every ring slot serves each tile once, so its phase is the tile count.  The release
+    // of a tile's last key slot is that tile's sready, the release of its last value slot
+    // its odone: each tile takes three commits for the keys and two for the values.
+    uint64_t kfull[NKS];                // key ring (rank 0, both CTAs' bytes)
+    uint64_t kempty[NKS - 1];           // release of key slots 0 and 1 (both CTAs)
+    uint64_t sready[2];                 // the scores of a tile are in tensor memory (score buffer =
+                                        // tile parity; both CTAs)
+    uint64_t vfull[NVS];                // value ring (rank 0)
+    uint64_t vempty[NVS - 1];           // release of value slot 0 (both CTAs)
+    uint64_t odone[2];                  // the value product of a tile (parity) is done (both CTAs)
+    uint64_t qfull;                     // shared-memory query chunks of both CTAs landed (rank 0)
+    uint64_t qtm;                       // tensor-memory query columns written in both CTAs (rank 0)
     uint64_t qempty;                    // every score product of the piece has read Q (both CTAs)
-    uint64_t sready[2];                 // scores of a tile (parity) in tensor memory (both CTAs)
     uint64_t sfree[2];                  // both CTAs have read them (rank 0: 4 warps x 2 CTAs)
-    uint64_t pready;                    // weights written, O rescaled, in both CTAs (rank 0)
-    uint64_t odone;                     // value product of a tile finished (both CTAs)
+    uint64_t pready[2];                 // weights of a tile (parity) written, O rescaled, in both CTAs (rank 0)
     uint64_t ofree;                     // both CTAs' epilogues have read O (rank 0)
     uint64_t mxbar[2];                  // the four softmax warps' tile maxima written (tile parity)
     uint64_t lxbar;                     // the four softmax warps' row sums written (end of a piece)
@@ -162,176 +184,284 @@ __device__ __forceinline__ HalfSrc half_source(const MlaParams &p, int b, int le
     return s;
 }
 
-// ------------------------------------------------------------------ producer (warp 0, lane 0)
-// Both CTAs load, in the order the MMAs consume: the query block of a sequence, then the
-// key chunks of tile k0, and for every tile k of the piece the key chunks of tile k + 1
-// followed by the value chunks of tile k.  Completions go to rank 0's barriers, which
-// rank 0 arms with the bytes of both CTAs.
-__device__ __forceinline__ void producer(const MlaParams &p, const MlaMaps &m, const Ctx &c) {
+// ------------------------------------------------------------------ producers
+// Two threads per CTA, one per ring, each loading in the order the MMAs consume its
+// ring: the key producer (warp 0) the shared-memory query chunks of a sequence, then the
+// key chunks of every tile of the piece; the value producer (warp 2) the value chunks of
+// every tile.  Completions go to rank 0's barriers, which rank 0 arms with the bytes of
+// both CTAs.
+__device__ __forceinline__ void key_producer(const MlaParams &p, const MlaMaps &m, const Ctx &c) {
     Bars *bars = c.bars;
-    const uint64_t pol_keep = l2_policy_evict_normal();   // keys: the latent columns are read again
-    const uint64_t pol_last = l2_policy_evict_first();    // values: last read
+    const uint64_t pol_keep = l2_policy_evict_normal();   // the latent columns are read again as values
     const bool lead = c.r == 0;
     const uint32_t qfull0 = map_to_rank(smem_u32(&bars->qfull), 0);
-    int sidx = 0, vidx = 0, pi = 0;
+    int nld = 0, pi = 0;
     bool ok = true;
     for (long long pos = c.p0; pos < c.p1 && ok; ++pi) {
         const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
         pos = pc.ustart + pc.lt1;
         const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
-        const int nt = pc.lt1 - pc.lt0;
-        // this CTA's 64 query rows: 8 latent chunks and the RoPE chunk
+        // this CTA's 64 query rows: latent chunks 4..7 and the RoPE chunk
         if (pi > 0 && !mbar_wait(&bars->qempty, (uint32_t)(pi - 1) & 1u, FLAG_EMPTY_WAIT, c.abort_flag)) {
             ok = false;
             break;
         }
-        if (lead) mbar_arrive_expect_tx(&bars->qfull, 2 * NQC * CHUNK);
-        for (int ch = 0; ch < 8; ++ch)
-            tma_load_3d_pair(c.smem + OFF_Q + ch * CHUNK, &m.qlat, qfull0, 64 * ch, HC * (int)c.r, pc.b, pol_keep);
-        tma_load_3d_pair(c.smem + OFF_Q + 8 * CHUNK, &m.qrope, qfull0, 0, HC * (int)c.r, pc.b, pol_keep);
-
-        auto load_keys = [&](int lt) -> bool {
+        if (lead) mbar_arrive_expect_tx(&bars->qfull, 2 * NQS * CHUNK);
+        for (int ch = 0; ch < NQS - 1; ++ch)
+            tma_load_3d_pair(c.smem + OFF_Q + ch * CHUNK, &m.qlat, qfull0, 64 * (NQT + ch), HC * (int)c.r, pc.b,
+                             pol_keep);
+        tma_load_3d_pair(c.smem + OFF_Q + (NQS - 1) * CHUNK, &m.qrope, qfull0, 0, HC * (int)c.r, pc.b, pol_keep);
+        for (int lt = pc.lt0; lt < pc.lt1 && ok; ++lt) {
             const HalfSrc hs = half_source(p, pc.b, len, lt, (int)c.r);
-            for (int ch = 0; ch < NQC; ++ch, ++sidx) {
-                const int s = sidx % NSS;
-                if (!mbar_wait(&bars->sempty[s], ((uint32_t)(sidx / NSS) & 1u) ^ 1u, FLAG_EMPTY_WAIT, c.abort_flag))
-                    return false;
-                if (lead) mbar_arrive_expect_tx(&bars->sfull[s], 2 * CHUNK);
-                const uint32_t bar = map_to_rank(smem_u32(&bars->sfull[s]), 0);
-                if (ch < 8)
-                    tma_load_3d_pair(c.smem + OFF_SR + s * CHUNK, &m.lat, bar, 64 * ch, hs.y, hs.page, pol_keep);
-                else
-                    tma_load_3d_pair(c.smem + OFF_SR + s * CHUNK, &m.rope, bar, 0, hs.y, hs.page, pol_keep);
-            }
-            return true;
-        };
-        auto load_values = [&](int lt) -> bool {
-            for (int j = 0; j < 2; ++j)
-                for (int h = 0; h < 2; ++h, ++vidx) {
-                    const HalfSrc hs = half_source(p, pc.b, len, lt, h);
-                    const int s = vidx % NPV;
-                    if (!mbar_wait(&bars->vempty[s], ((uint32_t)(vidx / NPV) & 1u) ^ 1u, FLAG_EMPTY_WAIT,
-                                   c.abort_flag))
-                        return false;
-                    if (lead) mbar_arrive_expect_tx(&bars->vfull[s], 4 * CHUNK);
-                    const uint32_t bar = map_to_rank(smem_u32(&bars->vfull[s]), 0);
-                    uint8_t *dst = c.smem + OFF_PV + s * 2 * CHUNK;
-                    const int x = 256 * j + 128 * (int)c.r;
-                    tma_load_3d_pair(dst, &m.lat, bar, x, hs.y, hs.page, pol_last);
-                    tma_load_3d_pair(dst + CHUNK, &m.lat, bar, x + 64, hs.y, hs.page, pol_last);
+            for (int s = 0; s < NKS; ++s, ++nld) {
+                // slot s of the previous tile must have been read: slots 0 and 1 have their
+                // own release barrier, the last slot's is the previous tile's sready
+                const int kt = nld / NKS;
+                const bool freed = s < NKS - 1
+                    ? mbar_wait(&bars->kempty[s], ((uint32_t)kt & 1u) ^ 1u, FLAG_EMPTY_WAIT, c.abort_flag)
+                    : (kt == 0 || mbar_wait(&bars->sready[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u,
+                                            FLAG_EMPTY_WAIT, c.abort_flag));
+                if (!freed) {
+                    ok = false;
+                    break;
                 }
-            return true;
-        };
-        if (!load_keys(pc.lt0)) { ok = false; break; }
-        for (int t = 0; t < nt; ++t) {
-            if (t + 1 < nt && !load_keys(pc.lt0 + t + 1)) { ok = false; break; }
-            if (!load_values(pc.lt0 + t)) { ok = false; break; }
+                if (lead) mbar_arrive_expect_tx(&bars->kfull[s], 2 * KSLOT);
+                const uint32_t bar = map_to_rank(smem_u32(&bars->kfull[s]), 0);
+                uint8_t *dst = c.smem + OFF_SR + s * KSLOT;
+                for (int e = 0; e < 3; ++e) {
+                    const int ch = 3 * s + e;
+                    if (ch < 8)
+                        tma_load_3d_pair(dst + e * CHUNK, &m.lat, bar, 64 * ch, hs.y, hs.page, pol_keep);
+                    else
+                        tma_load_3d_pair(dst + e * CHUNK, &m.rope, bar, 0, hs.y, hs.page, pol_keep);
+                }
+            }
         }
     }
     if (!ok && lead) {
         // Let the copies already issued land before the CTAs can exit.
-        for (int i = (sidx > NSS ? sidx - NSS : 0); i < sidx; ++i)
-            mbar_wait_sleep(&bars->sfull[i % NSS], (uint32_t)(i / NSS) & 1u, FLAG_FULL_WAIT, nullptr);
-        for (int i = (vidx > NPV ? vidx - NPV : 0); i < vidx; ++i)
-            mbar_wait_sleep(&bars->vfull[i % NPV], (uint32_t)(i / NPV) & 1u, FLAG_FULL_WAIT, nullptr);
+        for (int i = (nld > NKS ? nld - NKS : 0); i < nld; ++i)
+            mbar_wait_sleep(&bars->kfull[i % NKS], (uint32_t)(i / NKS) & 1u, FLAG_FULL_WAIT, nullptr);
+        if (pi > 0) mbar_wait_sleep(&bars->qfull, (uint32_t)(pi - 1) & 1u, FLAG_FULL_WAIT, nullptr);
     }
 }
 
-// ------------------------------------------------------------------ MMA issuer (rank 0, warp 1, lane 0)
-__device__ __forceinline__ bool wait_remote(uint64_t *bar, uint32_t parity, const Ctx &c) {
-    return mbar_spin<true>(bar, parity, FLAG_PEER_WAIT, c.abort_flag);
+__device__ __forceinline__ void value_producer(const MlaParams &p, const MlaMaps &m, const Ctx &c) {
+    Bars *bars = c.bars;
+    const uint64_t pol_last = l2_policy_evict_first();    // the values' read is the last one
+    const bool lead = c.r == 0;
+    int nld = 0;
+    bool ok = true;
+    for (long long pos = c.p0; pos < c.p1 && ok;) {
+        const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
+        pos = pc.ustart + pc.lt1;
+        const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
+        for (int lt = pc.lt0; lt < pc.lt1 && ok; ++lt) {
+            const HalfSrc hsrc[2] = {half_source(p, pc.b, len, lt, 0), half_source(p, pc.b, len, lt, 1)};
+            for (int j = 0; j < NVS; ++j, ++nld) {
+                // slot j of the previous tile must have been read: slot 0 has its own release
+                // barrier, the last slot's is the previous tile's odone
+                const int kt = nld / NVS;
+                const bool freed = j < NVS - 1
+                    ? mbar_wait(&bars->vempty[j], ((uint32_t)kt & 1u) ^ 1u, FLAG_EMPTY_WAIT, c.abort_flag)
+                    : (kt == 0 || mbar_wait(&bars->odone[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u,
+                                            FLAG_EMPTY_WAIT, c.abort_flag));
+                if (!freed) {
+                    ok = false;
+                    break;
+                }
+                if (lead) mbar_arrive_expect_tx(&bars->vfull[j], 2 * VSLOT);
+                const uint32_t bar = map_to_rank(smem_u32(&bars->vfull[j]), 0);
+                uint8_t *dst = c.smem + OFF_PV + j * VSLOT;
+                const int x = 256 * j + 128 * (int)c.r;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    tma_load_3d_pair(dst + 2 * h * CHUNK, &m.lat, bar, x, hsrc[h].y, hsrc[h].page, pol_last);
+                    tma_load_3d_pair(dst + (2 * h + 1) * CHUNK, &m.lat, bar, x + 64, hsrc[h].y, hsrc[h].page, pol_last);
+                }
+            }
+        }
+    }
+    if (!ok && lead)
+        for (int i = (nld > NVS ? nld - NVS : 0); i < nld; ++i)
+            mbar_wait_sleep(&bars->vfull[i % NVS], (uint32_t)(i / NVS) & 1u, FLAG_FULL_WAIT, nullptr);
 }
 
-__device__ __forceinline__ void mma_issuer(const MlaParams &p, const Ctx &c) {
+// ------------------------------------------------------------------ MMA issuer (rank 0, warp 1, lane 0)
+// Waits of the issuing threads on barriers that the softmax warps of both CTAs arrive on.
+// The issuers share their SM sub-partitions with softmax warps, so they wait with
+// try_wait (which suspends the thread for a while between tests) rather than polling.
+__device__ __forceinline__ bool wait_remote(uint64_t *bar, uint32_t parity, const Ctx &c) {
+    return mbar_wait(bar, parity, FLAG_PEER_WAIT, c.abort_flag);
+}
+
+// Two issuing threads: the score products (warp 1) and the value products (warp 3).  A
+// thread can issue a tcgen05.mma only every ~60 cycles, about the tensor time of one
+// N = 128 pair MMA, so one thread could not keep the tensor pipe busy with both streams;
+// the two streams use different accumulators and each thread commits its own MMAs.
+// Shared-memory descriptors are formed once; an operand's descriptor is the template
+// plus its address in 16-byte units (the start field never carries: shared addresses
+// are below 2^18), so the issue loops add constants only.
+
+// S of every tile into score buffer kt & 1: 9 chunks x 4 K-steps of 16.
+__device__ __forceinline__ void score_issuer(const MlaParams &p, const Ctx &c) {
     Bars *bars = c.bars;
     constexpr uint32_t id_s = idesc_f16(128, TILE, 1, 1, 0);   // K-major A and B
-    constexpr uint32_t id_v = idesc_f16(128, 256, 1, 1, 1);    // B (the latents) MN-major
-    const uint32_t q_base = smem_u32(c.smem + OFF_Q);
-    const uint32_t p_base = smem_u32(c.smem + OFF_P);
-    int sidx = 0, vidx = 0;
-
-    // S of tile kt into score buffer kt & 1: 9 chunks x 4 K-steps of 16.
-    auto issue_scores = [&](int kt) -> bool {
-        const int sb = kt & 1;
-        if (kt >= 2 && !wait_remote(&bars->sfree[sb], (uint32_t)((kt >> 1) - 1) & 1u, c)) return false;
-        for (int ch = 0; ch < NQC; ++ch, ++sidx) {
-            const int s = sidx % NSS;
-            if (!mbar_wait(&bars->sfull[s], (uint32_t)(sidx / NSS) & 1u, FLAG_FULL_WAIT, c.abort_flag)) return false;
-            tc_fence_after();
-            const uint32_t kb = smem_u32(c.smem + OFF_SR + s * CHUNK);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_pair_ss(c.tmem + TM_S + 64 * sb, smem_desc_sw128(q_base + ch * CHUNK + kk * 32, 16, 1024),
-                             smem_desc_sw128(kb + kk * 32, 16, 1024), id_s, (ch | kk) != 0);
-            umma_pair_commit_both(&bars->sempty[s]);
-        }
-        umma_pair_commit_both(&bars->sready[sb]);
-        return true;
-    };
-    // O += P_hi C + P_lo C for tile kt: latent blocks j, token halves h, K-steps of 16.
-    auto issue_values = [&](int kt, bool first) -> bool {
-        if (!wait_remote(&bars->pready, (uint32_t)kt & 1u, c)) return false;
-        for (int j = 0; j < 2; ++j)
-            for (int h = 0; h < 2; ++h, ++vidx) {
-                const int s = vidx % NPV;
-                if (!mbar_wait(&bars->vfull[s], (uint32_t)(vidx / NPV) & 1u, FLAG_FULL_WAIT, c.abort_flag))
-                    return false;
-                tc_fence_after();
-                const uint32_t vb = smem_u32(c.smem + OFF_PV + s * 2 * CHUNK);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(vb + kk * 2048, CHUNK, 1024);
-                    const uint32_t pa = p_base + h * CHUNK + kk * 32;
-                    umma_pair_ss(c.tmem + TM_O + 128 * j, smem_desc_sw128(pa, 16, 1024), bd, id_v,
-                                 (!first || h > 0 || kk > 0) ? 1u : 0u);
-                    umma_pair_ss(c.tmem + TM_O + 128 * j, smem_desc_sw128(pa + 2 * CHUNK, 16, 1024), bd, id_v, 1u);
-                }
-                umma_pair_commit_both(&bars->vempty[s]);
-            }
-        umma_pair_commit_both(&bars->odone);
-        return true;
-    };
-
+    const uint64_t k_tmpl = smem_desc_sw128(0, 16, 1024);       // K-major, 128-byte swizzle
+    const uint64_t q_desc = k_tmpl + (smem_u32(c.smem + OFF_Q) >> 4);
+    const uint64_t kr_desc = k_tmpl + (smem_u32(c.smem + OFF_SR) >> 4);
+    const uint32_t tm_q = c.tmem + TM_Q;
     int k = 0, pi = 0;
     for (long long pos = c.p0; pos < c.p1; ++pi) {
         const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
         pos = pc.ustart + pc.lt1;
         const int nt = pc.lt1 - pc.lt0;
         if (!mbar_wait(&bars->qfull, (uint32_t)pi & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
-        if (!issue_scores(k)) return;
-        if (nt == 1) umma_pair_commit_both(&bars->qempty);
-        for (int t = 0; t < nt; ++t) {
-            const int kt = k + t;
-            if (t + 1 < nt) {
-                if (!issue_scores(kt + 1)) return;
-                if (t + 2 == nt) umma_pair_commit_both(&bars->qempty);   // the piece's last score product
+        if (!wait_remote(&bars->qtm, (uint32_t)pi & 1u, c)) return;
+        tc_fence_after();
+        for (int kt = k; kt < k + nt; ++kt) {
+            const int sb = kt & 1;
+            const uint32_t d = c.tmem + TM_S + 64 * sb;
+            if (kt >= 2 && !wait_remote(&bars->sfree[sb], (uint32_t)((kt >> 1) - 1) & 1u, c)) return;
+            for (int s = 0; s < NKS; ++s) {
+                if (!mbar_wait(&bars->kfull[s], (uint32_t)kt & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
+                tc_fence_after();
+#pragma unroll
+                for (int e = 0; e < 3; ++e) {
+                    const int ch = 3 * s + e;
+                    const uint64_t bd = kr_desc + (uint64_t)((s * KSLOT + e * CHUNK) >> 4);
+                    if (ch < NQT) {
+                        const uint32_t a = tm_q + 32 * ch;
+                        umma_pair_ts(d, a, bd, id_s, ch != 0);
+                        umma_pair_ts(d, a + 8, bd + 2, id_s, 1u);
+                        umma_pair_ts(d, a + 16, bd + 4, id_s, 1u);
+                        umma_pair_ts(d, a + 24, bd + 6, id_s, 1u);
+                    } else {
+                        const uint64_t ad = q_desc + (uint64_t)((ch - NQT) * (CHUNK >> 4));
+                        umma_pair_ss(d, ad, bd, id_s, 1u);
+                        umma_pair_ss(d, ad + 2, bd + 2, id_s, 1u);
+                        umma_pair_ss(d, ad + 4, bd + 4, id_s, 1u);
+                        umma_pair_ss(d, ad + 6, bd + 6, id_s, 1u);
+                    }
+                }
+                if (s < NKS - 1)
+                    umma_pair_commit_both(&bars->kempty[s]);
+                else
+                    umma_pair_commit_both(&bars->sready[sb]);   // releases the last slot too
             }
-            // the previous piece's epilogue must have read O before the first product overwrites it
-            if (t == 0 && pi > 0 && !wait_remote(&bars->ofree, (uint32_t)(pi - 1) & 1u, c)) return;
-            if (!issue_values(kt, t == 0)) return;
+        }
+        umma_pair_commit_both(&bars->qempty);   // the piece's score products are done with Q
+        k += nt;
+    }
+}
+
+// O += P_hi C + P_lo C for every tile kt: latent blocks j, token halves h, K-steps of 16
+// tokens.
+__device__ __forceinline__ void value_issuer(const MlaParams &p, const Ctx &c) {
+    Bars *bars = c.bars;
+    constexpr uint32_t id_v = idesc_f16(128, 256, 1, 1, 1);    // B (the latents) MN-major
+    const uint64_t k_tmpl = smem_desc_sw128(0, 16, 1024);       // K-major, 128-byte swizzle
+    const uint64_t v_tmpl = smem_desc_sw128(0, CHUNK, 1024);    // MN-major: the two 64-column chunks 8 KB apart
+    const uint64_t p_desc = k_tmpl + (smem_u32(c.smem + OFF_P) >> 4);
+    const uint64_t vr_desc = v_tmpl + (smem_u32(c.smem + OFF_PV) >> 4);
+    int k = 0, pi = 0;
+    for (long long pos = c.p0; pos < c.p1; ++pi) {
+        const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
+        pos = pc.ustart + pc.lt1;
+        const int nt = pc.lt1 - pc.lt0;
+        // the previous piece's epilogue must have read O before the first product overwrites it
+        if (pi > 0 && !wait_remote(&bars->ofree, (uint32_t)(pi - 1) & 1u, c)) return;
+        for (int kt = k; kt < k + nt; ++kt) {
+            const bool first = kt == k;
+            if (!wait_remote(&bars->pready[kt & 1], (uint32_t)(kt >> 1) & 1u, c)) return;
+            for (int jb = 0; jb < NVS; ++jb) {
+                const uint32_t d = c.tmem + TM_O + 128 * jb;
+                if (!mbar_wait(&bars->vfull[jb], (uint32_t)kt & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
+                tc_fence_after();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint64_t bd = vr_desc + (uint64_t)((jb * VSLOT + h * 2 * CHUNK) >> 4);
+                    const uint64_t hi = p_desc + (uint64_t)(h * (CHUNK >> 4));
+                    const uint64_t lo = hi + (uint64_t)(2 * (CHUNK >> 4));
+                    umma_pair_ss(d, hi, bd, id_v, (!first || h > 0) ? 1u : 0u);
+                    umma_pair_ss(d, lo, bd, id_v, 1u);
+#pragma unroll
+                    for (int kk = 1; kk < 4; ++kk) {   // next 16 tokens: +32 B in the weights, +2 KB in the latents
+                        umma_pair_ss(d, hi + 2 * kk, bd + 128 * kk, id_v, 1u);
+                        umma_pair_ss(d, lo + 2 * kk, bd + 128 * kk, id_v, 1u);
+                    }
+                }
+                if (jb < NVS - 1)
+                    umma_pair_commit_both(&bars->vempty[jb]);
+                else
+                    umma_pair_commit_both(&bars->odone[kt & 1]);   // releases the last slot too
+            }
         }
         k += nt;
     }
 }
 
-// ------------------------------------------------------------------ softmax (warps 4-7)
+// ------------------------------------------------------------------ softmax (warps 4-11)
+// Two warps per tensor-memory lane quadrant: warp 4 + 4cg + q takes score columns
+// [32cg, 32cg + 32) of the lanes of quadrant q, i.e. 32 of the 64 tokens of its tile half.
+// The four partial tile maxima of a head (two halves x two column groups) meet in shared
+// memory, as do its four partial row sums at the end of a piece.  Column group cg also
+// owns O's block j = cg in the lane (its rescale, its epilogue) and half of the lane's
+// query columns in tensor memory.
+// Waits use try_wait (the thread is suspended between tests) so that waiting softmax
+// warps leave the issue slots to the producer and MMA threads on the same sub-partition.
+__device__ __forceinline__ bool wait_local(uint64_t *bar, uint32_t parity, unsigned int flag, const Ctx &c) {
+    return warp_all(mbar_wait(bar, parity, flag, c.abort_flag));
+}
+
 __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, int warp, int lane) {
     Bars *bars = c.bars;
     const int q = warp & 3;                     // tensor-memory lane quadrant
+    const int cg = (warp - 4) >> 2;             // column group: score columns [32cg, 32cg + 32)
     const int L = 32 * q + lane;                // tensor-memory lane
     const int hh = L & (HC - 1);                // head row of this CTA
     const int half = L >> 6;                    // tile half whose scores the lane holds
+    const int part = 2 * half + cg;             // this thread's share of the head's tile
     const int head = HC * (int)c.r + hh;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    float *mx_buf = reinterpret_cast<float *>(c.smem + OFF_MX);
-    float *lx_buf = reinterpret_cast<float *>(c.smem + OFF_LX);
+    float *mx_buf = reinterpret_cast<float *>(c.smem + OFF_MX);   // [2 tiles][4 parts][64]
+    float *lx_buf = reinterpret_cast<float *>(c.smem + OFF_LX);   // [4 parts][64]
     const uint32_t sfree0 = map_to_rank(smem_u32(&bars->sfree[0]), 0);
     const uint32_t sfree1 = map_to_rank(smem_u32(&bars->sfree[1]), 0);
-    const uint32_t pready0 = map_to_rank(smem_u32(&bars->pready), 0);
+    const uint32_t pready0 = map_to_rank(smem_u32(&bars->pready[0]), 0);
+    const uint32_t pready1 = map_to_rank(smem_u32(&bars->pready[1]), 0);
     const uint32_t ofree0 = map_to_rank(smem_u32(&bars->ofree), 0);
-    uint8_t *row_hi = c.smem + OFF_P + half * CHUNK + hh * 128;   // this row of the weights (K-major, swizzled)
+    const uint32_t qtm0 = map_to_rank(smem_u32(&bars->qtm), 0);
+    // this thread's 32 tokens of the weights: row hh of the half's K-major chunk, 16-byte
+    // units 4cg .. 4cg + 3 (128-byte swizzle)
+    uint8_t *row_hi = c.smem + OFF_P + half * CHUNK + hh * 128;
     uint8_t *row_lo = row_hi + 2 * CHUNK;
     const float sl2 = p.scale_log2;
+
+    // Query latent columns [64cg, 64cg + 64) (bf16 pairs) of this lane's head of sequence
+    // b into tensor memory; both lanes of a head hold the row.
+    auto write_q = [&](int b) -> bool {
+        const bool realq = head < p.H;
+        const uint4 *qrow =
+            reinterpret_cast<const uint4 *>(p.q_latent + ((size_t)b * p.H + (realq ? head : 0)) * 512) + 16 * cg;
+        tc_fence_after();
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            uint32_t v[32];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                uint4 x = make_uint4(0, 0, 0, 0);
+                if (realq) x = __ldg(qrow + 8 * w + e);
+                v[4 * e] = x.x; v[4 * e + 1] = x.y; v[4 * e + 2] = x.z; v[4 * e + 3] = x.w;
+            }
+            tmem_st32(c.tmem + lane_base + TM_Q + 64 * cg + 32 * w, v);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(qtm0);
+        return true;
+    };
 
     int k = 0, pi = 0;
     for (long long pos = c.p0; pos < c.p1; ++pi) {
@@ -339,86 +469,99 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         pos = pc.ustart + pc.lt1;
         const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
         const int nt = pc.lt1 - pc.lt0;
-        float m_ref = -INFINITY;      // running max (log2 units), shared by the two halves of the head
-        float l = 0.f;                // row sum of this half's weights, relative to m_ref
+        if (pi == 0 && !write_q(pc.b)) return;
+        float m_ref = -INFINITY;      // running max (log2 units), shared by the four parts of the head
+        float l = 0.f;                // row sum of this thread's weights, relative to m_ref
         for (int t = 0; t < nt; ++t) {
             const int kt = k + t;
             const int sb = kt & 1;
-            const int lo = half_source(p, pc.b, len, pc.lt0 + t, half).lo;
-            // ---- scores of this lane (64 tokens of its half)
-            if (!warp_all(mbar_spin<false>(&bars->sready[sb], (uint32_t)(kt >> 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
-                return;
+            // first valid column of this thread's 32 (masked: rows of the half below lo)
+            const int lo = half_source(p, pc.b, len, pc.lt0 + t, half).lo - 32 * cg;
+            // ---- this thread's 32 scores
+            if (!wait_local(&bars->sready[sb], (uint32_t)(kt >> 1) & 1u, FLAG_MMA_WAIT, c)) return;
             tc_fence_after();
-            float sv[64];
+            float sv[32];
             {
-                uint32_t a[32], b[32];
-                tmem_ld32(c.tmem + lane_base + TM_S + 64 * sb, a);
-                tmem_ld32(c.tmem + lane_base + TM_S + 64 * sb + 32, b);
+                uint32_t a[32];
+                tmem_ld32(c.tmem + lane_base + TM_S + 64 * sb + 32 * cg, a);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    sv[j] = __uint_as_float(a[j]);
-                    sv[32 + j] = __uint_as_float(b[j]);
-                }
+                for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(a[j]);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(sb ? sfree1 : sfree0);
-            // ---- scaled (log2 units), masked, tile maximum of this half
-            float mx = -INFINITY;
-            if (lo == 0) {
+            // ---- partial tile maximum (log2 units; masked columns excluded)
+            if (lo > 0) {
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    sv[i] *= sl2;
-                    mx = fmaxf(mx, sv[i]);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    sv[i] = i >= lo ? sv[i] * sl2 : -INFINITY;
-                    mx = fmaxf(mx, sv[i]);
-                }
+                for (int i = 0; i < 32; ++i) sv[i] = i >= lo ? sv[i] : (sl2 >= 0.f ? -INFINITY : INFINITY);
             }
-            // ---- the head's tile maximum over both halves, then the running max
-            mx_buf[(sb * 2 + half) * HC + hh] = mx;
+            float mx;
+            {
+                float m8[8];
+#pragma unroll
+                for (int g = 0; g < 8; ++g) m8[g] = sv[g];
+                if (sl2 >= 0.f) {
+#pragma unroll
+                    for (int i = 8; i < 32; ++i) m8[i & 7] = fmaxf(m8[i & 7], sv[i]);
+                } else {   // a negative scale turns the smallest raw score into the largest
+#pragma unroll
+                    for (int i = 8; i < 32; ++i) m8[i & 7] = fminf(m8[i & 7], sv[i]);
+                }
+                mx = fmaxf(fmaxf(fmaxf(m8[0] * sl2, m8[1] * sl2), fmaxf(m8[2] * sl2, m8[3] * sl2)),
+                           fmaxf(fmaxf(m8[4] * sl2, m8[5] * sl2), fmaxf(m8[6] * sl2, m8[7] * sl2)));
+                if (mx != mx) mx = -INFINITY;   // every column masked: (+-inf) * 0 is not a maximum
+            }
+            // ---- the head's tile maximum over its four parts, then the running max
+            mx_buf[(sb * 4 + part) * HC + hh] = mx;
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->mxbar[sb]);
-            if (!warp_all(mbar_spin<false>(&bars->mxbar[sb], (uint32_t)(kt >> 1) & 1u, FLAG_FULL_WAIT, c.abort_flag)))
-                return;
-            const float M = fmaxf(mx, mx_buf[(sb * 2 + (half ^ 1)) * HC + hh]);
+            if (!wait_local(&bars->mxbar[sb], (uint32_t)(kt >> 1) & 1u, FLAG_FULL_WAIT, c)) return;
+            const float *mxs = mx_buf + sb * 4 * HC + hh;
+            const float M = fmaxf(fmaxf(mxs[0], mxs[HC]), fmaxf(mxs[2 * HC], mxs[3 * HC]));
             const float m_new = (t == 0 || M > m_ref + RESCALE_LOG2) ? M : m_ref;
             const bool rescale = t > 0 && m_new != m_ref;
             const float alpha = rescale ? fast_exp2(m_ref - m_new) : 1.f;
             m_ref = m_new;
-            // ---- weights 2^(s - m): a bf16 high part and a bf16 remainder
-            uint32_t whi[32], wlo[32];
-            float ls = 0.f;
+            // ---- weights 2^(s * scale - m): a bf16 high part and a bf16 remainder
+            uint32_t whi[16], wlo[16];
+            float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+            if (lo <= 0) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float a = fast_exp2(sv[2 * j] - m_new);
-                const float b = fast_exp2(sv[2 * j + 1] - m_new);
-                ls += a + b;
-                split_bf16x2(a, b, whi[j], wlo[j]);
+                for (int j = 0; j < 16; ++j) {
+                    const float a = fast_exp2(fmaf(sv[2 * j], sl2, -m_new));
+                    const float b = fast_exp2(fmaf(sv[2 * j + 1], sl2, -m_new));
+                    ls4[j & 3] += a + b;
+                    split_bf16x2(a, b, whi[j], wlo[j]);
+                }
+            } else {   // masked columns get weight 0 (whatever the scale)
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float a = 2 * j >= lo ? fast_exp2(fmaf(sv[2 * j], sl2, -m_new)) : 0.f;
+                    const float b = 2 * j + 1 >= lo ? fast_exp2(fmaf(sv[2 * j + 1], sl2, -m_new)) : 0.f;
+                    ls4[j & 3] += a + b;
+                    split_bf16x2(a, b, whi[j], wlo[j]);
+                }
             }
-            l = l * alpha + ls;
-            // ---- the previous value product must be done with the weights and with O
-            if (kt > 0 && !warp_all(mbar_spin<false>(&bars->odone, (uint32_t)(kt - 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
+            l = l * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
+            // ---- the value product of tile kt - 1 must be done with the weights and with O
+            if (kt >= 1 && !wait_local(&bars->odone[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u, FLAG_MMA_WAIT, c))
                 return;
             tc_fence_after();
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int slot = (u ^ (hh & 7)) * 16;
+            for (int u = 0; u < 4; ++u) {
+                const int slot = ((4 * cg + u) ^ (hh & 7)) * 16;
                 *reinterpret_cast<uint4 *>(row_hi + slot) =
                     make_uint4(whi[4 * u], whi[4 * u + 1], whi[4 * u + 2], whi[4 * u + 3]);
                 *reinterpret_cast<uint4 *>(row_lo + slot) =
                     make_uint4(wlo[4 * u], wlo[4 * u + 1], wlo[4 * u + 2], wlo[4 * u + 3]);
             }
-            // rescale this lane's 256 columns of O (warp-collective: the whole warp takes
-            // the branch when any of its rows needs it, with factor 1 for the others)
+            // rescale block cg of this lane's O (warp-collective: the whole warp takes the
+            // branch when any of its rows needs it, with factor 1 for the others)
             if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-                for (int cc = 0; cc < 8; ++cc) {
-                    const uint32_t addr = c.tmem + lane_base + TM_O + 32 * cc;
+                for (int cc = 0; cc < 4; ++cc) {
+                    const uint32_t addr = c.tmem + lane_base + TM_O + 128 * cg + 32 * cc;
                     uint32_t ov[32];
                     tmem_ld32(addr, ov);
                     tmem_wait_ld();
@@ -431,39 +574,45 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(pready0);
+            if (lane == 0) mbar_arrive_remote(sb ? pready1 : pready0);
         }
-        // ---- end of the piece: the head's row sum, normalise, write
+        // ---- end of the piece.  First the next piece's query, so that its score products
+        //      can start while this epilogue runs (this piece's have read Q: qempty).
+        if (pos < c.p1) {
+            const Piece nx = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
+            if (!wait_local(&bars->qempty, (uint32_t)pi & 1u, FLAG_MMA_WAIT, c)) return;
+            if (!write_q(nx.b)) return;
+        }
+        // ---- the head's row sum (four parts), normalise, write block cg of the lane
         const int klast = k + nt - 1;
         k += nt;
-        lx_buf[half * HC + hh] = l;
+        lx_buf[part * HC + hh] = l;
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->lxbar);
-        if (!warp_all(mbar_spin<false>(&bars->lxbar, (uint32_t)pi & 1u, FLAG_FULL_WAIT, c.abort_flag))) return;
-        const float ltot = l + lx_buf[(half ^ 1) * HC + hh];
+        if (!wait_local(&bars->lxbar, (uint32_t)pi & 1u, FLAG_FULL_WAIT, c)) return;
+        const float ltot = (lx_buf[hh] + lx_buf[HC + hh]) + (lx_buf[2 * HC + hh] + lx_buf[3 * HC + hh]);
         const float lse_v = ltot > 0.f ? (m_ref + __log2f(ltot)) * 0.69314718055994531f : -INFINITY;
         const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-        if (!warp_all(mbar_spin<false>(&bars->odone, (uint32_t)klast & 1u, FLAG_MMA_WAIT, c.abort_flag))) return;
+        if (!wait_local(&bars->odone[klast & 1], (uint32_t)(klast >> 1) & 1u, FLAG_MMA_WAIT, c)) return;
         tc_fence_after();
         const bool real = head < p.H;
         float *dst = pc.whole ? p.out + ((size_t)pc.b * p.H + (real ? head : 0)) * 512
                               : p.ws_o + (((size_t)c.worker * 2 + pc.slot) * HR + head) * 512;
+        dst += 256 * cg + 128 * half;   // block j = cg, the lane's 128 columns of it
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int cc = 0; cc < 4; ++cc) {
+            uint32_t ov[32];
+            tmem_ld32(c.tmem + lane_base + TM_O + 128 * cg + 32 * cc, ov);
+            tmem_wait_ld();
+            if (real) {
+                float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * cc);
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t ov[32];
-                tmem_ld32(c.tmem + lane_base + TM_O + 128 * j + 32 * cc, ov);
-                tmem_wait_ld();
-                if (real) {
-                    float4 *d4 = reinterpret_cast<float4 *>(dst + 256 * j + 128 * half + 32 * cc);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        d4[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
-                                            __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
-                }
+                for (int e = 0; e < 8; ++e)
+                    d4[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
+                                        __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
             }
-        if (real && half == 0) {
+        }
+        if (real && part == 0) {
             if (pc.whole)
                 p.lse[(size_t)pc.b * p.H + head] = lse_v;
             else
@@ -490,26 +639,25 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        for (int s = 0; s < NSS; ++s) {
-            mbar_init(&bars->sfull[s], 1);
-            mbar_init(&bars->sempty[s], 1);
-        }
-        for (int s = 0; s < NPV; ++s) {
-            mbar_init(&bars->vfull[s], 1);
-            mbar_init(&bars->vempty[s], 1);
-        }
+        for (int g = 0; g < NKS; ++g) mbar_init(&bars->kfull[g], 1);
+        for (int g = 0; g < NKS - 1; ++g) mbar_init(&bars->kempty[g], 1);
+        for (int j = 0; j < NVS; ++j) mbar_init(&bars->vfull[j], 1);
+        for (int j = 0; j < NVS - 1; ++j) mbar_init(&bars->vempty[j], 1);
         mbar_init(&bars->qfull, 1);
+        mbar_init(&bars->qtm, 2 * NSOFT);    // one arrival per softmax warp of either CTA
         mbar_init(&bars->qempty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->sready[i], 1);
-            mbar_init(&bars->sfree[i], 8);   // one arrival per softmax warp of either CTA
+            mbar_init(&bars->sfree[i], 2 * NSOFT);
         }
-        mbar_init(&bars->pready, 8);
-        mbar_init(&bars->odone, 1);
-        mbar_init(&bars->ofree, 8);
-        mbar_init(&bars->mxbar[0], 4);
-        mbar_init(&bars->mxbar[1], 4);
-        mbar_init(&bars->lxbar, 4);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->odone[i], 1);
+            mbar_init(&bars->pready[i], 2 * NSOFT);
+        }
+        mbar_init(&bars->ofree, 2 * NSOFT);
+        mbar_init(&bars->mxbar[0], NSOFT);
+        mbar_init(&bars->mxbar[1], NSOFT);
+        mbar_init(&bars->lxbar, NSOFT);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -549,8 +697,10 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
     c.p1 = (c.p0 + W < total) ? c.p0 + W : total;
 
     if (c.p0 < total) {
-        if (warp == 0 && lane == 0) producer(p, maps, c);
-        if (warp == 1 && lane == 0 && c.r == 0) mma_issuer(p, c);
+        if (warp == 0 && lane == 0) key_producer(p, maps, c);
+        if (warp == 2 && lane == 0) value_producer(p, maps, c);
+        if (warp == 1 && lane == 0 && c.r == 0) score_issuer(p, c);
+        if (warp == 3 && lane == 0 && c.r == 0) value_issuer(p, c);
         if (warp >= 4) softmax_warps(p, c, warp, lane);
     }
 

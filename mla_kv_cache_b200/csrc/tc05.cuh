@@ -349,6 +349,17 @@ __device__ __forceinline__ void umma_pair_ss(uint32_t d_tmem, uint64_t a_desc, u
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// Same with A from tensor memory: each CTA holds its 64 rows of A twice, in lanes
+// [0, 64) and [64, 128) (row m in lanes m and 64 + m), two bf16 per 32-bit column.
+__device__ __forceinline__ void umma_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // Once every pair MMA issued so far by this thread has completed, arrive on the mbarrier
 // at this shared-memory offset in both CTAs of the pair.
 __device__ __forceinline__ void umma_pair_commit_both(uint64_t *bar) {
@@ -358,9 +369,13 @@ __device__ __forceinline__ void umma_pair_commit_both(uint64_t *bar) {
         "h"((uint16_t)3)
         : "memory");
 }
-// Arrive (release at cluster scope) on an mbarrier given by its shared::cluster address,
-// which may lie in either CTA of the cluster.
+// Arrive on an mbarrier given by its shared::cluster address, which may lie in either CTA
+// of the cluster, with the default semantics (release at CTA scope).  A release at
+// cluster scope costs about a microsecond per arrival on this path (measured), and the
+// pair pipelines do not need it: the data a pair barrier guards is either already in
+// the arriving thread's registers or made visible to the tensor cores by a proxy fence
+// before the arrival.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 }  // namespace kvattn
