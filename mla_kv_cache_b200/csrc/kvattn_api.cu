@@ -615,6 +615,7 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
     p.max_pages = cache.max_pages;
     p.page_size = cache.page_size;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.out_align32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
     const int smem = mla::smem_bytes(batch);
     if (smem > dev->max_smem_optin) {
         snprintf(t_detail, sizeof(t_detail), "needs %d B shared memory", smem);

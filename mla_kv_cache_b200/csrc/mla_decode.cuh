@@ -31,9 +31,11 @@
 //     B = the latent columns [256j + 128r, 256j + 128r + 128) of all 128 tokens (MN-major,
 //     loaded by CTA r for both halves: the B columns it supplies).  Lane m holds head
 //     64r + m's output columns 256j + [0, 128), lane 64 + m columns 256j + [128, 256).
-//   The weights enter as a bf16 high part (the top 16 bits of each fp32 weight) plus a
-//     bf16 remainder, two MMAs per K step, so they keep ~16 significant bits (a plain
-//     bf16 weight, 8 bits, misses the 2e-3 relative tolerance on sharp softmaxes).
+//     It runs in two steps, token half 0 then token half 1, each committed on its own
+//     barrier: the weights and the value slot of half 0 are free as soon as the first
+//     step is done, so the next tile's half-0 weights are written while the second step
+//     still runs, and the next tile's first step can follow this tile's second one
+//     without a gap.
 // Latent columns are thus read twice per pair (once as keys by the half's owner, once as
 // values by each CTA for its columns), the second time from L2.
 //
@@ -41,9 +43,9 @@
 //   warp 0, one thread   key producer (both CTAs): the shared-memory part of the query
 //                        block once per sequence and a ring of three 24 KB key slots (one
 //                        tile); completions signal rank 0's barriers.
-//   warp 2, one thread   value producer (both CTAs): a ring of two 32 KB value slots (one
-//                        tile), independent of the key stream; its loads hit L2 (the keys'
-//                        latent columns, loaded by the pair moments before).
+//   warp 2, one thread   value producer (both CTAs): two 32 KB value slots, one per token
+//                        half of a tile, independent of the key stream; its loads hit L2
+//                        (the keys' latent columns, loaded by the pair moments before).
 // Each slot release is one tcgen05.commit, which costs the issuing thread ~300 cycles
 // (measured, against ~56 for an MMA), so the slots are a few chunks each.
 //   warp 1, one thread   score MMA issuer (rank 0 only), running ahead of the softmax by
@@ -55,7 +57,8 @@
 //                        (moves only when a tile's maximum exceeds it by more than 2^8;
 //                        then this CTA's rows of O are rescaled in tensor memory), weights
 //                        into shared memory, row sums; at the end of a piece the
-//                        normalised result.
+//                        normalised result.  The warps of token half 0 (lanes 0-63) write
+//                        the half-0 weights, those of half 1 the half-1 weights.
 // Every wait is bounded; every wait ahead of a warp-collective instruction is made
 // warp-uniform.  No TMA load uses multicast.
 #pragma once
@@ -75,7 +78,7 @@ constexpr int NQC = 9;                   // query / key chunks of 64 columns: 8 
 constexpr int NQT = 4;                   // query chunks held in tensor memory (latent columns [0, 256))
 constexpr int NQS = NQC - NQT;           // query chunks in shared memory (latent [256, 512) + RoPE)
 constexpr int NKS = 3;                   // key ring: 3 slots of 3 chunks (192 columns), one tile
-constexpr int NVS = 2;                   // value ring: 2 slots (latent block j: 128 columns of both halves), one tile
+constexpr int NVS = 2;                   // value slots: one per token half (this CTA's 256 latent columns)
 constexpr int KSLOT = 3 * CHUNK;         // 24 KB
 constexpr int VSLOT = 4 * CHUNK;         // 32 KB
 constexpr int NTHREADS = 384;            // warps 0-3: producers and MMA issuers, 4-11: softmax
@@ -102,23 +105,25 @@ static_assert(smem_bytes(MAX_BATCH) <= 232448, "shared memory of the MLA kernel 
 
 struct Bars {
     // Every ring slot serves each tile once, so its phase is the tile count.  The release
-    // of a tile's last key slot is that tile's sready, the release of its last value slot
-    // its odone: each tile takes three commits for the keys and two for the values.
+    // of a tile's last key slot is that tile's sready; a value slot and the weights of its
+    // token half are released by that half's odone.
     uint64_t kfull[NKS];                // key ring (rank 0, both CTAs' bytes)
     uint64_t kempty[NKS - 1];           // release of key slots 0 and 1 (both CTAs)
     uint64_t sready[2];                 // the scores of a tile are in tensor memory (score buffer =
                                         // tile parity; both CTAs)
-    uint64_t vfull[NVS];                // value ring (rank 0)
-    uint64_t vempty[NVS - 1];           // release of value slot 0 (both CTAs)
-    uint64_t odone[2];                  // the value product of a tile (parity) is done (both CTAs)
+    uint64_t vfull[NVS];                // value slot of token half h (rank 0)
+    uint64_t odone[2][2];               // [h][tile parity]: the half-h step of a tile's value product
+                                        // is done (both CTAs); h = 1: the whole product
     uint64_t qfull;                     // shared-memory query chunks of both CTAs landed (rank 0)
     uint64_t qtm;                       // tensor-memory query columns written in both CTAs (rank 0)
     uint64_t qempty;                    // every score product of the piece has read Q (both CTAs)
-    uint64_t sfree[2];                  // both CTAs have read them (rank 0: 4 warps x 2 CTAs)
-    uint64_t pready[2];                 // weights of a tile (parity) written, O rescaled, in both CTAs (rank 0)
+    uint64_t sfree[2];                  // both CTAs have read them (rank 0: 8 warps x 2 CTAs)
+    uint64_t pready[2][2];              // [h][tile parity], rank 0: the half-h weights are written
+                                        // (h = 0 also: every rescale of O is done; all 16 softmax
+                                        // warps arrive) -- h = 1: the 8 warps of half 1
     uint64_t ofree;                     // both CTAs' epilogues have read O (rank 0)
-    uint64_t mxbar[2];                  // the four softmax warps' tile maxima written (tile parity)
-    uint64_t lxbar;                     // the four softmax warps' row sums written (end of a piece)
+    uint64_t mxbar[2];                  // the softmax warps' tile maxima written (tile parity)
+    uint64_t lxbar;                     // the softmax warps' row sums written (end of a piece)
 };
 static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
 
@@ -140,6 +145,7 @@ struct MlaParams {
     const int32_t *block_table; // [B, max_pages] physical pages (paged cache); null: contiguous
     int max_pages;              // block-table columns
     int page_size;              // rows per page (T_max when contiguous)
+    int out_align32;            // out is 32-byte aligned (else the epilogue stores 16 bytes at a time)
 };
 
 struct MlaMaps {
@@ -257,27 +263,23 @@ __device__ __forceinline__ void value_producer(const MlaParams &p, const MlaMaps
         pos = pc.ustart + pc.lt1;
         const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
         for (int lt = pc.lt0; lt < pc.lt1 && ok; ++lt) {
-            const HalfSrc hsrc[2] = {half_source(p, pc.b, len, lt, 0), half_source(p, pc.b, len, lt, 1)};
-            for (int j = 0; j < NVS; ++j, ++nld) {
-                // slot j of the previous tile must have been read: slot 0 has its own release
-                // barrier, the last slot's is the previous tile's odone
+            for (int h = 0; h < NVS; ++h, ++nld) {
+                // slot h is free once the previous tile's half-h step is done
                 const int kt = nld / NVS;
-                const bool freed = j < NVS - 1
-                    ? mbar_wait(&bars->vempty[j], ((uint32_t)kt & 1u) ^ 1u, FLAG_EMPTY_WAIT, c.abort_flag)
-                    : (kt == 0 || mbar_wait(&bars->odone[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u,
-                                            FLAG_EMPTY_WAIT, c.abort_flag));
-                if (!freed) {
+                if (kt > 0 && !mbar_wait(&bars->odone[h][(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u,
+                                         FLAG_EMPTY_WAIT, c.abort_flag)) {
                     ok = false;
                     break;
                 }
-                if (lead) mbar_arrive_expect_tx(&bars->vfull[j], 2 * VSLOT);
-                const uint32_t bar = map_to_rank(smem_u32(&bars->vfull[j]), 0);
-                uint8_t *dst = c.smem + OFF_PV + j * VSLOT;
-                const int x = 256 * j + 128 * (int)c.r;
+                const HalfSrc hs = half_source(p, pc.b, len, lt, h);
+                if (lead) mbar_arrive_expect_tx(&bars->vfull[h], 2 * VSLOT);
+                const uint32_t bar = map_to_rank(smem_u32(&bars->vfull[h]), 0);
+                uint8_t *dst = c.smem + OFF_PV + h * VSLOT;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    tma_load_3d_pair(dst + 2 * h * CHUNK, &m.lat, bar, x, hsrc[h].y, hsrc[h].page, pol_last);
-                    tma_load_3d_pair(dst + (2 * h + 1) * CHUNK, &m.lat, bar, x + 64, hsrc[h].y, hsrc[h].page, pol_last);
+                for (int j = 0; j < 2; ++j) {   // latent block j: this CTA's 128 columns of it
+                    const int x = 256 * j + 128 * (int)c.r;
+                    tma_load_3d_pair(dst + 2 * j * CHUNK, &m.lat, bar, x, hs.y, hs.page, pol_last);
+                    tma_load_3d_pair(dst + (2 * j + 1) * CHUNK, &m.lat, bar, x + 64, hs.y, hs.page, pol_last);
                 }
             }
         }
@@ -355,8 +357,8 @@ __device__ __forceinline__ void score_issuer(const MlaParams &p, const Ctx &c) {
     }
 }
 
-// O += P_hi C + P_lo C for every tile kt: latent blocks j, token halves h, K-steps of 16
-// tokens.
+// O += P_hi C + P_lo C for every tile kt: token halves h (one commit each), latent
+// blocks j, K-steps of 16 tokens.
 __device__ __forceinline__ void value_issuer(const MlaParams &p, const Ctx &c) {
     Bars *bars = c.bars;
     constexpr uint32_t id_v = idesc_f16(128, 256, 1, 1, 1);    // B (the latents) MN-major
@@ -373,16 +375,17 @@ __device__ __forceinline__ void value_issuer(const MlaParams &p, const Ctx &c) {
         if (pi > 0 && !wait_remote(&bars->ofree, (uint32_t)(pi - 1) & 1u, c)) return;
         for (int kt = k; kt < k + nt; ++kt) {
             const bool first = kt == k;
-            if (!wait_remote(&bars->pready[kt & 1], (uint32_t)(kt >> 1) & 1u, c)) return;
-            for (int jb = 0; jb < NVS; ++jb) {
-                const uint32_t d = c.tmem + TM_O + 128 * jb;
-                if (!mbar_wait(&bars->vfull[jb], (uint32_t)kt & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                if (!wait_remote(&bars->pready[h][kt & 1], (uint32_t)(kt >> 1) & 1u, c)) return;
+                if (!mbar_wait(&bars->vfull[h], (uint32_t)kt & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
                 tc_fence_after();
+                const uint64_t hi = p_desc + (uint64_t)(h * (CHUNK >> 4));
+                const uint64_t lo = hi + (uint64_t)(2 * (CHUNK >> 4));
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint64_t bd = vr_desc + (uint64_t)((jb * VSLOT + h * 2 * CHUNK) >> 4);
-                    const uint64_t hi = p_desc + (uint64_t)(h * (CHUNK >> 4));
-                    const uint64_t lo = hi + (uint64_t)(2 * (CHUNK >> 4));
+                for (int jb = 0; jb < 2; ++jb) {
+                    const uint32_t d = c.tmem + TM_O + 128 * jb;
+                    const uint64_t bd = vr_desc + (uint64_t)((h * VSLOT + jb * 2 * CHUNK) >> 4);
                     umma_pair_ss(d, hi, bd, id_v, (!first || h > 0) ? 1u : 0u);
                     umma_pair_ss(d, lo, bd, id_v, 1u);
 #pragma unroll
@@ -391,10 +394,7 @@ __device__ __forceinline__ void value_issuer(const MlaParams &p, const Ctx &c) {
                         umma_pair_ss(d, lo + 2 * kk, bd + 128 * kk, id_v, 1u);
                     }
                 }
-                if (jb < NVS - 1)
-                    umma_pair_commit_both(&bars->vempty[jb]);
-                else
-                    umma_pair_commit_both(&bars->odone[kt & 1]);   // releases the last slot too
+                umma_pair_commit_both(&bars->odone[h][kt & 1]);   // frees value slot h and the half-h weights
             }
         }
         k += nt;
@@ -428,8 +428,12 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
     float *lx_buf = reinterpret_cast<float *>(c.smem + OFF_LX);   // [4 parts][64]
     const uint32_t sfree0 = map_to_rank(smem_u32(&bars->sfree[0]), 0);
     const uint32_t sfree1 = map_to_rank(smem_u32(&bars->sfree[1]), 0);
-    const uint32_t pready0 = map_to_rank(smem_u32(&bars->pready[0]), 0);
-    const uint32_t pready1 = map_to_rank(smem_u32(&bars->pready[1]), 0);
+    // the weights-ready barriers this thread arrives on (rank 0), by tile parity: the
+    // first step's (every warp) and its own half's
+    const uint32_t pready_first0 = map_to_rank(smem_u32(&bars->pready[0][0]), 0);
+    const uint32_t pready_first1 = map_to_rank(smem_u32(&bars->pready[0][1]), 0);
+    const uint32_t pready_own0 = map_to_rank(smem_u32(&bars->pready[half][0]), 0);
+    const uint32_t pready_own1 = map_to_rank(smem_u32(&bars->pready[half][1]), 0);
     const uint32_t ofree0 = map_to_rank(smem_u32(&bars->ofree), 0);
     const uint32_t qtm0 = map_to_rank(smem_u32(&bars->qtm), 0);
     // this thread's 32 tokens of the weights: row hh of the half's K-major chunk, 16-byte
@@ -439,28 +443,47 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
     const float sl2 = p.scale_log2;
 
     // Query latent columns [64cg, 64cg + 64) (bf16 pairs) of this lane's head of sequence
-    // b into tensor memory; both lanes of a head hold the row.
-    auto write_q = [&](int b) -> bool {
-        const bool realq = head < p.H;
-        const uint4 *qrow =
-            reinterpret_cast<const uint4 *>(p.q_latent + ((size_t)b * p.H + (realq ? head : 0)) * 512) + 16 * cg;
-        tc_fence_after();
+    // b: loaded into registers, then (once the previous piece's score products are done
+    // with the columns) written to tensor memory; both lanes of a head hold the row.
+    const bool realq = head < p.H;
+    auto q_row = [&](int b) {
+        return reinterpret_cast<const uint4 *>(p.q_latent + ((size_t)b * p.H + (realq ? head : 0)) * 512) + 16 * cg;
+    };
+    auto load_q = [&](int b, uint32_t (&v0)[32], uint32_t (&v1)[32]) {
+        const uint4 *qrow = q_row(b);
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
-            uint32_t v[32];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                uint4 x = make_uint4(0, 0, 0, 0);
-                if (realq) x = __ldg(qrow + 8 * w + e);
-                v[4 * e] = x.x; v[4 * e + 1] = x.y; v[4 * e + 2] = x.z; v[4 * e + 3] = x.w;
+        for (int e = 0; e < 8; ++e) {
+            uint4 x = make_uint4(0, 0, 0, 0), y = make_uint4(0, 0, 0, 0);
+            if (realq) {
+                x = __ldg(qrow + e);
+                y = __ldg(qrow + 8 + e);
             }
-            tmem_st32(c.tmem + lane_base + TM_Q + 64 * cg + 32 * w, v);
+            v0[4 * e] = x.x; v0[4 * e + 1] = x.y; v0[4 * e + 2] = x.z; v0[4 * e + 3] = x.w;
+            v1[4 * e] = y.x; v1[4 * e + 1] = y.y; v1[4 * e + 2] = y.z; v1[4 * e + 3] = y.w;
         }
+    };
+    auto store_q = [&](uint32_t (&v0)[32], uint32_t (&v1)[32]) {
+        tc_fence_after();
+        tmem_st32(c.tmem + lane_base + TM_Q + 64 * cg, v0);
+        tmem_st32(c.tmem + lane_base + TM_Q + 64 * cg + 32, v1);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(qtm0);
-        return true;
+    };
+    // Rescale block cg of this lane's O by alpha (warp-collective).
+    auto rescale_o = [&](float alpha) {
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+            const uint32_t addr = c.tmem + lane_base + TM_O + 128 * cg + 32 * cc;
+            uint32_t ov[32];
+            tmem_ld32(addr, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+            tmem_st32(addr, ov);
+        }
+        tmem_wait_st();
     };
 
     int k = 0, pi = 0;
@@ -469,12 +492,24 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         pos = pc.ustart + pc.lt1;
         const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
         const int nt = pc.lt1 - pc.lt0;
-        if (pi == 0 && !write_q(pc.b)) return;
+        if (pi == 0) {
+            uint32_t v0[32], v1[32];
+            load_q(pc.b, v0, v1);
+            store_q(v0, v1);
+        }
+        // the next piece's sequence (-1: none); its query rows are fetched into L2 during
+        // this piece's last tile
+        const int next_b = pos < c.p1 ? piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0).b : -1;
         float m_ref = -INFINITY;      // running max (log2 units), shared by the four parts of the head
         float l = 0.f;                // row sum of this thread's weights, relative to m_ref
         for (int t = 0; t < nt; ++t) {
             const int kt = k + t;
             const int sb = kt & 1;
+            if (t == nt - 1 && next_b >= 0 && realq) {
+                const uint4 *qn = q_row(next_b);
+                prefetch_l2(qn);
+                prefetch_l2(qn + 8);
+            }
             // first valid column of this thread's 32 (masked: rows of the half below lo)
             const int lo = half_source(p, pc.b, len, pc.lt0 + t, half).lo - 32 * cg;
             // ---- this thread's 32 scores
@@ -544,44 +579,60 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
                 }
             }
             l = l * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
-            // ---- the value product of tile kt - 1 must be done with the weights and with O
-            if (kt >= 1 && !wait_local(&bars->odone[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u, FLAG_MMA_WAIT, c))
-                return;
-            tc_fence_after();
+            // ---- the weights into shared memory.  The half-h weights of tile kt - 1 are free
+            //      once the half-h step of its value product is done; a rescale of O needs
+            //      the whole product done, and must be finished before tile kt's first step,
+            //      which is why every warp arrives on the first step's barrier.
+            const int kp = kt - 1;
+            const bool any_rescale = __any_sync(0xffffffffu, rescale);   // only when t > 0, so kp >= 0
+            auto store_p = [&]() {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int slot = ((4 * cg + u) ^ (hh & 7)) * 16;
-                *reinterpret_cast<uint4 *>(row_hi + slot) =
-                    make_uint4(whi[4 * u], whi[4 * u + 1], whi[4 * u + 2], whi[4 * u + 3]);
-                *reinterpret_cast<uint4 *>(row_lo + slot) =
-                    make_uint4(wlo[4 * u], wlo[4 * u + 1], wlo[4 * u + 2], wlo[4 * u + 3]);
-            }
-            // rescale block cg of this lane's O (warp-collective: the whole warp takes the
-            // branch when any of its rows needs it, with factor 1 for the others)
-            if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    const uint32_t addr = c.tmem + lane_base + TM_O + 128 * cg + 32 * cc;
-                    uint32_t ov[32];
-                    tmem_ld32(addr, ov);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-                    tmem_st32(addr, ov);
+                for (int u = 0; u < 4; ++u) {
+                    const int slot = ((4 * cg + u) ^ (hh & 7)) * 16;
+                    *reinterpret_cast<uint4 *>(row_hi + slot) =
+                        make_uint4(whi[4 * u], whi[4 * u + 1], whi[4 * u + 2], whi[4 * u + 3]);
+                    *reinterpret_cast<uint4 *>(row_lo + slot) =
+                        make_uint4(wlo[4 * u], wlo[4 * u + 1], wlo[4 * u + 2], wlo[4 * u + 3]);
                 }
-                tmem_wait_st();
+                fence_proxy_async_smem();
+            };
+            if (half == 0) {
+                if (kt >= 1 && !wait_local(&bars->odone[0][kp & 1], (uint32_t)(kp >> 1) & 1u, FLAG_MMA_WAIT, c))
+                    return;
+                if (any_rescale) {
+                    if (!wait_local(&bars->odone[1][kp & 1], (uint32_t)(kp >> 1) & 1u, FLAG_MMA_WAIT, c)) return;
+                    tc_fence_after();
+                    rescale_o(alpha);
+                }
+                store_p();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(sb ? pready_own1 : pready_own0);
+            } else {
+                const bool need_prev = kt >= 1;
+                if (any_rescale) {
+                    if (!wait_local(&bars->odone[1][kp & 1], (uint32_t)(kp >> 1) & 1u, FLAG_MMA_WAIT, c)) return;
+                    tc_fence_after();
+                    rescale_o(alpha);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(sb ? pready_first1 : pready_first0);   // O of these lanes is settled
+                if (need_prev && !any_rescale &&
+                    !wait_local(&bars->odone[1][kp & 1], (uint32_t)(kp >> 1) & 1u, FLAG_MMA_WAIT, c))
+                    return;
+                store_p();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(sb ? pready_own1 : pready_own0);
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(sb ? pready1 : pready0);
         }
         // ---- end of the piece.  First the next piece's query, so that its score products
         //      can start while this epilogue runs (this piece's have read Q: qempty).
-        if (pos < c.p1) {
-            const Piece nx = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
+        if (next_b >= 0) {
+            uint32_t v0[32], v1[32];
+            load_q(next_b, v0, v1);
             if (!wait_local(&bars->qempty, (uint32_t)pi & 1u, FLAG_MMA_WAIT, c)) return;
-            if (!write_q(nx.b)) return;
+            store_q(v0, v1);
         }
         // ---- the head's row sum (four parts), normalise, write block cg of the lane
         const int klast = k + nt - 1;
@@ -593,18 +644,27 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         const float ltot = (lx_buf[hh] + lx_buf[HC + hh]) + (lx_buf[2 * HC + hh] + lx_buf[3 * HC + hh]);
         const float lse_v = ltot > 0.f ? (m_ref + __log2f(ltot)) * 0.69314718055994531f : -INFINITY;
         const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-        if (!wait_local(&bars->odone[klast & 1], (uint32_t)(klast >> 1) & 1u, FLAG_MMA_WAIT, c)) return;
+        if (!wait_local(&bars->odone[1][klast & 1], (uint32_t)(klast >> 1) & 1u, FLAG_MMA_WAIT, c)) return;
         tc_fence_after();
-        const bool real = head < p.H;
+        const bool real = realq;
         float *dst = pc.whole ? p.out + ((size_t)pc.b * p.H + (real ? head : 0)) * 512
                               : p.ws_o + (((size_t)c.worker * 2 + pc.slot) * HR + head) * 512;
         dst += 256 * cg + 128 * half;   // block j = cg, the lane's 128 columns of it
+        const bool wide = !pc.whole || p.out_align32;   // the workspace is 256-byte aligned
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
             uint32_t ov[32];
             tmem_ld32(c.tmem + lane_base + TM_O + 128 * cg + 32 * cc, ov);
             tmem_wait_ld();
-            if (real) {
+            if (real && wide) {   // 32-byte stores: whole sectors
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float o8[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) o8[i] = __uint_as_float(ov[8 * e + i]) * inv;
+                    st_global_v8(dst + 32 * cc + 8 * e, o8);
+                }
+            } else if (real) {
                 float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * cc);
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
@@ -642,7 +702,6 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
         for (int g = 0; g < NKS; ++g) mbar_init(&bars->kfull[g], 1);
         for (int g = 0; g < NKS - 1; ++g) mbar_init(&bars->kempty[g], 1);
         for (int j = 0; j < NVS; ++j) mbar_init(&bars->vfull[j], 1);
-        for (int j = 0; j < NVS - 1; ++j) mbar_init(&bars->vempty[j], 1);
         mbar_init(&bars->qfull, 1);
         mbar_init(&bars->qtm, 2 * NSOFT);    // one arrival per softmax warp of either CTA
         mbar_init(&bars->qempty, 1);
@@ -651,8 +710,10 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
             mbar_init(&bars->sfree[i], 2 * NSOFT);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars->odone[i], 1);
-            mbar_init(&bars->pready[i], 2 * NSOFT);
+            mbar_init(&bars->odone[0][i], 1);
+            mbar_init(&bars->odone[1][i], 1);
+            mbar_init(&bars->pready[0][i], 2 * NSOFT);   // every softmax warp of either CTA
+            mbar_init(&bars->pready[1][i], NSOFT);       // the half-1 warps of either CTA
         }
         mbar_init(&bars->ofree, 2 * NSOFT);
         mbar_init(&bars->mxbar[0], NSOFT);

@@ -31,7 +31,7 @@ def _reset_knob():
     assert kb.kvattn_read_device_flags() == 0, "a bounded wait ran out on the device"
 
 
-def run_case(cfg, seed=0, poison=True, q_gain=1.0, lat_gain=1.0):
+def run_case(cfg, seed=0, poison=True, q_gain=1.0, lat_gain=1.0, out_offset=0):
     x = wl.make_mla_inputs(cfg, seed=seed, poison_tail=poison)
     if q_gain != 1.0:  # a power of two keeps the bf16 values exact
         x["q_latent"] = (x["q_latent"].float() * q_gain).to(torch.bfloat16)
@@ -40,8 +40,12 @@ def run_case(cfg, seed=0, poison=True, q_gain=1.0, lat_gain=1.0):
         x["latent_cache"] = (x["latent_cache"].float() * lat_gain).to(torch.bfloat16)
         x["q_latent"] = (x["q_latent"].float() / lat_gain).to(torch.bfloat16)
     d = {k: v.cuda() for k, v in x.items()}
+    out = None
+    if out_offset:  # an output buffer that starts out_offset floats into an allocation
+        B, H = cfg.batch, cfg.n_heads
+        out = torch.full((B * H * 512 + out_offset,), float("nan"), device="cuda")[out_offset:].view(B, H, 512)
     out, lse = kb.kvattn_mla_decode(d["q_latent"], d["q_rope"], d["latent_cache"], d["rope_cache"],
-                                    d["seq_lens"], cfg.scale)
+                                    d["seq_lens"], cfg.scale, out=out)
     torch.cuda.synchronize()
     ro, rl = oracle.mla_decode(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"],
                                x["seq_lens"], cfg.scale)
@@ -81,6 +85,11 @@ def test_latents_beyond_fp16_range():
     the values stay bf16 all the way through the value product, and the output (divided
     by the gain, like the oracle's) meets the base case's tolerance."""
     run_case(mla("big", 2, 128, 700, lens=[700, 129]), lat_gain=2.0 ** 17)
+
+
+def test_output_16_byte_aligned():
+    """An output 16 but not 32 bytes aligned (the epilogue's 32-byte stores need 32)."""
+    run_case(mla("out16", 3, 128, 500, lens=[500, 77, 260]), out_offset=4)
 
 
 @pytest.mark.parametrize("workers,min_tiles", [(1, 1), (2, 1), (3, 1), (7, 1), (40, 1)])
