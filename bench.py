@@ -377,6 +377,11 @@ def oracle_step(cfg, x, ids):
     return oracle.gqa_decode(x["q"], x["k_cache"], x["v_cache"], x["seq_lens"], cfg.scale, batch_ids=ids)
 
 
+def is_mla(cfg):
+    """The MLA path is one kernel per call; the GQA paths launch a decode and a combine kernel."""
+    return isinstance(cfg, wl.MLAConfig)
+
+
 def flush_l2(buf):
     """Evict the step's data from L2: write a buffer twice the L2 size, then read it
     back, so that L2 holds clean lines (no dirty write-back of the flush itself lands
@@ -547,11 +552,13 @@ def gpu_arm(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
                      "peak_source": pk["source"] + " burst copy bandwidth",
-                     "timed_unit": "one library call: decode kernel + PDL-chained combine kernel"},
+                     "timed_unit": "one library call: " + ("the decode kernel (partials merged inside it)"
+                                                           if is_mla(head_cfg) else
+                                                           "decode kernel + PDL-chained combine kernel")},
         "e2e": {"value": nb["total"] * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "per step: pinned host q/seq_lens -> device, library call, out/lse -> pinned host; KV cache resident in HBM"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (1 if is_mla(head_cfg) else 2) * args.steps,
         "clocks": clocks,
         "configs": dict(extras, **{args.config: res}),
     }

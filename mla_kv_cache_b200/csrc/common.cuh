@@ -180,13 +180,6 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-// One 32-byte store (a whole sector); p is 32-byte aligned.
-__device__ __forceinline__ void st_global_v8(float *p, const float (&v)[8]) {
-    asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
-                 ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
-                 : "memory");
-}
-
 // 2^x with the hardware approximation (flushes subnormal results to zero).
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/kvattn.h"
@@ -42,6 +43,7 @@ struct DeviceState {
     } funcs[64] = {};
     int n_funcs = 0;
     int mla_clusters = 0;   // co-resident MLA CTA pairs (0: not queried yet)
+    std::atomic<unsigned int> mla_calls{0};   // MLA decode calls issued (tags the merge counters)
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -615,7 +617,9 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
     p.max_pages = cache.max_pages;
     p.page_size = cache.page_size;
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    p.out_align32 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
+    unsigned int epoch = ++dev->mla_calls;
+    if (epoch == 0) epoch = ++dev->mla_calls;   // 0 is the counters' state at load
+    p.epoch = epoch;
     const int smem = mla::smem_bytes(batch);
     if (smem > dev->max_smem_optin) {
         snprintf(t_detail, sizeof(t_detail), "needs %d B shared memory", smem);
@@ -654,44 +658,23 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
     if (workers < 1) workers = 1;
     p.workers = (int)workers;
 
+    // Partial results of the sequences cut by a worker boundary, merged inside the kernel
+    // by the last worker to finish each block.
     void *ws = nullptr;
-    const size_t meta_bytes = ((16 + (size_t)(batch + 1) * 4) + 255) & ~size_t(255);
     const size_t wlse_bytes = (((size_t)p.workers * 2 * mla::HR * 4) + 255) & ~size_t(255);
     const size_t wo_bytes = (size_t)p.workers * 2 * mla::HR * 512 * 4;
     {
         std::lock_guard<std::mutex> lk(g_mutex);
-        st = ensure_workspace(dev, meta_bytes + wlse_bytes + wo_bytes, &ws);
+        st = ensure_workspace(dev, wlse_bytes + wo_bytes, &ws);
         if (st != KVATTN_OK) return st;
     }
-    p.ws_meta = ws;
-    p.ws_lse = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes);
-    p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + meta_bytes + wlse_bytes);
+    p.ws_lse = reinterpret_cast<float *>(ws);
+    p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + wlse_bytes);
 
     mla_decode_kernel<<<2 * p.workers, mla::NTHREADS, smem, s>>>(p, maps);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e, "mla decode launch");
-
-    CombineParams cp;
-    cp.seq_lens = p.seq_lens;
-    cp.ws_lse = p.ws_lse;
-    cp.ws_o = p.ws_o;
-    cp.out = out;
-    cp.lse = lse;
-    cp.B = batch;
-    cp.n_q = n_heads;
-    cp.units_per_seq = 1;
-    cp.heads_per_unit = mla::HR;
-    cp.n_hb = 1;
-    cp.n_kv = 1;
-    cp.g = n_heads;
-    cp.T_max = p.T_max;
-    cp.tile = mla::TILE;
-    cp.workers = p.workers;
-    cp.min_tiles = p.min_tiles;
-    cp.q_len = 1;
-    cp.window = 0;
-    return launch_combine(512, cp, batch, n_heads, s,
-                          combine_warps((cache.capacity + mla::TILE - 1) / mla::TILE, max_tiles, p.workers));
+    return KVATTN_OK;
 }
 
 // Argument checks of kvattn_gqa_decode (and of kvattn_gqa_decode_noalloc, which takes the

@@ -59,6 +59,14 @@
 //                        into shared memory, row sums; at the end of a piece the
 //                        normalised result.  The warps of token half 0 (lanes 0-63) write
 //                        the half-0 weights, those of half 1 the half-1 weights.
+// End of a piece.  Each softmax warp owns a 32-head x 128-column block of O; it normalises
+// the block and writes it row-contiguously (transposed through its own 4 KB of the
+// weights buffer, so that eight lanes store one row's 128 bytes).  A sequence cut by a
+// worker boundary leaves one partial block (and log-sum-exp) per worker in the
+// workspace; the warp then counts itself in at a per-(sequence, rank, warp) counter, and
+// the last of the sequence's workers to arrive merges that block's partials by
+// log-sum-exp into the output.  No worker waits for another, and there is no second
+// kernel.  Empty sequences (no worker) get out = 0, lse = -inf, spread over the workers.
 // Every wait is bounded; every wait ahead of a warp-collective instruction is made
 // warp-uniform.  No TMA load uses multicast.
 #pragma once
@@ -135,7 +143,6 @@ struct MlaParams {
     const int32_t *seq_lens;
     float *out;        // [B, H, 512]
     float *lse;        // [B, H]
-    void *ws_meta;
     float *ws_lse;     // [workers, 2, 128]
     float *ws_o;       // [workers, 2, 128, 512]
     int B, H, T_max;
@@ -145,7 +152,7 @@ struct MlaParams {
     const int32_t *block_table; // [B, max_pages] physical pages (paged cache); null: contiguous
     int max_pages;              // block-table columns
     int page_size;              // rows per page (T_max when contiguous)
-    int out_align32;            // out is 32-byte aligned (else the epilogue stores 16 bytes at a time)
+    unsigned int epoch;         // number of this call (never 0), tags the merge counters
 };
 
 struct MlaMaps {
@@ -162,8 +169,47 @@ struct Ctx {
     uint32_t tmem;
     uint32_t r;        // rank in the pair
     int worker;
+    long long W;       // tiles per worker
     long long p0, p1;
 };
+
+// Tiles per worker for a batch whose sequences all have n tiles, given the balanced
+// share w0: n / k for the largest k dividing n with n / k >= w0, or the smallest multiple
+// of n not below w0 -- kept only if it adds at most max(2, w0 / 4) tiles to the share.
+__device__ __forceinline__ long long uniform_tiles_per_worker(long long w0, int n) {
+    long long w = n;
+    if (w0 >= n) {
+        w = ((w0 + n - 1) / n) * n;
+    } else {
+        for (int k = (int)(n / w0); k > 1; --k)
+            if (n % k == 0) {
+                w = n / k;
+                break;
+            }
+    }
+    const long long slack = w0 / 4 > 2 ? w0 / 4 : 2;
+    return w - w0 <= slack ? w : w0;
+}
+
+// Merge counters of the split sequences: one per (sequence, CTA rank, softmax warp), each
+// counting the workers whose partial block of that warp has been written in the call
+// numbered by its high 32 bits.  Zero at load; a call's first arrival re-tags it.
+__device__ unsigned long long g_mla_merge_count[MAX_BATCH * 2 * NSOFT];
+
+// One arrival of this call at a merge counter; true for the last of n arrivals.  The
+// compare-and-swap loop retries only when another arrival got in between.
+__device__ __forceinline__ bool merge_arrive_last(unsigned long long *cnt, unsigned int epoch, int n) {
+    unsigned long long cur = *reinterpret_cast<volatile unsigned long long *>(cnt);
+    unsigned long long nxt = 0;
+    for (int i = 0; i < (1 << 20); ++i) {
+        nxt = (unsigned int)(cur >> 32) == epoch ? cur + 1 : ((unsigned long long)epoch << 32) | 1ull;
+        const unsigned long long prev = atomicCAS(cnt, cur, nxt);
+        if (prev == cur) return (unsigned int)(nxt & 0xffffffffull) == (unsigned int)n;
+        cur = prev;
+    }
+    atomicOr(&g_device_flags, FLAG_PEER_WAIT);
+    return false;
+}
 
 // Where half h of tile lt of a sequence of length len is loaded from, and which of its 64
 // rows are tokens of that half.  A half is a 64-token sub-tile (pages hold whole
@@ -486,6 +532,127 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         tmem_wait_st();
     };
 
+    // This warp's block of O: rows head0 + [0, 32) (this CTA's heads 32 (q & 1) + ..), columns
+    // col0 + [0, 128) of the 512.
+    const int head0 = HC * (int)c.r + 32 * (q & 1);
+    const int col0 = 256 * cg + 128 * half;
+    // 16-byte unit u (0..7) of row rr of the warp's 4 KB transpose scratch: the warp's own
+    // units of the weights buffer (row 32 (q & 1) + rr of its half's chunk, units 4cg..4cg+3
+    // of the high part for u < 4, of the remainder for u >= 4)
+    auto scratch_unit = [&](int rr, int u) -> uint8_t * {
+        const int row = 32 * (q & 1) + rr;
+        return c.smem + OFF_P + half * CHUNK + (u >> 2) * 2 * CHUNK + row * 128 +
+               (((4 * cg + (u & 3)) ^ (row & 7)) * 16);
+    };
+    // Merge of the partial blocks of sequence b written by its n_parts workers (all
+    // arrived): out = sum_c exp(lse_c - lse) o_c, lse = log sum_c exp(lse_c).  Lane L
+    // takes the log-sum-exp of row L and puts the row's weights exp(lse_c - lse) in the
+    // warp's scratch (32 parts at a time); each load instruction then reads four rows'
+    // 128 contiguous bytes (eight lanes per row), two parts' loads in flight together.
+    // The partials are read through L2 (other SMs wrote them).
+    auto merge_block = [&](int b, long long ustart, int n_parts) {
+        const long long c_first = ustart / c.W;
+        auto part_row = [&](int j, int h) -> size_t {
+            const long long cw = c_first + j;
+            const int slot = (ustart <= cw * c.W) ? 0 : 1;
+            return ((size_t)cw * 2 + slot) * HR + h;
+        };
+        const int hl = head0 + lane;
+        float M = -INFINITY;
+        for (int j0 = 0; j0 < n_parts; j0 += 4) {
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = j0 + u < n_parts ? __ldcg(p.ws_lse + part_row(j0 + u, hl)) : -INFINITY;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) M = fmaxf(M, v[u]);
+        }
+        float S = 0.f;
+        if (M != -INFINITY)
+            for (int j0 = 0; j0 < n_parts; j0 += 4) {
+                float v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) v[u] = j0 + u < n_parts ? __ldcg(p.ws_lse + part_row(j0 + u, hl)) : -INFINITY;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) S += v[u] == -INFINITY ? 0.f : fast_exp2((v[u] - M) * 1.4426950408889634f);
+            }
+        const float lse_all = S > 0.f ? M + __logf(S) : -INFINITY;
+        // the scratch as [32 parts][32 rows] floats (its 4 KB are the warp's own units of the
+        // weights buffer: scratch_unit(r, u) for r < 32, u < 8 -- 8 floats per (r, u))
+        auto wslot = [&](int j, int rr) -> float * {   // weight of part j (< 32) for row rr
+            return reinterpret_cast<float *>(scratch_unit(j, rr >> 2)) + (rr & 3);
+        };
+        for (int jb = 0; jb < n_parts; jb += 32) {
+            const int nj = n_parts - jb < 32 ? n_parts - jb : 32;
+            __syncwarp();
+            for (int j = 0; j < nj; ++j) {
+                const float lj = __ldcg(p.ws_lse + part_row(jb + j, hl));
+                *wslot(j, lane) = (lse_all == -INFINITY || lj == -INFINITY)
+                                      ? 0.f : fast_exp2((lj - lse_all) * 1.4426950408889634f);
+            }
+            __syncwarp();
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                float4 acc[8];
+                if (jb == 0) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else {   // more than 32 parts: continue from what the earlier parts stored
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        acc[i] = __ldcg(reinterpret_cast<const float4 *>(
+                            p.out + ((size_t)b * p.H + (head0 + 4 * i + (lane >> 3) < p.H ? head0 + 4 * i + (lane >> 3) : 0)) * 512 +
+                            col0 + 32 * cc + 4 * (lane & 7)));
+                }
+#pragma unroll 1
+                for (int j = 0; j < nj; j += 2) {
+                    const bool two = j + 1 < nj;
+                    float4 x0[8], x1[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int rr = 4 * i + (lane >> 3);
+                        const size_t off = (size_t)col0 + 32 * cc + 4 * (lane & 7);
+                        x0[i] = __ldcg(reinterpret_cast<const float4 *>(p.ws_o + part_row(jb + j, head0 + rr) * 512 + off));
+                        x1[i] = two ? __ldcg(reinterpret_cast<const float4 *>(p.ws_o + part_row(jb + j + 1, head0 + rr) * 512 + off))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int rr = 4 * i + (lane >> 3);
+                        const float w0 = *wslot(j, rr);
+                        const float w1 = two ? *wslot(j + 1, rr) : 0.f;
+                        acc[i].x = fmaf(w1, x1[i].x, fmaf(w0, x0[i].x, acc[i].x));
+                        acc[i].y = fmaf(w1, x1[i].y, fmaf(w0, x0[i].y, acc[i].y));
+                        acc[i].z = fmaf(w1, x1[i].z, fmaf(w0, x0[i].z, acc[i].z));
+                        acc[i].w = fmaf(w1, x1[i].w, fmaf(w0, x0[i].w, acc[i].w));
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int h_r = head0 + 4 * i + (lane >> 3);
+                    if (h_r < p.H)
+                        *reinterpret_cast<float4 *>(p.out + ((size_t)b * p.H + h_r) * 512 + col0 + 32 * cc +
+                                                    4 * (lane & 7)) = acc[i];
+                }
+            }
+            if (jb + 32 < n_parts) __threadfence_block();   // this warp reads its stores back
+        }
+        if (part == 0 && hl < p.H) p.lse[(size_t)b * p.H + hl] = lse_all;
+    };
+
+    // Empty sequences (no tile, no worker): out 0, lse -inf, spread over the workers.
+    for (int b = c.worker; b < p.B; b += p.workers) {
+        if (c.s_prefix[b + 1] != c.s_prefix[b]) continue;
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i) {
+            const int rr = (i >> 2) * 4 + (lane >> 3), cc = i & 3;
+            const int h_r = head0 + rr;
+            if (h_r < p.H)
+                *reinterpret_cast<float4 *>(p.out + ((size_t)b * p.H + h_r) * 512 + col0 + 32 * cc + 4 * (lane & 7)) =
+                    make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (part == 0 && realq) p.lse[(size_t)b * p.H + head] = -INFINITY;
+    }
+
     int k = 0, pi = 0;
     for (long long pos = c.p0; pos < c.p1; ++pi) {
         const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
@@ -634,7 +801,8 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             if (!wait_local(&bars->qempty, (uint32_t)pi & 1u, FLAG_MMA_WAIT, c)) return;
             store_q(v0, v1);
         }
-        // ---- the head's row sum (four parts), normalise, write block cg of the lane
+        // ---- the head's row sum (four parts), normalise, write this warp's block of O:
+        //      rows 32 (q & 1) + [0, 32) of this CTA's heads, columns col0 + [0, 128)
         const int klast = k + nt - 1;
         k += nt;
         lx_buf[part * HC + hh] = l;
@@ -646,33 +814,32 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
         if (!wait_local(&bars->odone[1][klast & 1], (uint32_t)(klast >> 1) & 1u, FLAG_MMA_WAIT, c)) return;
         tc_fence_after();
-        const bool real = realq;
-        float *dst = pc.whole ? p.out + ((size_t)pc.b * p.H + (real ? head : 0)) * 512
-                              : p.ws_o + (((size_t)c.worker * 2 + pc.slot) * HR + head) * 512;
-        dst += 256 * cg + 128 * half;   // block j = cg, the lane's 128 columns of it
-        const bool wide = !pc.whole || p.out_align32;   // the workspace is 256-byte aligned
-#pragma unroll
+        float *dst = pc.whole ? p.out + (size_t)pc.b * p.H * 512
+                              : p.ws_o + ((size_t)c.worker * 2 + pc.slot) * HR * 512;
+#pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
             uint32_t ov[32];
             tmem_ld32(c.tmem + lane_base + TM_O + 128 * cg + 32 * cc, ov);
             tmem_wait_ld();
-            if (real && wide) {   // 32-byte stores: whole sectors
+            // transpose through this warp's own bytes of the weights buffer (free: every
+            // value product of the piece is done), so that eight lanes store one row's
+            // 128 contiguous bytes
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float o8[8];
+            for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<float4 *>(scratch_unit(lane, u)) =
+                    make_float4(__uint_as_float(ov[4 * u]) * inv, __uint_as_float(ov[4 * u + 1]) * inv,
+                                __uint_as_float(ov[4 * u + 2]) * inv, __uint_as_float(ov[4 * u + 3]) * inv);
+            __syncwarp();
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) o8[i] = __uint_as_float(ov[8 * e + i]) * inv;
-                    st_global_v8(dst + 32 * cc + 8 * e, o8);
-                }
-            } else if (real) {
-                float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * cc);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    d4[e] = make_float4(__uint_as_float(ov[4 * e]) * inv, __uint_as_float(ov[4 * e + 1]) * inv,
-                                        __uint_as_float(ov[4 * e + 2]) * inv, __uint_as_float(ov[4 * e + 3]) * inv);
+            for (int i = 0; i < 8; ++i) {
+                const int rr = 4 * i + (lane >> 3), u = lane & 7;
+                const int h_r = head0 + rr;
+                const float4 x = *reinterpret_cast<const float4 *>(scratch_unit(rr, u));
+                if (h_r < p.H) *reinterpret_cast<float4 *>(dst + (size_t)h_r * 512 + col0 + 32 * cc + 4 * u) = x;
             }
+            __syncwarp();
         }
-        if (real && part == 0) {
+        if (realq && part == 0) {
             if (pc.whole)
                 p.lse[(size_t)pc.b * p.H + head] = lse_v;
             else
@@ -681,9 +848,25 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(ofree0);
+        // ---- a cut sequence: the last of its workers to finish this block merges the
+        //      block's partials (no waiting on the others)
+        if (!pc.whole) {
+            const long long ustart = c.s_prefix[pc.b];
+            const int n_parts = (int)((ustart + pc.n_tiles - 1) / c.W - ustart / c.W) + 1;
+            __threadfence();   // this warp's partial rows, before the arrival
+            __syncwarp();
+            bool last = false;
+            if (lane == 0)
+                last = merge_arrive_last(&g_mla_merge_count[((size_t)pc.b * 2 + c.r) * NSOFT + (warp - 4)], p.epoch,
+                                         n_parts);
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) {
+                __threadfence();   // the other workers' partials, after their arrivals
+                merge_block(pc.b, ustart, n_parts);
+            }
+        }
     }
 }
-
 }  // namespace mla
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::NTHREADS, 1)
@@ -747,13 +930,20 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
     c.r = cluster_ctarank();
     c.worker = blockIdx.x >> 1;
     const long long total = s_prefix[p.B];
-    const long long W = tiles_per_worker(total, p.workers, p.min_tiles);
-    if (blockIdx.x == 0) {
-        MetaView mv = meta_view(p.ws_meta);
-        if (tid == 0) { mv.w_total[0] = W; mv.w_total[1] = total; }
-        for (int i = tid; i <= p.B; i += NTHREADS) mv.prefix[i] = s_prefix[i];
+    // Tiles per worker.  When every sequence has the same number of tiles n, W may be
+    // rounded up so that worker boundaries fall on sequence or equal-part boundaries (each
+    // sequence in k equal parts, or whole sequences): a boundary inside a worker's range
+    // costs a partial result, its merge and a pipeline drain, more than the few tiles the
+    // coarser split adds.
+    long long W = tiles_per_worker(total, p.workers, p.min_tiles);
+    {
+        const int n0 = s_prefix[1] - s_prefix[0];
+        int same = 1;
+        for (int i = tid; i < p.B; i += NTHREADS) same &= (s_prefix[i + 1] - s_prefix[i]) == n0;
+        same = __syncthreads_and(same);
+        if (same && n0 > 0) W = uniform_tiles_per_worker(W, n0);
     }
-    pdl_launch_dependents();
+    c.W = W;
     c.p0 = (long long)c.worker * W;
     c.p1 = (c.p0 + W < total) ? c.p0 + W : total;
 
@@ -762,8 +952,8 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
         if (warp == 2 && lane == 0) value_producer(p, maps, c);
         if (warp == 1 && lane == 0 && c.r == 0) score_issuer(p, c);
         if (warp == 3 && lane == 0 && c.r == 0) value_issuer(p, c);
-        if (warp >= 4) softmax_warps(p, c, warp, lane);
     }
+    if (warp >= 4) softmax_warps(p, c, warp, lane);   // also the empty sequences
 
     tc_fence_before();
     __syncthreads();
