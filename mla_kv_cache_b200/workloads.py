@@ -197,6 +197,21 @@ def make_mla_inputs(cfg: MLAConfig, seed: int = 0, poison_tail: bool = False):
             "seq_lens": lens}
 
 
+def make_mla_inputs_fp8(cfg: MLAConfig, seed: int = 0, poison_tail: bool = False):
+    """The bf16 workload of make_mla_inputs (same draws), with the latent and RoPE caches
+    stored as E4M3 codes and one float scale per cache tensor.  Returns dict(q_latent,
+    q_rope, latent_cache, rope_cache, seq_lens, latent_scale, rope_scale); the caches are
+    float8_e4m3fn tensors."""
+    x = make_mla_inputs(cfg, seed, poison_tail=False)
+    lens = x["seq_lens"] if poison_tail else None
+    lat8, ls = quantize_e4m3(x["latent_cache"], lens, seq_axis=1)
+    del x["latent_cache"]
+    rope8, rs = quantize_e4m3(x["rope_cache"], lens, seq_axis=1)
+    del x["rope_cache"]
+    return {"q_latent": x["q_latent"], "q_rope": x["q_rope"], "latent_cache": lat8, "rope_cache": rope8,
+            "seq_lens": x["seq_lens"], "latent_scale": ls, "rope_scale": rs}
+
+
 def make_inputs(cfg, seed: int = 0, poison_tail: bool = False):
     if isinstance(cfg, MLAConfig):
         return make_mla_inputs(cfg, seed, poison_tail)

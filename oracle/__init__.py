@@ -288,6 +288,31 @@ def e4m3_quant(x, scale, lib=None):
     return out
 
 
+def mla_decode_fp8(q_latent, q_rope, latent_codes, rope_codes, seq_lens, scale, latent_scale, rope_scale,
+                   batch_ids=None, lib=None):
+    """Absorbed MLA over an E4M3 latent cache: attention on the dequantised latents
+    value(code) * latent_scale (keys' latent part and values alike) and RoPE keys
+    value(code) * rope_scale.  q_latent [B, H, d_c], q_rope [B, H, d_r] bf16; caches
+    [B, T_max, d_c] and [B, T_max, d_r] of codes; only the first seq_lens[b] rows of each
+    sequence are read.  Returns (out [B, H, d_c], lse [B, H])."""
+    lib = lib or load()
+    lens = _lens(seq_lens)
+    lc, rc = _codes(latent_codes), _codes(rope_codes)
+    T_max = lc.shape[1]
+    ids = range(q_latent.shape[0]) if batch_ids is None else batch_ids
+    outs, lses = [], []
+    for b in ids:
+        T = _rows(lens[b], T_max)
+        n = max(T, 1)
+        lat = e4m3_dequant(lc[b:b + 1, :n], latent_scale, lib=lib)
+        rope = e4m3_dequant(rc[b:b + 1, :n], rope_scale, lib=lib)
+        o, l = mla_decode_f64(q_latent[b:b + 1], q_rope[b:b + 1], lat, rope, np.array([T], dtype=np.int32),
+                              scale, lib=lib)
+        outs.append(o[0])
+        lses.append(l[0])
+    return np.stack(outs), np.stack(lses)
+
+
 def gqa_decode_fp8(q, k_codes, v_codes, seq_lens, scale, k_scale, v_scale, window=0, lib=None):
     """Decode over an E4M3 cache: attention on the dequantised keys value(k) * k_scale and
     values value(v) * v_scale.  q [B, n_q, d] (single token: returns out [B, n_q, d],

@@ -1,7 +1,7 @@
 """The oracle's per-sequence wrappers, pinned to its fp64 core (CPU only).
 
 The GPU parity tests call the wrappers (oracle.gqa_decode, oracle.mla_decode,
-oracle.gqa_decode_multi, oracle.gqa_decode_fp8): they take the bf16 (or E4M3) tensors,
+oracle.gqa_decode_multi, oracle.gqa_decode_fp8, oracle.mla_decode_fp8): they take the bf16 (or E4M3) tensors,
 convert only the rows a sequence attends to, and call the fp64 core one sequence at a
 time.  The core itself is pinned by tests/oracle_pins.py; here each wrapper must give
 exactly (bit for bit) what the core gives on the whole batch at once, on inputs whose
@@ -86,7 +86,31 @@ def check_fp8():
     assert np.isfinite(o).all()
 
 
-CHECKS = [check_mla, check_gqa, check_multi, check_fp8]
+def check_mla_fp8():
+    cfg = wl.MLAConfig("wrap_mla8", 4, 6, 32, 8, 19, 0.3, seq_lens=(19, 0, 1, 11))
+    x = wl.make_mla_inputs_fp8(cfg, seed=36, poison_tail=True)
+    lc = x["latent_cache"].view(torch.uint8)
+    rc = x["rope_cache"].view(torch.uint8)
+    lens = x["seq_lens"]
+    for b in range(cfg.batch):            # the tails carry the NaN code
+        assert torch.all((lc[b, int(lens[b]):] & 0x7F) == 0x7F)
+        assert torch.all((rc[b, int(lens[b]):] & 0x7F) == 0x7F)
+    lat = oracle.e4m3_dequant(lc, x["latent_scale"])
+    rope = oracle.e4m3_dequant(rc, x["rope_scale"])
+    lat[np.isnan(lat)] = 0
+    rope[np.isnan(rope)] = 0
+    o, l = oracle.mla_decode_fp8(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"], lens, cfg.scale,
+                                 x["latent_scale"], x["rope_scale"])
+    o2, l2 = oracle.mla_decode_f64(x["q_latent"], x["q_rope"], lat, rope, lens, cfg.scale)
+    assert np.array_equal(o, o2) and np.array_equal(l, l2), "mla fp8 wrapper differs from the core"
+    assert np.isfinite(o).all()
+    # the two scales are not interchangeable: swapping them changes the result
+    o3, _ = oracle.mla_decode_fp8(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"], lens, cfg.scale,
+                                  x["rope_scale"], x["latent_scale"])
+    assert not np.allclose(o3, o2)
+
+
+CHECKS = [check_mla, check_gqa, check_multi, check_fp8, check_mla_fp8]
 
 
 @pytest.mark.parametrize("check", CHECKS, ids=lambda c: c.__name__)
