@@ -177,6 +177,41 @@ int kvattn_gqa_decode_fp8_paged(const uint16_t *q, const uint8_t *k_pages, const
                                 float *out, float *lse, void *stream);
 
 /*
+ * kvattn_mla_decode over an E4M3 (fp8) latent cache, the MLA form of
+ * kvattn_gqa_decode_fp8 (same format; the pages list quantised caches among what the
+ * libraries add, "Attention variants: MQA, GQA, and MLA", section "Against the real
+ * libraries").  The cached latent of token t is value(latent_cache[b, t, :]) *
+ * latent_scale -- the key's latent part and the value alike -- and its RoPE key
+ * value(rope_cache[b, t, :]) * rope_scale; the result is kvattn_mla_decode on those
+ * dequantised rows.
+ *   q_latent, q_rope  device bf16 [batch, n_heads, 512], [batch, n_heads, 64]
+ *   latent_cache, rope_cache  device E4M3 codes [batch, max_seq_len, 512],
+ *                     [batch, max_seq_len, 64] (one byte each)
+ *   latent_scale, rope_scale  finite, > 0
+ *   out, lse    device fp32 [batch, n_heads, 512], [batch, n_heads]
+ * Everything else, the results' layout and the errors as for kvattn_mla_decode.  The
+ * query (each head's, after scaling by a power of two that puts its largest magnitude in
+ * [128, 256)) and the softmax weights enter the tensor-core products as an E4M3 high part
+ * plus an E4M3 remainder (~8 significant bits), the codes exactly; accumulation is fp32.
+ * Codes past a sequence's length are never read.
+ */
+int kvattn_mla_decode_fp8(const uint16_t *q_latent, const uint16_t *q_rope, const uint8_t *latent_cache,
+                          const uint8_t *rope_cache, const int32_t *seq_lens, int max_seq_len, int batch,
+                          int n_heads, int latent_dim, int rope_dim, float scale, float latent_scale,
+                          float rope_scale, float *out, float *lse, void *stream);
+
+/*
+ * kvattn_mla_decode_fp8 over a paged cache: latent_pages [num_pages, page_size, 512] and
+ * rope_pages [num_pages, page_size, 64] E4M3 codes, block_table and seq_lens as for
+ * kvattn_gqa_decode_paged, page_size a multiple of 64.
+ */
+int kvattn_mla_decode_fp8_paged(const uint16_t *q_latent, const uint16_t *q_rope, const uint8_t *latent_pages,
+                                const uint8_t *rope_pages, const int32_t *block_table, const int32_t *seq_lens,
+                                int num_pages, int page_size, int max_pages_per_seq, int batch, int n_heads,
+                                int latent_dim, int rope_dim, float scale, float latent_scale, float rope_scale,
+                                float *out, float *lse, void *stream);
+
+/*
  * kvattn_gqa_decode over a paged KV cache: the cache is a pool of pages and each
  * sequence lists its pages in a block table (the serving-engine layout the pages name,
  * "Attention variants: MQA, GQA, and MLA", section "Against the real libraries": vLLM's
@@ -269,6 +304,23 @@ int kvattn_mla_rope_append(uint16_t *q_rope, const uint16_t *latent_new, const u
                            const int32_t *positions, uint16_t *latent_cache, uint16_t *rope_cache,
                            int max_seq_len, int batch, int n_heads, int latent_dim, int rope_dim,
                            float rope_base, int interleaved, void *stream);
+
+/*
+ * kvattn_mla_rope_append into an E4M3 cache, the producer side of kvattn_mla_decode_fp8:
+ * q_rope is rotated in place (bf16); the rotated RoPE key is stored as E4M3 codes of
+ * key / rope_scale and the latent as codes of latent / latent_scale (the quotient taken
+ * in fp32, correctly rounded; nearest code, ties to even, saturated at 448, NaN to the
+ * NaN code), as kvattn_rope_append_fp8 encodes.
+ *   latent_cache, rope_cache  device E4M3 codes [batch, max_seq_len, latent_dim],
+ *                             [batch, max_seq_len, rope_dim]
+ *   latent_scale, rope_scale  finite, > 0
+ * Everything else as for kvattn_mla_rope_append.
+ */
+int kvattn_mla_rope_append_fp8(uint16_t *q_rope, const uint16_t *latent_new, const uint16_t *rope_new,
+                               const int32_t *positions, uint8_t *latent_cache, uint8_t *rope_cache,
+                               int max_seq_len, int batch, int n_heads, int latent_dim, int rope_dim,
+                               float rope_base, int interleaved, float latent_scale, float rope_scale,
+                               void *stream);
 
 /* Human-readable name of a kvattn_status value (static string, never NULL). */
 const char *kvattn_status_string(int status);

@@ -70,6 +70,19 @@ _SIGNATURES = {
                                               _c_u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                               ctypes.c_void_p]),
+    "kvattn_mla_decode_fp8": (ctypes.c_int, [_c_u16p, _c_u16p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_void_p,
+                                             ctypes.c_void_p, ctypes.c_void_p]),
+    "kvattn_mla_decode_fp8_paged": (ctypes.c_int, [_c_u16p, _c_u16p, ctypes.c_void_p, ctypes.c_void_p,
+                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "kvattn_mla_rope_append_fp8": (ctypes.c_int, [_c_u16p, _c_u16p, _c_u16p, ctypes.c_void_p, ctypes.c_void_p,
+                                                  ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+                                                  ctypes.c_float, ctypes.c_float, ctypes.c_void_p]),
     "kvattn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvattn_last_error_detail": (ctypes.c_char_p, []),
     "kvattn_version": (ctypes.c_int, []),
@@ -447,6 +460,86 @@ def kvattn_mla_decode_paged(q_latent, q_rope, latent_pages, rope_pages, block_ta
     if st != KVATTN_OK:
         raise KvattnError(st, "kvattn_mla_decode_paged")
     return out, lse
+
+
+def kvattn_mla_decode_fp8(q_latent, q_rope, latent_cache, rope_cache, seq_lens, scale, latent_scale, rope_scale,
+                          out=None, lse=None, stream=None):
+    """Absorbed-MLA decode over an E4M3 cache (include/kvattn.h, kvattn_mla_decode_fp8):
+    latent_cache [B, T, 512], rope_cache [B, T, 64] float8_e4m3fn (or uint8 codes), value =
+    code * latent_scale / rope_scale.  Returns (out [B, H, 512], lse [B, H]) fp32."""
+    import torch
+    B, H, dc = q_latent.shape
+    dr = q_rope.shape[2]
+    T = latent_cache.shape[1]
+    _check(q_latent, "q_latent", torch.bfloat16)
+    _check(q_rope, "q_rope", torch.bfloat16, (B, H, dr))
+    _check_e4m3(latent_cache, "latent_cache", (B, T, dc))
+    _check_e4m3(rope_cache, "rope_cache", (B, T, dr))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, H, dc), dtype=torch.float32, device=q_latent.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q_latent.device)
+    _check(out, "out", torch.float32, (B, H, dc))
+    _check(lse, "lse", torch.float32, (B, H))
+    st = lib().kvattn_mla_decode_fp8(q_latent.data_ptr(), q_rope.data_ptr(), latent_cache.data_ptr(),
+                                     rope_cache.data_ptr(), seq_lens.data_ptr(), T, B, H, dc, dr, float(scale),
+                                     float(latent_scale), float(rope_scale), out.data_ptr(), lse.data_ptr(),
+                                     _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_mla_decode_fp8")
+    return out, lse
+
+
+def kvattn_mla_decode_fp8_paged(q_latent, q_rope, latent_pages, rope_pages, block_table, seq_lens, scale,
+                                latent_scale, rope_scale, out=None, lse=None, stream=None):
+    """kvattn_mla_decode_fp8 over a paged cache (include/kvattn.h): latent_pages [P, page_size,
+    512], rope_pages [P, page_size, 64] E4M3 codes, block_table [B, max_pages] int32."""
+    import torch
+    B, H, dc = q_latent.shape
+    dr = q_rope.shape[2]
+    P, S = latent_pages.shape[0], latent_pages.shape[1]
+    M = block_table.shape[1]
+    _check(q_latent, "q_latent", torch.bfloat16)
+    _check(q_rope, "q_rope", torch.bfloat16, (B, H, dr))
+    _check_e4m3(latent_pages, "latent_pages", (P, S, dc))
+    _check_e4m3(rope_pages, "rope_pages", (P, S, dr))
+    _check(block_table, "block_table", torch.int32, (B, M))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, H, dc), dtype=torch.float32, device=q_latent.device)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q_latent.device)
+    _check(out, "out", torch.float32, (B, H, dc))
+    _check(lse, "lse", torch.float32, (B, H))
+    st = lib().kvattn_mla_decode_fp8_paged(q_latent.data_ptr(), q_rope.data_ptr(), latent_pages.data_ptr(),
+                                           rope_pages.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(), P,
+                                           S, M, B, H, dc, dr, float(scale), float(latent_scale),
+                                           float(rope_scale), out.data_ptr(), lse.data_ptr(), _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_mla_decode_fp8_paged")
+    return out, lse
+
+
+def kvattn_mla_rope_append_fp8(q_rope, latent_new, rope_new, positions, latent_cache, rope_cache, latent_scale,
+                               rope_scale, rope_base=10000.0, interleaved=False, stream=None):
+    """kvattn_mla_rope_append into an E4M3 cache (include/kvattn.h): latent_cache [B, T, c],
+    rope_cache [B, T, r] float8_e4m3fn (or uint8 codes)."""
+    import torch
+    B, H, r = q_rope.shape
+    T, c = latent_cache.shape[1], latent_cache.shape[2]
+    _check(q_rope, "q_rope", torch.bfloat16)
+    _check(latent_new, "latent_new", torch.bfloat16, (B, c))
+    _check(rope_new, "rope_new", torch.bfloat16, (B, r))
+    _check(positions, "positions", torch.int32, (B,))
+    _check_e4m3(latent_cache, "latent_cache", (B, T, c))
+    _check_e4m3(rope_cache, "rope_cache", (B, T, r))
+    st = lib().kvattn_mla_rope_append_fp8(q_rope.data_ptr(), latent_new.data_ptr(), rope_new.data_ptr(),
+                                          positions.data_ptr(), latent_cache.data_ptr(), rope_cache.data_ptr(),
+                                          T, B, H, c, r, float(rope_base), int(bool(interleaved)),
+                                          float(latent_scale), float(rope_scale), _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_mla_rope_append_fp8")
 
 
 def kvattn_gqa_decode_multi(q, k_cache, v_cache, seq_lens, scale, window=0, out=None, lse=None, stream=None):

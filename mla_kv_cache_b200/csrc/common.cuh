@@ -180,6 +180,35 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+// Two bf16 values (one 32-bit word) as float.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// E4M3 high part and remainder of two values (already scaled into E4M3's range): the
+// pair goes through f16 (exact for the 8-bit bf16 significands scaled by a power of
+// two), the high part is the nearest E4M3 pair, the remainder the nearest E4M3 pair
+// to what is left (exact in f16).  Element order is kept (x in the low byte).
+__device__ __forceinline__ void split_e4m3x2(float x, float y, uint16_t &hi, uint16_t &lo) {
+    const __half2 h = __floats2half2_rn(x, y);
+    const __half2_raw hr = h;
+    hi = __nv_cvt_halfraw2_to_fp8x2(hr, __NV_SATFINITE, __NV_E4M3);
+    const __half2 back = __half2(__nv_cvt_fp8x2_to_halfraw2(hi, __NV_E4M3));
+    const __half2_raw rr = __hsub2(h, back);
+    lo = __nv_cvt_halfraw2_to_fp8x2(rr, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Three E4M3 parts of two fp32 values (already scaled into E4M3's range), each the
+// nearest E4M3 pair to what the parts before it leave (the differences are exact in fp32):
+// about 12 significant bits.  Element order is kept (x in the low byte).
+__device__ __forceinline__ void split3_e4m3x2(float x, float y, uint16_t &hi, uint16_t &mid, uint16_t &lo) {
+    hi = __nv_cvt_float2_to_fp8x2(make_float2(x, y), __NV_SATFINITE, __NV_E4M3);
+    const float2 h = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(hi, __NV_E4M3)));
+    const float rx = x - h.x, ry = y - h.y;
+    mid = __nv_cvt_float2_to_fp8x2(make_float2(rx, ry), __NV_SATFINITE, __NV_E4M3);
+    const float2 m = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(mid, __NV_E4M3)));
+    lo = __nv_cvt_float2_to_fp8x2(make_float2(rx - m.x, ry - m.y), __NV_SATFINITE, __NV_E4M3);
+}
+
 // 2^x with the hardware approximation (flushes subnormal results to zero).
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;

@@ -288,23 +288,6 @@ __device__ __forceinline__ void producer(const GqaParams &p, const CUtensorMap *
 }
 
 // ------------------------------------------------------------------ E4M3 query split (warp 1)
-// Two bf16 values (one 32-bit word) as float.
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// E4M3 high part and remainder of two values (already scaled into E4M3's range): the
-// pair goes through f16 (exact for the 8-bit bf16 significands scaled by a power of
-// two), the high part is the nearest E4M3 pair, the remainder the nearest E4M3 pair
-// to what is left (exact in f16).  Element order is kept (x in the low byte).
-__device__ __forceinline__ void split_e4m3x2(float x, float y, uint16_t &hi, uint16_t &lo) {
-    const __half2 h = __floats2half2_rn(x, y);
-    const __half2_raw hr = h;
-    hi = __nv_cvt_halfraw2_to_fp8x2(hr, __NV_SATFINITE, __NV_E4M3);
-    const __half2 back = __half2(__nv_cvt_fp8x2_to_halfraw2(hi, __NV_E4M3));
-    const __half2_raw rr = __hsub2(h, back);
-    lo = __nv_cvt_halfraw2_to_fp8x2(rr, __NV_SATFINITE, __NV_E4M3);
-}
-
 // Splits the bf16 query block at qbase (two 128-byte-swizzled [NQ x 64] boxes) in place
 // into two E4M3 blocks of [NQ x 128] in the same swizzle: the high parts where the first
 // box was, the remainders where the second was.  Every value is first multiplied by

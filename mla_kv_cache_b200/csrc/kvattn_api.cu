@@ -577,12 +577,14 @@ int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq
 // A latent + rotary-key cache as the MLA kernel sees it (pages of page_size rows; a
 // contiguous cache is one page per sequence).
 struct MlaCache {
-    const uint16_t *lat, *rope;
+    const void *lat, *rope;       // bf16, or E4M3 codes (e4m3)
     const int32_t *block_table;   // [batch, max_pages] or null (contiguous)
     int capacity;
     int page_size;
     int max_pages;
     long long pages;
+    bool e4m3;
+    float latent_scale, rope_scale;   // E4M3: a code's value times these
 };
 
 int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaCache &cache,
@@ -593,16 +595,31 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
     if (st != KVATTN_OK) return st;
 
     MlaMaps maps;
-    st = make_map_3d(&maps.lat, cache.lat, 512, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != KVATTN_OK) return st;
-    st = make_map_3d(&maps.rope, cache.rope, 64, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != KVATTN_OK) return st;
-    st = make_map_3d(&maps.qlat, q_latent, 512, n_heads, batch, 64, mla::HC, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != KVATTN_OK) return st;
-    st = make_map_3d(&maps.qrope, q_rope, 64, n_heads, batch, 64, mla::HC, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (st != KVATTN_OK) return st;
+    if (cache.e4m3) {
+        // E4M3 codes, two to an element of the map: a box of [64 rows x 128 codes]; the
+        // RoPE map is 64 codes wide, so its box reads 64 codes and zero-fills the other 64
+        st = make_map_3d(&maps.lat, cache.lat, 256, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != KVATTN_OK) return st;
+        st = make_map_3d(&maps.rope, cache.rope, 32, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != KVATTN_OK) return st;
+        maps.qlat = maps.lat;   // (the query is read by the threads)
+        maps.qrope = maps.lat;
+    } else {
+        st = make_map_3d(&maps.lat, cache.lat, 512, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != KVATTN_OK) return st;
+        st = make_map_3d(&maps.rope, cache.rope, 64, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != KVATTN_OK) return st;
+        st = make_map_3d(&maps.qlat, q_latent, 512, n_heads, batch, 64, mla::HC, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != KVATTN_OK) return st;
+        st = make_map_3d(&maps.qrope, q_rope, 64, n_heads, batch, 64, mla::HC, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != KVATTN_OK) return st;
+    }
+    const void *kern = cache.e4m3 ? reinterpret_cast<const void *>(mla_decode_kernel<true>)
+                                  : reinterpret_cast<const void *>(mla_decode_kernel<false>);
 
     MlaParams p = {};
     p.q_latent = reinterpret_cast<const __nv_bfloat16 *>(q_latent);
@@ -620,13 +637,15 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
     unsigned int epoch = ++dev->mla_calls;
     if (epoch == 0) epoch = ++dev->mla_calls;   // 0 is the counters' state at load
     p.epoch = epoch;
+    p.latent_scale = cache.e4m3 ? cache.latent_scale : 1.f;
+    p.rope_scale = cache.e4m3 ? cache.rope_scale : 1.f;
     const int smem = mla::smem_bytes(batch);
     if (smem > dev->max_smem_optin) {
         snprintf(t_detail, sizeof(t_detail), "needs %d B shared memory", smem);
         return KVATTN_ERR_UNSUPPORTED;
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(mla_decode_kernel), dev, smem);
+    cudaError_t e = set_smem_limit(kern, dev, smem);
     if (e != cudaSuccess) return fail_cuda(e, "cudaFuncSetAttribute(mla)");
     // Workers are CTA pairs; a persistent grid must not exceed the pairs that can be
     // resident at once (a pair needs two SMs of one GPC).
@@ -643,7 +662,7 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        e = cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void *>(mla_decode_kernel), &cfg);
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
         if (e != cudaSuccess || n <= 0) {
             cudaGetLastError();
             n = dev->sms / 2;
@@ -671,7 +690,10 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
     p.ws_lse = reinterpret_cast<float *>(ws);
     p.ws_o = reinterpret_cast<float *>(static_cast<char *>(ws) + wlse_bytes);
 
-    mla_decode_kernel<<<2 * p.workers, mla::NTHREADS, smem, s>>>(p, maps);
+    if (cache.e4m3)
+        mla_decode_kernel<true><<<2 * p.workers, mla::NTHREADS, smem, s>>>(p, maps);
+    else
+        mla_decode_kernel<false><<<2 * p.workers, mla::NTHREADS, smem, s>>>(p, maps);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e, "mla decode launch");
     return KVATTN_OK;
@@ -863,73 +885,85 @@ int kvattn_gqa_decode_fp8_paged(const uint16_t *q, const uint8_t *k_pages, const
     return gqa_decode_impl(q, cache, seq_lens, batch, n_q_heads, n_kv_heads, head_dim, scale, out, lse, stream);
 }
 
+// Checks and launch shared by the four MLA entry points: a contiguous cache is one page
+// per sequence (block_table null, num_pages = batch, page_size = max_pages_per_seq =
+// max_seq_len).  code_bytes = 2 (bf16) or 1 (E4M3).
+static int mla_entry(const uint16_t *q_latent, const uint16_t *q_rope, const void *lat, const void *rope,
+              const int32_t *block_table, const int32_t *seq_lens, int num_pages, int page_size,
+              int max_pages_per_seq, int batch, int n_heads, int latent_dim, int rope_dim, float scale, bool e4m3,
+              float latent_scale, float rope_scale, float *out, float *lse, void *stream) {
+    const bool paged = block_table != nullptr;
+    if (!q_latent || !q_rope || !lat || !rope || !seq_lens || !out || !lse) return KVATTN_ERR_INVALID_ARG;
+    if (batch <= 0 || n_heads <= 0 || num_pages <= 0 || page_size <= 0 || max_pages_per_seq <= 0 ||
+        latent_dim <= 0 || rope_dim < 0)
+        return KVATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
+    if (e4m3 && (!std::isfinite(latent_scale) || !std::isfinite(rope_scale) || !(latent_scale > 0.f) ||
+                 !(rope_scale > 0.f)))
+        return KVATTN_ERR_INVALID_ARG;
+    if (latent_dim != 512 || rope_dim != 64 || n_heads > 128) return KVATTN_ERR_UNSUPPORTED;
+    if (paged && page_size % mla::SUB != 0) return KVATTN_ERR_UNSUPPORTED;
+    if (batch > mla::MAX_BATCH) return KVATTN_ERR_UNSUPPORTED;
+    if ((long long)num_pages * page_size >= (1ll << 31) || (long long)max_pages_per_seq * page_size >= (1ll << 31))
+        return KVATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q_latent) || !aligned16(q_rope) || !aligned16(lat) || !aligned16(rope) ||
+        (paged && !aligned16(block_table)) || !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
+        return KVATTN_ERR_MISALIGNED;
+    const size_t cb = e4m3 ? 1 : 2;
+    const size_t ql_bytes = (size_t)batch * n_heads * latent_dim * 2;
+    const size_t qr_bytes = (size_t)batch * n_heads * rope_dim * 2;
+    const size_t lat_bytes = (size_t)num_pages * page_size * latent_dim * cb;
+    const size_t rope_bytes = (size_t)num_pages * page_size * rope_dim * cb;
+    const size_t out_bytes = (size_t)batch * n_heads * latent_dim * 4;
+    const size_t lse_bytes = (size_t)batch * n_heads * 4;
+    const void *ins[6] = {q_latent, q_rope, lat, rope, seq_lens, block_table};
+    const size_t in_sz[6] = {ql_bytes, qr_bytes, lat_bytes, rope_bytes, (size_t)batch * 4,
+                             paged ? (size_t)batch * max_pages_per_seq * 4 : 0};
+    for (int i = 0; i < 6; ++i)
+        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
+            return KVATTN_ERR_INVALID_ARG;
+    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
+    const MlaCache cache{lat, rope, block_table, max_pages_per_seq * page_size, page_size, max_pages_per_seq,
+                         num_pages, e4m3, latent_scale, rope_scale};
+    return mla_decode_impl(q_latent, q_rope, cache, seq_lens, batch, n_heads, scale, out, lse, stream);
+}
+
 int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
                       const uint16_t *latent_cache, const uint16_t *rope_cache,
                       const int32_t *seq_lens, int max_seq_len, int batch, int n_heads,
                       int latent_dim, int rope_dim, float scale, float *out, float *lse,
                       void *stream) {
-    if (!q_latent || !q_rope || !latent_cache || !rope_cache || !seq_lens || !out || !lse)
-        return KVATTN_ERR_INVALID_ARG;
-    if (batch <= 0 || n_heads <= 0 || max_seq_len <= 0 || latent_dim <= 0 || rope_dim < 0)
-        return KVATTN_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
-    if (latent_dim != 512 || rope_dim != 64 || n_heads > 128) return KVATTN_ERR_UNSUPPORTED;
-    if (batch > mla::MAX_BATCH) return KVATTN_ERR_UNSUPPORTED;
-    if ((long long)batch * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
-    if (!aligned16(q_latent) || !aligned16(q_rope) || !aligned16(latent_cache) ||
-        !aligned16(rope_cache) || !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
-        return KVATTN_ERR_MISALIGNED;
-    const size_t ql_bytes = (size_t)batch * n_heads * latent_dim * 2;
-    const size_t qr_bytes = (size_t)batch * n_heads * rope_dim * 2;
-    const size_t lat_bytes = (size_t)batch * max_seq_len * latent_dim * 2;
-    const size_t rope_bytes = (size_t)batch * max_seq_len * rope_dim * 2;
-    const size_t out_bytes = (size_t)batch * n_heads * latent_dim * 4;
-    const size_t lse_bytes = (size_t)batch * n_heads * 4;
-    const void *ins[5] = {q_latent, q_rope, latent_cache, rope_cache, seq_lens};
-    const size_t in_sz[5] = {ql_bytes, qr_bytes, lat_bytes, rope_bytes, (size_t)batch * 4};
-    for (int i = 0; i < 5; ++i)
-        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
-            return KVATTN_ERR_INVALID_ARG;
-    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
-
-    const MlaCache cache{latent_cache, rope_cache, nullptr, max_seq_len, max_seq_len, 1, batch};
-    return mla_decode_impl(q_latent, q_rope, cache, seq_lens, batch, n_heads, scale, out, lse, stream);
+    return mla_entry(q_latent, q_rope, latent_cache, rope_cache, nullptr, seq_lens, batch, max_seq_len, max_seq_len,
+                     batch, n_heads, latent_dim, rope_dim, scale, false, 1.f, 1.f, out, lse, stream);
 }
 
 int kvattn_mla_decode_paged(const uint16_t *q_latent, const uint16_t *q_rope, const uint16_t *latent_pages,
                             const uint16_t *rope_pages, const int32_t *block_table, const int32_t *seq_lens,
                             int num_pages, int page_size, int max_pages_per_seq, int batch, int n_heads,
                             int latent_dim, int rope_dim, float scale, float *out, float *lse, void *stream) {
-    if (!q_latent || !q_rope || !latent_pages || !rope_pages || !block_table || !seq_lens || !out || !lse)
-        return KVATTN_ERR_INVALID_ARG;
-    if (batch <= 0 || n_heads <= 0 || num_pages <= 0 || page_size <= 0 || max_pages_per_seq <= 0 ||
-        latent_dim <= 0 || rope_dim < 0)
-        return KVATTN_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
-    if (latent_dim != 512 || rope_dim != 64 || n_heads > 128) return KVATTN_ERR_UNSUPPORTED;
-    if (page_size % mla::SUB != 0) return KVATTN_ERR_UNSUPPORTED;
-    if (batch > mla::MAX_BATCH) return KVATTN_ERR_UNSUPPORTED;
-    if ((long long)num_pages * page_size >= (1ll << 31) || (long long)max_pages_per_seq * page_size >= (1ll << 31))
-        return KVATTN_ERR_UNSUPPORTED;
-    if (!aligned16(q_latent) || !aligned16(q_rope) || !aligned16(latent_pages) || !aligned16(rope_pages) ||
-        !aligned16(block_table) || !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
-        return KVATTN_ERR_MISALIGNED;
-    const size_t ql_bytes = (size_t)batch * n_heads * latent_dim * 2;
-    const size_t qr_bytes = (size_t)batch * n_heads * rope_dim * 2;
-    const size_t lat_bytes = (size_t)num_pages * page_size * latent_dim * 2;
-    const size_t rope_bytes = (size_t)num_pages * page_size * rope_dim * 2;
-    const size_t out_bytes = (size_t)batch * n_heads * latent_dim * 4;
-    const size_t lse_bytes = (size_t)batch * n_heads * 4;
-    const void *ins[6] = {q_latent, q_rope, latent_pages, rope_pages, seq_lens, block_table};
-    const size_t in_sz[6] = {ql_bytes, qr_bytes, lat_bytes, rope_bytes, (size_t)batch * 4,
-                             (size_t)batch * max_pages_per_seq * 4};
-    for (int i = 0; i < 6; ++i)
-        if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
-            return KVATTN_ERR_INVALID_ARG;
-    if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
-    const MlaCache cache{latent_pages, rope_pages, block_table, max_pages_per_seq * page_size, page_size,
-                         max_pages_per_seq, num_pages};
-    return mla_decode_impl(q_latent, q_rope, cache, seq_lens, batch, n_heads, scale, out, lse, stream);
+    if (!block_table) return KVATTN_ERR_INVALID_ARG;
+    return mla_entry(q_latent, q_rope, latent_pages, rope_pages, block_table, seq_lens, num_pages, page_size,
+                     max_pages_per_seq, batch, n_heads, latent_dim, rope_dim, scale, false, 1.f, 1.f, out, lse,
+                     stream);
+}
+
+int kvattn_mla_decode_fp8(const uint16_t *q_latent, const uint16_t *q_rope, const uint8_t *latent_cache,
+                          const uint8_t *rope_cache, const int32_t *seq_lens, int max_seq_len, int batch,
+                          int n_heads, int latent_dim, int rope_dim, float scale, float latent_scale,
+                          float rope_scale, float *out, float *lse, void *stream) {
+    return mla_entry(q_latent, q_rope, latent_cache, rope_cache, nullptr, seq_lens, batch, max_seq_len, max_seq_len,
+                     batch, n_heads, latent_dim, rope_dim, scale, true, latent_scale, rope_scale, out, lse, stream);
+}
+
+int kvattn_mla_decode_fp8_paged(const uint16_t *q_latent, const uint16_t *q_rope, const uint8_t *latent_pages,
+                                const uint8_t *rope_pages, const int32_t *block_table, const int32_t *seq_lens,
+                                int num_pages, int page_size, int max_pages_per_seq, int batch, int n_heads,
+                                int latent_dim, int rope_dim, float scale, float latent_scale, float rope_scale,
+                                float *out, float *lse, void *stream) {
+    if (!block_table) return KVATTN_ERR_INVALID_ARG;
+    return mla_entry(q_latent, q_rope, latent_pages, rope_pages, block_table, seq_lens, num_pages, page_size,
+                     max_pages_per_seq, batch, n_heads, latent_dim, rope_dim, scale, true, latent_scale, rope_scale,
+                     out, lse, stream);
 }
 
 const char *kvattn_status_string(int status) {
@@ -1090,22 +1124,26 @@ int kvattn_rope_append_fp8(uint16_t *q, const uint16_t *k_new, const uint16_t *v
     return launch_rope_append(p, static_cast<cudaStream_t>(stream), true);
 }
 
-int kvattn_mla_rope_append(uint16_t *q_rope, const uint16_t *latent_new, const uint16_t *rope_new,
-                           const int32_t *positions, uint16_t *latent_cache, uint16_t *rope_cache,
-                           int max_seq_len, int batch, int n_heads, int latent_dim, int rope_dim,
-                           float rope_base, int interleaved, void *stream) {
+static int mla_append(uint16_t *q_rope, const uint16_t *latent_new, const uint16_t *rope_new,
+                      const int32_t *positions, void *latent_cache, void *rope_cache, int max_seq_len, int batch,
+                      int n_heads, int latent_dim, int rope_dim, float rope_base, int interleaved, bool e4m3,
+                      float latent_scale, float rope_scale, void *stream) {
     if (!q_rope || !latent_new || !rope_new || !positions || !latent_cache || !rope_cache)
         return KVATTN_ERR_INVALID_ARG;
     if (batch <= 0 || n_heads <= 0 || max_seq_len <= 0 || latent_dim <= 0 || rope_dim <= 0)
         return KVATTN_ERR_INVALID_ARG;
     if ((rope_dim & 1) || (latent_dim & 1) || rope_dim > 1024 || latent_dim > 4096) return KVATTN_ERR_UNSUPPORTED;
     if (!std::isfinite(rope_base) || rope_base <= 0.f) return KVATTN_ERR_INVALID_ARG;
+    if (e4m3 && (!std::isfinite(latent_scale) || !std::isfinite(rope_scale) || !(latent_scale > 0.f) ||
+                 !(rope_scale > 0.f)))
+        return KVATTN_ERR_INVALID_ARG;
+    const size_t cb = e4m3 ? 1 : 2;
     if (!aligned16(q_rope) || !aligned16(latent_new) || !aligned16(rope_new) || !aligned16(positions) ||
         !aligned16(latent_cache) || !aligned16(rope_cache))
         return KVATTN_ERR_MISALIGNED;
     const void *w[3] = {q_rope, latent_cache, rope_cache};
-    const size_t wn[3] = {(size_t)batch * n_heads * rope_dim * 2, (size_t)batch * max_seq_len * latent_dim * 2,
-                          (size_t)batch * max_seq_len * rope_dim * 2};
+    const size_t wn[3] = {(size_t)batch * n_heads * rope_dim * 2, (size_t)batch * max_seq_len * latent_dim * cb,
+                          (size_t)batch * max_seq_len * rope_dim * cb};
     const void *r[3] = {latent_new, rope_new, positions};
     const size_t rn[3] = {(size_t)batch * latent_dim * 2, (size_t)batch * rope_dim * 2, (size_t)batch * 4};
     for (int i = 0; i < 3; ++i) {
@@ -1119,8 +1157,10 @@ int kvattn_mla_rope_append(uint16_t *q_rope, const uint16_t *latent_new, const u
     p.k_new = reinterpret_cast<const __nv_bfloat16 *>(rope_new);
     p.v_new = reinterpret_cast<const __nv_bfloat16 *>(latent_new);
     p.positions = positions;
-    p.k_cache = reinterpret_cast<__nv_bfloat16 *>(rope_cache);
-    p.v_cache = reinterpret_cast<__nv_bfloat16 *>(latent_cache);
+    p.k_cache = rope_cache;
+    p.v_cache = latent_cache;
+    p.k_scale = e4m3 ? rope_scale : 1.f;
+    p.v_scale = e4m3 ? latent_scale : 1.f;
     p.B = batch;
     p.n_q = n_heads;
     p.n_kv = 1;                    // one shared latent / rotary key per token
@@ -1132,7 +1172,24 @@ int kvattn_mla_rope_append(uint16_t *q_rope, const uint16_t *latent_new, const u
     p.n_q_pairs = (long long)batch * n_heads * (rope_dim / 2);
     p.n_k_pairs = (long long)batch * (rope_dim / 2);
     p.n_v_words = (long long)batch * (latent_dim / 2);
-    return launch_rope_append(p, static_cast<cudaStream_t>(stream));
+    return launch_rope_append(p, static_cast<cudaStream_t>(stream), e4m3);
+}
+
+int kvattn_mla_rope_append(uint16_t *q_rope, const uint16_t *latent_new, const uint16_t *rope_new,
+                           const int32_t *positions, uint16_t *latent_cache, uint16_t *rope_cache,
+                           int max_seq_len, int batch, int n_heads, int latent_dim, int rope_dim,
+                           float rope_base, int interleaved, void *stream) {
+    return mla_append(q_rope, latent_new, rope_new, positions, latent_cache, rope_cache, max_seq_len, batch, n_heads,
+                      latent_dim, rope_dim, rope_base, interleaved, false, 1.f, 1.f, stream);
+}
+
+int kvattn_mla_rope_append_fp8(uint16_t *q_rope, const uint16_t *latent_new, const uint16_t *rope_new,
+                               const int32_t *positions, uint8_t *latent_cache, uint8_t *rope_cache,
+                               int max_seq_len, int batch, int n_heads, int latent_dim, int rope_dim,
+                               float rope_base, int interleaved, float latent_scale, float rope_scale,
+                               void *stream) {
+    return mla_append(q_rope, latent_new, rope_new, positions, latent_cache, rope_cache, max_seq_len, batch, n_heads,
+                      latent_dim, rope_dim, rope_base, interleaved, true, latent_scale, rope_scale, stream);
 }
 
 void kvattn_debug_set_workers(int workers, int min_tiles) {

@@ -102,14 +102,41 @@ constexpr int OFF_Q = 0;                               // query chunks [5][64 he
 constexpr int OFF_P = OFF_Q + NQS * CHUNK;             // weights of a tile: high h0, h1, remainder h0, h1
 constexpr int OFF_SR = OFF_P + 4 * CHUNK;              // key ring
 constexpr int OFF_PV = OFF_SR + NKS * KSLOT;           // value ring
-constexpr int OFF_MX = OFF_PV + NVS * VSLOT;           // [2 tiles][4 parts][64] partial tile maxima
+constexpr int OFF_END = OFF_PV + NVS * VSLOT;          // 208 KB
+constexpr int OFF_MX = OFF_END + 8192;                 // (after the E4M3 layout's 216 KB too)
+                                                       // [2 tiles][4 parts][64] partial tile maxima
 constexpr int OFF_LX = OFF_MX + 2 * 4 * HC * 4;        // [4 parts][64] partial row sums
-constexpr int OFF_BARS = OFF_LX + 4 * HC * 4;
+constexpr int OFF_QX = OFF_LX + 4 * HC * 4;            // [2][4 parts][64] partial query maxima (E4M3)
+constexpr int OFF_BARS = OFF_QX + 2 * 4 * HC * 4;
 constexpr int OFF_TMEMPTR = OFF_BARS + 512;
 constexpr int OFF_ABORT = OFF_TMEMPTR + 16;
 constexpr int OFF_PREFIX = OFF_ABORT + 16;
 constexpr int smem_bytes(int B) { return 1024 + OFF_PREFIX + (B + 1) * 4; }
 static_assert(smem_bytes(MAX_BATCH) <= 232448, "shared memory of the MLA kernel exceeds 227 KB");
+
+// The E4M3 cache (one byte per code; a box is [64 rows x 128 codes], 128-byte swizzle, 8 KB).
+// Shared memory: the query's high parts (5 boxes: latent codes 0-511, then the RoPE part in
+// the first 64 codes of a fifth box) and its remainders, the weights' three parts ([64
+// heads x 128 tokens] each), a key ring of two tiles (5 boxes per tile; the RoPE box is
+// read from a 64-code-wide tensor, its other 64 codes are the TMA's zero fill and are
+// never multiplied), and one value slot per token half (this CTA's 256 latent codes of
+// the half's 64 tokens: 2 boxes).  216 KB.
+namespace e4 {
+constexpr int QPART = 5 * CHUNK;               // 40 KB: one part of the query
+constexpr int OFF_Q = 0;
+constexpr int OFF_P = OFF_Q + 2 * QPART;       // high part, middle part, low part
+constexpr int NPP = 3;                         // parts of a weight
+constexpr int PPART = CHUNK;                   // 8 KB
+constexpr int OFF_SR = OFF_P + NPP * PPART;
+constexpr int NKS = 2;                         // key ring: two tiles
+constexpr int KSLOT = 5 * CHUNK;               // 40 KB
+constexpr int OFF_PV = OFF_SR + NKS * KSLOT;
+constexpr int VSLOT = 2 * CHUNK;               // 16 KB
+static_assert(OFF_PV + NVS * VSLOT == OFF_MX, "E4M3 layout");
+constexpr uint32_t TM_SR = 384;                // [384, 512): the RoPE part of the scores of two tiles
+constexpr float RESCALE_LOG2 = 2.f;            // the weights stay below 2^(6 + 2) = 256 < 448
+constexpr float P_LOG2 = 6.f;                  // the weights carry 2^6
+}  // namespace e4
 
 struct Bars {
     // Every ring slot serves each tile once, so its phase is the tile count.  The release
@@ -132,6 +159,7 @@ struct Bars {
     uint64_t ofree;                     // both CTAs' epilogues have read O (rank 0)
     uint64_t mxbar[2];                  // the softmax warps' tile maxima written (tile parity)
     uint64_t lxbar;                     // the softmax warps' row sums written (end of a piece)
+    uint64_t qxbar;                     // the softmax warps' query maxima written (E4M3 cache)
 };
 static_assert(sizeof(Bars) <= 512, "barrier block overflows its slot");
 
@@ -153,6 +181,8 @@ struct MlaParams {
     int max_pages;              // block-table columns
     int page_size;              // rows per page (T_max when contiguous)
     unsigned int epoch;         // number of this call (never 0), tags the merge counters
+    float latent_scale;         // E4M3 cache: a latent code's value is code * latent_scale
+    float rope_scale;           // E4M3 cache: a RoPE code's value is code * rope_scale
 };
 
 struct MlaMaps {
@@ -242,6 +272,7 @@ __device__ __forceinline__ HalfSrc half_source(const MlaParams &p, int b, int le
 // key chunks of every tile of the piece; the value producer (warp 2) the value chunks of
 // every tile.  Completions go to rank 0's barriers, which rank 0 arms with the bytes of
 // both CTAs.
+template <bool KV8>
 __device__ __forceinline__ void key_producer(const MlaParams &p, const MlaMaps &m, const Ctx &c) {
     Bars *bars = c.bars;
     const uint64_t pol_keep = l2_policy_evict_normal();   // the latent columns are read again as values
@@ -253,6 +284,27 @@ __device__ __forceinline__ void key_producer(const MlaParams &p, const MlaMaps &
         const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
         pos = pc.ustart + pc.lt1;
         const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
+        if constexpr (KV8) {
+            // one slot per tile, two slots: tile nld's slot last held tile nld - 2, whose
+            // score product's completion (sready of its parity) frees it
+            for (int lt = pc.lt0; lt < pc.lt1 && ok; ++lt, ++nld) {
+                const int slot = nld % e4::NKS;
+                if (nld >= e4::NKS && !mbar_wait(&bars->sready[nld & 1], (uint32_t)((nld - 2) >> 1) & 1u,
+                                                 FLAG_EMPTY_WAIT, c.abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const HalfSrc hs = half_source(p, pc.b, len, lt, (int)c.r);
+                if (lead) mbar_arrive_expect_tx(&bars->kfull[slot], 2 * e4::KSLOT);
+                const uint32_t bar = map_to_rank(smem_u32(&bars->kfull[slot]), 0);
+                uint8_t *dst = c.smem + e4::OFF_SR + slot * e4::KSLOT;
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch)   // (the maps count two codes as one element)
+                    tma_load_3d_pair(dst + ch * CHUNK, &m.lat, bar, 64 * ch, hs.y, hs.page, pol_keep);
+                tma_load_3d_pair(dst + 4 * CHUNK, &m.rope, bar, 0, hs.y, hs.page, pol_keep);
+            }
+            continue;
+        }
         // this CTA's 64 query rows: latent chunks 4..7 and the RoPE chunk
         if (pi > 0 && !mbar_wait(&bars->qempty, (uint32_t)(pi - 1) & 1u, FLAG_EMPTY_WAIT, c.abort_flag)) {
             ok = false;
@@ -292,12 +344,14 @@ __device__ __forceinline__ void key_producer(const MlaParams &p, const MlaMaps &
     }
     if (!ok && lead) {
         // Let the copies already issued land before the CTAs can exit.
-        for (int i = (nld > NKS ? nld - NKS : 0); i < nld; ++i)
-            mbar_wait_sleep(&bars->kfull[i % NKS], (uint32_t)(i / NKS) & 1u, FLAG_FULL_WAIT, nullptr);
-        if (pi > 0) mbar_wait_sleep(&bars->qfull, (uint32_t)(pi - 1) & 1u, FLAG_FULL_WAIT, nullptr);
+        constexpr int nks = KV8 ? e4::NKS : NKS;
+        for (int i = (nld > nks ? nld - nks : 0); i < nld; ++i)
+            mbar_wait_sleep(&bars->kfull[i % nks], (uint32_t)(i / nks) & 1u, FLAG_FULL_WAIT, nullptr);
+        if (!KV8 && pi > 0) mbar_wait_sleep(&bars->qfull, (uint32_t)(pi - 1) & 1u, FLAG_FULL_WAIT, nullptr);
     }
 }
 
+template <bool KV8>
 __device__ __forceinline__ void value_producer(const MlaParams &p, const MlaMaps &m, const Ctx &c) {
     Bars *bars = c.bars;
     const uint64_t pol_last = l2_policy_evict_first();    // the values' read is the last one
@@ -318,14 +372,20 @@ __device__ __forceinline__ void value_producer(const MlaParams &p, const MlaMaps
                     break;
                 }
                 const HalfSrc hs = half_source(p, pc.b, len, lt, h);
-                if (lead) mbar_arrive_expect_tx(&bars->vfull[h], 2 * VSLOT);
+                constexpr int vslot = KV8 ? e4::VSLOT : VSLOT;
+                if (lead) mbar_arrive_expect_tx(&bars->vfull[h], 2 * vslot);
                 const uint32_t bar = map_to_rank(smem_u32(&bars->vfull[h]), 0);
-                uint8_t *dst = c.smem + OFF_PV + h * VSLOT;
+                uint8_t *dst = c.smem + (KV8 ? e4::OFF_PV : OFF_PV) + h * vslot;
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {   // latent block j: this CTA's 128 columns of it
-                    const int x = 256 * j + 128 * (int)c.r;
-                    tma_load_3d_pair(dst + 2 * j * CHUNK, &m.lat, bar, x, hs.y, hs.page, pol_last);
-                    tma_load_3d_pair(dst + (2 * j + 1) * CHUNK, &m.lat, bar, x + 64, hs.y, hs.page, pol_last);
+                    if constexpr (KV8) {        // one box of 128 codes (64 two-code elements)
+                        tma_load_3d_pair(dst + j * CHUNK, &m.lat, bar, 128 * j + 64 * (int)c.r, hs.y, hs.page,
+                                         pol_last);
+                    } else {
+                        const int x = 256 * j + 128 * (int)c.r;
+                        tma_load_3d_pair(dst + 2 * j * CHUNK, &m.lat, bar, x, hs.y, hs.page, pol_last);
+                        tma_load_3d_pair(dst + (2 * j + 1) * CHUNK, &m.lat, bar, x + 64, hs.y, hs.page, pol_last);
+                    }
                 }
             }
         }
@@ -351,9 +411,52 @@ __device__ __forceinline__ bool wait_remote(uint64_t *bar, uint32_t parity, cons
 // plus its address in 16-byte units (the start field never carries: shared addresses
 // are below 2^18), so the issue loops add constants only.
 
-// S of every tile into score buffer kt & 1: 9 chunks x 4 K-steps of 16.
+// S of every tile into score buffer kt & 1: 9 chunks x 4 K-steps of 16 (E4M3: 4 latent
+// boxes x 4 K-steps of 32 codes, each times the query's high part and its remainder; the
+// RoPE box's 2 K-steps into a score buffer of their own, since the RoPE codes have their
+// own scale).
+template <bool KV8>
 __device__ __forceinline__ void score_issuer(const MlaParams &p, const Ctx &c) {
     Bars *bars = c.bars;
+    if constexpr (KV8) {
+        constexpr uint32_t id_s = idesc_e4m3(128, TILE, 0, 0);     // K-major A and B
+        const uint64_t tmpl = smem_desc_sw128(0, 16, 1024);
+        const uint64_t q_desc = tmpl + (smem_u32(c.smem + e4::OFF_Q) >> 4);
+        const uint64_t kr_desc = tmpl + (smem_u32(c.smem + e4::OFF_SR) >> 4);
+        int k = 0, pi = 0;
+        for (long long pos = c.p0; pos < c.p1; ++pi) {
+            const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
+            pos = pc.ustart + pc.lt1;
+            const int nt = pc.lt1 - pc.lt0;
+            // the query parts are written by the softmax warps of both CTAs
+            if (!wait_remote(&bars->qtm, (uint32_t)pi & 1u, c)) return;
+            tc_fence_after();
+            for (int kt = k; kt < k + nt; ++kt) {
+                const int sb = kt & 1, slot = kt % e4::NKS;
+                const uint32_t d = c.tmem + TM_S + 64 * sb;
+                if (kt >= 2 && !wait_remote(&bars->sfree[sb], (uint32_t)((kt >> 1) - 1) & 1u, c)) return;
+                if (!mbar_wait(&bars->kfull[slot], (uint32_t)(kt / e4::NKS) & 1u, FLAG_FULL_WAIT, c.abort_flag))
+                    return;
+                tc_fence_after();
+                const uint64_t kb = kr_desc + (uint64_t)((slot * e4::KSLOT) >> 4);
+#pragma unroll
+                for (int ch = 0; ch < 5; ++ch) {
+                    const uint32_t dd = ch < 4 ? d : c.tmem + e4::TM_SR + 64 * sb;
+#pragma unroll
+                    for (int kk = 0; kk < (ch < 4 ? 4 : 2); ++kk) {   // +32 bytes per K-step
+                        const uint64_t off = (uint64_t)((ch * CHUNK + kk * 32) >> 4);
+                        const uint32_t acc = ((ch & 3) | kk) != 0 ? 1u : 0u;   // (ch 4: a new accumulator)
+                        umma_pair_ss_f8(dd, q_desc + off, kb + off, id_s, acc);
+                        umma_pair_ss_f8(dd, q_desc + off + (uint64_t)(e4::QPART >> 4), kb + off, id_s, 1u);
+                    }
+                }
+                umma_pair_commit_both(&bars->sready[sb]);   // also frees the key slot
+            }
+            umma_pair_commit_both(&bars->qempty);
+            k += nt;
+        }
+        return;
+    }
     constexpr uint32_t id_s = idesc_f16(128, TILE, 1, 1, 0);   // K-major A and B
     const uint64_t k_tmpl = smem_desc_sw128(0, 16, 1024);       // K-major, 128-byte swizzle
     const uint64_t q_desc = k_tmpl + (smem_u32(c.smem + OFF_Q) >> 4);
@@ -404,14 +507,17 @@ __device__ __forceinline__ void score_issuer(const MlaParams &p, const Ctx &c) {
 }
 
 // O += P_hi C + P_lo C for every tile kt: token halves h (one commit each), latent
-// blocks j, K-steps of 16 tokens.
+// blocks j, K-steps of 16 tokens (E4M3: 32).
+template <bool KV8>
 __device__ __forceinline__ void value_issuer(const MlaParams &p, const Ctx &c) {
     Bars *bars = c.bars;
     constexpr uint32_t id_v = idesc_f16(128, 256, 1, 1, 1);    // B (the latents) MN-major
+    constexpr uint32_t id_v8 = idesc_e4m3(128, 256, 0, 1);
     const uint64_t k_tmpl = smem_desc_sw128(0, 16, 1024);       // K-major, 128-byte swizzle
-    const uint64_t v_tmpl = smem_desc_sw128(0, CHUNK, 1024);    // MN-major: the two 64-column chunks 8 KB apart
-    const uint64_t p_desc = k_tmpl + (smem_u32(c.smem + OFF_P) >> 4);
-    const uint64_t vr_desc = v_tmpl + (smem_u32(c.smem + OFF_PV) >> 4);
+    // MN-major: bf16 -- the two 64-column chunks 8 KB apart; E4M3 -- one 128-code row per token
+    const uint64_t v_tmpl = smem_desc_sw128(0, CHUNK, 1024);
+    const uint64_t p_desc = k_tmpl + (smem_u32(c.smem + (KV8 ? e4::OFF_P : OFF_P)) >> 4);
+    const uint64_t vr_desc = v_tmpl + (smem_u32(c.smem + (KV8 ? e4::OFF_PV : OFF_PV)) >> 4);
     int k = 0, pi = 0;
     for (long long pos = c.p0; pos < c.p1; ++pi) {
         const Piece pc = piece_at(c.s_prefix, p.B, 1, pos, c.p1, c.p0);
@@ -426,6 +532,26 @@ __device__ __forceinline__ void value_issuer(const MlaParams &p, const Ctx &c) {
                 if (!wait_remote(&bars->pready[h][kt & 1], (uint32_t)(kt >> 1) & 1u, c)) return;
                 if (!mbar_wait(&bars->vfull[h], (uint32_t)kt & 1u, FLAG_FULL_WAIT, c.abort_flag)) return;
                 tc_fence_after();
+                if constexpr (KV8) {
+                    // weights: K-major [64 heads x 128 tokens], half h = bytes [64h, 64h + 64) of
+                    // each row; values: MN-major, 32 tokens = 4 KB per K-step
+#pragma unroll
+                    for (int jb = 0; jb < 2; ++jb) {
+                        const uint32_t d = c.tmem + TM_O + 128 * jb;
+                        const uint64_t bd = vr_desc + (uint64_t)((h * e4::VSLOT + jb * CHUNK) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < 2; ++kk) {
+                            const uint64_t pa = p_desc + (uint64_t)(((2 * h + kk) * 32) >> 4);
+                            const uint64_t vb = bd + (uint64_t)((kk * 4096) >> 4);
+                            umma_pair_ss_f8(d, pa, vb, id_v8, (!first || h > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                            for (int pp = 1; pp < e4::NPP; ++pp)
+                                umma_pair_ss_f8(d, pa + (uint64_t)((pp * e4::PPART) >> 4), vb, id_v8, 1u);
+                        }
+                    }
+                    umma_pair_commit_both(&bars->odone[h][kt & 1]);
+                    continue;
+                }
                 const uint64_t hi = p_desc + (uint64_t)(h * (CHUNK >> 4));
                 const uint64_t lo = hi + (uint64_t)(2 * (CHUNK >> 4));
 #pragma unroll
@@ -460,8 +586,10 @@ __device__ __forceinline__ bool wait_local(uint64_t *bar, uint32_t parity, unsig
     return warp_all(mbar_wait(bar, parity, flag, c.abort_flag));
 }
 
+template <bool KV8>
 __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, int warp, int lane) {
     Bars *bars = c.bars;
+    constexpr float RESCALE = KV8 ? e4::RESCALE_LOG2 : RESCALE_LOG2;
     const int q = warp & 3;                     // tensor-memory lane quadrant
     const int cg = (warp - 4) >> 2;             // column group: score columns [32cg, 32cg + 32)
     const int L = 32 * q + lane;                // tensor-memory lane
@@ -486,7 +614,12 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
     // units 4cg .. 4cg + 3 (128-byte swizzle)
     uint8_t *row_hi = c.smem + OFF_P + half * CHUNK + hh * 128;
     uint8_t *row_lo = row_hi + 2 * CHUNK;
-    const float sl2 = p.scale_log2;
+    // E4M3: row hh of the weights' [64 heads x 128 tokens] parts, units 4 half + 2 cg + {0, 1}
+    uint8_t *row8_hi = c.smem + e4::OFF_P + hh * 128;
+    // score scale in log2 units (E4M3: the scores arrive scaled, sl2 = 1; sl2_lat / sl2_rope
+    // are the scale times the codes' scale and 2^-e of the head's query part)
+    const float sl2 = KV8 ? 1.f : p.scale_log2;
+    float sl2_lat = 0.f, sl2_rope = 0.f;
 
     // Query latent columns [64cg, 64cg + 64) (bf16 pairs) of this lane's head of sequence
     // b: loaded into registers, then (once the previous piece's score products are done
@@ -517,6 +650,84 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(qtm0);
     };
+    // E4M3 cache: the query of this thread's head as an E4M3 high part and remainder after
+    // scaling by 2^e (the largest magnitude of its latent part, and separately of its RoPE
+    // part, lands in [128, 256)), written into the shared-memory query boxes: exact for
+    // bf16 values (a bf16 significand's eight bits minus the high part's four leave a
+    // remainder of at most four).  The head's 36 16-code units (32 latent, 4 RoPE) are
+    // shared by its four threads, nine each; their maxima meet in shared memory.
+    float *qx_buf = reinterpret_cast<float *>(c.smem + OFF_QX);   // [latent / RoPE][4 parts][64]
+    int q8_uses = 0;
+    auto q8_load = [&](int b, uint4 (&x)[18]) {
+        const uint4 *ql = reinterpret_cast<const uint4 *>(p.q_latent + ((size_t)b * p.H + (realq ? head : 0)) * 512);
+        const uint4 *qr = reinterpret_cast<const uint4 *>(p.q_rope + ((size_t)b * p.H + (realq ? head : 0)) * 64);
+#pragma unroll
+        for (int i = 0; i < 18; ++i) {
+            const int unit = 9 * part + (i >> 1);
+            const uint4 *src = unit < 32 ? ql + 2 * unit + (i & 1) : qr + 2 * (unit - 32) + (i & 1);
+            x[i] = realq ? __ldg(src) : make_uint4(0, 0, 0, 0);
+        }
+    };
+    auto q8_store = [&](const uint4 (&x)[18]) -> bool {
+        // value 2t (+1) of 16-byte load i
+        auto val = [&](int i, int t, int odd) -> float {
+            const uint32_t w = t == 0 ? x[i].x : t == 1 ? x[i].y : t == 2 ? x[i].z : x[i].w;
+            return odd ? bf16_hi(w) : bf16_lo(w);
+        };
+        float mxl = 0.f, mxr = 0.f;   // latent and RoPE parts
+#pragma unroll
+        for (int i = 0; i < 18; ++i) {
+            float m = 0.f;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) m = fmaxf(m, fmaxf(fabsf(val(i, t, 0)), fabsf(val(i, t, 1))));
+            if (9 * part + (i >> 1) < 32) mxl = fmaxf(mxl, m); else mxr = fmaxf(mxr, m);
+        }
+        qx_buf[part * HC + hh] = mxl;
+        qx_buf[4 * HC + part * HC + hh] = mxr;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->qxbar);
+        if (!wait_local(&bars->qxbar, (uint32_t)q8_uses & 1u, FLAG_FULL_WAIT, c)) return false;
+        ++q8_uses;
+        // 2^e that puts a part's largest magnitude in [128, 256)
+        auto pow2_exp = [](float M) -> int {
+            int e = 0;
+            if (M > 0.f && M <= 3.0e38f) {
+                int ex;
+                frexpf(M, &ex);             // M in [2^(ex-1), 2^ex)
+                e = min(max(8 - ex, -120), 120);
+            }
+            return e;
+        };
+        const float* qr = qx_buf + 4 * HC;
+        const int el = pow2_exp(fmaxf(fmaxf(qx_buf[hh], qx_buf[HC + hh]), fmaxf(qx_buf[2 * HC + hh], qx_buf[3 * HC + hh])));
+        const int er = pow2_exp(fmaxf(fmaxf(qr[hh], qr[HC + hh]), fmaxf(qr[2 * HC + hh], qr[3 * HC + hh])));
+        sl2_lat = p.scale_log2 * p.latent_scale * __int_as_float((127 - el) << 23);
+        sl2_rope = p.scale_log2 * p.rope_scale * __int_as_float((127 - er) << 23);
+#pragma unroll
+        for (int i = 0; i < 9; ++i) {
+            const int unit = 9 * part + i;
+            const float up = __int_as_float((127 + (unit < 32 ? el : er)) << 23);
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {   // codes 4t .. 4t + 3 of the unit
+                const int li = 2 * i + (t >> 1), tt = 2 * (t & 1);
+                uint16_t h0, l0, h1, l1;
+                split_e4m3x2(val(li, tt, 0) * up, val(li, tt, 1) * up, h0, l0);
+                split_e4m3x2(val(li, tt + 1, 0) * up, val(li, tt + 1, 1) * up, h1, l1);
+                hw[t] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                lw[t] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+            }
+            const int box = unit < 32 ? unit >> 3 : 4;
+            const int g = unit < 32 ? unit & 7 : unit - 32;
+            uint8_t *dst = c.smem + e4::OFF_Q + box * CHUNK + hh * 128 + ((g ^ (hh & 7)) << 4);
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4 *>(dst + e4::QPART) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(qtm0);
+        return true;
+    };
     // Rescale block cg of this lane's O by alpha (warp-collective).
     auto rescale_o = [&](float alpha) {
 #pragma unroll 1
@@ -536,11 +747,17 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
     // col0 + [0, 128) of the 512.
     const int head0 = HC * (int)c.r + 32 * (q & 1);
     const int col0 = 256 * cg + 128 * half;
-    // 16-byte unit u (0..7) of row rr of the warp's 4 KB transpose scratch: the warp's own
-    // units of the weights buffer (row 32 (q & 1) + rr of its half's chunk, units 4cg..4cg+3
-    // of the high part for u < 4, of the remainder for u >= 4)
+    // 16-byte unit u (0 .. SU - 1) of row rr (0..31) of the warp's transpose scratch: the
+    // warp's own units of the weights buffer.  bf16: row 32 (q & 1) + rr of its half's
+    // chunk, units 4cg..4cg+3 of the high part for u < 4, of the remainder for u >= 4 (SU =
+    // 8, 4 KB).  E4M3: row 32 (q & 1) + rr, units 4 half + 2 cg + {0, 1} of the high part for
+    // u < 2, of the remainder for u >= 2 (SU = 4, 2 KB).
+    constexpr int SU = KV8 ? 4 : 8;
     auto scratch_unit = [&](int rr, int u) -> uint8_t * {
         const int row = 32 * (q & 1) + rr;
+        if constexpr (KV8)
+            return c.smem + e4::OFF_P + (u >> 1) * e4::PPART + row * 128 +
+                   (((4 * half + 2 * cg + (u & 1)) ^ (row & 7)) * 16);
         return c.smem + OFF_P + half * CHUNK + (u >> 2) * 2 * CHUNK + row * 128 +
                (((4 * cg + (u & 3)) ^ (row & 7)) * 16);
     };
@@ -576,13 +793,15 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
                 for (int u = 0; u < 4; ++u) S += v[u] == -INFINITY ? 0.f : fast_exp2((v[u] - M) * 1.4426950408889634f);
             }
         const float lse_all = S > 0.f ? M + __logf(S) : -INFINITY;
-        // the scratch as [32 parts][32 rows] floats (its 4 KB are the warp's own units of the
-        // weights buffer: scratch_unit(r, u) for r < 32, u < 8 -- 8 floats per (r, u))
-        auto wslot = [&](int j, int rr) -> float * {   // weight of part j (< 32) for row rr
-            return reinterpret_cast<float *>(scratch_unit(j, rr >> 2)) + (rr & 3);
+        // the scratch as [JB parts][32 rows] floats (the warp's own units of the weights
+        // buffer: scratch_unit(r, u), 4 floats each)
+        constexpr int JB = 4 * SU;
+        auto wslot = [&](int j, int rr) -> float * {   // weight of part j (< JB) for row rr
+            const int e = 32 * j + rr;
+            return reinterpret_cast<float *>(scratch_unit(e / (4 * SU), (e % (4 * SU)) >> 2)) + (e & 3);
         };
-        for (int jb = 0; jb < n_parts; jb += 32) {
-            const int nj = n_parts - jb < 32 ? n_parts - jb : 32;
+        for (int jb = 0; jb < n_parts; jb += JB) {
+            const int nj = n_parts - jb < JB ? n_parts - jb : JB;
             __syncwarp();
             for (int j = 0; j < nj; ++j) {
                 const float lj = __ldcg(p.ws_lse + part_row(jb + j, hl));
@@ -634,7 +853,7 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
                                                     4 * (lane & 7)) = acc[i];
                 }
             }
-            if (jb + 32 < n_parts) __threadfence_block();   // this warp reads its stores back
+            if (jb + JB < n_parts) __threadfence_block();   // this warp reads its stores back
         }
         if (part == 0 && hl < p.H) p.lse[(size_t)b * p.H + hl] = lse_all;
     };
@@ -660,9 +879,15 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         const int len = clamp_len(__ldg(p.seq_lens + pc.b), p.T_max);
         const int nt = pc.lt1 - pc.lt0;
         if (pi == 0) {
-            uint32_t v0[32], v1[32];
-            load_q(pc.b, v0, v1);
-            store_q(v0, v1);
+            if constexpr (KV8) {
+                uint4 x[18];
+                q8_load(pc.b, x);
+                if (!q8_store(x)) return;
+            } else {
+                uint32_t v0[32], v1[32];
+                load_q(pc.b, v0, v1);
+                store_q(v0, v1);
+            }
         }
         // the next piece's sequence (-1: none); its query rows are fetched into L2 during
         // this piece's last tile
@@ -686,9 +911,19 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             {
                 uint32_t a[32];
                 tmem_ld32(c.tmem + lane_base + TM_S + 64 * sb + 32 * cg, a);
-                tmem_wait_ld();
+                if constexpr (KV8) {   // latent and RoPE parts, each with its scale: log2 units
+                    tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(a[j]);
+                    for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(a[j]) * sl2_lat;
+                    tmem_ld32(c.tmem + lane_base + e4::TM_SR + 64 * sb + 32 * cg, a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) sv[j] = fmaf(__uint_as_float(a[j]), sl2_rope, sv[j]);
+                } else {
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(a[j]);
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -721,28 +956,47 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             if (!wait_local(&bars->mxbar[sb], (uint32_t)(kt >> 1) & 1u, FLAG_FULL_WAIT, c)) return;
             const float *mxs = mx_buf + sb * 4 * HC + hh;
             const float M = fmaxf(fmaxf(mxs[0], mxs[HC]), fmaxf(mxs[2 * HC], mxs[3 * HC]));
-            const float m_new = (t == 0 || M > m_ref + RESCALE_LOG2) ? M : m_ref;
+            const float m_new = (t == 0 || M > m_ref + RESCALE) ? M : m_ref;
             const bool rescale = t > 0 && m_new != m_ref;
             const float alpha = rescale ? fast_exp2(m_ref - m_new) : 1.f;
             m_ref = m_new;
-            // ---- weights 2^(s * scale - m): a bf16 high part and a bf16 remainder
-            uint32_t whi[16], wlo[16];
+            // ---- weights 2^(s * scale - m): a bf16 high part and a bf16 remainder (E4M3 cache:
+            //      2^6 times that, as three E4M3 parts, four codes per word)
+            uint32_t whi[16], wlo[16], wmid[8];
             float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+            const float m_off = KV8 ? e4::P_LOG2 - m_new : -m_new;
+            auto put = [&](int j, float a, float b) {
+                if constexpr (KV8) {
+                    uint16_t h2, m2, l2;
+                    split3_e4m3x2(a, b, h2, m2, l2);
+                    if (j & 1) {
+                        whi[j >> 1] |= (uint32_t)h2 << 16;
+                        wmid[j >> 1] |= (uint32_t)m2 << 16;
+                        wlo[j >> 1] |= (uint32_t)l2 << 16;
+                    } else {
+                        whi[j >> 1] = h2;
+                        wmid[j >> 1] = m2;
+                        wlo[j >> 1] = l2;
+                    }
+                } else {
+                    split_bf16x2(a, b, whi[j], wlo[j]);
+                }
+            };
             if (lo <= 0) {
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float a = fast_exp2(fmaf(sv[2 * j], sl2, -m_new));
-                    const float b = fast_exp2(fmaf(sv[2 * j + 1], sl2, -m_new));
+                    const float a = fast_exp2(fmaf(sv[2 * j], sl2, m_off));
+                    const float b = fast_exp2(fmaf(sv[2 * j + 1], sl2, m_off));
                     ls4[j & 3] += a + b;
-                    split_bf16x2(a, b, whi[j], wlo[j]);
+                    put(j, a, b);
                 }
             } else {   // masked columns get weight 0 (whatever the scale)
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const float a = 2 * j >= lo ? fast_exp2(fmaf(sv[2 * j], sl2, -m_new)) : 0.f;
-                    const float b = 2 * j + 1 >= lo ? fast_exp2(fmaf(sv[2 * j + 1], sl2, -m_new)) : 0.f;
+                    const float a = 2 * j >= lo ? fast_exp2(fmaf(sv[2 * j], sl2, m_off)) : 0.f;
+                    const float b = 2 * j + 1 >= lo ? fast_exp2(fmaf(sv[2 * j + 1], sl2, m_off)) : 0.f;
                     ls4[j & 3] += a + b;
-                    split_bf16x2(a, b, whi[j], wlo[j]);
+                    put(j, a, b);
                 }
             }
             l = l * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
@@ -753,13 +1007,26 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             const int kp = kt - 1;
             const bool any_rescale = __any_sync(0xffffffffu, rescale);   // only when t > 0, so kp >= 0
             auto store_p = [&]() {
+                if constexpr (KV8) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int slot = ((4 * cg + u) ^ (hh & 7)) * 16;
-                    *reinterpret_cast<uint4 *>(row_hi + slot) =
-                        make_uint4(whi[4 * u], whi[4 * u + 1], whi[4 * u + 2], whi[4 * u + 3]);
-                    *reinterpret_cast<uint4 *>(row_lo + slot) =
-                        make_uint4(wlo[4 * u], wlo[4 * u + 1], wlo[4 * u + 2], wlo[4 * u + 3]);
+                    for (int u = 0; u < 2; ++u) {
+                        const int slot = ((4 * half + 2 * cg + u) ^ (hh & 7)) * 16;
+                        *reinterpret_cast<uint4 *>(row8_hi + slot) =
+                            make_uint4(whi[4 * u], whi[4 * u + 1], whi[4 * u + 2], whi[4 * u + 3]);
+                        *reinterpret_cast<uint4 *>(row8_hi + e4::PPART + slot) =
+                            make_uint4(wmid[4 * u], wmid[4 * u + 1], wmid[4 * u + 2], wmid[4 * u + 3]);
+                        *reinterpret_cast<uint4 *>(row8_hi + 2 * e4::PPART + slot) =
+                            make_uint4(wlo[4 * u], wlo[4 * u + 1], wlo[4 * u + 2], wlo[4 * u + 3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int slot = ((4 * cg + u) ^ (hh & 7)) * 16;
+                        *reinterpret_cast<uint4 *>(row_hi + slot) =
+                            make_uint4(whi[4 * u], whi[4 * u + 1], whi[4 * u + 2], whi[4 * u + 3]);
+                        *reinterpret_cast<uint4 *>(row_lo + slot) =
+                            make_uint4(wlo[4 * u], wlo[4 * u + 1], wlo[4 * u + 2], wlo[4 * u + 3]);
+                    }
                 }
                 fence_proxy_async_smem();
             };
@@ -796,10 +1063,17 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         // ---- end of the piece.  First the next piece's query, so that its score products
         //      can start while this epilogue runs (this piece's have read Q: qempty).
         if (next_b >= 0) {
-            uint32_t v0[32], v1[32];
-            load_q(next_b, v0, v1);
-            if (!wait_local(&bars->qempty, (uint32_t)pi & 1u, FLAG_MMA_WAIT, c)) return;
-            store_q(v0, v1);
+            if constexpr (KV8) {
+                uint4 x[18];
+                q8_load(next_b, x);
+                if (!wait_local(&bars->qempty, (uint32_t)pi & 1u, FLAG_MMA_WAIT, c)) return;
+                if (!q8_store(x)) return;
+            } else {
+                uint32_t v0[32], v1[32];
+                load_q(next_b, v0, v1);
+                if (!wait_local(&bars->qempty, (uint32_t)pi & 1u, FLAG_MMA_WAIT, c)) return;
+                store_q(v0, v1);
+            }
         }
         // ---- the head's row sum (four parts), normalise, write this warp's block of O:
         //      rows 32 (q & 1) + [0, 32) of this CTA's heads, columns col0 + [0, 128)
@@ -810,8 +1084,10 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         if (lane == 0) mbar_arrive(&bars->lxbar);
         if (!wait_local(&bars->lxbar, (uint32_t)pi & 1u, FLAG_FULL_WAIT, c)) return;
         const float ltot = (lx_buf[hh] + lx_buf[HC + hh]) + (lx_buf[2 * HC + hh] + lx_buf[3 * HC + hh]);
-        const float lse_v = ltot > 0.f ? (m_ref + __log2f(ltot)) * 0.69314718055994531f : -INFINITY;
-        const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+        // (E4M3 cache: the weights and their sum carry 2^6; a value code counts latent_scale)
+        const float lse_v =
+            ltot > 0.f ? (m_ref + __log2f(ltot) - (KV8 ? e4::P_LOG2 : 0.f)) * 0.69314718055994531f : -INFINITY;
+        const float inv = ltot > 0.f ? (KV8 ? p.latent_scale : 1.f) / ltot : 0.f;
         if (!wait_local(&bars->odone[1][klast & 1], (uint32_t)(klast >> 1) & 1u, FLAG_MMA_WAIT, c)) return;
         tc_fence_after();
         float *dst = pc.whole ? p.out + (size_t)pc.b * p.H * 512
@@ -822,22 +1098,28 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             tmem_ld32(c.tmem + lane_base + TM_O + 128 * cg + 32 * cc, ov);
             tmem_wait_ld();
             // transpose through this warp's own bytes of the weights buffer (free: every
-            // value product of the piece is done), so that eight lanes store one row's
-            // 128 contiguous bytes
+            // value product of the piece is done), SU * 4 columns at a time, so that SU
+            // lanes store one row's SU * 16 contiguous bytes
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                *reinterpret_cast<float4 *>(scratch_unit(lane, u)) =
-                    make_float4(__uint_as_float(ov[4 * u]) * inv, __uint_as_float(ov[4 * u + 1]) * inv,
-                                __uint_as_float(ov[4 * u + 2]) * inv, __uint_as_float(ov[4 * u + 3]) * inv);
-            __syncwarp();
+            for (int ps = 0; ps < 8 / SU; ++ps) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int rr = 4 * i + (lane >> 3), u = lane & 7;
-                const int h_r = head0 + rr;
-                const float4 x = *reinterpret_cast<const float4 *>(scratch_unit(rr, u));
-                if (h_r < p.H) *reinterpret_cast<float4 *>(dst + (size_t)h_r * 512 + col0 + 32 * cc + 4 * u) = x;
+                for (int u = 0; u < SU; ++u) {
+                    const int o = 4 * SU * ps + 4 * u;
+                    *reinterpret_cast<float4 *>(scratch_unit(lane, u)) =
+                        make_float4(__uint_as_float(ov[o]) * inv, __uint_as_float(ov[o + 1]) * inv,
+                                    __uint_as_float(ov[o + 2]) * inv, __uint_as_float(ov[o + 3]) * inv);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < SU; ++i) {
+                    const int rr = (32 / SU) * i + lane / SU, u = lane % SU;
+                    const int h_r = head0 + rr;
+                    const float4 x = *reinterpret_cast<const float4 *>(scratch_unit(rr, u));
+                    if (h_r < p.H)
+                        *reinterpret_cast<float4 *>(dst + (size_t)h_r * 512 + col0 + 32 * cc + 4 * SU * ps + 4 * u) = x;
+                }
+                __syncwarp();
             }
-            __syncwarp();
         }
         if (realq && part == 0) {
             if (pc.whole)
@@ -869,6 +1151,7 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
 }
 }  // namespace mla
 
+template <bool KV8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::NTHREADS, 1)
 mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
     using namespace mla;
@@ -884,6 +1167,7 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
     if (tid == 0) {
         for (int g = 0; g < NKS; ++g) mbar_init(&bars->kfull[g], 1);
         for (int g = 0; g < NKS - 1; ++g) mbar_init(&bars->kempty[g], 1);
+        mbar_init(&bars->qxbar, NSOFT);
         for (int j = 0; j < NVS; ++j) mbar_init(&bars->vfull[j], 1);
         mbar_init(&bars->qfull, 1);
         mbar_init(&bars->qtm, 2 * NSOFT);    // one arrival per softmax warp of either CTA
@@ -913,8 +1197,10 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
     if (warp == 0 && lane == 0) {
         prefetch_tensormap(&maps.lat);
         prefetch_tensormap(&maps.rope);
-        prefetch_tensormap(&maps.qlat);
-        prefetch_tensormap(&maps.qrope);
+        if (!KV8) {
+            prefetch_tensormap(&maps.qlat);
+            prefetch_tensormap(&maps.qrope);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -948,12 +1234,12 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
     c.p1 = (c.p0 + W < total) ? c.p0 + W : total;
 
     if (c.p0 < total) {
-        if (warp == 0 && lane == 0) key_producer(p, maps, c);
-        if (warp == 2 && lane == 0) value_producer(p, maps, c);
-        if (warp == 1 && lane == 0 && c.r == 0) score_issuer(p, c);
-        if (warp == 3 && lane == 0 && c.r == 0) value_issuer(p, c);
+        if (warp == 0 && lane == 0) key_producer<KV8>(p, maps, c);
+        if (warp == 2 && lane == 0) value_producer<KV8>(p, maps, c);
+        if (warp == 1 && lane == 0 && c.r == 0) score_issuer<KV8>(p, c);
+        if (warp == 3 && lane == 0 && c.r == 0) value_issuer<KV8>(p, c);
     }
-    if (warp >= 4) softmax_warps(p, c, warp, lane);   // also the empty sequences
+    if (warp >= 4) softmax_warps<KV8>(p, c, warp, lane);   // also the empty sequences
 
     tc_fence_before();
     __syncthreads();
