@@ -81,7 +81,7 @@ def step_bytes(cfg, lens):
     lens = [min(max(int(x), 0), cfg.max_seq_len) for x in lens]
     if isinstance(cfg, wl.MLAConfig):
         q = cfg.batch * cfg.n_heads * (cfg.latent_dim + cfg.rope_dim) * 2
-        kv = sum(lens) * (cfg.latent_dim + cfg.rope_dim) * 2
+        kv = sum(lens) * (cfg.latent_dim + cfg.rope_dim) * (1 if KV8 else 2)
         out = cfg.batch * cfg.n_heads * cfg.latent_dim * 4
         lse = cfg.batch * cfg.n_heads * 4
     else:
@@ -281,8 +281,10 @@ def to_pages(cache, page_size, seq_axis, perm):
 
 def host_inputs(cfg, seed):
     """The workload's seeded inputs (CPU) with the variant applied."""
-    if (KV8 or QLEN > 1 or WINDOW) and isinstance(cfg, wl.MLAConfig):
-        raise ValueError("E4M3 cache, several new tokens and windows: GQA workloads only")
+    if (QLEN > 1 or WINDOW) and isinstance(cfg, wl.MLAConfig):
+        raise ValueError("several new tokens and windows: GQA workloads only")
+    if isinstance(cfg, wl.MLAConfig):
+        return wl.make_mla_inputs_fp8(cfg, seed=seed) if KV8 else wl.make_mla_inputs(cfg, seed=seed)
     x = wl.make_gqa_inputs_fp8(cfg, seed=seed) if KV8 else wl.make_inputs(cfg, seed=seed)
     if QLEN > 1:
         g = torch.Generator().manual_seed(seed + 29)
@@ -318,6 +320,15 @@ def device_inputs(cfg, seed):
 
 def make_call(cfg, d, out, lse, stream):
     from mla_kv_cache_b200 import binding as kb
+    if KV8 and isinstance(cfg, wl.MLAConfig):
+        if PAGED:
+            return lambda: kb.kvattn_mla_decode_fp8_paged(d["q_latent"], d["q_rope"], d["latent_cache_pages"],
+                                                          d["rope_cache_pages"], d["block_table"], d["seq_lens"],
+                                                          cfg.scale, d["latent_scale"], d["rope_scale"], out=out,
+                                                          lse=lse, stream=stream)
+        return lambda: kb.kvattn_mla_decode_fp8(d["q_latent"], d["q_rope"], d["latent_cache"], d["rope_cache"],
+                                                d["seq_lens"], cfg.scale, d["latent_scale"], d["rope_scale"],
+                                                out=out, lse=lse, stream=stream)
     if KV8 and PAGED:
         if QLEN > 1 or WINDOW:
             raise ValueError("the paged E4M3 entry point takes one new token and no window")
@@ -361,6 +372,10 @@ def oracle_step(cfg, x, ids):
     """The oracle on sequences `ids` of the workload (variant applied)."""
     import oracle
     if isinstance(cfg, wl.MLAConfig):
+        if KV8:
+            return oracle.mla_decode_fp8(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"],
+                                         x["seq_lens"], cfg.scale, x["latent_scale"], x["rope_scale"],
+                                         batch_ids=ids)
         return oracle.mla_decode(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"],
                                  x["seq_lens"], cfg.scale, batch_ids=ids)
     if KV8:
@@ -490,8 +505,11 @@ def measure_config(cfg, steps, warmup, flush, stream, seed, pk, world):
            "flops_per_step": fl}
     if isinstance(cfg, wl.MLAConfig):
         t_hbm = nb["total"] / (pk["hbm_gbs"] * 1e9)
-        t_tc = fl / (pk["bf16_tflops"] * 1e12)
+        # E4M3 operands: the tensor pipe's fp8 rate, twice the measured bf16 one (the
+        # nominal dense ratio, 4.5 / 2.25 PFLOP/s)
+        t_tc = fl / (pk["bf16_tflops"] * (2.0 if KV8 else 1.0) * 1e12)
         res["roofline_us"] = max(t_hbm, t_tc) * 1e6
+        res["roofline_bound"] = "hbm" if t_hbm >= t_tc else "tensor"
         res["roofline_frac"] = res["roofline_us"] / res["us_per_step"]
     return x, d, res, times
 

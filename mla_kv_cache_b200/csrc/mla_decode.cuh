@@ -658,30 +658,28 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
     // shared by its four threads, nine each; their maxima meet in shared memory.
     float *qx_buf = reinterpret_cast<float *>(c.smem + OFF_QX);   // [latent / RoPE][4 parts][64]
     int q8_uses = 0;
-    auto q8_load = [&](int b, uint4 (&x)[18]) {
-        const uint4 *ql = reinterpret_cast<const uint4 *>(p.q_latent + ((size_t)b * p.H + (realq ? head : 0)) * 512);
-        const uint4 *qr = reinterpret_cast<const uint4 *>(p.q_rope + ((size_t)b * p.H + (realq ? head : 0)) * 64);
-#pragma unroll
-        for (int i = 0; i < 18; ++i) {
-            const int unit = 9 * part + (i >> 1);
-            const uint4 *src = unit < 32 ? ql + 2 * unit + (i & 1) : qr + 2 * (unit - 32) + (i & 1);
-            x[i] = realq ? __ldg(src) : make_uint4(0, 0, 0, 0);
-        }
+    auto q8_src = [&](int b, int i) -> const uint4 * {   // 16-byte load i (0..17) of this thread's units
+        const int unit = 9 * part + (i >> 1);
+        const size_t row = (size_t)b * p.H + (realq ? head : 0);
+        return unit < 32 ? reinterpret_cast<const uint4 *>(p.q_latent + row * 512) + 2 * unit + (i & 1)
+                         : reinterpret_cast<const uint4 *>(p.q_rope + row * 64) + 2 * (unit - 32) + (i & 1);
     };
-    auto q8_store = [&](const uint4 (&x)[18]) -> bool {
-        // value 2t (+1) of 16-byte load i
-        auto val = [&](int i, int t, int odd) -> float {
-            const uint32_t w = t == 0 ? x[i].x : t == 1 ? x[i].y : t == 2 ? x[i].z : x[i].w;
-            return odd ? bf16_hi(w) : bf16_lo(w);
-        };
-        float mxl = 0.f, mxr = 0.f;   // latent and RoPE parts
+    // first pass: the largest magnitudes of this thread's latent and RoPE values
+    auto q8_load = [&](int b, float &mxl, float &mxr) {
+        mxl = 0.f;
+        mxr = 0.f;
 #pragma unroll
         for (int i = 0; i < 18; ++i) {
+            const uint4 x = realq ? __ldg(q8_src(b, i)) : make_uint4(0, 0, 0, 0);
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
             float m = 0.f;
 #pragma unroll
-            for (int t = 0; t < 4; ++t) m = fmaxf(m, fmaxf(fabsf(val(i, t, 0)), fabsf(val(i, t, 1))));
+            for (int t = 0; t < 4; ++t) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[t])), fabsf(bf16_hi(w[t]))));
             if (9 * part + (i >> 1) < 32) mxl = fmaxf(mxl, m); else mxr = fmaxf(mxr, m);
         }
+    };
+    // second pass (the query loaded again, from L1): the head's scales, the split, the stores
+    auto q8_store = [&](int b, float mxl, float mxr) -> bool {
         qx_buf[part * HC + hh] = mxl;
         qx_buf[4 * HC + part * HC + hh] = mxr;
         __syncwarp();
@@ -698,22 +696,26 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             }
             return e;
         };
-        const float* qr = qx_buf + 4 * HC;
+        const float *qr = qx_buf + 4 * HC;
         const int el = pow2_exp(fmaxf(fmaxf(qx_buf[hh], qx_buf[HC + hh]), fmaxf(qx_buf[2 * HC + hh], qx_buf[3 * HC + hh])));
         const int er = pow2_exp(fmaxf(fmaxf(qr[hh], qr[HC + hh]), fmaxf(qr[2 * HC + hh], qr[3 * HC + hh])));
         sl2_lat = p.scale_log2 * p.latent_scale * __int_as_float((127 - el) << 23);
         sl2_rope = p.scale_log2 * p.rope_scale * __int_as_float((127 - er) << 23);
-#pragma unroll
+#pragma unroll 3
         for (int i = 0; i < 9; ++i) {
             const int unit = 9 * part + i;
             const float up = __int_as_float((127 + (unit < 32 ? el : er)) << 23);
+            uint4 xs[2];
+            xs[0] = realq ? __ldg(q8_src(b, 2 * i)) : make_uint4(0, 0, 0, 0);
+            xs[1] = realq ? __ldg(q8_src(b, 2 * i + 1)) : make_uint4(0, 0, 0, 0);
             uint32_t hw[4], lw[4];
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {   // codes 4t .. 4t + 3 of the unit
-                const int li = 2 * i + (t >> 1), tt = 2 * (t & 1);
+            for (int t = 0; t < 4; ++t) {   // codes 4t .. 4t + 3 of the unit: words 2t, 2t + 1 of the pair
+                const uint4 &x = xs[t >> 1];
+                const uint32_t w0 = (t & 1) ? x.z : x.x, w1 = (t & 1) ? x.w : x.y;
                 uint16_t h0, l0, h1, l1;
-                split_e4m3x2(val(li, tt, 0) * up, val(li, tt, 1) * up, h0, l0);
-                split_e4m3x2(val(li, tt + 1, 0) * up, val(li, tt + 1, 1) * up, h1, l1);
+                split_e4m3x2(bf16_lo(w0) * up, bf16_hi(w0) * up, h0, l0);
+                split_e4m3x2(bf16_lo(w1) * up, bf16_hi(w1) * up, h1, l1);
                 hw[t] = (uint32_t)h0 | ((uint32_t)h1 << 16);
                 lw[t] = (uint32_t)l0 | ((uint32_t)l1 << 16);
             }
@@ -880,9 +882,9 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         const int nt = pc.lt1 - pc.lt0;
         if (pi == 0) {
             if constexpr (KV8) {
-                uint4 x[18];
-                q8_load(pc.b, x);
-                if (!q8_store(x)) return;
+                float mxl, mxr;
+                q8_load(pc.b, mxl, mxr);
+                if (!q8_store(pc.b, mxl, mxr)) return;
             } else {
                 uint32_t v0[32], v1[32];
                 load_q(pc.b, v0, v1);
@@ -1064,10 +1066,10 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         //      can start while this epilogue runs (this piece's have read Q: qempty).
         if (next_b >= 0) {
             if constexpr (KV8) {
-                uint4 x[18];
-                q8_load(next_b, x);
+                float mxl, mxr;
+                q8_load(next_b, mxl, mxr);
                 if (!wait_local(&bars->qempty, (uint32_t)pi & 1u, FLAG_MMA_WAIT, c)) return;
-                if (!q8_store(x)) return;
+                if (!q8_store(next_b, mxl, mxr)) return;
             } else {
                 uint32_t v0[32], v1[32];
                 load_q(next_b, v0, v1);
