@@ -131,8 +131,13 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
  *             are not read.
  *   out       device fp32 [batch, q_len, n_q_heads, head_dim];  lse fp32 [batch, q_len, n_q_heads]
  * A query with no visible position (p < 0) gets out = 0 and lse = -inf.  q_len == 1 and
- * window == 0 is exactly kvattn_gqa_decode.  Otherwise head_dim must be 128 and
- * (n_q_heads / n_kv_heads) * q_len <= 64 (KVATTN_ERR_UNSUPPORTED if not).
+ * window == 0 is exactly kvattn_gqa_decode.  head_dim 64 or 128; a window needs head_dim
+ * 128 and n_q_heads / n_kv_heads <= 64; batch * q_len <= 4096 (KVATTN_ERR_UNSUPPORTED
+ * otherwise).  With head_dim 128 and (n_q_heads / n_kv_heads) * q_len <= 64 one kernel
+ * scores a group's heads at all q_len positions against each cache tile; otherwise the
+ * call runs as batch * q_len single-token sequences (query i of sequence b is a sequence
+ * of length seq_lens[b] - q_len + 1 + i over b's cache rows), which reads the cache once
+ * per new token (the repeats mostly from L2).
  */
 int kvattn_gqa_decode_multi(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
                             const int32_t *seq_lens, int max_seq_len, int batch, int q_len,
@@ -153,8 +158,8 @@ int kvattn_gqa_decode_multi(const uint16_t *q, const uint16_t *k_cache, const ui
  *               [batch, n_kv_heads, max_seq_len, head_dim]
  *   k_scale, v_scale  finite, > 0
  *   out, lse    device fp32 [batch, q_len, n_q_heads, head_dim], [batch, q_len, n_q_heads]
- * head_dim must be 128 and (n_q_heads / n_kv_heads) * q_len <= 64 (else
- * KVATTN_ERR_UNSUPPORTED); everything else as for kvattn_gqa_decode_multi.  The query
+ * head_dim must be 128 and n_q_heads / n_kv_heads <= 64 (else KVATTN_ERR_UNSUPPORTED);
+ * everything else as for kvattn_gqa_decode_multi.  The query
  * and the softmax weights enter the tensor-core products as two E4M3 parts each (~8
  * significant bits), the codes exactly; accumulation is fp32.  Codes past a sequence's
  * length are never read.
@@ -199,6 +204,25 @@ int kvattn_mla_decode_fp8(const uint16_t *q_latent, const uint16_t *q_rope, cons
                           const uint8_t *rope_cache, const int32_t *seq_lens, int max_seq_len, int batch,
                           int n_heads, int latent_dim, int rope_dim, float scale, float latent_scale,
                           float rope_scale, float *out, float *lse, void *stream);
+
+/*
+ * Several new tokens per sequence for absorbed MLA (the causal mask as for
+ * kvattn_gqa_decode_multi; no window): query i of sequence b, at position
+ * p = seq_lens[b] - q_len + i, attends to the cached tokens t <= p.
+ *   q_latent, q_rope  device bf16 [batch, q_len, n_heads, 512], [batch, q_len, n_heads, 64]
+ *   latent_cache, rope_cache  device [batch, max_seq_len, 512], [batch, max_seq_len, 64]:
+ *             bf16 (e4m3 == 0) or E4M3 codes with latent_scale / rope_scale as for
+ *             kvattn_mla_decode_fp8 (e4m3 != 0; the scales are ignored otherwise)
+ *   out, lse  device fp32 [batch, q_len, n_heads, 512], [batch, q_len, n_heads]
+ * A query with no visible position gets out = 0 and lse = -inf.  batch * q_len <= 1024.
+ * The call runs as batch * q_len single-token sequences over b's cache rows (the cache
+ * read once per new token, the repeats mostly from L2); q_len == 1 is kvattn_mla_decode
+ * (kvattn_mla_decode_fp8).  Everything else as for kvattn_mla_decode.
+ */
+int kvattn_mla_decode_multi(const uint16_t *q_latent, const uint16_t *q_rope, const void *latent_cache,
+                            const void *rope_cache, const int32_t *seq_lens, int max_seq_len, int batch, int q_len,
+                            int n_heads, int latent_dim, int rope_dim, float scale, int e4m3, float latent_scale,
+                            float rope_scale, float *out, float *lse, void *stream);
 
 /*
  * kvattn_mla_decode_fp8 over a paged cache: latent_pages [num_pages, page_size, 512] and

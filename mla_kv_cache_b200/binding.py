@@ -83,6 +83,10 @@ _SIGNATURES = {
                                                   ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                                   ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
                                                   ctypes.c_float, ctypes.c_float, ctypes.c_void_p]),
+    "kvattn_mla_decode_multi": (ctypes.c_int, [_c_u16p, _c_u16p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_float,
+                                               ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "kvattn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvattn_last_error_detail": (ctypes.c_char_p, []),
     "kvattn_version": (ctypes.c_int, []),
@@ -540,6 +544,41 @@ def kvattn_mla_rope_append_fp8(q_rope, latent_new, rope_new, positions, latent_c
                                           float(latent_scale), float(rope_scale), _stream_handle(stream))
     if st != KVATTN_OK:
         raise KvattnError(st, "kvattn_mla_rope_append_fp8")
+
+
+def kvattn_mla_decode_multi(q_latent, q_rope, latent_cache, rope_cache, seq_lens, scale, latent_scale=None,
+                            rope_scale=None, out=None, lse=None, stream=None):
+    """Several new tokens per sequence for MLA (include/kvattn.h, kvattn_mla_decode_multi):
+    q_latent [B, L, H, 512], q_rope [B, L, H, 64] bf16; caches [B, T, 512] / [B, T, 64] bf16,
+    or float8_e4m3fn codes with latent_scale / rope_scale.  Returns (out [B, L, H, 512],
+    lse [B, L, H]) fp32."""
+    import torch
+    B, L, H, dc = q_latent.shape
+    dr = q_rope.shape[3]
+    T = latent_cache.shape[1]
+    e4m3 = latent_cache.dtype != torch.bfloat16
+    _check(q_latent, "q_latent", torch.bfloat16)
+    _check(q_rope, "q_rope", torch.bfloat16, (B, L, H, dr))
+    if e4m3:
+        _check_e4m3(latent_cache, "latent_cache", (B, T, dc))
+        _check_e4m3(rope_cache, "rope_cache", (B, T, dr))
+    else:
+        _check(latent_cache, "latent_cache", torch.bfloat16, (B, T, dc))
+        _check(rope_cache, "rope_cache", torch.bfloat16, (B, T, dr))
+    _check(seq_lens, "seq_lens", torch.int32, (B,))
+    if out is None:
+        out = torch.empty((B, L, H, dc), dtype=torch.float32, device=q_latent.device)
+    if lse is None:
+        lse = torch.empty((B, L, H), dtype=torch.float32, device=q_latent.device)
+    _check(out, "out", torch.float32, (B, L, H, dc))
+    _check(lse, "lse", torch.float32, (B, L, H))
+    st = lib().kvattn_mla_decode_multi(q_latent.data_ptr(), q_rope.data_ptr(), latent_cache.data_ptr(),
+                                       rope_cache.data_ptr(), seq_lens.data_ptr(), T, B, L, H, dc, dr, float(scale),
+                                       int(e4m3), float(latent_scale or 1.0), float(rope_scale or 1.0),
+                                       out.data_ptr(), lse.data_ptr(), _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_mla_decode_multi")
+    return out, lse
 
 
 def kvattn_gqa_decode_multi(q, k_cache, v_cache, seq_lens, scale, window=0, out=None, lse=None, stream=None):

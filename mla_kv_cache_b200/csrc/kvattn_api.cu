@@ -37,6 +37,8 @@ struct DeviceState {
     int max_smem_optin = 0;
     void *ws = nullptr;
     size_t ws_bytes = 0;
+    void *aux = nullptr;          // the virtual batch of a multi-token call (lengths, block table)
+    size_t aux_bytes = 0;
     struct Func {
         const void *kern;
         int smem;
@@ -470,7 +472,70 @@ struct GqaCache {
     long long pages;              // pages in the pool (contiguous: batch)
     bool e4m3 = false;            // E4M3 codes (value = code * scale) instead of bf16
     float k_scale = 1.f, v_scale = 1.f;
+    bool one_page = false;        // every sequence's rows lie in its first page
 };
+
+// ---------------------------------------------------------------------------------------
+// Several new tokens through the single-token kernels.  New token i (0 <= i < L) of
+// sequence b sits at position len_b - L + i and attends, causally, to the cache rows
+// [0, len_b - L + i] (optionally the last `window` of them): exactly a single-token decode
+// of a sequence of length len_b - L + 1 + i over the same cache.  The call becomes a
+// batch of B * L such virtual sequences (v = b * L + i, so q [B, L, ...] and out / lse
+// [B, L, ...] are already in its layout), each reading sequence b's pages through a
+// block table built here on the device.  A contiguous cache is one page per sequence.
+// The cache is read once per new token; the L readers of a page run side by side in the
+// work split, so the repeats mostly come from L2.
+// ---------------------------------------------------------------------------------------
+__global__ void virtual_batch_kernel(const int32_t *seq_lens, const int32_t *block_table, int B, int L,
+                                     int max_pages, int capacity, int32_t *vlens, int32_t *vtable) {
+    const long long n = (long long)B * L;
+    for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n; v += (long long)gridDim.x * blockDim.x) {
+        const int b = (int)(v / L), i = (int)(v % L);
+        int len = __ldg(seq_lens + b);
+        len = len < 0 ? 0 : (len > capacity ? capacity : len);
+        const int lv = len - L + 1 + i;
+        vlens[v] = lv > 0 ? lv : 0;
+        if (block_table)
+            for (int m = 0; m < max_pages; ++m) vtable[v * max_pages + m] = __ldg(block_table + (size_t)b * max_pages + m);
+        else
+            vtable[v] = b;
+    }
+}
+
+// Builds the virtual batch's lengths and block table in the device's aux buffer.
+int virtual_batch(DeviceState *dev, const int32_t *seq_lens, const int32_t *block_table, int B, int L,
+                  int max_pages, int capacity, cudaStream_t s, int32_t **vlens, int32_t **vtable) {
+    const int mp = block_table ? max_pages : 1;
+    const size_t lens_bytes = (((size_t)B * L * 4) + 255) & ~size_t(255);
+    const size_t need = lens_bytes + (size_t)B * L * mp * 4;
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        if (dev->aux_bytes < need) {
+            if (dev->aux) {
+                cudaError_t e = cudaDeviceSynchronize();
+                if (e != cudaSuccess) return fail_cuda(e, "cudaDeviceSynchronize (aux grow)");
+                cudaFree(dev->aux);
+                dev->aux = nullptr;
+                dev->aux_bytes = 0;
+            }
+            cudaError_t e = cudaMalloc(&dev->aux, need);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                snprintf(t_detail, sizeof(t_detail), "cudaMalloc(%zu): %s", need, cudaGetErrorString(e));
+                return KVATTN_ERR_NO_MEMORY;
+            }
+            dev->aux_bytes = need;
+        }
+    }
+    *vlens = static_cast<int32_t *>(dev->aux);
+    *vtable = reinterpret_cast<int32_t *>(static_cast<char *>(dev->aux) + lens_bytes);
+    const long long n = (long long)B * L;
+    const int blocks = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+    virtual_batch_kernel<<<blocks, 256, 0, s>>>(seq_lens, block_table, B, L, mp, capacity, *vlens, *vtable);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail_cuda(e, "virtual batch launch");
+    return KVATTN_OK;
+}
 
 // noalloc: the warp-level kernel with its scratch in the static array (one new token,
 // no window, bf16 contiguous cache).
@@ -483,7 +548,34 @@ int gqa_decode_impl(const uint16_t *q, const GqaCache &cache, const int32_t *seq
 
     const int g = n_q_heads / n_kv_heads;
     // a paged cache needs pages made of whole 128-token tiles for the tcgen05 kernel
-    const bool tiles_fit = cache.block_table == nullptr || cache.page_size % gqatc::TILE == 0;
+    const bool tiles_fit = cache.block_table == nullptr || cache.one_page || cache.page_size % gqatc::TILE == 0;
+    // several new tokens the multi-token kernel cannot take (head_dim 64, g * q_len > 64,
+    // pages it cannot tile): a virtual batch of single-token sequences (windows only where
+    // the tcgen05 kernel serves the single-token form)
+    if (q_len > 1 && !noalloc &&
+        !(tiles_fit && head_dim == 128 && g * q_len <= gqatc::HB && gqatc::smem_bytes(batch) <= dev->max_smem_optin)) {
+        if ((long long)batch * q_len > kMaxBatch) {
+            snprintf(t_detail, sizeof(t_detail), "batch * q_len exceeds %d", kMaxBatch);
+            return KVATTN_ERR_UNSUPPORTED;
+        }
+        const bool tc1 = head_dim == 128 && g <= gqatc::HB &&
+                         gqatc::smem_bytes(batch * q_len) <= dev->max_smem_optin;
+        if ((window > 0 || cache.e4m3) && !tc1) {
+            snprintf(t_detail, sizeof(t_detail), "a window or an E4M3 cache needs head_dim 128 and g <= %d",
+                     gqatc::HB);
+            return KVATTN_ERR_UNSUPPORTED;
+        }
+        int32_t *vlens = nullptr, *vtable = nullptr;
+        st = virtual_batch(dev, seq_lens, cache.block_table, batch, q_len, cache.max_pages, cache.capacity,
+                           static_cast<cudaStream_t>(stream), &vlens, &vtable);
+        if (st != KVATTN_OK) return st;
+        GqaCache vc = cache;
+        vc.block_table = vtable;
+        vc.max_pages = cache.block_table ? cache.max_pages : 1;
+        vc.one_page = cache.block_table == nullptr;
+        return gqa_decode_impl(q, vc, vlens, batch * q_len, n_q_heads, n_kv_heads, head_dim, scale, out, lse,
+                               stream, 1, window);
+    }
     if (!noalloc && g_gqa_kernel == 2 && !(tiles_fit && use_tc_kernel(head_dim, g, batch, dev))) {
         snprintf(t_detail, sizeof(t_detail),
                  "tcgen05 GQA kernel needs head_dim 128, batch <= %d and pages of multiples of 128 rows",
@@ -789,9 +881,8 @@ int kvattn_gqa_decode_multi(const uint16_t *q, const uint16_t *k_cache, const ui
     if (n_q_heads % n_kv_heads != 0) return KVATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale)) return KVATTN_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return KVATTN_ERR_UNSUPPORTED;
-    if ((q_len > 1 || window > 0) && (head_dim != 128 || (n_q_heads / n_kv_heads) * q_len > gqatc::HB))
-        return KVATTN_ERR_UNSUPPORTED;
-    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
+    if (window > 0 && (head_dim != 128 || n_q_heads / n_kv_heads > gqatc::HB)) return KVATTN_ERR_UNSUPPORTED;
+    if (batch > kMaxBatch || (long long)batch * q_len > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
     if ((long long)batch * n_kv_heads * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seq_lens) ||
         !aligned16(out) || !aligned16(lse))
@@ -822,8 +913,8 @@ int kvattn_gqa_decode_fp8(const uint16_t *q, const uint8_t *k_cache, const uint8
     if (!std::isfinite(scale) || !std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) ||
         !(v_scale > 0.f))
         return KVATTN_ERR_INVALID_ARG;
-    if (head_dim != 128 || (n_q_heads / n_kv_heads) * q_len > gqatc::HB) return KVATTN_ERR_UNSUPPORTED;
-    if (batch > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
+    if (head_dim != 128 || n_q_heads / n_kv_heads > gqatc::HB) return KVATTN_ERR_UNSUPPORTED;
+    if (batch > kMaxBatch || (long long)batch * q_len > kMaxBatch) return KVATTN_ERR_UNSUPPORTED;
     if ((long long)batch * n_kv_heads * max_seq_len >= (1ll << 31)) return KVATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(seq_lens) ||
         !aligned16(out) || !aligned16(lse))
@@ -891,8 +982,10 @@ int kvattn_gqa_decode_fp8_paged(const uint16_t *q, const uint8_t *k_pages, const
 static int mla_entry(const uint16_t *q_latent, const uint16_t *q_rope, const void *lat, const void *rope,
               const int32_t *block_table, const int32_t *seq_lens, int num_pages, int page_size,
               int max_pages_per_seq, int batch, int n_heads, int latent_dim, int rope_dim, float scale, bool e4m3,
-              float latent_scale, float rope_scale, float *out, float *lse, void *stream) {
+              float latent_scale, float rope_scale, float *out, float *lse, void *stream, int q_len = 1) {
     const bool paged = block_table != nullptr;
+    if (q_len <= 0) return KVATTN_ERR_INVALID_ARG;
+    if ((long long)batch * q_len > mla::MAX_BATCH) return KVATTN_ERR_UNSUPPORTED;
     if (!q_latent || !q_rope || !lat || !rope || !seq_lens || !out || !lse) return KVATTN_ERR_INVALID_ARG;
     if (batch <= 0 || n_heads <= 0 || num_pages <= 0 || page_size <= 0 || max_pages_per_seq <= 0 ||
         latent_dim <= 0 || rope_dim < 0)
@@ -910,12 +1003,12 @@ static int mla_entry(const uint16_t *q_latent, const uint16_t *q_rope, const voi
         (paged && !aligned16(block_table)) || !aligned16(seq_lens) || !aligned16(out) || !aligned16(lse))
         return KVATTN_ERR_MISALIGNED;
     const size_t cb = e4m3 ? 1 : 2;
-    const size_t ql_bytes = (size_t)batch * n_heads * latent_dim * 2;
-    const size_t qr_bytes = (size_t)batch * n_heads * rope_dim * 2;
+    const size_t ql_bytes = (size_t)batch * q_len * n_heads * latent_dim * 2;
+    const size_t qr_bytes = (size_t)batch * q_len * n_heads * rope_dim * 2;
     const size_t lat_bytes = (size_t)num_pages * page_size * latent_dim * cb;
     const size_t rope_bytes = (size_t)num_pages * page_size * rope_dim * cb;
-    const size_t out_bytes = (size_t)batch * n_heads * latent_dim * 4;
-    const size_t lse_bytes = (size_t)batch * n_heads * 4;
+    const size_t out_bytes = (size_t)batch * q_len * n_heads * latent_dim * 4;
+    const size_t lse_bytes = (size_t)batch * q_len * n_heads * 4;
     const void *ins[6] = {q_latent, q_rope, lat, rope, seq_lens, block_table};
     const size_t in_sz[6] = {ql_bytes, qr_bytes, lat_bytes, rope_bytes, (size_t)batch * 4,
                              paged ? (size_t)batch * max_pages_per_seq * 4 : 0};
@@ -923,9 +1016,20 @@ static int mla_entry(const uint16_t *q_latent, const uint16_t *q_rope, const voi
         if (overlaps(out, out_bytes, ins[i], in_sz[i]) || overlaps(lse, lse_bytes, ins[i], in_sz[i]))
             return KVATTN_ERR_INVALID_ARG;
     if (overlaps(out, out_bytes, lse, lse_bytes)) return KVATTN_ERR_INVALID_ARG;
-    const MlaCache cache{lat, rope, block_table, max_pages_per_seq * page_size, page_size, max_pages_per_seq,
-                         num_pages, e4m3, latent_scale, rope_scale};
-    return mla_decode_impl(q_latent, q_rope, cache, seq_lens, batch, n_heads, scale, out, lse, stream);
+    MlaCache cache{lat, rope, block_table, max_pages_per_seq * page_size, page_size, max_pages_per_seq,
+                   num_pages, e4m3, latent_scale, rope_scale};
+    if (q_len == 1) return mla_decode_impl(q_latent, q_rope, cache, seq_lens, batch, n_heads, scale, out, lse, stream);
+    // several new tokens: a virtual batch of single-token sequences over the same pages
+    DeviceState *dev = nullptr;
+    int st = device_state(&dev);
+    if (st != KVATTN_OK) return st;
+    int32_t *vlens = nullptr, *vtable = nullptr;
+    st = virtual_batch(dev, seq_lens, block_table, batch, q_len, max_pages_per_seq, cache.capacity,
+                       static_cast<cudaStream_t>(stream), &vlens, &vtable);
+    if (st != KVATTN_OK) return st;
+    cache.block_table = vtable;
+    if (!paged) cache.max_pages = 1;   // one page (the whole capacity) per sequence
+    return mla_decode_impl(q_latent, q_rope, cache, vlens, batch * q_len, n_heads, scale, out, lse, stream);
 }
 
 int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
@@ -933,7 +1037,7 @@ int kvattn_mla_decode(const uint16_t *q_latent, const uint16_t *q_rope,
                       const int32_t *seq_lens, int max_seq_len, int batch, int n_heads,
                       int latent_dim, int rope_dim, float scale, float *out, float *lse,
                       void *stream) {
-    return mla_entry(q_latent, q_rope, latent_cache, rope_cache, nullptr, seq_lens, batch, max_seq_len, max_seq_len,
+    return mla_entry(q_latent, q_rope, latent_cache, rope_cache, nullptr, seq_lens, batch, max_seq_len, 1,
                      batch, n_heads, latent_dim, rope_dim, scale, false, 1.f, 1.f, out, lse, stream);
 }
 
@@ -951,8 +1055,17 @@ int kvattn_mla_decode_fp8(const uint16_t *q_latent, const uint16_t *q_rope, cons
                           const uint8_t *rope_cache, const int32_t *seq_lens, int max_seq_len, int batch,
                           int n_heads, int latent_dim, int rope_dim, float scale, float latent_scale,
                           float rope_scale, float *out, float *lse, void *stream) {
-    return mla_entry(q_latent, q_rope, latent_cache, rope_cache, nullptr, seq_lens, batch, max_seq_len, max_seq_len,
+    return mla_entry(q_latent, q_rope, latent_cache, rope_cache, nullptr, seq_lens, batch, max_seq_len, 1,
                      batch, n_heads, latent_dim, rope_dim, scale, true, latent_scale, rope_scale, out, lse, stream);
+}
+
+int kvattn_mla_decode_multi(const uint16_t *q_latent, const uint16_t *q_rope, const void *latent_cache,
+                            const void *rope_cache, const int32_t *seq_lens, int max_seq_len, int batch, int q_len,
+                            int n_heads, int latent_dim, int rope_dim, float scale, int e4m3, float latent_scale,
+                            float rope_scale, float *out, float *lse, void *stream) {
+    return mla_entry(q_latent, q_rope, latent_cache, rope_cache, nullptr, seq_lens, batch, max_seq_len, 1,
+                     batch, n_heads, latent_dim, rope_dim, scale, e4m3 != 0, e4m3 ? latent_scale : 1.f,
+                     e4m3 ? rope_scale : 1.f, out, lse, stream, q_len);
 }
 
 int kvattn_mla_decode_fp8_paged(const uint16_t *q_latent, const uint16_t *q_rope, const uint8_t *latent_pages,
@@ -993,6 +1106,13 @@ void kvattn_release_workspace(void) {
             cudaFree(g_dev[d].ws);
             g_dev[d].ws = nullptr;
             g_dev[d].ws_bytes = 0;
+        }
+        if (g_dev[d].aux) {
+            cudaSetDevice(d);
+            cudaDeviceSynchronize();
+            cudaFree(g_dev[d].aux);
+            g_dev[d].aux = nullptr;
+            g_dev[d].aux_bytes = 0;
         }
     }
     cudaSetDevice(cur);

@@ -194,6 +194,32 @@ def mla_decode(q_latent, q_rope, latent_cache, rope_cache, seq_lens, scale, batc
     return np.stack(outs), np.stack(lses)
 
 
+def _causal_rows(length, q_len, i, capacity):
+    """Cache rows query i (0-based, oldest first) of q_len new tokens sees: the tokens at
+    positions <= len - q_len + i ("Attention variants: MQA, GQA, and MLA", section
+    "Implementation, twice": no query sees a later token)."""
+    return max(_rows(length, capacity) - q_len + 1 + i, 0)
+
+
+def mla_decode_multi(q_latent, q_rope, latent_cache, rope_cache, seq_lens, scale, lib=None):
+    """Absorbed MLA with q_len new tokens per sequence under the causal mask.  q_latent
+    [B, L, H, d_c], q_rope [B, L, H, d_r] bf16; caches [B, T_max, d_c], [B, T_max, d_r]
+    (bf16, or fp64 arrays already dequantised).  Returns (out [B, L, H, d_c], lse [B, L, H]);
+    a query that sees no token gets out 0, lse -inf."""
+    lens = _lens(seq_lens)
+    B, L, H, d_c = q_latent.shape
+    T_max = latent_cache.shape[1]
+    out = np.zeros((B, L, H, d_c))
+    lse = np.zeros((B, L, H))
+    for b in range(B):
+        for i in range(L):
+            n = _causal_rows(lens[b], L, i, T_max)
+            o, l = mla_decode_f64(q_latent[b:b + 1, i], q_rope[b:b + 1, i], latent_cache[b:b + 1, :max(n, 1)],
+                                  rope_cache[b:b + 1, :max(n, 1)], np.array([n], dtype=np.int32), scale, lib=lib)
+            out[b, i], lse[b, i] = o[0], l[0]
+    return out, lse
+
+
 def rope_f64(x, positions, base, interleaved, lib=None):
     """Rotary embedding of the last axis of x (fp64 result, same shape).  positions
     holds one position per vector, broadcast over x's leading axes (e.g. [B] for x of

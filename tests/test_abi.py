@@ -206,10 +206,27 @@ def test_mla_paged_rejects_bad_arguments(lib, kw, expected):
 
 @pytest.mark.parametrize("kw,expected", [
     (dict(L=0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(L=513), kb.KVATTN_ERR_UNSUPPORTED),                # batch * q_len > 1024
+    (dict(dc=256), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(e4m3=1, ls=0.0), kb.KVATTN_ERR_INVALID_ARG),
+    (dict(out=A + 16), kb.KVATTN_ERR_INVALID_ARG),           # output overlaps q_latent
+])
+def test_mla_multi_rejects_bad_arguments(lib, kw, expected):
+    a = dict(ql=A, qr=2 * A, lat=3 * A, rope=4 * A, lens=5 * A, T=4096, B=2, L=4, H=128, dc=512, dr=64, e4m3=0,
+             ls=1.0, rs=1.0, out=6 * A, lse=7 * A)
+    a.update(kw)
+    st = lib.kvattn_mla_decode_multi(a["ql"], a["qr"], a["lat"], a["rope"], a["lens"], a["T"], a["B"], a["L"], a["H"],
+                                     a["dc"], a["dr"], 0.0722, a["e4m3"], a["ls"], a["rs"], a["out"], a["lse"], None)
+    assert st == expected
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(L=0), kb.KVATTN_ERR_INVALID_ARG),
     (dict(window=-1), kb.KVATTN_ERR_INVALID_ARG),
-    (dict(L=2, nq=64, nkv=1), kb.KVATTN_ERR_UNSUPPORTED),   # 64 heads x 2 positions > 64 columns
-    (dict(L=2, d=64), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(L=2049), kb.KVATTN_ERR_UNSUPPORTED),               # batch * q_len > 4096
+    (dict(d=96), kb.KVATTN_ERR_UNSUPPORTED),
     (dict(window=5, d=64), kb.KVATTN_ERR_UNSUPPORTED),
+    (dict(window=3, nq=128, nkv=1), kb.KVATTN_ERR_UNSUPPORTED),   # a window needs groups of <= 64
     (dict(q=A + 4), kb.KVATTN_ERR_MISALIGNED),
     (dict(out=A + 16), kb.KVATTN_ERR_INVALID_ARG),          # output overlaps q
 ])
@@ -224,7 +241,8 @@ def test_gqa_multi_rejects_bad_arguments(lib, kw, expected):
 
 @pytest.mark.parametrize("kw,expected", [
     (dict(d=64), kb.KVATTN_ERR_UNSUPPORTED),                 # E4M3 path: head_dim 128 only
-    (dict(L=3, nq=64, nkv=2), kb.KVATTN_ERR_UNSUPPORTED),    # 32 heads x 3 positions > 64 columns
+    (dict(nq=128, nkv=1), kb.KVATTN_ERR_UNSUPPORTED),        # groups of more than 64 heads
+    (dict(L=2049), kb.KVATTN_ERR_UNSUPPORTED),               # batch * q_len > 4096
     (dict(ks=0.0), kb.KVATTN_ERR_INVALID_ARG),
     (dict(vs=-1.0), kb.KVATTN_ERR_INVALID_ARG),
     (dict(ks=float("inf")), kb.KVATTN_ERR_INVALID_ARG),
