@@ -132,3 +132,15 @@ def test_fp8_paged(page_size):
     assert_close(lse.cpu().numpy(), rl, "fp8 paged lse")
     assert torch.equal(out, oc) and torch.equal(lse, lc), "paged and contiguous results differ"
 
+
+
+def test_fp8_multi_token_beyond_64_columns():
+    """32-head groups at 3 new tokens (96 columns): a virtual batch of single-token
+    sequences through the E4M3 kernel."""
+    lens = [1500, 2, 700]
+    cfg, x = fp8_inputs(len(lens), 64, 2, 1500, lens, seed=64)
+    g = torch.Generator().manual_seed(65)
+    q = torch.randn((len(lens), 3, 64, 128), generator=g).to(torch.bfloat16)
+    out, lse, ro, rl = run_fp8(cfg, x, q=q)
+    assert_close(out.cpu().numpy(), ro, "fp8 multi out")
+    assert_close(lse.cpu().numpy(), rl, "fp8 multi lse")

@@ -100,3 +100,34 @@ def test_forced_splits(workers, min_tiles):
 
 def test_workload_full_size():
     run_case(wl.CONFIGS["mla_b32_h128_c512_r64_t4096"])
+
+
+@pytest.mark.parametrize("L", [2, 4])
+def test_multi_token(L):
+    """L new tokens per sequence (causal), including sequences shorter than L (their first
+    queries see nothing)."""
+    cfg = mla("multi", 4, 128, 900, lens=[900, 1, 3, 500])
+    x = wl.make_mla_inputs(cfg, seed=17, poison_tail=True)
+    g = torch.Generator().manual_seed(18)
+    ql = torch.randn((cfg.batch, L, 128, 512), generator=g).to(torch.bfloat16)
+    qr = torch.randn((cfg.batch, L, 128, 64), generator=g).to(torch.bfloat16)
+    out, lse = kb.kvattn_mla_decode_multi(ql.cuda(), qr.cuda(), x["latent_cache"].cuda(), x["rope_cache"].cuda(),
+                                          x["seq_lens"].cuda(), cfg.scale)
+    torch.cuda.synchronize()
+    ro, rl = oracle.mla_decode_multi(ql, qr, x["latent_cache"], x["rope_cache"], x["seq_lens"], cfg.scale)
+    assert_close(out.cpu().numpy(), ro, f"mla multi L{L} out")
+    assert_close(lse.cpu().numpy(), rl, f"mla multi L{L} lse")
+
+
+def test_lengths_past_the_capacity_are_clamped():
+    """seq_lens above max_seq_len attend to the whole cache (clamped), no further."""
+    cfg = mla("clamp", 2, 128, 300, lens=[300, 120])
+    x = wl.make_mla_inputs(cfg, seed=19)
+    d = {k: v.cuda() for k, v in x.items()}
+    big = torch.tensor([5000, 120], dtype=torch.int32, device="cuda")
+    out, lse = kb.kvattn_mla_decode(d["q_latent"], d["q_rope"], d["latent_cache"], d["rope_cache"], big, cfg.scale)
+    torch.cuda.synchronize()
+    ro, rl = oracle.mla_decode(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"], x["seq_lens"],
+                               cfg.scale)
+    assert_close(out.cpu().numpy(), ro, "clamped out")
+    assert_close(lse.cpu().numpy(), rl, "clamped lse")

@@ -172,3 +172,20 @@ def test_append_fp8_then_decode_matches_oracle():
                                    x["rope_scale"])
     assert_close(out.cpu().numpy(), ro, "mla fp8 step out")
     assert_close(lse.cpu().numpy(), rl, "mla fp8 step lse")
+
+
+def test_multi_token_fp8():
+    """Three new tokens per sequence over the E4M3 cache (causal)."""
+    cfg = mla8("multi8", 3, 128, 800, [800, 2, 450])
+    x = wl.make_mla_inputs_fp8(cfg, seed=21, poison_tail=True)
+    g = torch.Generator().manual_seed(22)
+    ql = torch.randn((cfg.batch, 3, 128, 512), generator=g).to(torch.bfloat16)
+    qr = torch.randn((cfg.batch, 3, 128, 64), generator=g).to(torch.bfloat16)
+    out, lse = kb.kvattn_mla_decode_multi(ql.cuda(), qr.cuda(), x["latent_cache"].cuda(), x["rope_cache"].cuda(),
+                                          x["seq_lens"].cuda(), cfg.scale, x["latent_scale"], x["rope_scale"])
+    torch.cuda.synchronize()
+    lat = oracle.e4m3_dequant(x["latent_cache"], x["latent_scale"])
+    rope = oracle.e4m3_dequant(x["rope_cache"], x["rope_scale"])
+    ro, rl = oracle.mla_decode_multi(ql, qr, lat, rope, x["seq_lens"], cfg.scale)
+    assert_close(out.cpu().numpy(), ro, "mla fp8 multi out")
+    assert_close(lse.cpu().numpy(), rl, "mla fp8 multi lse")

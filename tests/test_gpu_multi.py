@@ -32,8 +32,7 @@ def _knobs():
     assert kb.kvattn_read_device_flags() == 0
 
 
-def run_multi(B, L, n_q, n_kv, T, lens, window, seed=0, poison_before=False):
-    d = 128
+def run_multi(B, L, n_q, n_kv, T, lens, window, seed=0, poison_before=False, d=128):
     cfg = wl.GQAConfig("multi", B, n_q, n_kv, d, T, 1.0 / math.sqrt(d), seq_lens=tuple(lens))
     x = wl.make_gqa_inputs(cfg, seed=seed, poison_tail=True)
     g = torch.Generator().manual_seed(seed + 1)
@@ -96,3 +95,21 @@ def test_single_token_matches_decode():
     o2, l2 = kb.kvattn_gqa_decode(d["q"], d["k_cache"], d["v_cache"], d["seq_lens"], cfg.scale)
     torch.cuda.synchronize()
     assert torch.equal(o1[:, 0], o2) and torch.equal(l1[:, 0], l2)
+
+
+# Shapes the multi-token kernel does not take (head_dim 64; a group's heads times the new
+# tokens above 64 columns): the call runs as a virtual batch of single-token sequences.
+VIRTUAL = [
+    # (B, L, n_q, n_kv, T, lens, window, d)
+    (3, 3, 16, 4, 700, (700, 2, 333), 0, 64),
+    (2, 5, 64, 4, 1500, (1500, 3), 0, 128),        # 16 heads x 5 tokens = 80 columns
+    (2, 5, 64, 4, 1500, (1500, 777), 200, 128),    # the same with a window
+    (2, 4, 32, 1, 3000, (3000, 1), 0, 128),        # MQA, 32 heads x 4 tokens
+    (2, 2, 128, 2, 600, (600, 1), 0, 128),         # 64-head groups x 2 tokens
+]
+
+
+@pytest.mark.parametrize("B,L,n_q,n_kv,T,lens,window,d", VIRTUAL,
+                         ids=[f"d{c[7]}_g{c[2] // c[3]}_L{c[1]}_w{c[6]}" for c in VIRTUAL])
+def test_multi_as_virtual_batch(B, L, n_q, n_kv, T, lens, window, d):
+    run_multi(B, L, n_q, n_kv, T, list(lens), window, seed=7, poison_before=window > 0, d=d)
