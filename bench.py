@@ -80,10 +80,10 @@ def step_bytes(cfg, lens):
     """Algorithmic bytes of one step: q + touched cache rows + out (fp32) + lse (fp32)."""
     lens = [min(max(int(x), 0), cfg.max_seq_len) for x in lens]
     if isinstance(cfg, wl.MLAConfig):
-        q = cfg.batch * cfg.n_heads * (cfg.latent_dim + cfg.rope_dim) * 2
+        q = QLEN * cfg.batch * cfg.n_heads * (cfg.latent_dim + cfg.rope_dim) * 2
         kv = sum(lens) * (cfg.latent_dim + cfg.rope_dim) * (1 if KV8 else 2)
-        out = cfg.batch * cfg.n_heads * cfg.latent_dim * 4
-        lse = cfg.batch * cfg.n_heads * 4
+        out = QLEN * cfg.batch * cfg.n_heads * cfg.latent_dim * 4
+        lse = QLEN * cfg.batch * cfg.n_heads * 4
     else:
         q = QLEN * cfg.batch * cfg.n_q_heads * cfg.head_dim * 2
         kv = 2 * sum(active_rows(n) for n in lens) * cfg.n_kv_heads * cfg.head_dim * (1 if KV8 else 2)
@@ -96,7 +96,8 @@ def step_flops(cfg, lens):
     """Algorithmic flops: 2 per multiply-add of the score and the value products."""
     lens = [min(max(int(x), 0), cfg.max_seq_len) for x in lens]
     if isinstance(cfg, wl.MLAConfig):
-        return sum(lens) * cfg.n_heads * 2 * ((cfg.latent_dim + cfg.rope_dim) + cfg.latent_dim)
+        vis = sum(max(0, n - QLEN + 1 + i) for n in lens for i in range(QLEN))
+        return vis * cfg.n_heads * 2 * ((cfg.latent_dim + cfg.rope_dim) + cfg.latent_dim)
     return sum(visible_pairs(n) for n in lens) * cfg.n_q_heads * 4 * cfg.head_dim
 
 
@@ -281,10 +282,16 @@ def to_pages(cache, page_size, seq_axis, perm):
 
 def host_inputs(cfg, seed):
     """The workload's seeded inputs (CPU) with the variant applied."""
-    if (QLEN > 1 or WINDOW) and isinstance(cfg, wl.MLAConfig):
-        raise ValueError("several new tokens and windows: GQA workloads only")
+    if WINDOW and isinstance(cfg, wl.MLAConfig):
+        raise ValueError("windows: GQA workloads only")
     if isinstance(cfg, wl.MLAConfig):
-        return wl.make_mla_inputs_fp8(cfg, seed=seed) if KV8 else wl.make_mla_inputs(cfg, seed=seed)
+        x = wl.make_mla_inputs_fp8(cfg, seed=seed) if KV8 else wl.make_mla_inputs(cfg, seed=seed)
+        if QLEN > 1:
+            g = torch.Generator().manual_seed(seed + 29)
+            x["q_latent"] = torch.randn((cfg.batch, QLEN, cfg.n_heads, cfg.latent_dim),
+                                        generator=g).to(torch.bfloat16)
+            x["q_rope"] = torch.randn((cfg.batch, QLEN, cfg.n_heads, cfg.rope_dim), generator=g).to(torch.bfloat16)
+        return x
     x = wl.make_gqa_inputs_fp8(cfg, seed=seed) if KV8 else wl.make_inputs(cfg, seed=seed)
     if QLEN > 1:
         g = torch.Generator().manual_seed(seed + 29)
@@ -320,6 +327,12 @@ def device_inputs(cfg, seed):
 
 def make_call(cfg, d, out, lse, stream):
     from mla_kv_cache_b200 import binding as kb
+    if QLEN > 1 and isinstance(cfg, wl.MLAConfig):
+        if PAGED:
+            raise ValueError("the MLA multi-token entry point takes a contiguous cache")
+        return lambda: kb.kvattn_mla_decode_multi(d["q_latent"], d["q_rope"], d["latent_cache"], d["rope_cache"],
+                                                  d["seq_lens"], cfg.scale, d.get("latent_scale"),
+                                                  d.get("rope_scale"), out=out, lse=lse, stream=stream)
     if KV8 and isinstance(cfg, wl.MLAConfig):
         if PAGED:
             return lambda: kb.kvattn_mla_decode_fp8_paged(d["q_latent"], d["q_rope"], d["latent_cache_pages"],
@@ -362,6 +375,8 @@ def make_call(cfg, d, out, lse, stream):
 
 def out_shapes(cfg):
     if isinstance(cfg, wl.MLAConfig):
+        if QLEN > 1:
+            return (cfg.batch, QLEN, cfg.n_heads, cfg.latent_dim), (cfg.batch, QLEN, cfg.n_heads)
         return (cfg.batch, cfg.n_heads, cfg.latent_dim), (cfg.batch, cfg.n_heads)
     if q4d():
         return (cfg.batch, QLEN, cfg.n_q_heads, cfg.head_dim), (cfg.batch, QLEN, cfg.n_q_heads)
@@ -371,6 +386,14 @@ def out_shapes(cfg):
 def oracle_step(cfg, x, ids):
     """The oracle on sequences `ids` of the workload (variant applied)."""
     import oracle
+    if isinstance(cfg, wl.MLAConfig) and QLEN > 1:
+        lat, rope = x["latent_cache"], x["rope_cache"]
+        if KV8:
+            lat = oracle.e4m3_dequant(lat, x["latent_scale"])
+            rope = oracle.e4m3_dequant(rope, x["rope_scale"])
+        sel = list(ids)
+        return oracle.mla_decode_multi(x["q_latent"][sel], x["q_rope"][sel], lat[sel], rope[sel],
+                                       x["seq_lens"][sel], cfg.scale)
     if isinstance(cfg, wl.MLAConfig):
         if KV8:
             return oracle.mla_decode_fp8(x["q_latent"], x["q_rope"], x["latent_cache"], x["rope_cache"],
