@@ -181,6 +181,76 @@ int encode_map_3d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t di
     return KVATTN_OK;
 }
 
+// A strided view of a 16-bit tensor (rank 3..5): dims[0] contiguous, strides[i] the byte
+// stride of dims[i + 1] -- not necessarily increasing, e.g. a [rows][chunks][64] view of
+// rows whose chunk dimension strides 128 bytes inside a row, so that one copy moves
+// several 64-column chunks of a row block.  Cached like make_map_3d.
+struct ViewKey {
+    const void *base;
+    int rank;
+    uint64_t dims[5], strides[4];
+    uint32_t box[5];
+    bool operator==(const ViewKey &o) const {
+        if (base != o.base || rank != o.rank) return false;
+        for (int i = 0; i < 5; ++i)
+            if (dims[i] != o.dims[i] || box[i] != o.box[i]) return false;
+        for (int i = 0; i < 4; ++i)
+            if (strides[i] != o.strides[i]) return false;
+        return true;
+    }
+};
+struct ViewEntry {
+    ViewKey key;
+    CUtensorMap map;
+    bool valid;
+};
+constexpr int kViewCache = 16;
+thread_local ViewEntry t_views[kViewCache];
+thread_local int t_view_next = 0;
+
+int make_map_view(CUtensorMap *map, const void *base, int rank, const uint64_t *dims, const uint64_t *strides,
+                  const uint32_t *box) {
+    ViewKey key = {};
+    key.base = base;
+    key.rank = rank;
+    for (int i = 0; i < rank; ++i) {
+        key.dims[i] = dims[i];
+        key.box[i] = box[i];
+        if (i + 1 < rank) key.strides[i] = strides[i];
+    }
+    for (int i = 0; i < kViewCache; ++i)
+        if (t_views[i].valid && t_views[i].key == key) {
+            *map = t_views[i].map;
+            return KVATTN_OK;
+        }
+    auto fn = encode_fn();
+    if (!fn) {
+        snprintf(t_detail, sizeof(t_detail), "cuTensorMapEncodeTiled unavailable");
+        return KVATTN_ERR_CUDA;
+    }
+    cuuint64_t d[5], st[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+        if (i + 1 < rank) st[i] = strides[i];
+    }
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), d, st, bx, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(t_detail, sizeof(t_detail), "cuTensorMapEncodeTiled (%d-D view) failed (%d)", rank, (int)r);
+        return KVATTN_ERR_CUDA;
+    }
+    ViewEntry &e = t_views[t_view_next];
+    t_view_next = (t_view_next + 1) % kViewCache;
+    e.key = key;
+    e.map = *map;
+    e.valid = true;
+    return KVATTN_OK;
+}
+
 // 4-D bf16 tensor [dim3][dim2][dim1][dim0] (dim0 fastest, densely packed), box
 // {box0, box1, box2, 1}.  Not cached (used once per call).
 int make_map_4d(CUtensorMap *map, const void *base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint64_t dim3,
@@ -690,24 +760,52 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
     if (cache.e4m3) {
         // E4M3 codes, two to an element of the map: a box of [64 rows x 128 codes]; the
         // RoPE map is 64 codes wide, so its box reads 64 codes and zero-fills the other 64
-        st = make_map_3d(&maps.lat, cache.lat, 256, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
-                         CU_TENSOR_MAP_SWIZZLE_128B);
-        if (st != KVATTN_OK) return st;
         st = make_map_3d(&maps.rope, cache.rope, 32, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
                          CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != KVATTN_OK) return st;
-        maps.qlat = maps.lat;   // (the query is read by the threads)
-        maps.qrope = maps.lat;
-    } else {
-        st = make_map_3d(&maps.lat, cache.lat, 512, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
-                         CU_TENSOR_MAP_SWIZZLE_128B);
+        // key slot: the 4 latent chunks of a row block in one copy; value slot: chunks r and
+        // 2 + r (128-byte units of a 512-byte row) in one copy
+        const uint64_t rowb = 512, pageb = rowb * (uint64_t)cache.page_size;
+        const uint64_t kd[4] = {64, (uint64_t)cache.page_size, 4, (uint64_t)cache.pages};
+        const uint64_t ks[3] = {rowb, 128, pageb};
+        const uint32_t kb[4] = {64, (uint32_t)mla::SUB, 4, 1};
+        st = make_map_view(&maps.latk, cache.lat, 4, kd, ks, kb);
         if (st != KVATTN_OK) return st;
+        maps.latk2 = maps.latk;
+        const uint64_t vd[5] = {64, (uint64_t)cache.page_size, 2, 2, (uint64_t)cache.pages};
+        const uint64_t vs[4] = {rowb, 128, 256, pageb};
+        const uint32_t vb[5] = {64, (uint32_t)mla::SUB, 1, 2, 1};
+        st = make_map_view(&maps.latv, cache.lat, 5, vd, vs, vb);
+        if (st != KVATTN_OK) return st;
+        maps.qlatc = maps.latk;   // (the query is read by the threads)
+        maps.qrope = maps.latk;
+    } else {
         st = make_map_3d(&maps.rope, cache.rope, 64, cache.page_size, (uint64_t)cache.pages, 64, mla::SUB,
                          CU_TENSOR_MAP_SWIZZLE_128B);
         if (st != KVATTN_OK) return st;
-        st = make_map_3d(&maps.qlat, q_latent, 512, n_heads, batch, 64, mla::HC, CU_TENSOR_MAP_SWIZZLE_128B);
-        if (st != KVATTN_OK) return st;
         st = make_map_3d(&maps.qrope, q_rope, 64, n_heads, batch, 64, mla::HC, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (st != KVATTN_OK) return st;
+        // [rows][8 chunks][64] views of the latent rows: key slots of 3 and 2 chunks, the
+        // value slot (chunks 4j + 2r + {0, 1}, j = 0, 1) and the query's chunks 4..7, each
+        // in one copy
+        const uint64_t rowb = 1024, pageb = rowb * (uint64_t)cache.page_size;
+        const uint64_t kd[4] = {64, (uint64_t)cache.page_size, 8, (uint64_t)cache.pages};
+        const uint64_t ks[3] = {rowb, 128, pageb};
+        const uint32_t kb3[4] = {64, (uint32_t)mla::SUB, 3, 1};
+        const uint32_t kb2[4] = {64, (uint32_t)mla::SUB, 2, 1};
+        st = make_map_view(&maps.latk, cache.lat, 4, kd, ks, kb3);
+        if (st != KVATTN_OK) return st;
+        st = make_map_view(&maps.latk2, cache.lat, 4, kd, ks, kb2);
+        if (st != KVATTN_OK) return st;
+        const uint64_t vd[5] = {64, (uint64_t)cache.page_size, 4, 2, (uint64_t)cache.pages};
+        const uint64_t vs[4] = {rowb, 128, 512, pageb};
+        const uint32_t vb[5] = {64, (uint32_t)mla::SUB, 2, 2, 1};
+        st = make_map_view(&maps.latv, cache.lat, 5, vd, vs, vb);
+        if (st != KVATTN_OK) return st;
+        const uint64_t qd[4] = {64, (uint64_t)n_heads, 8, (uint64_t)batch};
+        const uint64_t qs[3] = {1024, 128, 1024 * (uint64_t)n_heads};
+        const uint32_t qb[4] = {64, (uint32_t)mla::HC, (uint32_t)mla::NQS - 1, 1};
+        st = make_map_view(&maps.qlatc, q_latent, 4, qd, qs, qb);
         if (st != KVATTN_OK) return st;
     }
     const void *kern = cache.e4m3 ? reinterpret_cast<const void *>(mla_decode_kernel<true>)

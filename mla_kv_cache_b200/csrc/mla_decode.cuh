@@ -185,8 +185,13 @@ struct MlaParams {
     float rope_scale;           // E4M3 cache: a RoPE code's value is code * rope_scale
 };
 
+// rope / qrope: [pages][page rows][columns] boxes of [64 rows x 128 bytes]; latk / latk2:
+// views [pages][chunk][page rows][64] whose chunk dimension strides 128 bytes inside a row
+// (one copy moves a key slot's latent chunks: 3 and 2 of them in bf16, 4 in E4M3); latv: a
+// 5-D view that moves a value slot in one copy; qlatc: the query's shared-memory latent
+// chunks (bf16) in one copy.
 struct MlaMaps {
-    CUtensorMap lat, rope, qlat, qrope;
+    CUtensorMap rope, qrope, latk, latk2, latv, qlatc;
 };
 
 namespace mla {
@@ -298,9 +303,7 @@ __device__ __forceinline__ void key_producer(const MlaParams &p, const MlaMaps &
                 if (lead) mbar_arrive_expect_tx(&bars->kfull[slot], 2 * e4::KSLOT);
                 const uint32_t bar = map_to_rank(smem_u32(&bars->kfull[slot]), 0);
                 uint8_t *dst = c.smem + e4::OFF_SR + slot * e4::KSLOT;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch)   // (the maps count two codes as one element)
-                    tma_load_3d_pair(dst + ch * CHUNK, &m.lat, bar, 64 * ch, hs.y, hs.page, pol_keep);
+                tma_load_4d_pair(dst, &m.latk, bar, 0, hs.y, 0, hs.page, pol_keep);   // latent chunks 0..3
                 tma_load_3d_pair(dst + 4 * CHUNK, &m.rope, bar, 0, hs.y, hs.page, pol_keep);
             }
             continue;
@@ -311,9 +314,7 @@ __device__ __forceinline__ void key_producer(const MlaParams &p, const MlaMaps &
             break;
         }
         if (lead) mbar_arrive_expect_tx(&bars->qfull, 2 * NQS * CHUNK);
-        for (int ch = 0; ch < NQS - 1; ++ch)
-            tma_load_3d_pair(c.smem + OFF_Q + ch * CHUNK, &m.qlat, qfull0, 64 * (NQT + ch), HC * (int)c.r, pc.b,
-                             pol_keep);
+        tma_load_4d_pair(c.smem + OFF_Q, &m.qlatc, qfull0, 0, HC * (int)c.r, NQT, pc.b, pol_keep);   // chunks 4..7
         tma_load_3d_pair(c.smem + OFF_Q + (NQS - 1) * CHUNK, &m.qrope, qfull0, 0, HC * (int)c.r, pc.b, pol_keep);
         for (int lt = pc.lt0; lt < pc.lt1 && ok; ++lt) {
             const HalfSrc hs = half_source(p, pc.b, len, lt, (int)c.r);
@@ -332,12 +333,11 @@ __device__ __forceinline__ void key_producer(const MlaParams &p, const MlaMaps &
                 if (lead) mbar_arrive_expect_tx(&bars->kfull[s], 2 * KSLOT);
                 const uint32_t bar = map_to_rank(smem_u32(&bars->kfull[s]), 0);
                 uint8_t *dst = c.smem + OFF_SR + s * KSLOT;
-                for (int e = 0; e < 3; ++e) {
-                    const int ch = 3 * s + e;
-                    if (ch < 8)
-                        tma_load_3d_pair(dst + e * CHUNK, &m.lat, bar, 64 * ch, hs.y, hs.page, pol_keep);
-                    else
-                        tma_load_3d_pair(dst + e * CHUNK, &m.rope, bar, 0, hs.y, hs.page, pol_keep);
+                if (s < NKS - 1) {   // latent chunks 3s .. 3s + 2
+                    tma_load_4d_pair(dst, &m.latk, bar, 0, hs.y, 3 * s, hs.page, pol_keep);
+                } else {             // latent chunks 6, 7 and the RoPE chunk
+                    tma_load_4d_pair(dst, &m.latk2, bar, 0, hs.y, 6, hs.page, pol_keep);
+                    tma_load_3d_pair(dst + 2 * CHUNK, &m.rope, bar, 0, hs.y, hs.page, pol_keep);
                 }
             }
         }
@@ -376,17 +376,9 @@ __device__ __forceinline__ void value_producer(const MlaParams &p, const MlaMaps
                 if (lead) mbar_arrive_expect_tx(&bars->vfull[h], 2 * vslot);
                 const uint32_t bar = map_to_rank(smem_u32(&bars->vfull[h]), 0);
                 uint8_t *dst = c.smem + (KV8 ? e4::OFF_PV : OFF_PV) + h * vslot;
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {   // latent block j: this CTA's 128 columns of it
-                    if constexpr (KV8) {        // one box of 128 codes (64 two-code elements)
-                        tma_load_3d_pair(dst + j * CHUNK, &m.lat, bar, 128 * j + 64 * (int)c.r, hs.y, hs.page,
-                                         pol_last);
-                    } else {
-                        const int x = 256 * j + 128 * (int)c.r;
-                        tma_load_3d_pair(dst + 2 * j * CHUNK, &m.lat, bar, x, hs.y, hs.page, pol_last);
-                        tma_load_3d_pair(dst + (2 * j + 1) * CHUNK, &m.lat, bar, x + 64, hs.y, hs.page, pol_last);
-                    }
-                }
+                // this CTA's columns of latent blocks j = 0, 1 in one copy: bf16 chunks
+                // 4j + 2r + {0, 1}, E4M3 128-code chunks 2j + r; shared memory [j][chunk]
+                tma_load_5d_pair(dst, &m.latv, bar, 0, hs.y, (KV8 ? 1 : 2) * (int)c.r, 0, hs.page, pol_last);
             }
         }
     }
@@ -664,13 +656,29 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         return unit < 32 ? reinterpret_cast<const uint4 *>(p.q_latent + row * 512) + 2 * unit + (i & 1)
                          : reinterpret_cast<const uint4 *>(p.q_rope + row * 64) + 2 * (unit - 32) + (i & 1);
     };
-    // first pass: the largest magnitudes of this thread's latent and RoPE values
+    // The 16 bytes of unit u's high part; its remainder's are e4::QPART further on.  The
+    // unit's 32 raw bytes (bf16) are first parked in those same bytes, which no other
+    // thread reads or writes, and converted in place.
+    auto q8_dst = [&](int u) -> uint8_t * {
+        const int box = u < 32 ? u >> 3 : 4;
+        const int g = u < 32 ? u & 7 : u - 32;
+        return c.smem + e4::OFF_Q + box * CHUNK + hh * 128 + ((g ^ (hh & 7)) << 4);
+    };
+    // First pass (the query boxes free): the 18 asynchronous copies all in flight at once,
+    // then the largest magnitudes of this thread's latent and RoPE values.
     auto q8_load = [&](int b, float &mxl, float &mxr) {
+#pragma unroll
+        for (int i = 0; i < 18; ++i) {
+            uint8_t *d = q8_dst(9 * part + (i >> 1)) + (i & 1) * e4::QPART;
+            if (realq) cp_async16(d, q8_src(b, i));
+            else *reinterpret_cast<uint4 *>(d) = make_uint4(0, 0, 0, 0);
+        }
+        cp_async_wait_all();
         mxl = 0.f;
         mxr = 0.f;
 #pragma unroll
         for (int i = 0; i < 18; ++i) {
-            const uint4 x = realq ? __ldg(q8_src(b, i)) : make_uint4(0, 0, 0, 0);
+            const uint4 x = *reinterpret_cast<const uint4 *>(q8_dst(9 * part + (i >> 1)) + (i & 1) * e4::QPART);
             const uint32_t w[4] = {x.x, x.y, x.z, x.w};
             float m = 0.f;
 #pragma unroll
@@ -678,8 +686,8 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             if (9 * part + (i >> 1) < 32) mxl = fmaxf(mxl, m); else mxr = fmaxf(mxr, m);
         }
     };
-    // second pass (the query loaded again, from L1): the head's scales, the split, the stores
-    auto q8_store = [&](int b, float mxl, float mxr) -> bool {
+    // Second pass: the head's scales, then each parked unit split in place.
+    auto q8_store = [&](float mxl, float mxr) -> bool {
         qx_buf[part * HC + hh] = mxl;
         qx_buf[4 * HC + part * HC + hh] = mxr;
         __syncwarp();
@@ -705,9 +713,9 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         for (int i = 0; i < 9; ++i) {
             const int unit = 9 * part + i;
             const float up = __int_as_float((127 + (unit < 32 ? el : er)) << 23);
-            uint4 xs[2];
-            xs[0] = realq ? __ldg(q8_src(b, 2 * i)) : make_uint4(0, 0, 0, 0);
-            xs[1] = realq ? __ldg(q8_src(b, 2 * i + 1)) : make_uint4(0, 0, 0, 0);
+            uint8_t *dst = q8_dst(unit);
+            const uint4 xs[2] = {*reinterpret_cast<const uint4 *>(dst),
+                                 *reinterpret_cast<const uint4 *>(dst + e4::QPART)};
             uint32_t hw[4], lw[4];
 #pragma unroll
             for (int t = 0; t < 4; ++t) {   // codes 4t .. 4t + 3 of the unit: words 2t, 2t + 1 of the pair
@@ -719,9 +727,6 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
                 hw[t] = (uint32_t)h0 | ((uint32_t)h1 << 16);
                 lw[t] = (uint32_t)l0 | ((uint32_t)l1 << 16);
             }
-            const int box = unit < 32 ? unit >> 3 : 4;
-            const int g = unit < 32 ? unit & 7 : unit - 32;
-            uint8_t *dst = c.smem + e4::OFF_Q + box * CHUNK + hh * 128 + ((g ^ (hh & 7)) << 4);
             *reinterpret_cast<uint4 *>(dst) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
             *reinterpret_cast<uint4 *>(dst + e4::QPART) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
@@ -884,7 +889,7 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             if constexpr (KV8) {
                 float mxl, mxr;
                 q8_load(pc.b, mxl, mxr);
-                if (!q8_store(pc.b, mxl, mxr)) return;
+                if (!q8_store(mxl, mxr)) return;
             } else {
                 uint32_t v0[32], v1[32];
                 load_q(pc.b, v0, v1);
@@ -899,10 +904,16 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         for (int t = 0; t < nt; ++t) {
             const int kt = k + t;
             const int sb = kt & 1;
-            if (t == nt - 1 && next_b >= 0 && realq) {
-                const uint4 *qn = q_row(next_b);
-                prefetch_l2(qn);
-                prefetch_l2(qn + 8);
+            if (t == nt - 1 && next_b >= 0 && realq) {   // the next query into L2
+                if constexpr (KV8) {
+                    prefetch_l2(q8_src(next_b, 0));
+                    prefetch_l2(q8_src(next_b, 8));
+                    prefetch_l2(q8_src(next_b, 16));
+                } else {
+                    const uint4 *qn = q_row(next_b);
+                    prefetch_l2(qn);
+                    prefetch_l2(qn + 8);
+                }
             }
             // first valid column of this thread's 32 (masked: rows of the half below lo)
             const int lo = half_source(p, pc.b, len, pc.lt0 + t, half).lo - 32 * cg;
@@ -967,18 +978,19 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             uint32_t whi[16], wlo[16], wmid[8];
             float ls4[4] = {0.f, 0.f, 0.f, 0.f};
             const float m_off = KV8 ? e4::P_LOG2 - m_new : -m_new;
+            uint32_t ph = 0, pm = 0, pl = 0;   // E4M3: the codes of the previous (even) pair
             auto put = [&](int j, float a, float b) {
                 if constexpr (KV8) {
                     uint16_t h2, m2, l2;
                     split3_e4m3x2(a, b, h2, m2, l2);
                     if (j & 1) {
-                        whi[j >> 1] |= (uint32_t)h2 << 16;
-                        wmid[j >> 1] |= (uint32_t)m2 << 16;
-                        wlo[j >> 1] |= (uint32_t)l2 << 16;
+                        whi[j >> 1] = ph | ((uint32_t)h2 << 16);
+                        wmid[j >> 1] = pm | ((uint32_t)m2 << 16);
+                        wlo[j >> 1] = pl | ((uint32_t)l2 << 16);
                     } else {
-                        whi[j >> 1] = h2;
-                        wmid[j >> 1] = m2;
-                        wlo[j >> 1] = l2;
+                        ph = h2;
+                        pm = m2;
+                        pl = l2;
                     }
                 } else {
                     split_bf16x2(a, b, whi[j], wlo[j]);
@@ -1067,9 +1079,9 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         if (next_b >= 0) {
             if constexpr (KV8) {
                 float mxl, mxr;
-                q8_load(next_b, mxl, mxr);
                 if (!wait_local(&bars->qempty, (uint32_t)pi & 1u, FLAG_MMA_WAIT, c)) return;
-                if (!q8_store(next_b, mxl, mxr)) return;
+                q8_load(next_b, mxl, mxr);
+                if (!q8_store(mxl, mxr)) return;
             } else {
                 uint32_t v0[32], v1[32];
                 load_q(next_b, v0, v1);
@@ -1197,10 +1209,12 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
     }
     if (warp == 2) build_tile_prefix(p.seq_lens, p.B, p.T_max, TILE, s_prefix, lane);
     if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&maps.lat);
+        prefetch_tensormap(&maps.latk);
+        prefetch_tensormap(&maps.latv);
         prefetch_tensormap(&maps.rope);
+        if (!KV8) prefetch_tensormap(&maps.latk2);
         if (!KV8) {
-            prefetch_tensormap(&maps.qlat);
+            prefetch_tensormap(&maps.qlatc);
             prefetch_tensormap(&maps.qrope);
         }
     }
