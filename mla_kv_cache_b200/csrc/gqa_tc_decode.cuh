@@ -117,8 +117,7 @@ struct Bars {
     uint64_t qconv[2];    // E4M3 cache: the MMA warp has split that block (and its 2^-e)
     uint64_t sready[2];   // scores of a tile in TMEM buffer (tile & 1)
     uint64_t sfree[2];    // the softmax threads have read that buffer
-    uint64_t pready[2];   // P^T written (and O^T rescaled): the value product may run
-    uint64_t odone[2];    // value product of a tile (parity tile & 1) finished
+    uint64_t pready[4];   // P^T of tile kt (index kt & 3) written, O^T rescaled: its value product may run
     uint64_t ofree;       // the epilogue has read O^T
     uint64_t grp[2];      // barrier of a softmax group's four warps
     uint64_t hand[2];     // running max after a tile of group g published (two groups)
@@ -422,16 +421,19 @@ __device__ __forceinline__ void issue_values(const Ctx &c, int kt, bool first) {
             umma_ss(c.tmem + L::TM_O, a, b, idesc_pv, (!first || kk > 0) ? 1u : 0u);
         }
     }
-    umma_commit(&c.bars->empty[s]);
-    umma_commit(&c.bars->odone[kt & 1]);
+    umma_commit(&c.bars->empty[s]);   // frees the stage; also tells the softmax that O^T has this tile
 }
 
 // The issuer never blocks on one product while the other could go: it tests whether
 // the next score product (its tile landed, its TMEM buffer free) or the next value
 // product (P^T written; at a piece start, O^T read out) may run and issues whatever is
-// ready.  Score products run at most two tiles ahead of value products -- the order a
-// blocking loop would give -- which keeps every tested barrier within one phase of the
-// tested parity.  Idle time is bounded like every other wait.  The whole warp runs the
+// ready.  Score products run at most three tiles ahead of value products, so a softmax
+// group finds its next tile's scores waiting when it finishes a tile (the two TMEM score
+// buffers are guarded by sfree); with four P^T-ready barriers (tile & 3) every tested
+// barrier stays within one phase of the tested parity.  A value product ends with one
+// commit, on its stage's empty barrier, which the softmax warps also wait on before they
+// touch O^T (a commit costs the issuing thread ~300 cycles).  Idle time is bounded like
+// every other wait.  The whole warp runs the
 // loop over pieces (with an E4M3 cache its 32 lanes split each query block); lane 0
 // alone issues.
 template <int NR, bool KV8>
@@ -459,7 +461,7 @@ __device__ __forceinline__ void mma_issuer(const GqaParams &p, const Ctx &c, int
             long long idle_since = clock64();
             while (nv < nt) {
                 bool progressed = false;
-                if (nq < nt && nq < nv + 2) {
+                if (nq < nt && nq < nv + 3) {
                     const int kt = k + nq;
                     if (mbar_test(&bars->full[kt % NST], (uint32_t)(kt / NST) & 1u) &&
                         (kt < 2 || mbar_test(&bars->sfree[kt & 1], (uint32_t)((kt >> 1) - 1) & 1u))) {
@@ -471,7 +473,7 @@ __device__ __forceinline__ void mma_issuer(const GqaParams &p, const Ctx &c, int
                 }
                 if (nv < nq) {
                     const int kt = k + nv;
-                    if (mbar_test(&bars->pready[kt & 1], (uint32_t)(kt >> 1) & 1u) &&
+                    if (mbar_test(&bars->pready[kt & 3], (uint32_t)(kt >> 2) & 1u) &&
                         (nv > 0 || pi == 0 || mbar_test(&bars->ofree, (uint32_t)(pi - 1) & 1u))) {
                         issue_values<NR, KV8>(c, kt, nv == 0);
                         ++nv;
@@ -725,7 +727,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
             fence_proxy_async_smem();
             // ---- rescale the affected columns of O^T (after the previous tile's value product)
             if (any_o != 0) {
-                if (!warp_all(mbar_wait(&bars->odone[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u, FLAG_MMA_WAIT,
+                if (!warp_all(mbar_wait(&bars->empty[(kt - 1) % NST], (uint32_t)((kt - 1) / NST) & 1u, FLAG_MMA_WAIT,
                                         c.abort_flag)))
                     return;
                 tc_fence_after();
@@ -754,7 +756,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
                 tmem_wait_st();
             }
             tc_fence_before();
-            warp_arrive(&bars->pready[sb], lane);
+            warp_arrive(&bars->pready[kt & 3], lane);
         }
         k += nt;
 
@@ -801,7 +803,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
         }
         if (!all_sync()) return;
         const int klast = k - 1;
-        if (!warp_all(mbar_wait(&bars->odone[klast & 1], (uint32_t)(klast >> 1) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
+        if (!warp_all(mbar_wait(&bars->empty[klast % NST], (uint32_t)(klast / NST) & 1u, FLAG_MMA_WAIT, c.abort_flag)))
             return;
         tc_fence_after();
         // 16-column chunks of O^T, taken by the groups in turn
@@ -858,7 +860,7 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
             mbar_init(&bars->sready[i], 1);
             mbar_init(&bars->sfree[i], 4);        // the four warps of the tile's group
             mbar_init(&bars->pready[i], 4);
-            mbar_init(&bars->odone[i], 1);
+            mbar_init(&bars->pready[2 + i], 4);
             mbar_init(&bars->grp[i], 4);
             mbar_init(&bars->hand[i], (NR + 31) / 32);   // the group's warps holding owners
         }

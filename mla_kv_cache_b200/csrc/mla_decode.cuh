@@ -208,24 +208,6 @@ struct Ctx {
     long long p0, p1;
 };
 
-// Tiles per worker for a batch whose sequences all have n tiles, given the balanced
-// share w0: n / k for the largest k dividing n with n / k >= w0, or the smallest multiple
-// of n not below w0 -- kept only if it adds at most max(2, w0 / 4) tiles to the share.
-__device__ __forceinline__ long long uniform_tiles_per_worker(long long w0, int n) {
-    long long w = n;
-    if (w0 >= n) {
-        w = ((w0 + n - 1) / n) * n;
-    } else {
-        for (int k = (int)(n / w0); k > 1; --k)
-            if (n % k == 0) {
-                w = n / k;
-                break;
-            }
-    }
-    const long long slack = w0 / 4 > 2 ? w0 / 4 : 2;
-    return w - w0 <= slack ? w : w0;
-}
-
 // Merge counters of the split sequences: one per (sequence, CTA rank, softmax warp), each
 // counting the workers whose partial block of that warp has been written in the call
 // numbered by its high 32 bits.  Zero at load; a call's first arrival re-tags it.
@@ -1237,14 +1219,7 @@ mla_decode_kernel(const MlaParams p, const __grid_constant__ MlaMaps maps) {
     // sequence in k equal parts, or whole sequences): a boundary inside a worker's range
     // costs a partial result, its merge and a pipeline drain, more than the few tiles the
     // coarser split adds.
-    long long W = tiles_per_worker(total, p.workers, p.min_tiles);
-    {
-        const int n0 = s_prefix[1] - s_prefix[0];
-        int same = 1;
-        for (int i = tid; i < p.B; i += NTHREADS) same &= (s_prefix[i + 1] - s_prefix[i]) == n0;
-        same = __syncthreads_and(same);
-        if (same && n0 > 0) W = uniform_tiles_per_worker(W, n0);
-    }
+    const long long W = split_tiles(total, p.workers, p.min_tiles, uniform_tile_count(s_prefix, p.B));
     c.W = W;
     c.p0 = (long long)c.worker * W;
     c.p1 = (c.p0 + W < total) ? c.p0 + W : total;

@@ -128,6 +128,42 @@ __device__ __forceinline__ long long tiles_per_worker(long long total, int worke
     return w;
 }
 
+// When every sequence has the same number of tiles n (per unit), the share w0 may be
+// rounded so that worker boundaries fall on unit boundaries or cut units into equal
+// parts (a multiple or a divisor of n), if that adds at most max(2, w0 / 4) tiles: a
+// boundary inside a worker's range costs a partial result, its merge and a pipeline
+// restart, more than the few tiles the coarser split adds.
+__device__ __forceinline__ long long uniform_tiles_per_worker(long long w0, int n) {
+    long long w = n;
+    if (w0 >= n) {
+        w = ((w0 + n - 1) / n) * n;
+    } else {
+        for (int k = (int)(n / w0); k > 1; --k)
+            if (n % k == 0) {
+                w = n / k;
+                break;
+            }
+    }
+    const long long slack = w0 / 4 > 2 ? w0 / 4 : 2;
+    return w - w0 <= slack ? w : w0;
+}
+// The MLA kernel's work split: tiles_per_worker, rounded as above when n_uniform (the
+// common tile count of every sequence) is > 0.  (The GQA kernels keep tiles_per_worker:
+// measured, the rounding cost them more than the cuts it removed.)
+__device__ __forceinline__ long long split_tiles(long long total, int workers, int min_tiles, int n_uniform) {
+    const long long w = tiles_per_worker(total, workers, min_tiles);
+    return n_uniform > 0 ? uniform_tiles_per_worker(w, n_uniform) : w;
+}
+// The common tile count of every sequence from a tile prefix (0 if they differ or are
+// empty); block-wide (every thread of the block must call it).
+__device__ __forceinline__ int uniform_tile_count(const int *s_prefix, int B) {
+    const int n0 = s_prefix[1] - s_prefix[0];
+    int same = 1;
+    for (int i = threadIdx.x; i < B; i += blockDim.x) same &= (s_prefix[i + 1] - s_prefix[i]) == n0;
+    same = __syncthreads_and(same);
+    return same && n0 > 0 ? n0 : 0;
+}
+
 // Layout of the published decomposition at the start of the workspace.
 struct MetaView {
     long long *w_total;  // [0] = W, [1] = total
