@@ -46,6 +46,7 @@ struct GqaParams {
     int q_len;                  // new tokens per sequence (1: single-token decode)
     int window;                 // sliding window in tokens (0: none)
     float k_scale, v_scale;     // E4M3 cache: value = code * scale (1 for a bf16 cache)
+    int unit_mode;              // warp kernel: worker u takes exactly unit u (no partials, no combine)
 };
 
 template <int D, int MT>
@@ -119,7 +120,7 @@ gqa_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap,
 
     const long long total = (long long)s_prefix[p.B] * U;
     const long long W = tiles_per_worker(total, p.workers, p.min_tiles);
-    if (blockIdx.x == 0) {
+    if (blockIdx.x == 0 && !p.unit_mode) {
         MetaView mv = meta_view(p.ws_meta);
         if (tid == 0) { mv.w_total[0] = W; mv.w_total[1] = total; }
         for (int i = tid; i <= p.B; i += C::NTHREADS) mv.prefix[i] = s_prefix[i];
@@ -127,8 +128,29 @@ gqa_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap,
     // The combine kernel may be scheduled now; it waits for this grid to finish.
     pdl_launch_dependents();
 
-    const long long p0 = (long long)blockIdx.x * W;
-    const long long p1 = (p0 + W < total) ? p0 + W : total;
+    long long p0 = (long long)blockIdx.x * W;
+    long long p1 = (p0 + W < total) ? p0 + W : total;
+    if (p.unit_mode) {
+        // one worker per unit (B * U workers): the unit's own tile range, so that every
+        // piece is the whole unit and is written as the final result; a unit without
+        // tiles writes out = 0, lse = -inf for its rows
+        const int u = blockIdx.x, b = u / U, i = u % U;
+        const int n = s_prefix[b + 1] - s_prefix[b];
+        p0 = (long long)s_prefix[b] * U + (long long)i * n;
+        p1 = p0 + n;
+        if (n == 0) {
+            const int j = i / p.n_hb, hb = i % p.n_hb;
+            for (int e = tid; e < C::HEADS * D; e += C::NTHREADS) {
+                const int r = e / D, col = e - r * D;
+                const int hg = hb * C::HEADS + r;
+                if (hg >= p.g) continue;
+                const size_t gh = (size_t)b * p.n_q + (size_t)j * p.g + hg;
+                p.out[gh * D + col] = 0.f;
+                if (col == 0) p.lse[gh] = -INFINITY;
+            }
+            return;
+        }
+    }
     if (p0 >= total) return;
 
     if (warp == C::NCW) {

@@ -412,6 +412,21 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
     if (g_force_workers <= 0 && workers > by_size) workers = by_size;
     if (workers < 1) workers = 1;
     p.workers = (int)workers;
+    // Small problems: one worker per unit when every unit fits on its own SM and a unit's
+    // whole cache is at most 256 KB -- a split would save less than the combine launch
+    // costs; each unit is then finished in its CTA and no combine runs.
+    const long long units = (long long)p.B * units_per_seq;
+    const long long unit_bytes = (long long)((p.T_max + C::TILE - 1) / C::TILE) * C::STAGE_BYTES;
+    p.unit_mode = g_force_workers <= 0 && units <= dev->sms && unit_bytes <= (256 << 10) ? 1 : 0;
+    if (p.unit_mode) {
+        p.workers = (int)units;
+        auto kern = gqa_decode_kernel<D, MT>;
+        cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), dev, smem);
+        if (e != cudaSuccess) return fail_cuda(e, "cudaFuncSetAttribute(gqa)");
+        kern<<<p.workers, C::NTHREADS, smem, stream>>>(p, kmap, vmap);
+        e = cudaGetLastError();
+        return e == cudaSuccess ? KVATTN_OK : fail_cuda(e, "gqa decode launch");
+    }
 
     void *ws = nullptr;
     const size_t meta_bytes = ((16 + (size_t)(p.B + 1) * 4) + 255) & ~size_t(255);
