@@ -369,6 +369,16 @@ int kvattn_read_device_flags(unsigned int *flags);
 int kvattn_clear_device_flags(void);
 
 /*
+ * Test hook for the bounded waits: launches one CTA on `stream` (a cudaStream_t, NULL:
+ * the default stream) whose thread waits, with the same bounded wait the kernels use but
+ * cut to about limit_us microseconds of SM clock (1 .. 1000000), for a shared-memory
+ * barrier that nothing completes.  The wait runs out, sets bit 0 of the device flags and
+ * the kernel returns: no fault, no trap, the context stays usable.  Returns
+ * KVATTN_ERR_INVALID_ARG for a limit out of range, else the launch status.
+ */
+int kvattn_debug_wait_probe(int limit_us, void *stream);
+
+/*
  * Test and tuning knob (process-wide): when workers > 0 the next calls use exactly
  * that many workers (CTAs or CTA pairs) and at least min_tiles tiles per worker,
  * which forces the split/combine path on small inputs.  workers == 0 restores the

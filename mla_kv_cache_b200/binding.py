@@ -93,6 +93,7 @@ _SIGNATURES = {
     "kvattn_release_workspace": (None, []),
     "kvattn_read_device_flags": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint)]),
     "kvattn_clear_device_flags": (ctypes.c_int, []),
+    "kvattn_debug_wait_probe": (ctypes.c_int, [ctypes.c_int, ctypes.c_void_p]),
     "kvattn_debug_set_workers": (None, [ctypes.c_int, ctypes.c_int]),
     "kvattn_debug_set_gqa_kernel": (None, [ctypes.c_int]),
 }
@@ -264,6 +265,14 @@ def kvattn_clear_device_flags():
     st = lib().kvattn_clear_device_flags()
     if st != KVATTN_OK:
         raise KvattnError(st, "kvattn_clear_device_flags")
+
+
+def kvattn_debug_wait_probe(limit_us, stream=None):
+    """Test hook (include/kvattn.h, kvattn_debug_wait_probe): one bounded wait on a barrier
+    nothing completes, cut to about limit_us; it runs out and sets bit 0 of the device flags."""
+    st = lib().kvattn_debug_wait_probe(int(limit_us), _stream_handle(stream))
+    if st != KVATTN_OK:
+        raise KvattnError(st, "kvattn_debug_wait_probe")
 
 
 def kvattn_debug_set_workers(workers, min_tiles=0):

@@ -63,17 +63,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
     return ok != 0;
 }
 // Waits until the phase with the given parity has completed.  Gives up after
-// kWaitLimitCycles, or earlier when *abort becomes non-zero; returns false then (and
-// records `flag` when it timed out).
+// `limit` cycles (kWaitLimitCycles), or earlier when *abort becomes non-zero; returns
+// false then (and records `flag` when it timed out).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int flag,
-                                          volatile int *abort) {
+                                          volatile int *abort, long long limit = kWaitLimitCycles) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(a, parity)) return true;
         if (abort != nullptr && *abort) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             atomicOr(&g_device_flags, flag);
             if (abort != nullptr) *abort = 1;
             return false;

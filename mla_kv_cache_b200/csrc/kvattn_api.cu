@@ -1245,6 +1245,34 @@ int kvattn_clear_device_flags(void) {
     return KVATTN_OK;
 }
 
+// ---- test hook: a bounded wait that runs out
+namespace kvattn {
+// One thread waits, with the kernels' own bounded wait cut to `limit` cycles, for the
+// first phase of a shared-memory barrier that nothing arrives on; the wait gives up,
+// records FLAG_FULL_WAIT and the kernel returns.
+__global__ void wait_probe_kernel(long long limit) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0u, FLAG_FULL_WAIT, nullptr, limit);
+}
+}  // namespace kvattn
+
+int kvattn_debug_wait_probe(int limit_us, void *stream) {
+    if (limit_us <= 0 || limit_us > 1000000) return KVATTN_ERR_INVALID_ARG;
+    DeviceState *dev = nullptr;
+    int st = device_state(&dev);
+    if (st != KVATTN_OK) return st;
+    int khz = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev->id);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaDeviceGetAttribute(clock rate)");
+    const long long limit = (long long)limit_us * (khz > 0 ? khz : 2000000) / 1000;
+    kvattn::wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? KVATTN_OK : fail_cuda(e, "wait probe launch");
+}
+
 // ---- rotary embedding of the new token + cache append
 static int launch_rope_append(RopeAppendParams &p, cudaStream_t s, bool kv8 = false) {
     DeviceState *dev = nullptr;
