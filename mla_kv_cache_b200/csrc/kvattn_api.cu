@@ -413,11 +413,13 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
     if (workers < 1) workers = 1;
     p.workers = (int)workers;
     // Small problems: one worker per unit when every unit fits on its own SM and a unit's
-    // whole cache is at most 256 KB -- a split would save less than the combine launch
-    // costs; each unit is then finished in its CTA and no combine runs.
+    // whole cache is at most 128 KB -- a split would save less than the combine launch
+    // costs (measured: a unit's tiles cost ~0.5 us each in a row on one SM, so at 16 tiles
+    // of d = 64 the split with its combine is faster); each unit is then finished in its
+    // CTA and no combine runs.
     const long long units = (long long)p.B * units_per_seq;
     const long long unit_bytes = (long long)((p.T_max + C::TILE - 1) / C::TILE) * C::STAGE_BYTES;
-    p.unit_mode = g_force_workers <= 0 && units <= dev->sms && unit_bytes <= (256 << 10) ? 1 : 0;
+    p.unit_mode = g_force_workers <= 0 && units <= dev->sms && unit_bytes <= (128 << 10) ? 1 : 0;
     if (p.unit_mode) {
         p.workers = (int)units;
         auto kern = gqa_decode_kernel<D, MT>;
