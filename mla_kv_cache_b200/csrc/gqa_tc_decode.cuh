@@ -125,7 +125,7 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 256, "barrier block overflows its slot");
 
-template <int NR>
+template <int NR, bool KV8 = false>
 struct Cfg {
     static_assert(NR == 8 || NR == 16 || NR == 32 || NR == 64, "head columns per unit");
     static constexpr int NQ = NR < 16 ? 16 : NR;           // score-product N (and columns read)
@@ -137,9 +137,11 @@ struct Cfg {
     // current piece still reads its own
     static constexpr int NQB = 2 * QBLOCK <= QREGION ? 2 : 1;
     // softmax groups: two, taking alternate tiles, for 16 and 32 columns (where one
-    // group's per-tile work paces the kernel); one for 8 columns (the data's arrival
-    // paces it, measured) and for 64 (a thread's registers do not allow 320 threads)
-    static constexpr int NG = (NR == 16 || NR == 32) ? 2 : 1;
+    // group's per-tile work paces the kernel) and for 8 over an E4M3 cache (half the bytes
+    // per tile: 52.2 vs 56.3 us on the ragged GQA workload, 189 vs 200 us on MHA); one for
+    // 8 over bf16 (the data's arrival paces it, measured) and for 64 (a thread's registers
+    // do not allow 320 threads)
+    static constexpr int NG = (NR == 16 || NR == 32 || (KV8 && NR == 8)) ? 2 : 1;
     static constexpr int NTHREADS = 64 + 128 * NG;
 };
 
@@ -512,7 +514,7 @@ __device__ __forceinline__ void mma_issuer(const GqaParams &p, const Ctx &c, int
 // single-token MQA workload ~4 us per step (measured) even where it does not run.
 template <int NR, bool KV8, bool MULTI>
 __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, int warp, int lane) {
-    using C = Cfg<NR>;
+    using C = Cfg<NR, KV8>;
     using L = Kv<KV8>;
     constexpr int NQ = C::NQ;
     constexpr int NST = L::NST;
@@ -831,7 +833,7 @@ __device__ __forceinline__ void softmax_warps(const GqaParams &p, const Ctx &c, 
 }  // namespace gqatc
 
 template <int NR, bool KV8, bool MULTI>
-__global__ void __launch_bounds__(gqatc::Cfg<NR>::NTHREADS, 1)
+__global__ void __launch_bounds__(gqatc::Cfg<NR, KV8>::NTHREADS, 1)
 gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap qmap) {
     using namespace gqatc;
@@ -855,7 +857,7 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
             mbar_init(&bars->qempty[i], 1);
             mbar_init(&bars->qconv[i], 32);
         }
-        constexpr int NG = Cfg<NR>::NG;
+        constexpr int NG = Cfg<NR, KV8>::NG;
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->sready[i], 1);
             mbar_init(&bars->sfree[i], 4);        // the four warps of the tile's group
@@ -877,7 +879,7 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
     // query buffers start zeroed: rows a unit's block does not fill stay finite (a
     // single-token block is a full box: the TMA fills its rows past the heads with zeros)
     if constexpr (MULTI)
-        for (int i = tid; i < QREGION / 16; i += Cfg<NR>::NTHREADS)
+        for (int i = tid; i < QREGION / 16; i += Cfg<NR, KV8>::NTHREADS)
             reinterpret_cast<uint4 *>(smem + OFF_Q)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
     if (warp == 0 && lane == 0) {
@@ -901,7 +903,7 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
     if (blockIdx.x == 0) {
         MetaView mv = meta_view(p.ws_meta);
         if (tid == 0) { mv.w_total[0] = W; mv.w_total[1] = total; }
-        for (int i = tid; i <= p.B; i += Cfg<NR>::NTHREADS) mv.prefix[i] = s_prefix[i];
+        for (int i = tid; i <= p.B; i += Cfg<NR, KV8>::NTHREADS) mv.prefix[i] = s_prefix[i];
     }
     // The combine kernel may be scheduled now; it waits for this grid to finish.
     pdl_launch_dependents();

@@ -510,7 +510,7 @@ int run_gqa_tc(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap
     auto kern = (p.q_len > 1 || p.window > 0) ? gqa_tc_decode_kernel<NR, KV8, true> : gqa_tc_decode_kernel<NR, KV8, false>;
     cudaError_t e = set_smem_limit(reinterpret_cast<const void *>(kern), dev, smem);
     if (e != cudaSuccess) return fail_cuda(e, "cudaFuncSetAttribute(gqa tc)");
-    kern<<<p.workers, gqatc::Cfg<NR>::NTHREADS, smem, stream>>>(p, kmap, vmap, qmap);
+    kern<<<p.workers, gqatc::Cfg<NR, KV8>::NTHREADS, smem, stream>>>(p, kmap, vmap, qmap);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e, "gqa tc decode launch");
 
