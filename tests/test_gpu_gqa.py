@@ -91,6 +91,14 @@ def test_all_empty():
     assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
 
 
+def test_small_problem_one_worker_per_unit():
+    """A batch small enough for one worker per unit (every unit's cache <= 128 KB): empty,
+    one-token, partial-tile and full sequences in one call, each unit finished in its own
+    CTA with no combine."""
+    run_case(small("unit_mode", 5, 8, 2, 64, 512, lens=[512, 0, 1, 100, 0]))
+    run_case(small("unit_mode128", 3, 8, 4, 128, 256, lens=[0, 256, 65]))
+
+
 def test_sharp_softmax():
     # keys scaled by 8: a few tokens dominate each head (the P-rounding worst case)
     run_case(small("sharp", 2, 16, 2, 128, 200, lens=[200, 3], key_scale=8.0))
