@@ -39,11 +39,11 @@
 // Latent columns are thus read twice per pair (once as keys by the half's owner, once as
 // values by each CTA for its columns), the second time from L2.
 //
-// Warp roles (256 threads per CTA):
+// Warp roles (384 threads per CTA):
 //   warp 0, one thread   key producer (both CTAs): the shared-memory part of the query
 //                        block once per sequence and a ring of three 24 KB key slots (one
-//                        tile); completions signal rank 0's barriers.
-//   warp 2, one thread   value producer (both CTAs): two 32 KB value slots, one per token
+//                        tile, one multi-chunk copy a slot); completions to rank 0.
+//   warp 2, one thread   value producer (both CTAs): two 32 KB value slots (one copy each), one per token
 //                        half of a tile, independent of the key stream; its loads hit L2
 //                        (the keys' latent columns, loaded by the pair moments before).
 // Each slot release is one tcgen05.commit, which costs the issuing thread ~300 cycles
