@@ -6,9 +6,9 @@ cannot afford cudaMalloc's implicit synchronisation.  Its scratch is a fixed arr
 inside the library shared by every call.
 
 The test calls it through the C ABI (ctypes, no Python wrapper) twice in a row on
-different workloads and checks both results against kvattn_gqa_decode's at the
-library's tolerance; the second call runs on a scratch array that still holds the
-first call's contents.  It also checks that a plan too large for the array is refused
+different workloads and checks both results against the fp64 oracle and against
+kvattn_gqa_decode's at the library's tolerance; the second call runs on a scratch array
+that still holds the first call's contents.  It also checks that a plan too large for the array is refused
 with a clear error.  This file is collected last on purpose, and it must pass both on
 its own in a fresh process (the first call on the device does the one-time set-up) and
 after the other tests.
@@ -19,6 +19,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from mla_kv_cache_b200 import binding as kb
 from mla_kv_cache_b200 import workloads as wl
 from tests.parity import assert_close
@@ -44,7 +45,8 @@ def _inputs(cfg, seed):
     B, n_q, hd = d["q"].shape
     nan = float("nan")
     bufs = {"out": torch.full((B, n_q, hd), nan, dtype=torch.float32, device="cuda"),
-            "lse": torch.full((B, n_q), nan, dtype=torch.float32, device="cuda")}
+            "lse": torch.full((B, n_q), nan, dtype=torch.float32, device="cuda"),
+            "host": x}
     return d, bufs
 
 
@@ -69,6 +71,10 @@ def test_noalloc_matches_allocating_entry_point_twice():
         assert _c_call("kvattn_gqa_decode_noalloc", d, cfg, got["out"], got["lse"], stream) == kb.KVATTN_OK
     torch.cuda.synchronize()
     for cfg, _, ref, got in cases:
+        x = got["host"]
+        ro, rl = oracle.gqa_decode(x["q"], x["k_cache"], x["v_cache"], x["seq_lens"], cfg.scale)
+        assert_close(got["out"].cpu().numpy(), ro, f"{cfg.name} out vs oracle")
+        assert_close(got["lse"].cpu().numpy(), rl, f"{cfg.name} lse vs oracle")
         assert_close(got["out"].cpu().numpy(), ref["out"].cpu().numpy().astype(np.float64),
                      f"{cfg.name} out")
         assert_close(got["lse"].cpu().numpy(), ref["lse"].cpu().numpy().astype(np.float64),
