@@ -98,6 +98,20 @@ def test_forced_splits(workers, min_tiles):
     run_case(mla("split", 4, 128, 2000, lens=[2000, 1, 0, 777]))
 
 
+def test_many_short_ragged_sequences():
+    """300 sequences of 0-400 tokens: every worker runs pieces of several sequences, and
+    the sequences cut by worker boundaries are merged by their last worker."""
+    lens = np.random.default_rng(31).integers(0, 401, size=300).tolist()
+    run_case(mla("many", 300, 128, 400, lens=lens))
+
+
+def test_largest_batch():
+    """1024 sequences (the largest batch) of at most 64 tokens: one tile each, ~14 pieces
+    per worker, the merge counters of every sequence in use."""
+    lens = np.random.default_rng(32).integers(1, 65, size=1024).tolist()
+    run_case(mla("b1024", 1024, 128, 64, lens=lens))
+
+
 def test_workload_full_size():
     run_case(wl.CONFIGS["mla_b32_h128_c512_r64_t4096"])
 
