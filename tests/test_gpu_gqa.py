@@ -99,6 +99,18 @@ def test_small_problem_one_worker_per_unit():
     run_case(small("unit_mode128", 3, 8, 4, 128, 256, lens=[0, 256, 65]))
 
 
+@pytest.mark.parametrize("which", [1, 2], ids=["warp_kernel", "tcgen05_kernel"])
+def test_many_short_sequences(which):
+    """1000 sequences of 0-200 tokens (group 4, head_dim 128): many pieces per worker and
+    many units cut by worker boundaries, on each kernel."""
+    kb.kvattn_debug_set_gqa_kernel(which)
+    try:
+        lens = np.random.default_rng(34 + which).integers(0, 201, size=1000).tolist()
+        run_case(small("many", 1000, 32, 8, 128, 200, lens=lens))
+    finally:
+        kb.kvattn_debug_set_gqa_kernel(0)
+
+
 def test_sharp_softmax():
     # keys scaled by 8: a few tokens dominate each head (the P-rounding worst case)
     run_case(small("sharp", 2, 16, 2, 128, 200, lens=[200, 3], key_scale=8.0))

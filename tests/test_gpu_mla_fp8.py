@@ -103,6 +103,13 @@ def test_forced_splits(workers, min_tiles):
     run_case(mla8("split", 4, 128, 2000, [2000, 1, 0, 777]))
 
 
+def test_many_short_ragged_sequences():
+    """300 sequences of 0-400 tokens over the E4M3 cache: several pieces per worker (each
+    with its own query split) and the merges of the cut sequences."""
+    lens = np.random.default_rng(33).integers(0, 401, size=300).tolist()
+    run_case(mla8("many8", 300, 128, 400, lens))
+
+
 def test_workload_full_size():
     """The DeepSeek-shaped workload (batch 32, 128 heads, context 4096) with its cache in
     E4M3, every sequence, in the bench's launch configuration."""
