@@ -574,6 +574,13 @@ def gpu_arm(args):
         torch.cuda.synchronize()
         dist_barrier()
     clocks = clk.summary()
+    # the library's own count of the kernels one step enqueues (decode, and a combine only
+    # when units are cut between workers)
+    from mla_kv_cache_b200 import binding as kb
+    n0 = kb.kvattn_kernel_launches()
+    call()
+    torch.cuda.synchronize()
+    launches_per_step = kb.kvattn_kernel_launches() - n0
     ms = dist_max(sum(times) / len(times))
     lens = x["seq_lens"].tolist()
     nb = step_bytes(head_cfg, lens)
@@ -593,13 +600,17 @@ def gpu_arm(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
                      "peak_source": pk["source"] + " burst copy bandwidth",
-                     "timed_unit": "one library call: " + ("the decode kernel (partials merged inside it)"
+                     "timed_unit": "one library call: " + (("the decode kernel (partials merged inside it)"
+                                                            + (" after the virtual-batch kernel"
+                                                               if launches_per_step > 1 else ""))
                                                            if is_mla(head_cfg) else
-                                                           "decode kernel + PDL-chained combine kernel")},
+                                                           "decode kernel + PDL-chained combine kernel"
+                                                           if launches_per_step > 1 else
+                                                           "the decode kernel (no unit cut: no combine)")},
         "e2e": {"value": nb["total"] * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "note": "per step: pinned host q/seq_lens -> device, library call, out/lse -> pinned host; KV cache resident in HBM"},
-        "gpu_launches": (1 if is_mla(head_cfg) else 2) * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "configs": dict(extras, **{args.config: res}),
     }

@@ -369,6 +369,15 @@ int kvattn_read_device_flags(unsigned int *flags);
 int kvattn_clear_device_flags(void);
 
 /*
+ * Kernels this library has launched (enqueued successfully) from the calling host thread
+ * since the library was loaded: a decode call adds one (the decode kernel), or two when a
+ * combine kernel merges units cut between workers, plus one when several new tokens run
+ * as a virtual batch; an append adds one.  Read it before and after a call to count that
+ * call's kernels.
+ */
+unsigned long long kvattn_kernel_launches(void);
+
+/*
  * Test hook for the bounded waits: launches one CTA on `stream` (a cudaStream_t, NULL:
  * the default stream) whose thread waits, with the same bounded wait the kernels use but
  * cut to about limit_us microseconds of SM clock (1 .. 1000000), for a shared-memory

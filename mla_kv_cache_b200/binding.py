@@ -94,6 +94,7 @@ _SIGNATURES = {
     "kvattn_read_device_flags": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint)]),
     "kvattn_clear_device_flags": (ctypes.c_int, []),
     "kvattn_debug_wait_probe": (ctypes.c_int, [ctypes.c_int, ctypes.c_void_p]),
+    "kvattn_kernel_launches": (ctypes.c_ulonglong, []),
     "kvattn_debug_set_workers": (None, [ctypes.c_int, ctypes.c_int]),
     "kvattn_debug_set_gqa_kernel": (None, [ctypes.c_int]),
 }
@@ -265,6 +266,11 @@ def kvattn_clear_device_flags():
     st = lib().kvattn_clear_device_flags()
     if st != KVATTN_OK:
         raise KvattnError(st, "kvattn_clear_device_flags")
+
+
+def kvattn_kernel_launches():
+    """Kernels the library has launched from this thread (include/kvattn.h)."""
+    return int(lib().kvattn_kernel_launches())
 
 
 def kvattn_debug_wait_probe(limit_us, stream=None):

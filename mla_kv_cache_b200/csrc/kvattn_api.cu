@@ -293,15 +293,21 @@ cudaError_t set_smem_limit(const void *kern, DeviceState *dev, int smem) {
     return e;
 }
 
+// Kernels this library has launched from the calling thread (kvattn_kernel_launches).
+thread_local unsigned long long t_launches = 0;
+
 template <int D>
 cudaError_t launch_combine_d(cudaLaunchConfig_t &cfg, const CombineParams &cp, int warps) {
     cfg.blockDim = dim3(warps * 32, 1, 1);
+    cudaError_t e;
     switch (warps) {
-        case 1: return cudaLaunchKernelEx(&cfg, combine_kernel<D, 1>, cp);
-        case 2: return cudaLaunchKernelEx(&cfg, combine_kernel<D, 2>, cp);
-        case 4: return cudaLaunchKernelEx(&cfg, combine_kernel<D, 4>, cp);
-        default: return cudaLaunchKernelEx(&cfg, combine_kernel<D, 8>, cp);
+        case 1: e = cudaLaunchKernelEx(&cfg, combine_kernel<D, 1>, cp); break;
+        case 2: e = cudaLaunchKernelEx(&cfg, combine_kernel<D, 2>, cp); break;
+        case 4: e = cudaLaunchKernelEx(&cfg, combine_kernel<D, 4>, cp); break;
+        default: e = cudaLaunchKernelEx(&cfg, combine_kernel<D, 8>, cp); break;
     }
+    if (e == cudaSuccess) ++t_launches;
+    return e;
 }
 
 // Warps per combine CTA from the partials one unit is expected to have (about four
@@ -427,7 +433,9 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
         if (e != cudaSuccess) return fail_cuda(e, "cudaFuncSetAttribute(gqa)");
         kern<<<p.workers, C::NTHREADS, smem, stream>>>(p, kmap, vmap);
         e = cudaGetLastError();
-        return e == cudaSuccess ? KVATTN_OK : fail_cuda(e, "gqa decode launch");
+        if (e != cudaSuccess) return fail_cuda(e, "gqa decode launch");
+        ++t_launches;
+        return KVATTN_OK;
     }
 
     void *ws = nullptr;
@@ -448,6 +456,7 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
     kern<<<p.workers, C::NTHREADS, smem, stream>>>(p, kmap, vmap);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e, "gqa decode launch");
+    ++t_launches;
 
     CombineParams cp;
     cp.seq_lens = p.seq_lens;
@@ -513,6 +522,7 @@ int run_gqa_tc(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap
     kern<<<p.workers, gqatc::Cfg<NR, KV8>::NTHREADS, smem, stream>>>(p, kmap, vmap, qmap);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e, "gqa tc decode launch");
+    ++t_launches;
 
     CombineParams cp;
     cp.seq_lens = p.seq_lens;
@@ -621,6 +631,7 @@ int virtual_batch(DeviceState *dev, const int32_t *seq_lens, const int32_t *bloc
     virtual_batch_kernel<<<blocks, 256, 0, s>>>(seq_lens, block_table, B, L, mp, capacity, *vlens, *vtable);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e, "virtual batch launch");
+    ++t_launches;
     return KVATTN_OK;
 }
 
@@ -903,6 +914,7 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
         mla_decode_kernel<false><<<2 * p.workers, mla::NTHREADS, smem, s>>>(p, maps);
     e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e, "mla decode launch");
+    ++t_launches;
     return KVATTN_OK;
 }
 
@@ -1261,6 +1273,8 @@ __global__ void wait_probe_kernel(long long limit) {
 }
 }  // namespace kvattn
 
+unsigned long long kvattn_kernel_launches(void) { return t_launches; }
+
 int kvattn_debug_wait_probe(int limit_us, void *stream) {
     if (limit_us <= 0 || limit_us > 1000000) return KVATTN_ERR_INVALID_ARG;
     DeviceState *dev = nullptr;
@@ -1272,7 +1286,9 @@ int kvattn_debug_wait_probe(int limit_us, void *stream) {
     const long long limit = (long long)limit_us * (khz > 0 ? khz : 2000000) / 1000;
     kvattn::wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit);
     e = cudaGetLastError();
-    return e == cudaSuccess ? KVATTN_OK : fail_cuda(e, "wait probe launch");
+    if (e != cudaSuccess) return fail_cuda(e, "wait probe launch");
+    ++t_launches;
+    return KVATTN_OK;
 }
 
 // ---- rotary embedding of the new token + cache append
@@ -1291,6 +1307,7 @@ static int launch_rope_append(RopeAppendParams &p, cudaStream_t s, bool kv8 = fa
         rope_append_kernel<false><<<(unsigned)blocks, 256, 0, s>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail_cuda(e, "rope append launch");
+    ++t_launches;
     return KVATTN_OK;
 }
 
