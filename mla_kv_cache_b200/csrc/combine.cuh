@@ -40,6 +40,7 @@ struct CombineParams {
     int min_tiles;         // the decode kernel's minimum tiles per worker
     int q_len;             // new tokens per sequence (rows of a unit: q_len x g)
     int window;            // sliding window (0: none)
+    int unit_split;        // the decode kernel cuts equal units into parts (unit_part_tiles)
 };
 
 // D columns, D / 32 floats per lane; NW warps share the partials of one output row.
@@ -65,25 +66,29 @@ __global__ void __launch_bounds__(NW * 32) combine_kernel(const CombineParams p)
     const int col = lane * VEC;
 
     // ---- the work split, from seq_lens (an input: readable before the decode grid ends)
-    int before = 0, all = 0;
+    const int l0 = clamp_len(__ldg(p.seq_lens), p.T_max);
+    const int t0 = tiles_of(l0 - active_start(l0, p.q_len, p.window), p.tile);
+    int before = 0, all = 0, same = 1;
     for (int x = threadIdx.x; x < p.B; x += blockDim.x) {
         const int lx = clamp_len(__ldg(p.seq_lens + x), p.T_max);
         const int t = tiles_of(lx - active_start(lx, p.q_len, p.window), p.tile);
         all += t;
+        same &= t == t0;
         if (x < b) before += t;
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) {
         before += __shfl_xor_sync(0xffffffffu, before, off);
         all += __shfl_xor_sync(0xffffffffu, all, off);
+        same &= __shfl_xor_sync(0xffffffffu, same, off);
     }
-    __shared__ int s_sum[2][kCombineWarps];
-    if (lane == 0) { s_sum[0][warp] = before; s_sum[1][warp] = all; }
+    __shared__ int s_sum[3][kCombineWarps];
+    if (lane == 0) { s_sum[0][warp] = before; s_sum[1][warp] = all; s_sum[2][warp] = same; }
     __syncthreads();
     before = 0;
     all = 0;
 #pragma unroll
-    for (int w = 0; w < kCombineWarps; ++w) { before += s_sum[0][w]; all += s_sum[1][w]; }
+    for (int w = 0; w < kCombineWarps; ++w) { before += s_sum[0][w]; all += s_sum[1][w]; same &= s_sum[2][w]; }
     const int len_b = clamp_len(__ldg(p.seq_lens + b), p.T_max);
     const int n_tiles = tiles_of(len_b - active_start(len_b, p.q_len, p.window), p.tile);
     const long long W = tiles_per_worker((long long)all * p.units_per_seq, p.workers, p.min_tiles);
@@ -94,8 +99,18 @@ __global__ void __launch_bounds__(NW * 32) combine_kernel(const CombineParams p)
         return;
     }
     const long long ustart = (long long)before * p.units_per_seq + (long long)i * n_tiles;
-    const long long c_first = ustart / W;
-    const long long c_last = (ustart + n_tiles - 1) / W;
+    long long c_first = ustart / W;
+    long long c_last = (ustart + n_tiles - 1) / W;
+    bool parts = false;   // the decode kernel's unit parts: workers u k .. u k + ceil(n / Wu) - 1, slot 0
+    if (p.unit_split && same) {
+        int k = 0;
+        const long long Wu = unit_part_tiles(t0, (long long)p.B * p.units_per_seq, p.workers, p.min_tiles, &k);
+        if (Wu > 0) {
+            parts = true;
+            c_first = (long long)u * k;
+            c_last = c_first + (t0 + Wu - 1) / Wu - 1;
+        }
+    }
     if (c_first == c_last) return;            // finished by its only worker
 
     pdl_wait_primary();
@@ -112,7 +127,7 @@ __global__ void __launch_bounds__(NW * 32) combine_kernel(const CombineParams p)
             const long long c = c0 + (long long)q * kCombineWarps;
             ls[q] = -INFINITY;
             if (c <= c_last) {
-                const int slot = (ustart <= c * W) ? 0 : 1;
+                const int slot = (parts || ustart <= c * W) ? 0 : 1;
                 const size_t part = ((size_t)c * 2 + slot) * p.heads_per_unit + r;
                 ls[q] = p.ws_lse[part];
                 const float4 *src = reinterpret_cast<const float4 *>(p.ws_o + part * D + col);

@@ -47,6 +47,7 @@ struct GqaParams {
     int window;                 // sliding window in tokens (0: none)
     float k_scale, v_scale;     // E4M3 cache: value = code * scale (1 for a bf16 cache)
     int unit_mode;              // warp kernel: worker u takes exactly unit u (no partials, no combine)
+    int unit_split;             // tcgen05 kernel: unit parts when every unit has the same tiles
 };
 
 template <int D, int MT>

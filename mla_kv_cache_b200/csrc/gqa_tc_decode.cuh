@@ -909,6 +909,21 @@ gqa_tc_decode_kernel(const GqaParams p, const __grid_constant__ CUtensorMap kmap
     pdl_launch_dependents();
     c.p0 = (long long)blockIdx.x * W;
     c.p1 = (c.p0 + W < total) ? c.p0 + W : total;
+    if (p.unit_split) {   // equal units: consecutive parts of one unit per worker (schedule.cuh)
+        const int n_uni = uniform_tile_count(s_prefix, p.B);
+        const long long units = (long long)p.B * U;
+        int k = 0;
+        const long long Wu = unit_part_tiles(n_uni, units, p.workers, p.min_tiles, &k);
+        if (Wu > 0) {
+            const long long u = blockIdx.x / k, i = blockIdx.x % k, ub = u * n_uni;
+            c.p0 = total;
+            c.p1 = total;
+            if (u < units && i * Wu < n_uni) {
+                c.p0 = ub + i * Wu;
+                c.p1 = (i + 1) * Wu < n_uni ? c.p0 + Wu : ub + n_uni;
+            }
+        }
+    }
 
     if (c.p0 < total) {
         if (warp == 0) {

@@ -477,6 +477,7 @@ int run_gqa(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &v
     cp.min_tiles = p.min_tiles;
     cp.q_len = 1;
     cp.window = 0;
+    cp.unit_split = 0;
     const int rows = p.g < C::HEADS ? p.g : C::HEADS;
     return launch_combine(D, cp, p.B * units_per_seq, rows, stream,
                           combine_warps((p.T_max + C::TILE - 1) / C::TILE, max_tiles, p.workers));
@@ -488,6 +489,7 @@ template <int NR, bool KV8>
 int run_gqa_tc(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap &vmap,
                const CUtensorMap &qmap, DeviceState *dev, int units_per_seq, cudaStream_t stream) {
     GqaParams p = base;
+    p.unit_split = 1;   // equal units are cut into parts of one unit each (schedule.cuh)
     const int smem = gqatc::smem_bytes(p.B);
     if (smem > dev->max_smem_optin) {
         snprintf(t_detail, sizeof(t_detail), "needs %d B shared memory", smem);
@@ -543,6 +545,7 @@ int run_gqa_tc(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap
     cp.min_tiles = p.min_tiles;
     cp.q_len = p.q_len;
     cp.window = p.window;
+    cp.unit_split = p.unit_split;
     const int rows = p.g * p.q_len < gqatc::HB ? p.g * p.q_len : gqatc::HB;
     return launch_combine(gqatc::D, cp, p.B * units_per_seq, rows, stream,
                           combine_warps((p.T_max + gqatc::TILE - 1) / gqatc::TILE, max_tiles, p.workers));

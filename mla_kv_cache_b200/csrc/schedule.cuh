@@ -164,6 +164,22 @@ __device__ __forceinline__ int uniform_tile_count(const int *s_prefix, int B) {
     return same && n0 > 0 ? n0 : 0;
 }
 
+// Unit parts (the tcgen05 GQA kernel and its combine): when every unit has the same
+// number of tiles n and there are at least as many workers as units, unit u is cut into
+// k consecutive parts of at most ceil(n / k) tiles (k = workers / units, parts of at least
+// min_tiles), worker u * k + i taking part i -- so no worker spans two units (a worker
+// that does pays a second query load, epilogue and pipeline restart and finishes last).
+// Returns the tiles per part and k, or 0 where it does not apply.
+__device__ __forceinline__ long long unit_part_tiles(int n, long long units, int workers, int min_tiles, int *k_out) {
+    if (n <= 0 || units <= 0 || units > workers) return 0;
+    long long k = workers / units;
+    const long long kmax = (n + (min_tiles > 0 ? min_tiles : 1) - 1) / (min_tiles > 0 ? min_tiles : 1);
+    if (k > kmax) k = kmax;
+    if (k < 1) k = 1;
+    *k_out = (int)k;
+    return (n + k - 1) / k;
+}
+
 // Layout of the published decomposition at the start of the workspace.
 struct MetaView {
     long long *w_total;  // [0] = W, [1] = total
