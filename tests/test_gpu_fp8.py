@@ -79,6 +79,23 @@ def test_fp8_sharp_keys_ragged():
     assert_close(lse.cpu().numpy(), rl, "fp8 sharp lse")
 
 
+@pytest.mark.parametrize("B,n_q,n_kv,T", [(2, 32, 1, 128 * 37), (3, 16, 2, 1000)],
+                         ids=["2units_37tiles", "6units_8tiles"])
+def test_fp8_equal_units_in_parts(B, n_q, n_kv, T):
+    """Every sequence of the same length and no more units than workers: each unit is cut
+    into consecutive parts of its own (the last one shorter), which the combine merges."""
+    cfg, x = fp8_inputs(B, n_q, n_kv, T, [T] * B, seed=66)
+    out, lse, ro, rl = run_fp8(cfg, x)
+    assert_close(out.cpu().numpy(), ro, "fp8 parts out")
+    assert_close(lse.cpu().numpy(), rl, "fp8 parts lse")
+    # several new tokens over equal lengths (the multi-token instantiation)
+    g = torch.Generator().manual_seed(67)
+    q = torch.randn((B, 2, n_q, 128), generator=g).to(torch.bfloat16)
+    out, lse, ro, rl = run_fp8(cfg, x, q=q)
+    assert_close(out.cpu().numpy(), ro, "fp8 parts multi out")
+    assert_close(lse.cpu().numpy(), rl, "fp8 parts multi lse")
+
+
 @pytest.mark.parametrize("L,window", [(4, 0), (8, 100), (2, 1), (16, 0)])
 def test_fp8_multi_token(L, window):
     lens = [1000, 0, 2, 129, 3000, 257]

@@ -111,6 +111,18 @@ def test_many_short_sequences(which):
         kb.kvattn_debug_set_gqa_kernel(0)
 
 
+@pytest.mark.parametrize("B,n_q,n_kv,T", [(2, 32, 1, 128 * 37), (3, 16, 2, 1000), (1, 64, 8, 4096)],
+                         ids=["2units_37tiles", "6units_8tiles", "8units_32tiles"])
+def test_equal_units_in_parts(B, n_q, n_kv, T):
+    """Equal lengths and no more units than workers on the tcgen05 kernel: each unit is
+    cut into consecutive parts of its own (the last one shorter), merged by the combine."""
+    kb.kvattn_debug_set_gqa_kernel(2)
+    try:
+        run_case(small("parts", B, n_q, n_kv, 128, T))
+    finally:
+        kb.kvattn_debug_set_gqa_kernel(0)
+
+
 def test_sharp_softmax():
     # keys scaled by 8: a few tokens dominate each head (the P-rounding worst case)
     run_case(small("sharp", 2, 16, 2, 128, 200, lens=[200, 3], key_scale=8.0))
