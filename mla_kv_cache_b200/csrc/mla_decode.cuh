@@ -754,9 +754,13 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
     // arrived): out = sum_c exp(lse_c - lse) o_c, lse = log sum_c exp(lse_c).  Lane L
     // takes the log-sum-exp of row L and puts the row's weights exp(lse_c - lse) in the
     // warp's scratch (32 parts at a time); each load instruction then reads four rows'
-    // 128 contiguous bytes (eight lanes per row), two parts' loads in flight together.
-    // The partials are read through L2 (other SMs wrote them).
-    auto merge_block = [&](int b, long long ustart, int n_parts) {
+    // 128 contiguous bytes (eight lanes per row).  The partials are read through L2
+    // (other SMs wrote them), and the merge is a chain of L2 round trips, so it keeps
+    // many loads in flight: up to NPR parts' log-sum-exps are read once, together; two
+    // parts (the usual cut), when `stage` (16 KB of shared memory no one else uses) is
+    // given, two column chunks at a time (32 copies in flight); otherwise two parts' loads
+    // of one chunk go together.
+    auto merge_block = [&](int b, long long ustart, int n_parts, uint8_t *stage) {
         const long long c_first = ustart / c.W;
         auto part_row = [&](int j, int h) -> size_t {
             const long long cw = c_first + j;
@@ -764,23 +768,40 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             return ((size_t)cw * 2 + slot) * HR + h;
         };
         const int hl = head0 + lane;
+        constexpr int NPR = 4;
+        const bool few = n_parts <= NPR;
+        float lv[NPR];
         float M = -INFINITY;
-        for (int j0 = 0; j0 < n_parts; j0 += 4) {
-            float v[4];
+        if (few) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = j0 + u < n_parts ? __ldcg(p.ws_lse + part_row(j0 + u, hl)) : -INFINITY;
+            for (int u = 0; u < NPR; ++u) lv[u] = u < n_parts ? __ldcg(p.ws_lse + part_row(u, hl)) : -INFINITY;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) M = fmaxf(M, v[u]);
-        }
-        float S = 0.f;
-        if (M != -INFINITY)
+            for (int u = 0; u < NPR; ++u) M = fmaxf(M, lv[u]);
+        } else {
             for (int j0 = 0; j0 < n_parts; j0 += 4) {
                 float v[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) v[u] = j0 + u < n_parts ? __ldcg(p.ws_lse + part_row(j0 + u, hl)) : -INFINITY;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) S += v[u] == -INFINITY ? 0.f : fast_exp2((v[u] - M) * 1.4426950408889634f);
+                for (int u = 0; u < 4; ++u) M = fmaxf(M, v[u]);
             }
+        }
+        float S = 0.f;
+        if (M != -INFINITY) {
+            if (few) {
+#pragma unroll
+                for (int u = 0; u < NPR; ++u)
+                    S += lv[u] == -INFINITY ? 0.f : fast_exp2((lv[u] - M) * 1.4426950408889634f);
+            } else {
+                for (int j0 = 0; j0 < n_parts; j0 += 4) {
+                    float v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) v[u] = j0 + u < n_parts ? __ldcg(p.ws_lse + part_row(j0 + u, hl)) : -INFINITY;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) S += v[u] == -INFINITY ? 0.f : fast_exp2((v[u] - M) * 1.4426950408889634f);
+                }
+            }
+        }
         const float lse_all = S > 0.f ? M + __logf(S) : -INFINITY;
         // the scratch as [JB parts][32 rows] floats (the warp's own units of the weights
         // buffer: scratch_unit(r, u), 4 floats each)
@@ -792,12 +813,62 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
         for (int jb = 0; jb < n_parts; jb += JB) {
             const int nj = n_parts - jb < JB ? n_parts - jb : JB;
             __syncwarp();
-            for (int j = 0; j < nj; ++j) {
-                const float lj = __ldcg(p.ws_lse + part_row(jb + j, hl));
-                *wslot(j, lane) = (lse_all == -INFINITY || lj == -INFINITY)
-                                      ? 0.f : fast_exp2((lj - lse_all) * 1.4426950408889634f);
+            if (few) {   // (jb = 0, nj = n_parts)
+#pragma unroll
+                for (int u = 0; u < NPR; ++u)
+                    if (u < nj)
+                        *wslot(u, lane) = (lse_all == -INFINITY || lv[u] == -INFINITY)
+                                              ? 0.f : fast_exp2((lv[u] - lse_all) * 1.4426950408889634f);
+            } else {
+                for (int j = 0; j < nj; ++j) {
+                    const float lj = __ldcg(p.ws_lse + part_row(jb + j, hl));
+                    *wslot(j, lane) = (lse_all == -INFINITY || lj == -INFINITY)
+                                          ? 0.f : fast_exp2((lj - lse_all) * 1.4426950408889634f);
+                }
             }
             __syncwarp();
+            if (n_parts == 2 && stage != nullptr) {
+                // two column chunks of both parts in flight: copied by cp.async into this
+                // warp's 16 KB of idle shared memory (a lane reads back only its own copies,
+                // so its own wait is enough), then merged from there
+                // (a part's rows are consecutive: row head0 + rr of part j is rr rows after
+                // row head0)
+                const float *src0 = p.ws_o + part_row(0, head0 + (lane >> 3)) * 512 + col0 + 4 * (lane & 7);
+                const float *src1 = p.ws_o + part_row(1, head0 + (lane >> 3)) * 512 + col0 + 4 * (lane & 7);
+#pragma unroll 1
+                for (int cp = 0; cp < 2; ++cp) {   // column chunks 2cp, 2cp + 1
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int off = 4 * i * 512 + 32 * (2 * cp + e);
+                            uint8_t *d = stage + ((e * 8 + i) * 2 * 32 + lane) * 16;
+                            cp_async16(d, src0 + off);
+                            cp_async16(d + 32 * 16, src1 + off);
+                        }
+                    cp_async_wait_all();
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int rr = 4 * i + (lane >> 3);
+                            const uint8_t *d = stage + ((e * 8 + i) * 2 * 32 + lane) * 16;
+                            const float4 x0 = *reinterpret_cast<const float4 *>(d);
+                            const float4 x1 = *reinterpret_cast<const float4 *>(d + 32 * 16);
+                            const float w0 = *wslot(0, rr), w1 = *wslot(1, rr);
+                            float4 o;
+                            o.x = fmaf(w1, x1.x, w0 * x0.x);
+                            o.y = fmaf(w1, x1.y, w0 * x0.y);
+                            o.z = fmaf(w1, x1.z, w0 * x0.z);
+                            o.w = fmaf(w1, x1.w, w0 * x0.w);
+                            const int h_r = head0 + rr;
+                            if (h_r < p.H)
+                                *reinterpret_cast<float4 *>(p.out + ((size_t)b * p.H + h_r) * 512 + col0 +
+                                                            32 * (2 * cp + e) + 4 * (lane & 7)) = o;
+                        }
+                }
+                continue;
+            }
 #pragma unroll 1
             for (int cc = 0; cc < 4; ++cc) {
                 float4 acc[8];
@@ -1140,7 +1211,18 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             last = __shfl_sync(0xffffffffu, last, 0);
             if (last) {
                 __threadfence();   // the other workers' partials, after their arrivals
-                merge_block(pc.b, ustart, n_parts);
+                // After a worker's last piece its key ring and value slots are idle (every
+                // load of the piece has landed and every product that reads them is done:
+                // odone of the last tile): 16 KB of them per softmax warp stage the merge.
+                uint8_t *stage = nullptr;
+                if (next_b < 0) {
+                    const int w = warp - 4;
+                    if constexpr (KV8)
+                        stage = w < 5 ? c.smem + e4::OFF_Q + w * 16384 : c.smem + e4::OFF_SR + (w - 5) * 16384;
+                    else
+                        stage = c.smem + OFF_SR + w * 16384;
+                }
+                merge_block(pc.b, ustart, n_parts, stage);
             }
         }
     }
