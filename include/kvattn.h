@@ -41,8 +41,11 @@
  *  - Scratch memory: the library keeps one workspace per device, grown with
  *    cudaMalloc when a call needs more than it holds and kept until
  *    kvattn_release_workspace().  A call that grows it is not capturable in a CUDA
- *    graph; issue one call of the largest shape before capturing.  Calls that share a
- *    device must be ordered (same stream, or synchronised): they share the workspace.
+ *    graph; issue one call of the largest shape before capturing.  A captured decode
+ *    call may be replayed any number of times: its kernels derive the work split from
+ *    the device-side seq_lens at every launch, so the lengths (not the shapes or
+ *    pointers) may change between replays.  Calls that share a device must be ordered
+ *    (same stream, or synchronised): they share the workspace.
  *  - Thread safety: entry points may be called from several host threads; the
  *    workspace is guarded by a mutex, but see the ordering rule above.
  */

@@ -210,7 +210,10 @@ struct Ctx {
 
 // Merge counters of the split sequences: one per (sequence, CTA rank, softmax warp), each
 // counting the workers whose partial block of that warp has been written in the call
-// numbered by its high 32 bits.  Zero at load; a call's first arrival re-tags it.
+// numbered by its high 32 bits.  Zero at load; a call's first arrival re-tags it, and its
+// last arrival sets the count back to zero under the same tag, so that a launch replayed
+// with the same number (a captured CUDA graph) counts from zero again.  The tag keeps a
+// call that stopped early (an error flag set) from corrupting the next call's count.
 __device__ unsigned long long g_mla_merge_count[MAX_BATCH * 2 * NSOFT];
 
 // One arrival of this call at a merge counter; true for the last of n arrivals.  The
@@ -221,7 +224,13 @@ __device__ __forceinline__ bool merge_arrive_last(unsigned long long *cnt, unsig
     for (int i = 0; i < (1 << 20); ++i) {
         nxt = (unsigned int)(cur >> 32) == epoch ? cur + 1 : ((unsigned long long)epoch << 32) | 1ull;
         const unsigned long long prev = atomicCAS(cnt, cur, nxt);
-        if (prev == cur) return (unsigned int)(nxt & 0xffffffffull) == (unsigned int)n;
+        if (prev == cur) {
+            const bool last = (unsigned int)(nxt & 0xffffffffull) == (unsigned int)n;
+            // every arrival of this launch is in: no one reads the count again before the
+            // next launch
+            if (last) atomicExch(cnt, (unsigned long long)epoch << 32);
+            return last;
+        }
         cur = prev;
     }
     atomicOr(&g_device_flags, FLAG_PEER_WAIT);
