@@ -495,9 +495,11 @@ int run_gqa_tc(const GqaParams &base, const CUtensorMap &kmap, const CUtensorMap
         snprintf(t_detail, sizeof(t_detail), "needs %d B shared memory", smem);
         return KVATTN_ERR_UNSUPPORTED;
     }
-    const long long max_tiles =
-        (long long)p.B * units_per_seq * ((p.T_max + gqatc::TILE - 1) / gqatc::TILE);
-    p.min_tiles = g_force_min_tiles > 0 ? g_force_min_tiles : 2;
+    const int unit_tiles = (p.T_max + gqatc::TILE - 1) / gqatc::TILE;
+    const long long max_tiles = (long long)p.B * units_per_seq * unit_tiles;
+    // at least two tiles a worker, but never more than a unit can have: units shorter
+    // than that then get a worker each instead of sharing one in turn
+    p.min_tiles = g_force_min_tiles > 0 ? g_force_min_tiles : (unit_tiles < 2 ? (unit_tiles > 0 ? unit_tiles : 1) : 2);
     long long workers = g_force_workers > 0 ? g_force_workers : dev->sms;
     const long long by_size = (max_tiles + p.min_tiles - 1) / p.min_tiles;
     if (g_force_workers <= 0 && workers > by_size) workers = by_size;
@@ -890,8 +892,12 @@ int mla_decode_impl(const uint16_t *q_latent, const uint16_t *q_rope, const MlaC
         }
         dev->mla_clusters = n < dev->sms / 2 ? n : dev->sms / 2;
     }
-    const long long max_tiles = (long long)batch * ((cache.capacity + mla::TILE - 1) / mla::TILE);
-    p.min_tiles = g_force_min_tiles > 0 ? g_force_min_tiles : 4;
+    const int seq_tiles = (cache.capacity + mla::TILE - 1) / mla::TILE;
+    const long long max_tiles = (long long)batch * seq_tiles;
+    // at least four tiles a worker, but never more than a sequence can have: a batch of
+    // short sequences then gets a CTA pair per sequence instead of pairs that take
+    // several sequences in turn (a query load, a first tile and an epilogue each)
+    p.min_tiles = g_force_min_tiles > 0 ? g_force_min_tiles : (seq_tiles < 4 ? (seq_tiles > 0 ? seq_tiles : 1) : 4);
     long long workers = g_force_workers > 0 ? g_force_workers : dev->mla_clusters;
     const long long by_size = (max_tiles + p.min_tiles - 1) / p.min_tiles;
     if (g_force_workers <= 0 && workers > by_size) workers = by_size;
