@@ -11,7 +11,7 @@
 //    completion with tcgen05.commit on an mbarrier of its own CTA;
 //  - TMEM addresses are (lane << 16) | column; a warp may only touch the 32 lanes of its
 //    quadrant (warp_id % 4).
-// No TMA or bulk load in this library uses .multicast::cluster.
+// No TMA or bulk load in this library is multicast to the CTAs of a cluster.
 #pragma once
 #include "common.cuh"
 
