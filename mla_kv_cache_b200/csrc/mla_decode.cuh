@@ -65,7 +65,8 @@
 // worker boundary leaves one partial block (and log-sum-exp) per worker in the
 // workspace; the warp then counts itself in at a per-(sequence, rank, warp) counter, and
 // the last of the sequence's workers to arrive merges that block's partials by
-// log-sum-exp into the output.  No worker waits for another, and there is no second
+// log-sum-exp into the output (a sequence cut in two, after the worker's last piece:
+// its own block again from tensor memory, only the other part's from the workspace).  No worker waits for another, and there is no second
 // kernel.  Empty sequences (no worker) get out = 0, lse = -inf, spread over the workers.
 // Every wait is bounded; every wait ahead of a warp-collective instruction is made
 // warp-uniform.  No TMA load uses multicast.
@@ -765,11 +766,9 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
     // warp's scratch (32 parts at a time); each load instruction then reads four rows'
     // 128 contiguous bytes (eight lanes per row).  The partials are read through L2
     // (other SMs wrote them), and the merge is a chain of L2 round trips, so it keeps
-    // many loads in flight: up to NPR parts' log-sum-exps are read once, together; two
-    // parts (the usual cut), when `stage` (16 KB of shared memory no one else uses) is
-    // given, two column chunks at a time (32 copies in flight); otherwise two parts' loads
-    // of one chunk go together.
-    auto merge_block = [&](int b, long long ustart, int n_parts, uint8_t *stage) {
+    // many loads in flight: up to NPR parts' log-sum-exps are read once, together, and
+    // two parts' loads of one column chunk go together.
+    auto merge_block = [&](int b, long long ustart, int n_parts) {
         const long long c_first = ustart / c.W;
         auto part_row = [&](int j, int h) -> size_t {
             const long long cw = c_first + j;
@@ -836,48 +835,6 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
                 }
             }
             __syncwarp();
-            if (n_parts == 2 && stage != nullptr) {
-                // two column chunks of both parts in flight: copied by cp.async into this
-                // warp's 16 KB of idle shared memory (a lane reads back only its own copies,
-                // so its own wait is enough), then merged from there
-                // (a part's rows are consecutive: row head0 + rr of part j is rr rows after
-                // row head0)
-                const float *src0 = p.ws_o + part_row(0, head0 + (lane >> 3)) * 512 + col0 + 4 * (lane & 7);
-                const float *src1 = p.ws_o + part_row(1, head0 + (lane >> 3)) * 512 + col0 + 4 * (lane & 7);
-#pragma unroll 1
-                for (int cp = 0; cp < 2; ++cp) {   // column chunks 2cp, 2cp + 1
-#pragma unroll
-                    for (int e = 0; e < 2; ++e)
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int off = 4 * i * 512 + 32 * (2 * cp + e);
-                            uint8_t *d = stage + ((e * 8 + i) * 2 * 32 + lane) * 16;
-                            cp_async16(d, src0 + off);
-                            cp_async16(d + 32 * 16, src1 + off);
-                        }
-                    cp_async_wait_all();
-#pragma unroll
-                    for (int e = 0; e < 2; ++e)
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int rr = 4 * i + (lane >> 3);
-                            const uint8_t *d = stage + ((e * 8 + i) * 2 * 32 + lane) * 16;
-                            const float4 x0 = *reinterpret_cast<const float4 *>(d);
-                            const float4 x1 = *reinterpret_cast<const float4 *>(d + 32 * 16);
-                            const float w0 = *wslot(0, rr), w1 = *wslot(1, rr);
-                            float4 o;
-                            o.x = fmaf(w1, x1.x, w0 * x0.x);
-                            o.y = fmaf(w1, x1.y, w0 * x0.y);
-                            o.z = fmaf(w1, x1.z, w0 * x0.z);
-                            o.w = fmaf(w1, x1.w, w0 * x0.w);
-                            const int h_r = head0 + rr;
-                            if (h_r < p.H)
-                                *reinterpret_cast<float4 *>(p.out + ((size_t)b * p.H + h_r) * 512 + col0 +
-                                                            32 * (2 * cp + e) + 4 * (lane & 7)) = o;
-                        }
-                }
-                continue;
-            }
 #pragma unroll 1
             for (int cc = 0; cc < 4; ++cc) {
                 float4 acc[8];
@@ -925,6 +882,62 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
             if (jb + JB < n_parts) __threadfence_block();   // this warp reads its stores back
         }
         if (part == 0 && hl < p.H) p.lse[(size_t)b * p.H + hl] = lse_all;
+    };
+
+    // Merge of a sequence cut in two, by the warp that arrived last, after its worker's
+    // last piece (its block of O is still in tensor memory, and `stage`, 16 KB of shared
+    // memory, is idle): only the other part's block is read, with its log-sum-exp, in one
+    // round trip -- a copy instruction moves one row of the block, stored in `stage` with
+    // row rr's 16-byte unit u at unit u ^ rr, so that a lane then reads and rewrites its
+    // own row at the 16-byte minimum of bank conflicts -- and this warp's own block comes
+    // from tensor memory again (inv normalises it, lse_own is its log-sum-exp).  The
+    // merged rows go out one row per store instruction.
+    auto merge_pair_own = [&](int b, long long ustart, uint8_t *stage, float inv, float lse_own) {
+        const long long c_first = ustart / c.W;
+        const long long cw = c.worker == c_first ? c_first + 1 : c_first;   // the other part's worker
+        const int slot = (ustart <= cw * c.W) ? 0 : 1;
+        const size_t row0 = ((size_t)cw * 2 + slot) * HR + head0;
+        const float *src = p.ws_o + row0 * 512 + col0 + 4 * lane;
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) cp_async16(stage + rr * 512 + ((lane ^ rr) << 4), src + (size_t)rr * 512);
+        const float lse_oth = __ldcg(p.ws_lse + row0 + lane);
+        const float M = fmaxf(lse_own, lse_oth);
+        float lse_all = -INFINITY, w_own = 0.f, w_oth = 0.f;
+        if (M != -INFINITY) {
+            const float S = (lse_own == -INFINITY ? 0.f : fast_exp2((lse_own - M) * 1.4426950408889634f)) +
+                            (lse_oth == -INFINITY ? 0.f : fast_exp2((lse_oth - M) * 1.4426950408889634f));
+            lse_all = M + __logf(S);
+            w_own = lse_own == -INFINITY ? 0.f : fast_exp2((lse_own - lse_all) * 1.4426950408889634f);
+            w_oth = lse_oth == -INFINITY ? 0.f : fast_exp2((lse_oth - lse_all) * 1.4426950408889634f);
+        }
+        const float wi = w_own * inv;
+        cp_async_wait_all();
+        __syncwarp();   // every lane's copies, before any lane reads its row
+        tc_fence_after();
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+            uint32_t ov[32];
+            tmem_ld32(c.tmem + lane_base + TM_O + 128 * cg + 32 * cc, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4) {
+                float4 *sx = reinterpret_cast<float4 *>(stage + lane * 512 + (((8 * cc + k4) ^ lane) << 4));
+                float4 x = *sx;
+                x.x = fmaf(w_oth, x.x, wi * __uint_as_float(ov[4 * k4]));
+                x.y = fmaf(w_oth, x.y, wi * __uint_as_float(ov[4 * k4 + 1]));
+                x.z = fmaf(w_oth, x.z, wi * __uint_as_float(ov[4 * k4 + 2]));
+                x.w = fmaf(w_oth, x.w, wi * __uint_as_float(ov[4 * k4 + 3]));
+                *sx = x;
+            }
+        }
+        __syncwarp();
+        float *dst = p.out + ((size_t)b * p.H + head0) * 512 + col0 + 4 * lane;
+#pragma unroll 4
+        for (int rr = 0; rr < 32; ++rr)
+            if (head0 + rr < p.H)
+                *reinterpret_cast<float4 *>(dst + (size_t)rr * 512) =
+                    *reinterpret_cast<const float4 *>(stage + rr * 512 + ((lane ^ rr) << 4));
+        if (part == 0 && head0 + lane < p.H) p.lse[(size_t)b * p.H + head0 + lane] = lse_all;
     };
 
     // Empty sequences (no tile, no worker): out 0, lse -inf, spread over the workers.
@@ -1197,7 +1210,10 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
                 __syncwarp();
             }
         }
-        if (realq && part == 0) {
+        // a partial's log-sum-exp is written by every warp for its own rows (the four parts
+        // of a head hold the same value), so that this warp's arrival below orders it
+        // before the merging warp, the same warp of another worker, reads it
+        if (realq && (part == 0 || !pc.whole)) {
             if (pc.whole)
                 p.lse[(size_t)pc.b * p.H + head] = lse_v;
             else
@@ -1231,7 +1247,10 @@ __device__ __forceinline__ void softmax_warps(const MlaParams &p, const Ctx &c, 
                     else
                         stage = c.smem + OFF_SR + w * 16384;
                 }
-                merge_block(pc.b, ustart, n_parts, stage);
+                if (n_parts == 2 && stage != nullptr)
+                    merge_pair_own(pc.b, ustart, stage, inv, lse_v);
+                else
+                    merge_block(pc.b, ustart, n_parts);
             }
         }
     }
