@@ -73,3 +73,10 @@ def test_reference_arm_two_ranks_prints_once(oracle_lib):
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2
     assert rec["value"] > 0 and rec["cpu_baseline"]["kind"] == "oracle"
     assert rec["e2e"]["h2d_bytes_per_step"] == 0
+    # the reference arm's config object is the one the GPU arm prints for the same workload
+    import bench
+    from mla_kv_cache_b200 import workloads as wl
+    name = "gqa_b1_h8_kv2_d64_t512"
+    cfg = wl.CONFIGS[name]
+    lens = [cfg.max_seq_len] * cfg.batch
+    assert rec["config"] == bench.config_fields(name, cfg, bench.step_bytes(cfg, lens), 2)
